@@ -1,0 +1,545 @@
+"""Benchmark of the GQA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one gqa_forward call over the decode workload of a Mistral-7B-shaped
+layer (B=16, Hq=32, Hkv=8, Sq=1, Sk=4096 KV cache, D=128, bf16, q/k/v i.i.d.
+N(0,1) from the seeded generator, no mask, scale 1/sqrt(128)).  The metric is
+decode KV-read GB/s: the algorithmic bytes of q, k, v and out per call
+(268,697,600 B) over the device time.  Inputs are resident in HBM before the
+timed region; the timed launches rotate over enough copies of K/V that no
+launch finds its K/V in the 126 MB L2.
+
+Extra measurements on the same line (N=1 only): the long-context decode of a
+Llama-2-70B-shaped layer (GB/s), the causal prefill (TFLOP/s) and the padded
+masked prefill (TFLOP/s), each with its roofline fraction.
+
+N > 1 (one process per GPU under torchrun): every rank runs its own copy of the
+workload (weak scaling, no data-path collective); the timed region is bracketed
+by a barrier and a device synchronise, and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the correctness reference, not a
+tuned baseline) on bounded samples of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402  (seeded inputs; no attention arithmetic)
+
+DECODE = dict(name="decode_mistral7b_layer", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128,
+              causal=False, mask=False, seed=2)
+DECODE_LONG = dict(name="decode_llama2_70b_layer", B=16, Hq=64, Hkv=8, Sq=1, Sk=32768, D=128,
+                   causal=False, mask=False, seed=3)
+PREFILL_CAUSAL = dict(name="prefill_causal", B=4, Hq=32, Hkv=8, Sq=4096, Sk=4096, D=128,
+                      causal=True, mask=False, seed=4)
+PREFILL_MASKED = dict(name="prefill_padded_mask", B=8, Hq=12, Hkv=2, Sq=2048, Sk=2048, D=64,
+                      causal=False, mask=True, seed=5)
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return (float(pk["hbm_gbs"]), float(pk["bf16_tflops"]),
+                float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured")
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _traffic_for(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source is unchanged since it was captured; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec[workload]
+        src = os.path.join(ROOT, "grouped_query_attention_fwd_b200", "csrc", kernel_file)
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+        if ent.get("source_sha256") != h:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.rows = []
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self, t0=None, t1=None):
+        rows = [r for (t, r) in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        if not rows:
+            rows = [r for (_, r) in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = [n for i, n in enumerate(names)
+                   if any(len(r) > 4 + i and r[4 + i].lower().startswith("active") for r in rows)]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ inputs
+
+def _host_inputs(cfg, torch, pin=False):
+    """Seeded q, k, v (bf16) and mask as host tensors."""
+    B, Hq, Hkv, Sq, Sk, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sq", "Sk", "D"))
+    seed = cfg["seed"]
+
+    def gen(stream, shape):
+        t = torch.empty(shape, dtype=torch.bfloat16, pin_memory=pin)
+        synth.normal_bf16_into(seed, stream, t.data_ptr(), t.numel())
+        return t
+
+    q = gen(synth.STREAM_Q, (B, Hq, Sq, D))
+    k = gen(synth.STREAM_K, (B, Hkv, Sk, D))
+    v = gen(synth.STREAM_V, (B, Hkv, Sk, D))
+    mask = None
+    if cfg["mask"]:
+        lens = synth.uniform_int(seed, synth.STREAM_MASK, B, 256, Sk)
+        mask = torch.from_numpy(synth.mask_from_lengths(lens, Sq, Sk))
+        if pin:
+            mask = mask.pin_memory()
+    return q, k, v, mask
+
+
+def _visible_pairs(cfg, mask_host):
+    if mask_host is not None:
+        return float(mask_host.sum().item()) * cfg["Hq"]
+    if cfg["causal"]:
+        S = cfg["Sq"]
+        return cfg["B"] * cfg["Hq"] * S * (S + 1) / 2.0
+    return float(cfg["B"] * cfg["Hq"] * cfg["Sq"] * cfg["Sk"])
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
+    """Device-resident timing of one workload.  Returns a dict of numbers."""
+    q, k, v, mask = _host_inputs(cfg, torch)
+    qd = q.to(dev)
+    kv_bytes = 2 * k.numel() * 2
+    copies = max(1, math.ceil(rotate_to_bytes / kv_bytes)) if kv_bytes < rotate_to_bytes else 1
+    ks = [k.to(dev) for _ in range(copies)]
+    vs = [v.to(dev) for _ in range(copies)]
+    md = mask.to(dev) if mask is not None else None
+    out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
+    plan = gqa.query(qd, ks[0], vs[0], mask=md, causal=cfg["causal"])
+    ws = gqa.workspace_for(dev, plan["workspace_bytes"])
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warmup):
+        gqa.forward(qd, ks[i % copies], vs[i % copies], mask=md, causal=cfg["causal"], out=out,
+                    workspace=ws)
+    torch.cuda.synchronize(dev)
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after warm-up: %s" % gqa.status_string(st))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        gqa.forward(qd, ks[i % copies], vs[i % copies], mask=md, causal=cfg["causal"], out=out,
+                    workspace=ws)
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    total_ms = e0.elapsed_time(e1)
+    per = [a.elapsed_time(b) for a, b in ev]
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
+    res = dict(total_ms=total_ms, per_launch_ms=statistics.mean(per),
+               per_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
+               visible_pairs=_visible_pairs(cfg, mask))
+    del ks, vs, qd, md, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def _e2e(gqa, torch, cfg, steps, dev):
+    """Through the public call with host buffers: pinned host -> device copy
+    of the step's inputs, the forward, and a device -> host read of out."""
+    q, k, v, mask = _host_inputs(cfg, torch, pin=True)
+    qd, kd, vd = (torch.empty_like(x, device=dev) for x in (q, k, v))
+    md = torch.empty_like(mask, device=dev) if mask is not None else None
+    out_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    out_d = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        qd.copy_(q, non_blocking=True)
+        kd.copy_(k, non_blocking=True)
+        vd.copy_(v, non_blocking=True)
+        if md is not None:
+            md.copy_(mask, non_blocking=True)
+        gqa.forward(qd, kd, vd, mask=md, causal=cfg["causal"], out=out_d)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    h2d = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + (mask.numel() if mask is not None else 0)
+    return ms, h2d, out_h.numel() * 2
+
+
+def _cpu_baseline(cfg, budget_s=12.0):
+    """The fp64 oracle as it stands, single-threaded, on whole (batch, kv head)
+    groups of the workload until about ``budget_s`` of CPU time."""
+    import oracle
+    B, Hq, Hkv, Sq, Sk, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sq", "Sk", "D"))
+    g = Hq // Hkv
+    qb = synth.normal_bf16_bits(cfg["seed"], synth.STREAM_Q, B * Hq * Sq * D).reshape(B, Hq, Sq, D)
+    groups, nbytes, t_used = 0, 0, 0.0
+    order = [(b, kv) for b in range(B) for kv in range(Hkv)]
+    while t_used < budget_s and groups < len(order) * 4:
+        b, kv = order[groups % len(order)]
+        ks = synth.bf16_bits_to_f64(
+            synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_K, B, Hkv, Sk, D, b, kv))[None, None]
+        vs = synth.bf16_bits_to_f64(
+            synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_V, B, Hkv, Sk, D, b, kv))[None, None]
+        qs = synth.bf16_bits_to_f64(qb[b:b + 1, kv * g:(kv + 1) * g])
+        t0 = time.perf_counter()
+        oracle.forward(qs, ks, vs, causal=cfg["causal"])
+        t_used += time.perf_counter() - t0
+        groups += 1
+        nbytes += 2 * (qs.size * 2) + 2 * (Sk * D * 2)
+    return dict(value=nbytes / t_used / 1e9, unit="GB/s", cores=1, kind="oracle",
+                sample="%d (batch, kv-head) groups of %d query heads x %d keys (of %d groups), "
+                       "fp64 single-threaded, %.1f s" % (groups, g, Sk, B * Hkv, t_used))
+
+
+def _roofline_decode(res, hbm, peak_kind, workload, kernel_file="decode.cu"):
+    per_s = res["per_launch_ms"] / 1e3
+    ab = res["plan"]["algorithmic_bytes"]
+    achieved = ab / per_s / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
+            "traffic": _traffic_for(kernel_file, workload),
+            "algorithmic_bytes_per_launch": ab,
+            "launch_ms": round(res["per_launch_ms"], 5)}
+
+
+def _roofline_prefill(res, tflops, peak_kind, workload):
+    per_s = res["per_launch_ms"] / 1e3
+    fl = res["plan"]["algorithmic_flops"]
+    achieved = fl / per_s / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tflops, "unit": "TFLOP/s",
+            "frac": round(achieved / tflops, 4), "peak_source": peak_kind,
+            "traffic": _traffic_for("prefill.cu", workload),
+            "algorithmic_flops_per_launch": fl, "launch_ms": round(res["per_launch_ms"], 5)}
+
+
+def run_gpu(args):
+    import torch
+    import grouped_query_attention_fwd_b200 as gqa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    hbm, tf_burst, tf_sus, peak_kind = _peaks()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(props.uuid)
+    except Exception:
+        gpu_id = None
+
+    cfg = DECODE
+    q, k, v, _ = _host_inputs(cfg, torch)
+    qd = q.to(dev)
+    kv_bytes = 2 * k.numel() * 2
+    copies = max(1, math.ceil(3 * L2_BYTES / kv_bytes))
+    ks = [k.to(dev) for _ in range(copies)]
+    vs = [v.to(dev) for _ in range(copies)]
+    del q, k, v
+    out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
+    plan = gqa.query(qd, ks[0], vs[0])
+    ws = gqa.workspace_for(dev, plan["workspace_bytes"])
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(args.warmup):
+        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+    torch.cuda.synchronize(dev)
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after warm-up: %s" % gqa.status_string(st))
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    sampler.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    per_launch = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    del ks, vs
+    torch.cuda.empty_cache()
+
+    total_bytes = plan["algorithmic_bytes"] * args.steps * world
+    value = total_bytes / (elapsed_ms / 1e3) / 1e9
+    clocks = sampler.summary(t_wall0 - 0.2, t_wall1 + 0.2)
+
+    line = {
+        "metric": "GQA decode KV-read GB/s (% HBM peak); prefill TFLOP/s (% bf16 TC peak)",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: q/k/v i.i.d. N(0,1) from a seeded SplitMix64/Box-Muller generator, rounded to bf16",
+        "config": {
+            "workload": "decode, Mistral-7B-shaped layer: B=16 Hq=32 Hkv=8 (g=4) Sq=1 Sk=4096 "
+                        "D=128 bf16, no mask, scale=1/sqrt(128)",
+            "B": 16, "Hq": 32, "Hkv": 8, "Sq": 1, "Sk": 4096, "D": 128,
+            "parallelism": "replicas" if world == 1 else "dp%d (independent problems per rank)" % world,
+            "l2": "K/V rotated over %d device copies (%.0f MB) so no launch finds its K/V in L2"
+                  % (copies, copies * kv_bytes / 1e6),
+        },
+        "gpu_launches": args.steps * plan["launches"],
+        "clocks": {k_: v_ for k_, v_ in clocks.items()},
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(plan["algorithmic_bytes"] / (per_launch / 1e3) / 1e9, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(plan["algorithmic_bytes"] / (per_launch / 1e3) / 1e9 / hbm, 4),
+            "traffic": _traffic_for("decode.cu", DECODE["name"]),
+            "peak_source": peak_kind,
+            "kernel": "gqa_decode_kernel + gqa_decode_combine_kernel (timed together per call)",
+            "algorithmic_bytes_per_launch": plan["algorithmic_bytes"],
+            "launch_ms": round(per_launch, 5),
+        },
+    }
+
+    if rank == 0 and world == 1 and not args.skip_extra:
+        extra = {}
+        for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED):
+            try:
+                res = _time_config(gqa, torch, c, steps=max(3, min(args.steps, 50)),
+                                   warmup=max(3, min(args.warmup, 10)), dev=dev)
+            except Exception as e:  # report, keep the primary line
+                extra[c["name"]] = {"unavailable": "%s: %s" % (type(e).__name__, e)}
+                continue
+            if c["Sq"] == 1:
+                rf = _roofline_decode(res, hbm, peak_kind, c["name"])
+                extra[c["name"]] = {"value": rf["achieved"], "unit": "GB/s", "roofline": rf}
+            else:
+                rf = _roofline_prefill(res, tf_burst, peak_kind, c["name"])
+                vis = res["visible_pairs"] * 4 * c["D"] / (res["per_launch_ms"] / 1e3) / 1e12
+                extra[c["name"]] = {"value": rf["achieved"], "unit": "TFLOP/s", "roofline": rf,
+                                    "visible_pairs_tflops": round(vis, 1),
+                                    "frac_of_sustained_peak": round(rf["achieved"] / tf_sus, 4)}
+        line["extra"] = extra
+
+    if rank == 0 and not args.skip_e2e:
+        e2e_steps = max(3, min(args.steps, 20))
+        ms, h2d, d2h = _e2e(gqa, torch, DECODE, e2e_steps, dev)
+        line["e2e"] = {"value": round(plan["algorithmic_bytes"] / (ms / 1e3) / 1e9, 2),
+                       "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(ms, 4),
+                       "note": "pinned host q/k/v copied to the device, gqa_forward, out copied back, every step"}
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = _cpu_baseline(DECODE)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = DECODE
+    B, Hq, Hkv, Sk, D = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["Sk"], cfg["D"]
+    g = Hq // Hkv
+    qb = synth.normal_bf16_bits(cfg["seed"], synth.STREAM_Q, B * Hq * D).reshape(B, Hq, 1, D)
+    order = [(b, kv) for b in range(B) for kv in range(Hkv)]
+    cache = {}
+
+    def group(i):
+        b, kv = order[i % len(order)]
+        if (b, kv) not in cache:
+            ks = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_K, B, Hkv, Sk, D, b, kv))
+            vs = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_V, B, Hkv, Sk, D, b, kv))
+            cache[(b, kv)] = (synth.bf16_bits_to_f64(qb[b:b + 1, kv * g:(kv + 1) * g]),
+                              ks[None, None], vs[None, None])
+        return cache[(b, kv)]
+
+    # Calibrate one group, then size each step so that the run stays bounded.
+    t0 = time.perf_counter()
+    oracle.forward(*group(0))
+    t_group = max(time.perf_counter() - t0, 1e-4)
+    budget = 60.0
+    per_step = int(max(1, min(len(order), budget / ((args.steps + args.warmup) * t_group))))
+    group_bytes = 2 * g * D * 2 + 2 * Sk * D * 2
+    idx = 0
+    for _ in range(args.warmup):
+        for _ in range(per_step):
+            oracle.forward(*group(idx))
+            idx += 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(per_step):
+            oracle.forward(*group(idx))
+            idx += 1
+    el = time.perf_counter() - t0
+    value = group_bytes * per_step * args.steps / el / 1e9
+    sample = ("%d of %d (batch, kv-head) groups per step (g=%d query heads x %d keys each), "
+              "fp64 oracle, single thread" % (per_step, len(order), g, Sk))
+    line = {
+        "metric": "GQA decode KV-read GB/s (% HBM peak); prefill TFLOP/s (% bf16 TC peak)",
+        "impl": "reference",
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: same seeded inputs as the GPU arm",
+        "config": {"workload": "decode, Mistral-7B-shaped layer: B=16 Hq=32 Hkv=8 Sq=1 Sk=4096 "
+                               "D=128, bounded sample per step (see cpu_baseline.sample)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-extra", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+"""Grouped-query attention forward on B200 (sm_100a): Python binding.
+
+Argument marshalling over the C ABI declared in ``include/gqa.h``: tensors go
+in as device pointers, sizes and element strides; every step of the attention
+runs in the CUDA kernels of ``libgqa_b200.so``.  There is no CPU or PyTorch
+fallback: if the library is missing this module raises at import time.
+
+    out = forward(q, k, v, mask=None, causal=False, scale=None)
+
+q [B, Hq, Sq, D], k and v [B, Hkv, Sk, D] (CUDA tensors, bf16 or fp32, last
+dim contiguous), mask bool/uint8 [B, Sq, Sk] (True = attend, shared by all
+heads), ``scale`` defaults to 1/sqrt(D).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libgqa_b200.so is not built (run __graft_entry__.build() or "
+        "python -m grouped_query_attention_fwd_b200._build); there is no fallback path")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+GQA_OK = 0
+GQA_ERR_NULL, GQA_ERR_SHAPE, GQA_ERR_LAYOUT, GQA_ERR_UNSUPPORTED = 1, 2, 3, 4
+GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 5, 6, 7, 8, 9
+GQA_DTYPE_BF16, GQA_DTYPE_F32 = 0, 1
+KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero"}
+
+EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version")
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32), ("has_mask", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("batch", ctypes.c_int64), ("heads_q", ctypes.c_int64), ("heads_kv", ctypes.c_int64),
+        ("seq_q", ctypes.c_int64), ("seq_k", ctypes.c_int64), ("head_dim", ctypes.c_int64),
+        ("q_stride", ctypes.c_int64 * 4), ("k_stride", ctypes.c_int64 * 4),
+        ("v_stride", ctypes.c_int64 * 4), ("o_stride", ctypes.c_int64 * 4),
+        ("mask_stride", ctypes.c_int64 * 3),
+    ]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [
+        ("kernel", ctypes.c_int32), ("grid", ctypes.c_int32), ("block", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int32), ("launches", ctypes.c_int32),
+        ("work_units", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
+        ("algorithmic_bytes", ctypes.c_int64), ("algorithmic_flops", ctypes.c_double),
+    ]
+
+    def as_dict(self):
+        d = {f: getattr(self, f) for f, _ in self._fields_}
+        d["kernel_name"] = KERNEL_NAMES.get(self.kernel, "?")
+        return d
+
+
+_vp = ctypes.c_void_p
+_lib.gqa_query.argtypes = [ctypes.POINTER(Problem), ctypes.c_int, ctypes.POINTER(Plan)]
+_lib.gqa_query.restype = ctypes.c_int
+_lib.gqa_forward.argtypes = [ctypes.POINTER(Problem), _vp, _vp, _vp, _vp, _vp, _vp,
+                             ctypes.c_size_t, _vp]
+_lib.gqa_forward.restype = ctypes.c_int
+_lib.gqa_device_status.argtypes = [_vp, _vp]
+_lib.gqa_device_status.restype = ctypes.c_int
+_lib.gqa_status_string.argtypes = [ctypes.c_int]
+_lib.gqa_status_string.restype = ctypes.c_char_p
+_lib.gqa_version.argtypes = []
+_lib.gqa_version.restype = ctypes.c_int
+
+
+class GQAError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where or "gqa", status_string(status), status))
+
+
+def status_string(status: int) -> str:
+    return _lib.gqa_status_string(status).decode()
+
+
+def version() -> int:
+    return _lib.gqa_version()
+
+
+def make_problem(dtype: int, B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int,
+                 q_stride, k_stride, v_stride, o_stride, mask_stride=None,
+                 causal: bool = False, scale: float | None = None) -> Problem:
+    """Build the C problem descriptor from plain sizes and element strides."""
+    p = Problem()
+    p.dtype = dtype
+    p.causal = int(bool(causal))
+    p.has_mask = int(mask_stride is not None)
+    p.scale = float((1.0 / math.sqrt(D) if D > 0 else 1.0) if scale is None else scale)
+    p.batch, p.heads_q, p.heads_kv, p.seq_q, p.seq_k, p.head_dim = B, Hq, Hkv, Sq, Sk, D
+    for i in range(4):
+        p.q_stride[i], p.k_stride[i] = int(q_stride[i]), int(k_stride[i])
+        p.v_stride[i], p.o_stride[i] = int(v_stride[i]), int(o_stride[i])
+    if mask_stride is not None:
+        for i in range(3):
+            p.mask_stride[i] = int(mask_stride[i])
+    return p
+
+
+def query_problem(p: Problem, sm_count: int = 0) -> Plan:
+    plan = Plan()
+    rc = _lib.gqa_query(ctypes.byref(p), int(sm_count), ctypes.byref(plan))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_query")
+    return plan
+
+
+def forward_ptrs(p: Problem, q: int, k: int, v: int, mask: int | None, out: int,
+                 workspace: int, workspace_bytes: int, stream: int) -> None:
+    """Raw pointer form of gqa_forward (all device pointers)."""
+    rc = _lib.gqa_forward(ctypes.byref(p), q, k, v, mask, out, workspace,
+                          workspace_bytes, stream)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_forward")
+
+
+# --------------------------------------------------------------- torch glue
+# torch is used only to own device memory and to name the current stream.
+
+def _torch():
+    import torch
+    return torch
+
+
+_workspaces = {}
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return GQA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return GQA_DTYPE_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None) -> Problem:
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, S, D]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    B, Hq, Sq, D = q.shape
+    Bk, Hkv, Sk, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+        raise ValueError("k and v must be [B, Hkv, Sk, D] with q's B and D")
+    ost = out.stride() if out is not None else (Hq * Sq * D, Sq * D, D, 1)
+    mst = None
+    if mask is not None:
+        if tuple(mask.shape) != (B, Sq, Sk):
+            raise ValueError("mask must be [B, Sq, Sk]")
+        mst = mask.stride()
+    return make_problem(_dtype_code(q), B, Hq, Hkv, Sq, Sk, D, q.stride(), k.stride(),
+                        v.stride(), ost, mst, causal=causal, scale=scale)
+
+
+def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0) -> dict:
+    return query_problem(problem_for(q, k, v, mask, causal, scale), sm_count).as_dict()
+
+
+def workspace_for(device, nbytes: int):
+    """A zeroed, cached device workspace of at least ``nbytes`` for ``device``."""
+    torch = _torch()
+    key = torch.device(device).index if torch.device(device).index is not None else \
+        torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=torch.device("cuda", key))
+        _workspaces[key] = ws
+    return ws
+
+
+def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=None,
+            stream=None):
+    """out = softmax(mask(q k_{h/g}^T * scale)) v_{h/g} on the GPU."""
+    torch = _torch()
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors (there is no CPU path)")
+    if mask is not None:
+        if not mask.is_cuda:
+            raise ValueError("mask must be a CUDA tensor")
+        if mask.dtype == torch.bool:
+            mask = mask.view(torch.uint8)
+        elif mask.dtype != torch.uint8:
+            raise TypeError("mask must be bool or uint8")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    p = problem_for(q, k, v, mask, causal, scale, out)
+    plan = query_problem(p)
+    if workspace is None:
+        workspace = workspace_for(q.device, plan.workspace_bytes)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    forward_ptrs(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                 mask.data_ptr() if mask is not None else None, out.data_ptr(),
+                 workspace.data_ptr(), workspace.numel(), stream)
+    return out
+
+
+def device_status(workspace=None, stream=None) -> int:
+    """Synchronise and read/clear the workspace error word (GQA_OK or an error)."""
+    torch = _torch()
+    if workspace is None:
+        workspace = workspace_for(torch.cuda.current_device(), 256)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return _lib.gqa_device_status(workspace.data_ptr(), stream)

@@ -1,0 +1,337 @@
+// C-ABI layer: validation, planning, TMA descriptor encoding and dispatch.
+// Every entry point returns a status code; nothing throws across the ABI.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "gqa.h"
+#include "kernels.h"
+
+namespace gqa {
+namespace {
+
+constexpr int64_t kErrWordBytes = 256;  // workspace head reserved for the error word
+
+bool bf16_paths(const gqa_problem& p) { return p.dtype == GQA_DTYPE_BF16; }
+
+int validate(const gqa_problem* pp) {
+  if (pp == nullptr) return GQA_ERR_NULL;
+  const gqa_problem& p = *pp;
+  if (p.dtype != GQA_DTYPE_BF16 && p.dtype != GQA_DTYPE_F32) return GQA_ERR_ARG;
+  if (!std::isfinite(p.scale)) return GQA_ERR_ARG;
+  if (p.batch < 0 || p.seq_q < 0 || p.seq_k < 0) return GQA_ERR_SHAPE;
+  if (p.heads_q <= 0 || p.heads_kv <= 0 || p.head_dim <= 0) return GQA_ERR_SHAPE;
+  if (p.heads_q % p.heads_kv != 0) return GQA_ERR_SHAPE;
+  // Sizes must fit the kernels' 32-bit coordinates.
+  const int64_t lim = int64_t(1) << 31;
+  if (p.batch >= lim || p.heads_q >= lim || p.seq_q >= lim || p.seq_k >= lim) return GQA_ERR_SHAPE;
+  if (p.q_stride[3] != 1 || p.k_stride[3] != 1 || p.v_stride[3] != 1 || p.o_stride[3] != 1)
+    return GQA_ERR_LAYOUT;
+  if (p.has_mask && p.mask_stride[2] != 1) return GQA_ERR_LAYOUT;
+  for (int d = 0; d < 3; ++d)
+    if (p.q_stride[d] < 0 || p.k_stride[d] < 0 || p.v_stride[d] < 0 || p.o_stride[d] < 0 ||
+        (p.has_mask && p.mask_stride[d] < 0))
+      return GQA_ERR_LAYOUT;
+  if (p.causal && p.seq_q != p.seq_k) return GQA_ERR_UNSUPPORTED;
+  if (bf16_paths(p)) {
+    if (p.head_dim != 64 && p.head_dim != 128) return GQA_ERR_UNSUPPORTED;
+    // 16-byte rule of the TMA unit for every stride of a dimension longer than 1.
+    const int64_t qsz[3] = {p.batch, p.heads_q, p.seq_q};
+    const int64_t ksz[3] = {p.batch, p.heads_kv, p.seq_k};
+    for (int d = 0; d < 3; ++d) {
+      if (qsz[d] > 1 && (p.q_stride[d] % 8 != 0 || p.o_stride[d] % 8 != 0)) return GQA_ERR_LAYOUT;
+      if (ksz[d] > 1 && (p.k_stride[d] % 8 != 0 || p.v_stride[d] % 8 != 0)) return GQA_ERR_LAYOUT;
+    }
+    if (p.seq_q > 1) {
+      const int64_t g = p.heads_q / p.heads_kv;
+      if (g > 128) return GQA_ERR_UNSUPPORTED;  // one query position per 128-row tile at most
+    }
+  } else {
+    if (p.head_dim > 256) return GQA_ERR_UNSUPPORTED;
+  }
+  return GQA_OK;
+}
+
+int pick_kernel(const gqa_problem& p) {
+  if (p.batch == 0 || p.seq_q == 0) return GQA_KERNEL_NONE;
+  if (p.seq_k == 0) return GQA_KERNEL_ZERO;
+  if (p.dtype == GQA_DTYPE_F32) return GQA_KERNEL_F32;
+  return p.seq_q == 1 ? GQA_KERNEL_DECODE : GQA_KERNEL_PREFILL;
+}
+
+int device_sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  int sms = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_DEVICE;
+  }
+  if (major != 10) return GQA_ERR_DEVICE;
+  *out = sms;
+  return GQA_OK;
+}
+
+int64_t elem_bytes(const gqa_problem& p) { return p.dtype == GQA_DTYPE_F32 ? 4 : 2; }
+
+int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
+  std::memset(plan, 0, sizeof(*plan));
+  const int64_t eb = elem_bytes(p);
+  const int64_t qo = p.batch * p.heads_q * p.seq_q * p.head_dim * eb;
+  const int64_t kv = p.batch * p.heads_kv * p.seq_k * p.head_dim * eb;
+  plan->algorithmic_bytes = 2 * qo + 2 * kv + (p.has_mask ? p.batch * p.seq_q * p.seq_k : 0);
+  double flops = 4.0 * double(p.batch) * double(p.heads_q) * double(p.seq_q) * double(p.seq_k) *
+                 double(p.head_dim);
+  if (p.causal) flops *= 0.5;
+  plan->algorithmic_flops = flops;
+  plan->workspace_bytes = kErrWordBytes;
+  plan->kernel = pick_kernel(p);
+  switch (plan->kernel) {
+    case GQA_KERNEL_NONE:
+      break;
+    case GQA_KERNEL_ZERO:
+      plan->grid = 592;
+      plan->block = 256;
+      plan->launches = 1;
+      break;
+    case GQA_KERNEL_F32: {
+      const int64_t rows = p.batch * p.heads_q * p.seq_q;
+      plan->grid = static_cast<int32_t>((rows + 7) / 8);
+      plan->block = 256;
+      plan->launches = 1;
+      plan->work_units = static_cast<int32_t>(rows);
+      break;
+    }
+    case GQA_KERNEL_DECODE: {
+      const DecodeShape s = plan_decode(p, sm_count);
+      plan->grid = s.grid;
+      plan->block = kDecodeThreads;
+      plan->smem_bytes = s.smem_bytes;
+      plan->launches = 2;
+      plan->work_units = static_cast<int32_t>(s.units);
+      plan->workspace_bytes = kErrWordBytes + s.part_bytes;
+      break;
+    }
+    case GQA_KERNEL_PREFILL: {
+      const PrefillShape s = plan_prefill(p, sm_count);
+      plan->grid = s.grid;
+      plan->block = 192;
+      plan->smem_bytes = s.smem_bytes;
+      plan->launches = p.has_mask ? 2 : 1;
+      plan->work_units = static_cast<int32_t>(s.work);
+      plan->workspace_bytes = kErrWordBytes + s.summary_bytes;
+      break;
+    }
+  }
+  plan->workspace_bytes = (plan->workspace_bytes + 255) / 256 * 256;
+  return GQA_OK;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 4-D bf16 map over (d, s, h, b) of a tensor with element strides st[0..2]
+// for (b, h, s); box {64, box_s, box_h, 1} with 128-byte swizzle.
+int encode_bf16_map(CUtensorMap* map, const void* base, int64_t B, int64_t H, int64_t S,
+                    int64_t D, const int64_t st[4], uint32_t box_s, uint32_t box_h) {
+  auto enc = get_encoder();
+  if (enc == nullptr) return GQA_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  // Strides of length-1 dimensions are never stepped; give them a legal value.
+  int64_t sb = st[2] * 2, hb = st[1] * 2, bb = st[0] * 2;
+  if (S <= 1) sb = D * 2 < 16 ? 16 : ((D * 2 + 15) / 16) * 16;
+  if (H <= 1) hb = sb * (S > 0 ? S : 1);
+  if (B <= 1) bb = hb * (H > 0 ? H : 1);
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(sb), static_cast<cuuint64_t>(hb),
+                           static_cast<cuuint64_t>(bb)};
+  cuuint32_t box[4] = {64, box_s, box_h, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_LAYOUT;
+}
+
+bool aligned(const void* ptr, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" {
+
+GQA_API int gqa_version(void) { return 10000; }
+
+GQA_API const char* gqa_status_string(int status) {
+  switch (status) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_NULL: return "a required pointer is NULL";
+    case GQA_ERR_SHAPE: return "inconsistent or invalid sizes (heads_q must be a multiple of heads_kv)";
+    case GQA_ERR_LAYOUT: return "unsupported memory layout (innermost stride must be 1; bf16 bases and strides must be multiples of 16 bytes)";
+    case GQA_ERR_UNSUPPORTED: return "unsupported combination (bf16 needs head_dim 64 or 128; causal needs seq_q == seq_k)";
+    case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case GQA_ERR_CUDA: return "a CUDA runtime call failed";
+    case GQA_ERR_TIMEOUT: return "a kernel gave up on an internal wait; outputs are undefined";
+    case GQA_ERR_ARG: return "invalid scalar argument (scale must be finite; dtype must be known)";
+    case GQA_ERR_DEVICE: return "no usable sm_100 CUDA device";
+    default: return "unknown status";
+  }
+}
+
+GQA_API int gqa_query(const gqa_problem* p, int sm_count, gqa_plan* plan) {
+  if (plan == nullptr) return GQA_ERR_NULL;
+  const int rc = validate(p);
+  if (rc != GQA_OK) return rc;
+  if (sm_count <= 0) {
+    const int drc = device_sm_count(&sm_count);
+    if (drc != GQA_OK) return drc;
+  }
+  return fill_plan(*p, sm_count, plan);
+}
+
+GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, const void* v,
+                        const uint8_t* mask, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream_ptr) {
+  const int rc = validate(pp);
+  if (rc != GQA_OK) return rc;
+  const gqa_problem& p = *pp;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  gqa_plan plan;
+  int sms = 0;
+  {
+    const int drc = device_sm_count(&sms);
+    if (drc != GQA_OK) return drc;
+  }
+  fill_plan(p, sms, &plan);
+  if (plan.kernel == GQA_KERNEL_NONE) return GQA_OK;
+  if (out == nullptr) return GQA_ERR_NULL;
+  if (plan.kernel == GQA_KERNEL_ZERO) return launch_zero(p, out, stream);
+  if (q == nullptr || k == nullptr || v == nullptr) return GQA_ERR_NULL;
+  if (p.has_mask && mask == nullptr) return GQA_ERR_NULL;
+  if (workspace == nullptr) return GQA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || workspace_bytes < static_cast<size_t>(plan.workspace_bytes))
+    return GQA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+
+  if (plan.kernel == GQA_KERNEL_F32) {
+    if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
+      return GQA_ERR_LAYOUT;
+    return launch_f32(p, static_cast<const float*>(q), static_cast<const float*>(k),
+                      static_cast<const float*>(v), mask, static_cast<float*>(out), stream);
+  }
+
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return GQA_ERR_LAYOUT;
+  const float scale_log2 =
+      static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634073599);
+  const int64_t g = p.heads_q / p.heads_kv;
+
+  if (plan.kernel == GQA_KERNEL_DECODE) {
+    const DecodeShape s = plan_decode(p, sms);
+    CUtensorMap tmk, tmv;
+    int erc = encode_bf16_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride,
+                              kDecodeKeysPerTile, 1);
+    if (erc != GQA_OK) return erc;
+    erc = encode_bf16_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride,
+                          kDecodeKeysPerTile, 1);
+    if (erc != GQA_OK) return erc;
+    DecodeArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    for (int d = 0; d < 4; ++d) a.qs[d] = p.q_stride[d], a.os[d] = p.o_stride[d];
+    a.mask = p.has_mask ? mask : nullptr;
+    for (int d = 0; d < 3; ++d) a.ms[d] = p.mask_stride[d];
+    a.out = static_cast<uint16_t*>(out);
+    a.part_ml = reinterpret_cast<float2*>(ws + s.part_ml_offset);
+    a.part_o = reinterpret_cast<float*>(ws + s.part_o_offset);
+    a.err = err;
+    a.B = static_cast<int>(p.batch);
+    a.Hq = static_cast<int>(p.heads_q);
+    a.Hkv = static_cast<int>(p.heads_kv);
+    a.Sk = static_cast<int>(p.seq_k);
+    a.g = static_cast<int>(g);
+    a.scale_log2 = scale_log2;
+    return launch_decode(p, s, a, tmk, tmv, stream);
+  }
+
+  // Prefill.
+  const PrefillShape s = plan_prefill(p, sms);
+  CUtensorMap tmq, tmk, tmv;
+  int erc = encode_bf16_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
+                            static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g));
+  if (erc != GQA_OK) return erc;
+  erc = encode_bf16_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 128, 1);
+  if (erc != GQA_OK) return erc;
+  erc = encode_bf16_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128, 1);
+  if (erc != GQA_OK) return erc;
+  PrefillArgs a{};
+  a.mask = p.has_mask ? mask : nullptr;
+  for (int d = 0; d < 3; ++d) a.ms[d] = p.mask_stride[d];
+  a.out = static_cast<uint16_t*>(out);
+  for (int d = 0; d < 4; ++d) a.os[d] = p.o_stride[d];
+  a.summary = ws + s.summary_offset;
+  a.err = err;
+  a.B = static_cast<int>(p.batch);
+  a.Hq = static_cast<int>(p.heads_q);
+  a.Hkv = static_cast<int>(p.heads_kv);
+  a.Sq = static_cast<int>(p.seq_q);
+  a.Sk = static_cast<int>(p.seq_k);
+  a.g = static_cast<int>(g);
+  a.causal = p.causal;
+  a.has_mask = p.has_mask;
+  a.scale_log2 = scale_log2;
+  return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
+}
+
+GQA_API int gqa_device_status(void* workspace, void* stream_ptr) {
+  if (workspace == nullptr) return GQA_ERR_NULL;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  uint32_t word[4] = {0, 0, 0, 0};
+  if (cudaMemcpyAsync(word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  if (word[0] != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    return GQA_ERR_TIMEOUT;
+  }
+  return GQA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,467 @@
+// Split-K decode kernel (seq_q == 1) and its combine pass.
+//
+// Decoding re-reads the whole KV cache once per generated token and does
+// about one multiply-add per byte it reads, so its time is the KV bytes over
+// HBM bandwidth ("Multi-Query Attention", "Theory"; "Grouped-Query Attention
+// Explained Simply", "Why it matters").  The kernel is built around that
+// bound:
+//
+//  * Work unit = one 64-key tile of one (batch, kv head, head pass).  All units
+//    of the problem are laid end to end and cut into one contiguous range per
+//    CTA (a persistent grid of one CTA per SM), so every SM streams the same
+//    number of bytes whatever B * Hkv is; a range may start or end inside a
+//    kv head's key sequence (split-K), which leaves a partial softmax state.
+//  * A producer warp streams K and V tiles with TMA (128-byte swizzled boxes,
+//    so the ldmatrix reads below are bank-conflict free) into a ring of
+//    shared-memory stages guarded by mbarriers; each tile crosses HBM once.
+//  * Four consumer warps take 16 keys each of every staged tile and serve all
+//    g query heads of the group from it: the kv head is never expanded
+//    ("Multi-Query Attention": a zero stride over the head dimension).  The
+//    dot products run on the tensor cores as S^T = K Q^T with keys in the MMA
+//    M dimension and the group's heads in N (g <= 8 fills one 8-wide column
+//    tile), then O^T += V^T P^T; at g = 8 a CUDA-core version would need about
+//    as many FMA issue slots as the HBM time allows, the MMA needs a few %.
+//  * Online softmax in fp32 with warp-shuffle max/sum reductions; at the end
+//    of a range the four warps merge in shared memory and one partial
+//    (m, l, O) per head is written.  The combine kernel (launched with
+//    programmatic dependent launch so it is resident before the stream
+//    reaches it) merges the partials of each group and writes bf16 out.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int KT = kDecodeKeysPerTile;  // keys per tile
+constexpr int NCW = kDecodeConsumerWarps;
+constexpr int CHUNK_BYTES = KT * 128;   // one 64-wide bf16 column chunk of a tile
+
+__host__ __device__ inline int64_t range_start(int64_t c, int64_t T, int64_t P) {
+  return (c * T) / P;
+}
+
+template <int D, int NT>
+struct DecodeSmem {
+  static constexpr int kTileBytes = KT * D * 2;        // K (or V) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
+  static constexpr int HP = 8 * NT;
+  static constexpr int kScrRow = D + 4;                // padded head row (floats)
+  static constexpr int kScrOBytes = NCW * HP * kScrRow * 4;
+  static constexpr int kScrMLBytes = NCW * HP * 2 * 4;
+  static int bytes(int stages) {
+    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + kScrMLBytes +
+           2 * stages * 8 + 16;
+  }
+};
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    gqa_decode_kernel(const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const DecodeArgs a,
+                      const int tiles_per_group, const int passes, const int64_t units,
+                      const int segmax, const int stages) {
+  using L = DecodeSmem<D, NT>;
+  constexpr int HP = L::HP;
+  constexpr int KSTEPS = D / 16;
+  constexpr int CHUNKS = D / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem;
+  float* scr_o = reinterpret_cast<float*>(ring + stages * L::kStageBytes);
+  float* scr_ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scr_o) + L::kScrOBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scr_ml) +
+                                               L::kScrMLBytes);
+  uint64_t* empty = full + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t P = gridDim.x;
+  const int64_t u_begin = range_start(blockIdx.x, units, P);
+  const int64_t u_end = range_start(blockIdx.x + 1, units, P);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // Let the combine kernel launch and wait on this grid's completion.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == NCW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+      int64_t it = 0;
+      for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+        const int s = static_cast<int>(it % stages);
+        const uint32_t round = static_cast<uint32_t>(it / stages);
+        if (round > 0 &&
+            !mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, a.err, kErrDecodeWait))
+          break;
+        const int64_t grp = u / tiles_per_group;
+        const int t = static_cast<int>(u % tiles_per_group);
+        const int64_t bk = grp / passes;  // b * Hkv + kv
+        const int kv = static_cast<int>(bk % a.Hkv);
+        const int b = static_cast<int>(bk / a.Hkv);
+        uint8_t* st = ring + s * L::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, t * KT, kv, b);
+          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64, t * KT, kv,
+                      b);
+        }
+      }
+      // Unwind: make sure no copy is still landing in this CTA's shared memory.
+      if (*abort_flag) {
+        const int64_t issued = it;
+        for (int64_t j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+          mbar_wait_drain(&full[j % stages], static_cast<uint32_t>((j / stages) & 1));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    uint32_t bq[NT][KSTEPS][2];
+    float o[NT][KSTEPS][4];
+    float m_run[NT][2], l_run[NT][2];
+    int64_t cur = -1;
+    int seg = 0;
+    int b = 0, kv = 0, pass = 0;
+    const uint8_t* mrow = nullptr;
+
+    auto reset_state = [&]() {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) o[nt][mt][c] = 0.f;
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
+      }
+    };
+
+    auto load_q = [&]() {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hl = pass * HP + nt * 8 + (lane >> 2);  // head within the group
+        const bool ok = hl < a.g;
+        const uint16_t* qrow = a.q + b * a.qs[0] + (int64_t)(kv * a.g + (ok ? hl : 0)) * a.qs[1];
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int d0 = ks * 16 + (lane & 3) * 2;
+          bq[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+          bq[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+        }
+      }
+    };
+
+    // Merge the four warps' states of the finished range and write one partial.
+    auto flush = [&]() {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float l = l_run[nt][e];
+          l += __shfl_xor_sync(0xffffffffu, l, 4);
+          l += __shfl_xor_sync(0xffffffffu, l, 8);
+          l += __shfl_xor_sync(0xffffffffu, l, 16);
+          l_run[nt][e] = l;
+        }
+      float* my_o = scr_o + warp * HP * L::kScrRow;
+      float* my_ml = scr_ml + warp * HP * 2;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int h = nt * 8 + (lane & 3) * 2 + (c & 1);
+            const int d = mt * 16 + (lane >> 2) + ((c & 2) ? 8 : 0);
+            my_o[h * L::kScrRow + d] = o[nt][mt][c];
+          }
+        if (lane < 4) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = nt * 8 + lane * 2 + e;
+            my_ml[h * 2 + 0] = m_run[nt][e];
+            my_ml[h * 2 + 1] = l_run[nt][e];
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      const int64_t slot = (static_cast<int64_t>(blockIdx.x) * segmax + seg) * HP;
+      for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
+        const int h = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
+        float l = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            const float sc = fast_exp2(scr_ml[(w * HP + h) * 2] - M);
+            l += sc * scr_ml[(w * HP + h) * 2 + 1];
+            acc += sc * scr_o[(w * HP + h) * L::kScrRow + d];
+          }
+        }
+        a.part_o[(slot + h) * D + d] = acc;
+        if (d == 0) a.part_ml[slot + h] = make_float2(M, l);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+    };
+
+    int64_t it = 0;
+    bool ok = true;
+    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+      const int64_t grp = u / tiles_per_group;
+      const int t = static_cast<int>(u % tiles_per_group);
+      if (grp != cur) {
+        if (cur >= 0) {
+          flush();
+          ++seg;
+        }
+        cur = grp;
+        const int64_t bk = grp / passes;
+        pass = static_cast<int>(grp % passes);
+        kv = static_cast<int>(bk % a.Hkv);
+        b = static_cast<int>(bk / a.Hkv);
+        mrow = a.mask ? a.mask + b * a.ms[0] : nullptr;
+        load_q();
+        reset_state();
+      }
+      const int s = static_cast<int>(it % stages);
+      const uint32_t round = static_cast<uint32_t>(it / stages);
+      if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
+        ok = false;
+        break;
+      }
+      const uint32_t kbase = smem_u32(ring + s * L::kStageBytes);
+      const uint32_t vbase = kbase + L::kTileBytes;
+
+      // S^T[16 keys x 8 heads] = K[16 x D] Q^T[D x 8] per column tile.
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
+      {
+        const int mi = lane >> 3;
+        const int r = warp * 16 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int u16 = ((ks & 3) << 1) + (mi >> 1);
+          const uint32_t addr =
+              kbase + (ks >> 2) * CHUNK_BYTES + r * 128 + ((u16 ^ (r & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(a0, a1, a2, a3, addr);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(sc[nt], a0, a1, a2, a3, bq[nt][ks][0], bq[nt][ks][1]);
+        }
+      }
+
+      // Visibility of this thread's two keys.
+      const int64_t key0 = static_cast<int64_t>(t) * KT + warp * 16 + (lane >> 2);
+      const int64_t key1 = key0 + 8;
+      const bool vis0 = key0 < a.Sk && key_visible(mrow, key0, 0, 0);
+      const bool vis1 = key1 < a.Sk && key_visible(mrow, key1, 0, 0);
+
+      uint32_t pt0[NT], pt1[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float tv[4];
+        tv[0] = vis0 ? sc[nt][0] * a.scale_log2 : -INFINITY;
+        tv[1] = vis0 ? sc[nt][1] * a.scale_log2 : -INFINITY;
+        tv[2] = vis1 ? sc[nt][2] * a.scale_log2 : -INFINITY;
+        tv[3] = vis1 ? sc[nt][3] * a.scale_log2 : -INFINITY;
+        float alpha[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = fmaxf(tv[e], tv[e + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m_run[nt][e], mx);
+          const float ref = exp_ref(m_new);
+          alpha[e] = fast_exp2(m_run[nt][e] - ref);
+          m_run[nt][e] = m_new;
+          tv[e] = fast_exp2(tv[e] - ref);
+          tv[e + 2] = fast_exp2(tv[e + 2] - ref);
+          l_run[nt][e] = l_run[nt][e] * alpha[e] + tv[e] + tv[e + 2];
+        }
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          o[nt][mt][0] *= alpha[0];
+          o[nt][mt][1] *= alpha[1];
+          o[nt][mt][2] *= alpha[0];
+          o[nt][mt][3] *= alpha[1];
+        }
+        // P^T as the B operand: transpose the two 8x8 (keys x heads) blocks.
+        pt0[nt] = movmatrix_trans(pack_bf16x2(tv[0], tv[1]));
+        pt1[nt] = movmatrix_trans(pack_bf16x2(tv[2], tv[3]));
+      }
+
+      // O^T[D x 8] += V^T[D x 16 keys] P^T[16 keys x 8].
+      {
+        const int mi = lane >> 3;
+        const int key = warp * 16 + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          const int dcol = mt * 16 + (mi & 1) * 8;
+          const int u16 = (dcol & 63) >> 3;
+          const uint32_t addr =
+              vbase + (dcol >> 6) * CHUNK_BYTES + key * 128 + ((u16 ^ (key & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_trans(a0, a1, a2, a3, addr);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, pt0[nt], pt1[nt]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (ok && cur >= 0) flush();
+    if (!ok) {
+      // Keep the named barrier count consistent for warps still in flush():
+      // nothing else to do, the error word is already set.
+    }
+  }
+  __syncthreads();
+}
+
+// Merge the partial states of one (batch, kv head, pass) group and write
+// out[b, h, 0, :] for its heads.
+template <int D, int HP>
+__global__ void __launch_bounds__(128)
+    gqa_decode_combine_kernel(const DecodeArgs a, const int tiles_per_group, const int passes,
+                              const int64_t units, const int P, const int segmax) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t grp = blockIdx.x;
+  const int64_t bk = grp / passes;
+  const int pass = static_cast<int>(grp % passes);
+  const int kv = static_cast<int>(bk % a.Hkv);
+  const int b = static_cast<int>(bk / a.Hkv);
+  const int64_t u0 = grp * tiles_per_group, u1 = u0 + tiles_per_group;
+
+  // First CTA whose range contains u0.
+  int64_t c = (u0 * P) / units;
+  if (c > P - 1) c = P - 1;
+  while (c > 0 && range_start(c, units, P) > u0) --c;
+  while (c + 1 < P && range_start(c + 1, units, P) <= u0) ++c;
+  const int64_t c_lo = c;
+
+  for (int idx = threadIdx.x; idx < HP * D; idx += blockDim.x) {
+    const int h = idx / D, d = idx % D;
+    const int hl = pass * HP + h;
+    if (hl >= a.g) continue;
+    float M = -INFINITY;
+    for (int64_t cc = c_lo; cc < P && range_start(cc, units, P) < u1; ++cc) {
+      const int seg = static_cast<int>(grp - range_start(cc, units, P) / tiles_per_group);
+      M = fmaxf(M, a.part_ml[(cc * segmax + seg) * HP + h].x);
+    }
+    float l = 0.f, acc = 0.f;
+    if (M != -INFINITY) {
+      for (int64_t cc = c_lo; cc < P && range_start(cc, units, P) < u1; ++cc) {
+        const int seg = static_cast<int>(grp - range_start(cc, units, P) / tiles_per_group);
+        const int64_t slot = (cc * segmax + seg) * HP + h;
+        const float2 ml = a.part_ml[slot];
+        const float sc = fast_exp2(ml.x - M);
+        l += sc * ml.y;
+        acc += sc * a.part_o[slot * D + d];
+      }
+    }
+    const int hq = kv * a.g + hl;
+    a.out[b * a.os[0] + hq * a.os[1] + d] = bf16_bits_rn(acc / l);
+  }
+}
+
+template <int D, int NT>
+int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap& tmk,
+                    const CUtensorMap& tmv, cudaStream_t stream) {
+  auto kern = gqa_decode_kernel<D, NT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_bytes) !=
+      cudaSuccess)
+    return GQA_ERR_CUDA;
+  kern<<<s.grid, kDecodeThreads, s.smem_bytes, stream>>>(tmk, tmv, a, s.tiles_per_group,
+                                                          s.passes, s.units, s.segmax, s.stages);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(s.groups));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gqa_decode_combine_kernel<D, 8 * NT>, a, s.tiles_per_group,
+                         s.passes, s.units, s.grid, s.segmax) != cudaSuccess)
+    return GQA_ERR_CUDA;
+  return GQA_OK;
+}
+
+}  // namespace
+
+DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
+  DecodeShape s{};
+  const int64_t g = p.heads_q / p.heads_kv;
+  s.D = static_cast<int>(p.head_dim);
+  s.NT = g <= 8 ? 1 : 2;
+  s.HP = 8 * s.NT;
+  s.passes = static_cast<int>((g + s.HP - 1) / s.HP);
+  s.tiles_per_group = static_cast<int>((p.seq_k + KT - 1) / KT);
+  s.groups = p.batch * p.heads_kv * s.passes;
+  s.units = s.groups * s.tiles_per_group;
+  s.grid = static_cast<int>(s.units < sm_count ? s.units : sm_count);
+  if (s.grid < 1) s.grid = 1;
+  const int64_t per_cta = (s.units + s.grid - 1) / s.grid;
+  s.segmax = static_cast<int>((per_cta + s.tiles_per_group - 1) / s.tiles_per_group + 1);
+  const int stage_bytes = 2 * KT * s.D * 2;
+  if (s.D == 128)
+    s.stages = s.NT == 1 ? 6 : 5;
+  else
+    s.stages = 8;
+  if (s.D == 128 && s.NT == 1)
+    s.smem_bytes = DecodeSmem<128, 1>::bytes(s.stages);
+  else if (s.D == 128)
+    s.smem_bytes = DecodeSmem<128, 2>::bytes(s.stages);
+  else if (s.NT == 1)
+    s.smem_bytes = DecodeSmem<64, 1>::bytes(s.stages);
+  else
+    s.smem_bytes = DecodeSmem<64, 2>::bytes(s.stages);
+  (void)stage_bytes;
+  const int64_t slots = static_cast<int64_t>(s.grid) * s.segmax * s.HP;
+  s.part_ml_offset = 256;
+  s.part_o_offset = 256 + ((slots * 8 + 255) / 256) * 256;
+  s.part_bytes = (s.part_o_offset - 256) + slots * s.D * 4;
+  return s;
+}
+
+int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
+                  const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
+  (void)p;
+  if (s.D == 128 && s.NT == 1) return launch_decode_t<128, 1>(s, a, tmk, tmv, stream);
+  if (s.D == 128 && s.NT == 2) return launch_decode_t<128, 2>(s, a, tmk, tmv, stream);
+  if (s.D == 64 && s.NT == 1) return launch_decode_t<64, 1>(s, a, tmk, tmv, stream);
+  if (s.D == 64 && s.NT == 2) return launch_decode_t<64, 2>(s, a, tmk, tmv, stream);
+  return GQA_ERR_UNSUPPORTED;
+}
+
+}  // namespace gqa

@@ -1,0 +1,90 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gqa.h"
+
+namespace gqa {
+
+// ------------------------------------------------------------ decode
+// Keys per streamed tile and consumer warps per CTA of the decode kernel.
+constexpr int kDecodeKeysPerTile = 64;
+constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+
+struct DecodeShape {
+  int D;            // 64 or 128
+  int NT;           // 8-head MMA column tiles per pass (1 or 2)
+  int HP;           // heads per pass = 8 * NT
+  int passes;       // ceil(g / HP)
+  int tiles_per_group;
+  int64_t groups;   // batch * heads_kv * passes
+  int64_t units;    // groups * tiles_per_group
+  int grid;         // CTAs (<= units)
+  int segmax;       // partial segments per CTA
+  int stages;       // shared-memory ring depth
+  int smem_bytes;
+  int64_t part_o_offset, part_ml_offset, part_bytes;
+};
+
+DecodeShape plan_decode(const gqa_problem& p, int sm_count);
+
+struct DecodeArgs {
+  const uint16_t* q;
+  int64_t qs[4];
+  const uint8_t* mask;
+  int64_t ms[3];
+  uint16_t* out;
+  int64_t os[4];
+  float* part_o;
+  float2* part_ml;
+  uint32_t* err;
+  int B, Hq, Hkv, Sk, g;
+  float scale_log2;  // scale * log2(e)
+};
+
+int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
+                  const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream);
+
+// ------------------------------------------------------------ prefill
+struct PrefillShape {
+  int D;             // 64 or 128
+  int qpt;           // query positions per 128-row tile (rows = qpt * g)
+  int rows;          // qpt * g <= 128
+  int m_tiles;       // ceil(Sq / qpt)
+  int n_tiles;       // ceil(Sk / 128)
+  int64_t work;      // batch * heads_kv * m_tiles
+  int grid;
+  int smem_bytes;
+  int64_t summary_offset, summary_bytes;
+};
+
+PrefillShape plan_prefill(const gqa_problem& p, int sm_count);
+
+struct PrefillArgs {
+  const uint8_t* mask;
+  int64_t ms[3];
+  uint16_t* out;
+  int64_t os[4];
+  uint8_t* summary;  // [B][m_tiles][n_tiles]: 0 all hidden, 1 mixed, 2 all visible
+  uint32_t* err;
+  int B, Hq, Hkv, Sq, Sk, g;
+  int causal, has_mask;
+  float scale_log2;
+};
+
+int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
+                   const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                   cudaStream_t stream);
+
+// ------------------------------------------------------------ fp32 path
+int launch_f32(const gqa_problem& p, const float* q, const float* k, const float* v,
+               const uint8_t* mask, float* out, cudaStream_t stream);
+
+// ------------------------------------------------------------ zero fill (seq_k == 0)
+int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream);
+
+}  // namespace gqa

@@ -1,0 +1,117 @@
+// fp32 path on the CUDA cores, plus the zero fill used when seq_k == 0.
+//
+// The tensor cores have no fp32-operand mode with fp32 accuracy (tf32 keeps
+// 10 mantissa bits), so single precision runs here: one warp per output row
+// (b, h, i), lanes split the head dimension, online softmax in fp32 over the
+// keys of kv head h / g.  This path exists for exact-precision callers and the
+// small fp32 problems; the bf16 kernels carry the throughput.
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace gqa {
+namespace {
+
+constexpr int kMaxDPerLane = 8;  // head_dim <= 256
+
+__global__ void __launch_bounds__(256)
+    gqa_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                   const float* __restrict__ v, const uint8_t* __restrict__ mask,
+                   float* __restrict__ out, int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq,
+                   int64_t Sk, int64_t D, int64_t qs0, int64_t qs1, int64_t qs2, int64_t ks0,
+                   int64_t ks1, int64_t ks2, int64_t vs0, int64_t vs1, int64_t vs2, int64_t os0,
+                   int64_t os1, int64_t os2, int64_t ms0, int64_t ms1, int causal,
+                   float scale_log2) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= B * Hq * Sq) return;
+  const int64_t i = row % Sq;
+  const int64_t h = (row / Sq) % Hq;
+  const int64_t b = row / (Sq * Hq);
+  const int64_t g = Hq / Hkv;
+  const int64_t kv = h / g;
+
+  const float* qr = q + b * qs0 + h * qs1 + i * qs2;
+  const float* kb = k + b * ks0 + kv * ks1;
+  const float* vb = v + b * vs0 + kv * vs1;
+  const uint8_t* mrow = mask ? mask + b * ms0 + i * ms1 : nullptr;
+
+  float qv[kMaxDPerLane], acc[kMaxDPerLane];
+#pragma unroll
+  for (int e = 0; e < kMaxDPerLane; ++e) {
+    const int64_t d = lane + 32 * e;
+    qv[e] = d < D ? qr[d] : 0.f;
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int64_t jend = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;
+  for (int64_t j = 0; j < jend; ++j) {
+    if (!key_visible(mrow, j, i, causal)) continue;
+    const float* kr = kb + j * ks2;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < kMaxDPerLane; ++e) {
+      const int64_t d = lane + 32 * e;
+      if (d < D) dot = fmaf(qv[e], kr[d], dot);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    const float t = dot * scale_log2;
+    const float m_new = fmaxf(m, t);
+    const float alpha = exp2f(m - m_new);
+    const float p = exp2f(t - m_new);
+    l = l * alpha + p;
+    const float* vr = vb + j * vs2;
+#pragma unroll
+    for (int e = 0; e < kMaxDPerLane; ++e) {
+      const int64_t d = lane + 32 * e;
+      if (d < D) acc[e] = fmaf(p, vr[d], acc[e] * alpha);
+    }
+    m = m_new;
+  }
+  float* orow = out + b * os0 + h * os1 + i * os2;
+#pragma unroll
+  for (int e = 0; e < kMaxDPerLane; ++e) {
+    const int64_t d = lane + 32 * e;
+    if (d < D) orow[d] = acc[e] / l;  // l == 0 (no visible key): NaN
+  }
+}
+
+__global__ void gqa_zero_kernel(uint8_t* out, int64_t B, int64_t Hq, int64_t Sq, int64_t D,
+                                int64_t os0, int64_t os1, int64_t os2, int elem_bytes) {
+  const int64_t n = B * Hq * Sq * D;
+  for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; x < n;
+       x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t d = x % D, i = (x / D) % Sq, h = (x / (D * Sq)) % Hq, b = x / (D * Sq * Hq);
+    uint8_t* dst = out + (b * os0 + h * os1 + i * os2 + d) * elem_bytes;
+    for (int e = 0; e < elem_bytes; ++e) dst[e] = 0;
+  }
+}
+
+}  // namespace
+
+int launch_f32(const gqa_problem& p, const float* q, const float* k, const float* v,
+               const uint8_t* mask, float* out, cudaStream_t stream) {
+  const int64_t rows = p.batch * p.heads_q * p.seq_q;
+  const int warps_per_block = 8;
+  const int64_t blocks = (rows + warps_per_block - 1) / warps_per_block;
+  if (blocks > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
+  const float scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634);
+  gqa_f32_kernel<<<static_cast<unsigned>(blocks), warps_per_block * 32, 0, stream>>>(
+      q, k, v, p.has_mask ? mask : nullptr, out, p.batch, p.heads_q, p.heads_kv, p.seq_q,
+      p.seq_k, p.head_dim, p.q_stride[0], p.q_stride[1], p.q_stride[2], p.k_stride[0],
+      p.k_stride[1], p.k_stride[2], p.v_stride[0], p.v_stride[1], p.v_stride[2], p.o_stride[0],
+      p.o_stride[1], p.o_stride[2], p.mask_stride[0], p.mask_stride[1], p.causal, scale_log2);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream) {
+  const int elem = p.dtype == GQA_DTYPE_F32 ? 4 : 2;
+  gqa_zero_kernel<<<592, 256, 0, stream>>>(static_cast<uint8_t*>(out), p.batch, p.heads_q,
+                                           p.seq_q, p.head_dim, p.o_stride[0], p.o_stride[1],
+                                           p.o_stride[2], elem);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace gqa

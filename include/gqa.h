@@ -1,0 +1,155 @@
+/*
+ * gqa.h -- C ABI of the B200 (sm_100a) grouped-query attention forward.
+ *
+ * Operation (page "28. Grouped-Query Attention (GQA)", sections "Step-by-Step
+ * Approach" and "Reference solution"; causal form from "Grouped-Query Attention
+ * Explained Simply", "Minimal implementation"; bool attention mask from
+ * "Multi-Query Attention", "Implementation"):
+ *
+ *   g            = heads_q / heads_kv                 (must divide exactly)
+ *   s[b,h,i,j]   = scale * sum_d q[b,h,i,d] * k[b,h/g,j,d]
+ *                  -inf where has_mask and mask[b,i,j] == 0
+ *                  -inf where causal and j > i
+ *   out[b,h,i,:] = sum_j softmax_j(s[b,h,i,:]) * v[b,h/g,j,:]
+ *
+ * Query head h reads kv head h / g (the contiguous "repeat_interleave"
+ * grouping); the kv head is never expanded in memory -- each K/V tile is read
+ * once and serves all g query heads of its group ("Multi-Query Attention",
+ * remark under "Implementation": a zero stride over the head dimension).
+ *
+ * Conventions
+ *  - Tensors are described by sizes and element strides; the innermost
+ *    (head_dim) stride must be 1.  q and out are [batch, heads_q, seq_q,
+ *    head_dim]; k and v are [batch, heads_kv, seq_k, head_dim]; the optional
+ *    mask is uint8 [batch, seq_q, seq_k], nonzero = attend, shared by every
+ *    head.  Any other strides are allowed (e.g. a [B, S, H, D] buffer viewed as
+ *    [B, H, S, D]), subject to the 16-byte rules below on the bf16 paths.
+ *  - dtype: GQA_DTYPE_BF16 (compute in fp32, bf16 in/out, head_dim 64 or 128)
+ *    or GQA_DTYPE_F32 (fp32 throughout, head_dim 1..256).
+ *  - causal is top-left aligned (key j visible to query i iff j <= i) and
+ *    requires seq_q == seq_k.  With has_mask as well, a key must pass both.
+ *  - A row whose keys are all hidden yields NaN (the softmax of an all -inf
+ *    row).  seq_k == 0 yields zeros (an empty weighted sum).  batch == 0 or
+ *    seq_q == 0 is a no-op.
+ *  - Memory: every pointer passed to gqa_forward is DEVICE memory of the
+ *    current CUDA device, owned by the caller, and must stay valid until the
+ *    work queued on `stream` has finished.  The library allocates nothing and
+ *    keeps no state between calls.
+ *  - Execution: gqa_forward only validates, plans and enqueues kernels on
+ *    `stream` (a cudaStream_t; NULL = the legacy default stream); it returns
+ *    before the work is done.  Errors in the arguments are returned at once;
+ *    a kernel that gives up on an internal wait records it in the workspace's
+ *    error word, read by gqa_device_status.
+ *  - No function throws across this boundary; every function returns a status
+ *    code (or a string / number as documented).
+ */
+#ifndef GQA_B200_GQA_H
+#define GQA_B200_GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+/* Status codes. */
+#define GQA_OK 0
+#define GQA_ERR_NULL 1        /* a required pointer is NULL */
+#define GQA_ERR_SHAPE 2       /* sizes inconsistent, negative, or heads_q % heads_kv != 0 */
+#define GQA_ERR_LAYOUT 3      /* innermost stride != 1, or a base/stride the TMA unit cannot
+                                 address (bf16 paths: base and non-innermost strides must be
+                                 multiples of 16 bytes) */
+#define GQA_ERR_UNSUPPORTED 4 /* dtype / head_dim combination, or causal with seq_q != seq_k */
+#define GQA_ERR_WORKSPACE 5   /* workspace NULL, too small, or not 256-byte aligned */
+#define GQA_ERR_CUDA 6        /* a CUDA runtime call failed (launch, attribute, encode) */
+#define GQA_ERR_TIMEOUT 7     /* a kernel's bounded internal wait ran out (gqa_device_status) */
+#define GQA_ERR_ARG 8         /* scale not finite, or an unknown dtype */
+#define GQA_ERR_DEVICE 9      /* no usable CUDA device, or not an sm_100 device */
+
+#define GQA_DTYPE_BF16 0
+#define GQA_DTYPE_F32 1
+
+#define GQA_KERNEL_NONE 0     /* nothing to launch (empty problem) */
+#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1: split-K stream over the KV cache */
+#define GQA_KERNEL_PREFILL 2  /* bf16, seq_q >= 2: tcgen05 / tensor-memory tiles */
+#define GQA_KERNEL_F32 3      /* fp32 CUDA-core path */
+#define GQA_KERNEL_ZERO 4     /* seq_k == 0: the output is filled with zeros */
+
+/* One attention problem.  Strides are in elements. */
+typedef struct gqa_problem {
+  int32_t dtype;          /* GQA_DTYPE_BF16 or GQA_DTYPE_F32, for q, k, v and out */
+  int32_t causal;         /* nonzero: key j hidden from query i when j > i */
+  int32_t has_mask;       /* nonzero: a mask pointer is passed to gqa_forward */
+  float scale;            /* multiplies q.k; 1/sqrt(head_dim) reproduces the pages */
+  int64_t batch, heads_q, heads_kv, seq_q, seq_k, head_dim;
+  int64_t q_stride[4];    /* over (b, h, i, d) */
+  int64_t k_stride[4];    /* over (b, h_kv, j, d) */
+  int64_t v_stride[4];    /* over (b, h_kv, j, d) */
+  int64_t o_stride[4];    /* over (b, h, i, d) */
+  int64_t mask_stride[3]; /* over (b, i, j); the j stride must be 1 */
+} gqa_problem;
+
+/* What gqa_forward will do for a problem on a device. */
+typedef struct gqa_plan {
+  int32_t kernel;            /* GQA_KERNEL_* */
+  int32_t grid;              /* CTAs of the main kernel */
+  int32_t block;             /* threads per CTA of the main kernel */
+  int32_t smem_bytes;        /* dynamic shared memory per CTA of the main kernel */
+  int32_t launches;          /* kernels enqueued per call */
+  int32_t work_units;        /* decode: 64-key tiles streamed; prefill: 128-row tiles */
+  int64_t workspace_bytes;   /* bytes of device scratch gqa_forward needs (>= 256) */
+  int64_t algorithmic_bytes; /* bytes of q, k, v, out (and mask) the call must move once */
+  double algorithmic_flops;  /* 4*B*Hq*Sq*Sk*D, halved when causal */
+} gqa_plan;
+
+/*
+ * gqa_query -- validate `p` and describe the plan.
+ *   sm_count: number of SMs to plan for; <= 0 asks the current CUDA device.
+ * Returns GQA_OK, an argument error (checked before any device query), or
+ * GQA_ERR_DEVICE when sm_count <= 0 and no device is usable.  Pure host code;
+ * enqueues nothing.
+ */
+GQA_API int gqa_query(const gqa_problem* p, int sm_count, gqa_plan* plan);
+
+/*
+ * gqa_forward -- enqueue out = GQA(q, k, v, mask) on `stream`.
+ *   q, k, v, out: device pointers described by `p` (dtype, sizes, strides).
+ *   mask:         device uint8 pointer if p->has_mask, else ignored (may be NULL).
+ *   workspace:    device scratch of at least plan.workspace_bytes, 256-byte
+ *                 aligned.  Its first 16 bytes hold the error word: zero them
+ *                 once before first use (gqa_device_status re-zeroes them).
+ *                 Calls that share a workspace must be ordered on one stream.
+ *   stream:       cudaStream_t.
+ * Returns GQA_OK once the kernels are enqueued, or an error code with nothing
+ * enqueued.  Does not synchronise.
+ */
+GQA_API int gqa_forward(const gqa_problem* p, const void* q, const void* k, const void* v,
+                        const uint8_t* mask, void* out, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * gqa_device_status -- synchronise `stream`, read and clear the workspace's
+ * error word.  Returns GQA_OK, GQA_ERR_TIMEOUT if a kernel gave up on a wait
+ * (its outputs are then undefined), or GQA_ERR_CUDA if the stream reports a
+ * CUDA error.
+ */
+GQA_API int gqa_device_status(void* workspace, void* stream);
+
+/* Static English description of a status code (never NULL). */
+GQA_API const char* gqa_status_string(int status);
+
+/* ABI version of this library (major * 10000 + minor * 100 + patch). */
+GQA_API int gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_B200_GQA_H */

@@ -1,0 +1,143 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports what
+``include/gqa.h`` declares, validates arguments and plans without a device."""
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    import grouped_query_attention_fwd_b200 as m
+    return m
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "gqa.h")).read()
+    return sorted(set(re.findall(r"GQA_API\s+[\w\s\*]+?\b(gqa_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(gqa):
+    syms = _declared_symbols()
+    assert set(syms) == set(gqa.EXPORTS)
+    for s in syms:
+        assert hasattr(gqa._lib, s), s
+
+
+def test_status_strings(gqa):
+    for code in range(0, 10):
+        s = gqa.status_string(code)
+        assert s and s != "unknown status"
+    assert gqa.status_string(1234) == "unknown status"
+    assert gqa.version() >= 10000
+
+
+def _contig(B, H, S, D):
+    return (H * S * D, S * D, D, 1)
+
+
+def _p(gqa, B=2, Hq=8, Hkv=2, Sq=1, Sk=100, D=128, dtype=0, causal=False, mask=False,
+       scale=None, **over):
+    qs, ks, os_ = _contig(B, Hq, Sq, D), _contig(B, Hkv, Sk, D), _contig(B, Hq, Sq, D)
+    ms = (Sq * Sk, Sk, 1) if mask else None
+    p = gqa.make_problem(dtype, B, Hq, Hkv, Sq, Sk, D, over.pop("q_stride", qs),
+                         over.pop("k_stride", ks), over.pop("v_stride", ks),
+                         over.pop("o_stride", os_), over.pop("mask_stride", ms),
+                         causal=causal, scale=scale)
+    for k, v in over.items():
+        setattr(p, k, v)
+    return p
+
+
+def _rc(gqa, p, sms=148):
+    plan = gqa.Plan()
+    import ctypes
+    return gqa._lib.gqa_query(ctypes.byref(p), sms, ctypes.byref(plan)), plan
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=6, Hkv=4), 2),                       # Hq not a multiple of Hkv
+    (dict(B=-1), 2),
+    (dict(D=0), 2),
+    (dict(Hkv=0), 2),
+    (dict(D=96), 4),                              # bf16 needs 64 or 128
+    (dict(D=300, dtype=1), 4),                    # fp32 path: D <= 256
+    (dict(Sq=3, Sk=5, causal=True), 4),           # causal needs Sq == Sk
+    (dict(scale=float("nan")), 8),
+    (dict(scale=float("inf")), 8),
+    (dict(dtype=7), 8),
+    (dict(q_stride=(1024, 128, 128, 2)), 3),      # innermost stride != 1
+    (dict(k_stride=(25600, 12804, 128, 1)), 3),   # bf16 stride not a multiple of 16 bytes
+    (dict(mask=True, mask_stride=(100, 100, 2)), 3),
+    (dict(Sq=4, Sk=4, Hq=129 * 2, Hkv=2), 4),     # prefill packs at most 128 heads per tile
+])
+def test_validation_errors(gqa, kw, code):
+    rc, _ = _rc(gqa, _p(gqa, **kw))
+    assert rc == code, (kw, rc, gqa.status_string(rc))
+
+
+def test_null_arguments(gqa):
+    import ctypes
+    plan = gqa.Plan()
+    assert gqa._lib.gqa_query(None, 148, ctypes.byref(plan)) == gqa.GQA_ERR_NULL
+    assert gqa._lib.gqa_query(ctypes.byref(_p(gqa)), 148, None) == gqa.GQA_ERR_NULL
+    assert gqa._lib.gqa_device_status(None, None) == gqa.GQA_ERR_NULL
+
+
+def test_plans_for_the_five_workloads(gqa):
+    # page-1 toy, fp32
+    rc, pl = _rc(gqa, _p(gqa, B=1, Hq=4, Hkv=2, Sq=5, Sk=5, D=4, dtype=1, scale=0.5))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "f32"
+    # decode, Mistral-7B-shaped layer
+    rc, pl = _rc(gqa, _p(gqa, B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "decode"
+    assert pl.algorithmic_bytes == 268697600
+    assert pl.grid == 148 and pl.work_units == 16 * 8 * 64 and pl.launches == 2
+    assert pl.workspace_bytes > 256 and pl.workspace_bytes % 256 == 0
+    assert pl.smem_bytes <= 227 * 1024
+    # long-context decode, Llama-2-70B-shaped layer
+    rc, pl = _rc(gqa, _p(gqa, B=16, Hq=64, Hkv=8, Sq=1, Sk=32768, D=128))
+    assert rc == 0 and pl.algorithmic_bytes == 2148007936
+    assert math.isclose(pl.algorithmic_flops, 4 * 16 * 64 * 32768 * 128)
+    # causal prefill
+    rc, pl = _rc(gqa, _p(gqa, B=4, Hq=32, Hkv=8, Sq=4096, Sk=4096, D=128, causal=True))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "prefill"
+    assert math.isclose(pl.algorithmic_flops, 4 * 4 * 32 * 4096 * 4096 * 128 / 2)
+    # padded-batch prefill with an explicit mask
+    rc, pl = _rc(gqa, _p(gqa, B=8, Hq=12, Hkv=2, Sq=2048, Sk=2048, D=64, mask=True))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "prefill"
+    assert pl.algorithmic_bytes == 2 * 8 * 12 * 2048 * 64 * 2 + 2 * 8 * 2 * 2048 * 64 * 2 + 8 * 2048 * 2048
+
+
+def test_decode_grid_small_problem(gqa):
+    # Fewer 64-key tiles than SMs: one tile per CTA.
+    rc, pl = _rc(gqa, _p(gqa, B=1, Hq=4, Hkv=1, Sq=1, Sk=130, D=64))
+    assert rc == 0 and pl.work_units == 3 and pl.grid == 3
+    # g > 8 uses 16-head passes.
+    rc, pl = _rc(gqa, _p(gqa, B=1, Hq=40, Hkv=1, Sq=1, Sk=64, D=128))
+    assert rc == 0 and pl.work_units == 3  # ceil(40 / 16) passes x 1 tile
+
+
+def test_empty_problems(gqa):
+    rc, pl = _rc(gqa, _p(gqa, B=0))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "none"
+    rc, pl = _rc(gqa, _p(gqa, Sq=0, Sk=10))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "none"
+    rc, pl = _rc(gqa, _p(gqa, Sq=3, Sk=0))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "zero"
+
+
+def test_no_device_is_an_error_not_a_fallback(gqa):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc, _ = _rc(gqa, _p(gqa), sms=0)
+    assert rc == gqa.GQA_ERR_DEVICE
+    with pytest.raises(gqa.GQAError) as ei:
+        gqa.forward_ptrs(_p(gqa), 16, 16, 16, None, 16, 256, 1 << 20, 0)
+    assert ei.value.status == gqa.GQA_ERR_DEVICE
+    with pytest.raises(ValueError):
+        gqa.forward(torch.zeros(1, 2, 1, 64), torch.zeros(1, 1, 3, 64), torch.zeros(1, 1, 3, 64))

@@ -1,0 +1,177 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+from gpu_util import (BF16_ABS, BF16_REL_RMS, F32_ABS, assert_bf16_parity, bf16_inputs, bits_to_dev,
+                      f64, oracle_bf16, rel_rms, to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import grouped_query_attention_fwd_b200 as m
+    return m
+
+
+def _status_ok(gqa):
+    st = gqa.device_status()
+    assert st == 0, gqa.status_string(st)
+
+
+# ------------------------------------------------------------------ fp32
+
+def test_f32_page_toy(gqa):
+    """q (1,4,5,4), k, v (1,2,5,4): the page-1 example, fp32, scale 1/sqrt(4)."""
+    q, k, v = synth.qkv_f32(1, 1, 4, 2, 5, 5, 4)
+    out = gqa.forward(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(),
+                      torch.from_numpy(v).cuda(), scale=0.5)
+    assert tuple(out.shape) == (1, 4, 5, 4)
+    ref = oracle.forward(q, k, v, scale=0.5)
+    assert np.abs(out.cpu().numpy() - ref).max() <= F32_ABS
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal,masked", [
+    (2, 6, 3, 7, 9, 8, False, False),
+    (2, 8, 2, 33, 33, 64, True, False),
+    (3, 12, 2, 5, 70, 37, False, True),
+    (1, 4, 1, 1, 300, 128, False, False),
+    (2, 4, 4, 16, 16, 256, True, True),
+])
+def test_f32_shapes(gqa, B, Hq, Hkv, Sq, Sk, D, causal, masked):
+    q, k, v = synth.qkv_f32(B + Sk, B, Hq, Hkv, Sq, Sk, D)
+    mask = synth.mask_random(5, B, Sq, Sk, 0.5) if masked else None
+    out = gqa.forward(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(),
+                      torch.from_numpy(v).cuda(),
+                      mask=torch.from_numpy(mask).cuda() if masked else None, causal=causal)
+    ref = oracle.forward(q, k, v, mask=mask, causal=causal)
+    assert np.abs(out.cpu().numpy() - ref).max() <= F32_ABS
+
+
+# ------------------------------------------------------------------ decode
+
+DECODE_CASES = [
+    # B, Hq, Hkv, Sk, D
+    (1, 4, 2, 1, 128),
+    (2, 8, 2, 63, 128),
+    (2, 8, 2, 64, 128),
+    (2, 8, 2, 65, 128),
+    (3, 32, 8, 333, 128),
+    (2, 12, 2, 1000, 64),
+    (1, 8, 8, 200, 128),      # g = 1 (MHA)
+    (2, 8, 1, 517, 128),      # g = 8, one kv head (MQA)
+    (2, 6, 2, 129, 64),       # g = 3
+    (1, 24, 2, 700, 128),     # g = 12: two 8-wide column tiles
+    (1, 40, 1, 300, 64),      # g = 40: three 16-head passes
+    (5, 32, 8, 4096, 128),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sk,D", DECODE_CASES)
+def test_decode_parity(gqa, B, Hq, Hkv, Sk, D):
+    bits, (q, k, v) = bf16_inputs(100 + Sk, B, Hq, Hkv, 1, Sk, D)
+    out = gqa.forward(q, k, v)
+    _status_ok(gqa)
+    assert_bf16_parity(to_np(out), oracle_bf16(*bits), "decode %s" % ((B, Hq, Hkv, Sk, D),))
+
+
+@pytest.mark.parametrize("Sk", [77, 1500])
+def test_decode_masked(gqa, Sk):
+    B, Hq, Hkv, D = 3, 16, 4, 128
+    bits, (q, k, v) = bf16_inputs(7, B, Hq, Hkv, 1, Sk, D)
+    mask = synth.mask_random(8, B, 1, Sk, 0.3)
+    out = gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda())
+    _status_ok(gqa)
+    assert_bf16_parity(to_np(out), oracle_bf16(*bits, mask=mask), "decode masked")
+
+
+def test_decode_strided_bshd_views(gqa):
+    """K/V cache stored [B, Sk, Hkv, D] and viewed as [B, Hkv, Sk, D]; q and out too."""
+    B, Hq, Hkv, Sk, D = 2, 16, 4, 300, 128
+    qb, kb, vb = synth.qkv_bf16_bits(9, B, Hq, Hkv, 1, Sk, D)
+    q = bits_to_dev(qb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    k = bits_to_dev(kb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    v = bits_to_dev(vb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    assert not k.is_contiguous()
+    out = torch.empty(B, 1, Hq, D, dtype=torch.bfloat16, device="cuda").transpose(1, 2)
+    gqa.forward(q, k, v, out=out)
+    _status_ok(gqa)
+    assert_bf16_parity(to_np(out), oracle_bf16(qb, kb, vb), "decode strided")
+
+
+def test_decode_scale_and_determinism(gqa):
+    bits, (q, k, v) = bf16_inputs(10, 4, 32, 8, 1, 2000, 128)
+    a = gqa.forward(q, k, v, scale=0.3)
+    b = gqa.forward(q, k, v, scale=0.3)
+    _status_ok(gqa)
+    assert torch.equal(a, b)
+    assert_bf16_parity(to_np(a), oracle_bf16(*bits, scale=0.3), "decode scale")
+
+
+def test_decode_fully_hidden_row_is_nan(gqa):
+    bits, (q, k, v) = bf16_inputs(11, 2, 8, 2, 1, 100, 128)
+    mask = np.ones((2, 1, 100), dtype=np.uint8)
+    mask[1] = 0
+    out = to_np(gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda()))
+    _status_ok(gqa)
+    assert np.all(np.isnan(out[1])) and np.all(np.isfinite(out[0]))
+
+
+def test_empty_and_zero_length(gqa):
+    q = torch.zeros(0, 4, 1, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(0, 2, 10, 128, dtype=torch.bfloat16, device="cuda")
+    assert gqa.forward(q, k, k).shape == (0, 4, 1, 128)
+    q = torch.randn(2, 4, 3, 64, device="cuda").bfloat16()
+    k = torch.zeros(2, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((2, 4, 3, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    gqa.forward(q, k, k, out=out)
+    assert torch.count_nonzero(out).item() == 0  # empty weighted sum
+
+
+def test_bad_alignment_rejected(gqa):
+    base = torch.zeros(1 + 8 * 64, dtype=torch.bfloat16, device="cuda")
+    q = base[1:].view(1, 8, 1, 64)  # 2-byte offset: not 16-byte aligned
+    k = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gqa.GQAError) as ei:
+        gqa.forward(q, k, k)
+    assert ei.value.status == gqa.GQA_ERR_LAYOUT
+
+
+# ------------------------------------------------------ full-size decode
+
+def _full_decode(gqa, seed, B, Hq, Hkv, Sk, D, groups):
+    """Full-size decode on the GPU; the oracle recomputes the given (b, kv)
+    groups from their own slices of the seeded inputs."""
+    bits, (q, k, v) = bf16_inputs(seed, B, Hq, Hkv, 1, Sk, D)
+    out = to_np(gqa.forward(q, k, v))
+    _status_ok(gqa)
+    g = Hq // Hkv
+    qb = bits[0]
+    del bits
+    for (b, kv) in groups:
+        ks = synth.kv_slice_bf16_bits(seed, synth.STREAM_K, B, Hkv, Sk, D, b, kv)
+        vs = synth.kv_slice_bf16_bits(seed, synth.STREAM_V, B, Hkv, Sk, D, b, kv)
+        ref = oracle.forward(f64(qb[b:b + 1, kv * g:(kv + 1) * g]), f64(ks)[None, None],
+                             f64(vs)[None, None])
+        assert_bf16_parity(out[b:b + 1, kv * g:(kv + 1) * g], ref, "group %s" % ((b, kv),))
+    return out
+
+
+def test_decode_mistral7b_layer_full(gqa):
+    """B=16, Hq=32, Hkv=8, Sk=4096, D=128: the whole output against the oracle."""
+    bits, (q, k, v) = bf16_inputs(2, 16, 32, 8, 1, 4096, 128)
+    out = to_np(gqa.forward(q, k, v))
+    _status_ok(gqa)
+    ma, rr = assert_bf16_parity(out, oracle_bf16(*bits), "mistral-7b decode")
+    print("decode B16 Hq32 Hkv8 Sk4096: max_abs=%.3e rel_rms=%.3e" % (ma, rr))
+
+
+def test_decode_llama70b_layer_sampled(gqa):
+    """B=16, Hq=64, Hkv=8, Sk=32768, D=128 (2 GiB of K+V): sampled groups."""
+    _full_decode(gqa, 3, 16, 64, 8, 32768, 128, [(0, 0), (7, 3), (15, 7), (9, 5)])
