@@ -262,7 +262,7 @@ def _cpu_baseline(cfg, budget_s=12.0):
     qb = synth.normal_bf16_bits(cfg["seed"], synth.STREAM_Q, B * Hq * Sq * D).reshape(B, Hq, Sq, D)
     groups, nbytes, t_used = 0, 0, 0.0
     order = [(b, kv) for b in range(B) for kv in range(Hkv)]
-    while t_used < budget_s and groups < len(order) * 4:
+    while t_used < budget_s and groups < len(order) * 64:
         b, kv = order[groups % len(order)]
         ks = synth.bf16_bits_to_f64(
             synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_K, B, Hkv, Sk, D, b, kv))[None, None]
@@ -327,7 +327,7 @@ def run_gpu(args):
     q, k, v, _ = _host_inputs(cfg, torch)
     qd = q.to(dev)
     kv_bytes = 2 * k.numel() * 2
-    copies = max(1, math.ceil(3 * L2_BYTES / kv_bytes))
+    copies = max(3, math.ceil(3 * L2_BYTES / kv_bytes))
     ks = [k.to(dev) for _ in range(copies)]
     vs = [v.to(dev) for _ in range(copies)]
     del q, k, v

@@ -68,7 +68,7 @@ _lib.gqa_query.restype = ctypes.c_int
 _lib.gqa_forward.argtypes = [ctypes.POINTER(Problem), _vp, _vp, _vp, _vp, _vp, _vp,
                              ctypes.c_size_t, _vp]
 _lib.gqa_forward.restype = ctypes.c_int
-_lib.gqa_device_status.argtypes = [_vp, _vp]
+_lib.gqa_device_status.argtypes = [_vp, ctypes.c_size_t, _vp]
 _lib.gqa_device_status.restype = ctypes.c_int
 _lib.gqa_status_string.argtypes = [ctypes.c_int]
 _lib.gqa_status_string.restype = ctypes.c_char_p
@@ -215,4 +215,4 @@ def device_status(workspace=None, stream=None) -> int:
         workspace = workspace_for(torch.cuda.current_device(), 256)
     if stream is None:
         stream = torch.cuda.current_stream().cuda_stream
-    return _lib.gqa_device_status(workspace.data_ptr(), stream)
+    return _lib.gqa_device_status(workspace.data_ptr(), workspace.numel(), stream)

@@ -114,7 +114,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       plan->grid = s.grid;
       plan->block = kDecodeThreads;
       plan->smem_bytes = s.smem_bytes;
-      plan->launches = 2;
+      plan->launches = 1;
       plan->work_units = static_cast<int32_t>(s.units);
       plan->workspace_bytes = kErrWordBytes + s.part_bytes;
       break;
@@ -122,7 +122,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
     case GQA_KERNEL_PREFILL: {
       const PrefillShape s = plan_prefill(p, sm_count);
       plan->grid = s.grid;
-      plan->block = 192;
+      plan->block = 224;
       plan->smem_bytes = s.smem_bytes;
       plan->launches = p.has_mask ? 2 : 1;
       plan->work_units = static_cast<int32_t>(s.work);
@@ -270,6 +270,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     a.out = static_cast<uint16_t*>(out);
     a.part_ml = reinterpret_cast<float2*>(ws + s.part_ml_offset);
     a.part_o = reinterpret_cast<float*>(ws + s.part_o_offset);
+    a.counters = reinterpret_cast<uint32_t*>(ws + s.counters_offset);
     a.err = err;
     a.B = static_cast<int>(p.batch);
     a.Hq = static_cast<int>(p.heads_q);
@@ -309,7 +310,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
 }
 
-GQA_API int gqa_device_status(void* workspace, void* stream_ptr) {
+GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream_ptr) {
   if (workspace == nullptr) return GQA_ERR_NULL;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   if (cudaStreamSynchronize(stream) != cudaSuccess) {
@@ -324,7 +325,10 @@ GQA_API int gqa_device_status(void* workspace, void* stream_ptr) {
     return GQA_ERR_CUDA;
   }
   if (word[0] != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof(word), stream) != cudaSuccess ||
+    // A kernel gave up part-way: its split counters may be off.  Return the
+    // whole workspace to the all-zero state that the next call expects.
+    const size_t n = workspace_bytes > sizeof(word) ? workspace_bytes : sizeof(word);
+    if (cudaMemsetAsync(workspace, 0, n, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;

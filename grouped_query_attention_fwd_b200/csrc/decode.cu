@@ -1,4 +1,4 @@
-// Split-K decode kernel (seq_q == 1) and its combine pass.
+// Split-K decode kernel (seq_q == 1) with its split merge fused in.
 //
 // Decoding re-reads the whole KV cache once per generated token and does
 // about one multiply-add per byte it reads, so its time is the KV bytes over
@@ -22,10 +22,13 @@
 //    tile), then O^T += V^T P^T; at g = 8 a CUDA-core version would need about
 //    as many FMA issue slots as the HBM time allows, the MMA needs a few %.
 //  * Online softmax in fp32 with warp-shuffle max/sum reductions; at the end
-//    of a range the four warps merge in shared memory and one partial
-//    (m, l, O) per head is written.  The combine kernel (launched with
-//    programmatic dependent launch so it is resident before the stream
-//    reaches it) merges the partials of each group and writes bf16 out.
+//    of a range the four warps merge in shared memory.  A group handled by
+//    one CTA is normalised and written straight to `out`.  A group split over
+//    several CTAs leaves one partial (m, l, O) per head and CTA in the
+//    workspace; each contributor then takes a ticket from the group's counter
+//    and the last one merges all partials, writes bf16 `out` and resets the
+//    counter to zero (so the workspace is left as it was found).  No CTA
+//    ever waits for another one.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -42,6 +45,12 @@ constexpr int CHUNK_BYTES = KT * 128;   // one 64-wide bf16 column chunk of a ti
 
 __host__ __device__ inline int64_t range_start(int64_t c, int64_t T, int64_t P) {
   return (c * T) / P;
+}
+
+// The CTA whose range [range_start(c), range_start(c + 1)) holds unit u:
+// the largest c with floor(c T / P) <= u, i.e. ceil((u + 1) P / T) - 1.
+__host__ __device__ inline int64_t cta_of_unit(int64_t u, int64_t T, int64_t P) {
+  return ((u + 1) * P + T - 1) / T - 1;
 }
 
 template <int D, int NT>
@@ -63,7 +72,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a,
                       const int tiles_per_group, const int passes, const int64_t units,
-                      const int segmax, const int stages) {
+                      const int segmax, const int stages, uint32_t* __restrict__ counters) {
   using L = DecodeSmem<D, NT>;
   constexpr int HP = L::HP;
   constexpr int KSTEPS = D / 16;
@@ -79,6 +88,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                                L::kScrMLBytes);
   uint64_t* empty = full + stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -95,9 +105,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-
-  // Let the combine kernel launch and wait on this grid's completion.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
@@ -203,6 +210,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      // Which CTAs share this group?  Ranges are static, so every CTA can tell.
+      const int64_t g_u0 = cur * tiles_per_group, g_u1 = g_u0 + tiles_per_group;
+      const int64_t c_lo = cta_of_unit(g_u0, units, P);
+      const int64_t c_hi = cta_of_unit(g_u1 - 1, units, P);
+      const int hq0 = kv * a.g + pass * HP;  // first query head of this pass
+      uint16_t* obase = a.out + b * a.os[0];
+      if (c_lo == c_hi) {
+        // The whole group is in this CTA: normalise and write out.
+        for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
+          const int h = idx / D, d = idx % D;
+          if (pass * HP + h >= a.g) continue;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
+          float l = 0.f, acc = 0.f;
+          if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NCW; ++w) {
+              const float sc = fast_exp2(scr_ml[(w * HP + h) * 2] - M);
+              l += sc * scr_ml[(w * HP + h) * 2 + 1];
+              acc += sc * scr_o[(w * HP + h) * L::kScrRow + d];
+            }
+          }
+          obase[(hq0 + h) * a.os[1] + d] = bf16_bits_rn(acc / l);  // l == 0: NaN
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+        return;
+      }
+      // Split group: publish this CTA's partial, then take a ticket.
       const int64_t slot = (static_cast<int64_t>(blockIdx.x) * segmax + seg) * HP;
       for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
         const int h = idx / D, d = idx % D;
@@ -220,6 +256,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         a.part_o[(slot + h) * D + d] = acc;
         if (d == 0) a.part_ml[slot + h] = make_float2(M, l);
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      if (threadIdx.x == 0) {
+        const uint32_t n = static_cast<uint32_t>(c_hi - c_lo + 1);
+        const uint32_t old = atomicAdd(&counters[cur], 1u);
+        *last_flag = (old == n - 1) ? 1 : 0;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      if (*last_flag) {
+        // Last contributor: every other partial of the group is published.
+        __threadfence();
+        for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
+          const int h = idx / D, d = idx % D;
+          if (pass * HP + h >= a.g) continue;
+          float M = -INFINITY;
+          for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
+            const int sg = static_cast<int>(cur - range_start(cc, units, P) / tiles_per_group);
+            M = fmaxf(M, __ldcg(&a.part_ml[(cc * segmax + sg) * HP + h]).x);
+          }
+          float l = 0.f, acc = 0.f;
+          if (M != -INFINITY) {
+            for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
+              const int sg = static_cast<int>(cur - range_start(cc, units, P) / tiles_per_group);
+              const int64_t sl = (cc * segmax + sg) * HP + h;
+              const float2 ml = __ldcg(&a.part_ml[sl]);
+              const float sc = fast_exp2(ml.x - M);
+              l += sc * ml.y;
+              acc += sc * __ldcg(&a.part_o[sl * D + d]);
+            }
+          }
+          obase[(hq0 + h) * a.os[1] + d] = bf16_bits_rn(acc / l);  // l == 0: NaN
+        }
+        if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
     };
@@ -344,52 +414,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
 }
 
-// Merge the partial states of one (batch, kv head, pass) group and write
-// out[b, h, 0, :] for its heads.
-template <int D, int HP>
-__global__ void __launch_bounds__(128)
-    gqa_decode_combine_kernel(const DecodeArgs a, const int tiles_per_group, const int passes,
-                              const int64_t units, const int P, const int segmax) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int64_t grp = blockIdx.x;
-  const int64_t bk = grp / passes;
-  const int pass = static_cast<int>(grp % passes);
-  const int kv = static_cast<int>(bk % a.Hkv);
-  const int b = static_cast<int>(bk / a.Hkv);
-  const int64_t u0 = grp * tiles_per_group, u1 = u0 + tiles_per_group;
-
-  // First CTA whose range contains u0.
-  int64_t c = (u0 * P) / units;
-  if (c > P - 1) c = P - 1;
-  while (c > 0 && range_start(c, units, P) > u0) --c;
-  while (c + 1 < P && range_start(c + 1, units, P) <= u0) ++c;
-  const int64_t c_lo = c;
-
-  for (int idx = threadIdx.x; idx < HP * D; idx += blockDim.x) {
-    const int h = idx / D, d = idx % D;
-    const int hl = pass * HP + h;
-    if (hl >= a.g) continue;
-    float M = -INFINITY;
-    for (int64_t cc = c_lo; cc < P && range_start(cc, units, P) < u1; ++cc) {
-      const int seg = static_cast<int>(grp - range_start(cc, units, P) / tiles_per_group);
-      M = fmaxf(M, a.part_ml[(cc * segmax + seg) * HP + h].x);
-    }
-    float l = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-      for (int64_t cc = c_lo; cc < P && range_start(cc, units, P) < u1; ++cc) {
-        const int seg = static_cast<int>(grp - range_start(cc, units, P) / tiles_per_group);
-        const int64_t slot = (cc * segmax + seg) * HP + h;
-        const float2 ml = a.part_ml[slot];
-        const float sc = fast_exp2(ml.x - M);
-        l += sc * ml.y;
-        acc += sc * a.part_o[slot * D + d];
-      }
-    }
-    const int hq = kv * a.g + hl;
-    a.out[b * a.os[0] + hq * a.os[1] + d] = bf16_bits_rn(acc / l);
-  }
-}
-
 template <int D, int NT>
 int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap& tmk,
                     const CUtensorMap& tmv, cudaStream_t stream) {
@@ -398,23 +422,9 @@ int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap
       cudaSuccess)
     return GQA_ERR_CUDA;
   kern<<<s.grid, kDecodeThreads, s.smem_bytes, stream>>>(tmk, tmv, a, s.tiles_per_group,
-                                                          s.passes, s.units, s.segmax, s.stages);
-  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(s.groups));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gqa_decode_combine_kernel<D, 8 * NT>, a, s.tiles_per_group,
-                         s.passes, s.units, s.grid, s.segmax) != cudaSuccess)
-    return GQA_ERR_CUDA;
-  return GQA_OK;
+                                                          s.passes, s.units, s.segmax, s.stages,
+                                                          a.counters);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 }  // namespace
@@ -448,8 +458,9 @@ DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
     s.smem_bytes = DecodeSmem<64, 2>::bytes(s.stages);
   (void)stage_bytes;
   const int64_t slots = static_cast<int64_t>(s.grid) * s.segmax * s.HP;
-  s.part_ml_offset = 256;
-  s.part_o_offset = 256 + ((slots * 8 + 255) / 256) * 256;
+  s.counters_offset = 256;
+  s.part_ml_offset = s.counters_offset + ((s.groups * 4 + 255) / 256) * 256;
+  s.part_o_offset = s.part_ml_offset + ((slots * 8 + 255) / 256) * 256;
   s.part_bytes = (s.part_o_offset - 256) + slots * s.D * 4;
   return s;
 }

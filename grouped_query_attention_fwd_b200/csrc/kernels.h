@@ -27,7 +27,7 @@ struct DecodeShape {
   int segmax;       // partial segments per CTA
   int stages;       // shared-memory ring depth
   int smem_bytes;
-  int64_t part_o_offset, part_ml_offset, part_bytes;
+  int64_t counters_offset, part_o_offset, part_ml_offset, part_bytes;
 };
 
 DecodeShape plan_decode(const gqa_problem& p, int sm_count);
@@ -41,6 +41,7 @@ struct DecodeArgs {
   int64_t os[4];
   float* part_o;
   float2* part_ml;
+  uint32_t* counters;  // one ticket counter per group; zero between calls
   uint32_t* err;
   int B, Hq, Hkv, Sk, g;
   float scale_log2;  // scale * log2(e)

@@ -77,7 +77,7 @@ extern "C" {
 #define GQA_DTYPE_F32 1
 
 #define GQA_KERNEL_NONE 0     /* nothing to launch (empty problem) */
-#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1: split-K stream over the KV cache */
+#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1: split-K stream over the KV cache, one launch */
 #define GQA_KERNEL_PREFILL 2  /* bf16, seq_q >= 2: tcgen05 / tensor-memory tiles */
 #define GQA_KERNEL_F32 3      /* fp32 CUDA-core path */
 #define GQA_KERNEL_ZERO 4     /* seq_k == 0: the output is filled with zeros */
@@ -123,9 +123,15 @@ GQA_API int gqa_query(const gqa_problem* p, int sm_count, gqa_plan* plan);
  *   q, k, v, out: device pointers described by `p` (dtype, sizes, strides).
  *   mask:         device uint8 pointer if p->has_mask, else ignored (may be NULL).
  *   workspace:    device scratch of at least plan.workspace_bytes, 256-byte
- *                 aligned.  Its first 16 bytes hold the error word: zero them
- *                 once before first use (gqa_device_status re-zeroes them).
- *                 Calls that share a workspace must be ordered on one stream.
+ *                 aligned, owned by the caller.  It must be all zero before its
+ *                 first use.  The parts that must start at zero (the error word
+ *                 and the split-merge counters) are back at zero after every
+ *                 call that completes without error, and the rest needs no
+ *                 particular contents, so zeroing once at allocation is
+ *                 enough.  After gqa_device_status reports an error it
+ *                 re-zeroes the workspace itself.  Calls that share a
+ *                 workspace must be ordered on one stream; calls that overlap
+ *                 on the GPU race.
  *   stream:       cudaStream_t.
  * Returns GQA_OK once the kernels are enqueued, or an error code with nothing
  * enqueued.  Does not synchronise.
@@ -135,12 +141,13 @@ GQA_API int gqa_forward(const gqa_problem* p, const void* q, const void* k, cons
                         size_t workspace_bytes, void* stream);
 
 /*
- * gqa_device_status -- synchronise `stream`, read and clear the workspace's
- * error word.  Returns GQA_OK, GQA_ERR_TIMEOUT if a kernel gave up on a wait
- * (its outputs are then undefined), or GQA_ERR_CUDA if the stream reports a
- * CUDA error.
+ * gqa_device_status -- synchronise `stream` and read the workspace's error
+ * word.  Returns GQA_OK; or GQA_ERR_TIMEOUT if a kernel gave up on a wait (its
+ * outputs are then undefined), in which case the first `workspace_bytes` of
+ * the workspace are zeroed so that it can be used again; or GQA_ERR_CUDA if
+ * the stream reports a CUDA error.
  */
-GQA_API int gqa_device_status(void* workspace, void* stream);
+GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static English description of a status code (never NULL). */
 GQA_API const char* gqa_status_string(int status);

@@ -47,6 +47,9 @@ def test_f32_page_toy(gqa):
 def test_f32_shapes(gqa, B, Hq, Hkv, Sq, Sk, D, causal, masked):
     q, k, v = synth.qkv_f32(B + Sk, B, Hq, Hkv, Sq, Sk, D)
     mask = synth.mask_random(5, B, Sq, Sk, 0.5) if masked else None
+    if masked and causal:  # keep the diagonal so that no row is fully hidden
+        for i in range(min(Sq, Sk)):
+            mask[:, i, i] = 1
     out = gqa.forward(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(),
                       torch.from_numpy(v).cuda(),
                       mask=torch.from_numpy(mask).cuda() if masked else None, causal=causal)

@@ -1,0 +1,161 @@
+"""tcgen05 prefill kernel vs the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+from gpu_util import assert_bf16_parity, bf16_inputs, bits_to_dev, f64, oracle_bf16, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import grouped_query_attention_fwd_b200 as m
+    return m
+
+
+def _status_ok(gqa):
+    st = gqa.device_status()
+    assert st == 0, gqa.status_string(st)
+
+
+def _mask(kind, seed, B, Sq, Sk, causal):
+    if kind is None:
+        return None
+    if kind == "random":
+        m = synth.mask_random(seed, B, Sq, Sk, 0.5)
+    else:
+        lens = synth.uniform_int(seed, synth.STREAM_MASK, B, 1, Sk)
+        m = synth.mask_from_lengths(lens, Sq, Sk)
+    if causal:  # keep the diagonal so that no row is fully hidden
+        for i in range(min(Sq, Sk)):
+            m[:, i, i] = 1
+    return m
+
+
+PREFILL_CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, causal, mask
+    (1, 8, 2, 200, 200, 128, True, None),        # g=4: 32 queries x 4 heads per tile
+    (1, 8, 2, 200, 200, 128, False, None),
+    (2, 12, 2, 150, 300, 64, False, "random"),   # g=6: 21 x 6 = 126 rows + 2 pad
+    (1, 4, 4, 130, 130, 128, False, None),       # g=1 (MHA): 128 queries per tile
+    (2, 8, 1, 64, 64, 128, True, None),          # g=8 (MQA-like): 16 queries per tile
+    (1, 6, 2, 77, 513, 64, False, None),         # g=3: 42 x 3 = 126 rows
+    (1, 16, 1, 9, 257, 128, False, None),        # g=16: 8 queries per tile
+    (1, 128, 1, 5, 100, 64, False, None),        # g=128: one query per tile
+    (2, 8, 2, 256, 256, 128, True, "random"),    # causal and mask together
+    (1, 4, 2, 3, 1, 64, False, None),            # one key
+    (1, 4, 2, 2, 2, 128, True, None),            # smallest causal prefill
+    (3, 12, 2, 300, 300, 64, False, "lengths"),  # right-padded batch
+    (2, 32, 8, 384, 384, 128, True, None),       # several 128-key tiles, exact multiple
+    (1, 8, 2, 129, 1000, 128, False, "lengths"),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal,mask_kind", PREFILL_CASES)
+def test_prefill_parity(gqa, B, Hq, Hkv, Sq, Sk, D, causal, mask_kind):
+    seed = 1000 + Sq + Sk + Hq
+    bits, (q, k, v) = bf16_inputs(seed, B, Hq, Hkv, Sq, Sk, D)
+    mask = _mask(mask_kind, seed, B, Sq, Sk, causal)
+    out = gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda() if mask is not None else None,
+                      causal=causal)
+    _status_ok(gqa)
+    ref = oracle_bf16(*bits, mask=mask, causal=causal)
+    assert_bf16_parity(to_np(out), ref, "prefill %s" % ((B, Hq, Hkv, Sq, Sk, D, causal, mask_kind),))
+
+
+def test_prefill_strided_bshd(gqa):
+    B, Hq, Hkv, S, D = 2, 8, 2, 160, 128
+    qb, kb, vb = synth.qkv_bf16_bits(21, B, Hq, Hkv, S, S, D)
+    q = bits_to_dev(qb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    k = bits_to_dev(kb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    v = bits_to_dev(vb.transpose(0, 2, 1, 3).copy()).transpose(1, 2)
+    out = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device="cuda").transpose(1, 2)
+    gqa.forward(q, k, v, out=out, causal=True)
+    _status_ok(gqa)
+    assert_bf16_parity(to_np(out), oracle_bf16(qb, kb, vb, causal=True), "prefill strided")
+
+
+def test_prefill_determinism_and_scale(gqa):
+    bits, (q, k, v) = bf16_inputs(22, 2, 8, 2, 300, 300, 128)
+    a = gqa.forward(q, k, v, causal=True, scale=0.05)
+    b = gqa.forward(q, k, v, causal=True, scale=0.05)
+    _status_ok(gqa)
+    assert torch.equal(a, b)
+    assert_bf16_parity(to_np(a), oracle_bf16(*bits, causal=True, scale=0.05), "prefill scale")
+
+
+def test_prefill_large_scores_rescale(gqa):
+    """Scores that grow along the keys force the lazy O rescale path."""
+    B, Hq, Hkv, S, D = 1, 8, 2, 512, 64
+    qb, kb, vb = synth.qkv_bf16_bits(23, B, Hq, Hkv, S, S, D)
+    ramp = np.linspace(0.0, 6.0, S, dtype=np.float32)[None, None, :, None]
+    kf = (synth.bf16_bits_to_f64(kb).astype(np.float32) + ramp).astype(np.float32)
+    kb2 = synth.round_bf16_bits(kf)
+    q, k, v = bits_to_dev(qb), bits_to_dev(kb2), bits_to_dev(vb)
+    out = gqa.forward(q, k, v, scale=1.0)
+    _status_ok(gqa)
+    assert_bf16_parity(to_np(out), oracle_bf16(qb, kb2, vb, scale=1.0), "prefill rescale")
+
+
+def test_prefill_fully_hidden_rows_are_nan(gqa):
+    bits, (q, k, v) = bf16_inputs(24, 2, 8, 2, 70, 300, 128)
+    mask = np.ones((2, 70, 300), dtype=np.uint8)
+    mask[1, 5, :] = 0          # one hidden row
+    mask[0, 40:70, :] = 0      # a whole query tile hidden (no key tile visited)
+    out = to_np(gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda()))
+    _status_ok(gqa)
+    assert np.all(np.isnan(out[1, :, 5])) and np.all(np.isnan(out[0, :, 40:70]))
+    ok = np.ones(out.shape[:3], dtype=bool)
+    ok[1, :, 5] = False
+    ok[0, :, 40:70] = False
+    ref = oracle_bf16(*bits, mask=mask)
+    assert np.all(np.isfinite(out[ok]))
+    assert_bf16_parity(out[ok], ref[ok], "prefill visible rows")
+
+
+# ------------------------------------------------------------ full size
+
+def _sampled(gqa, seed, B, Hq, Hkv, S, D, causal, mask_lens, samples):
+    bits, (q, k, v) = bf16_inputs(seed, B, Hq, Hkv, S, S, D)
+    mask = None
+    if mask_lens:
+        lens = synth.uniform_int(seed, synth.STREAM_MASK, B, 256, S)
+        mask = synth.mask_from_lengths(lens, S, S)
+    out = to_np(gqa.forward(q, k, v, causal=causal,
+                            mask=torch.from_numpy(mask).cuda() if mask is not None else None))
+    _status_ok(gqa)
+    qb, kb, vb = bits
+    g = Hq // Hkv
+    got, ref = [], []
+    for (b, kv, rows) in samples:
+        qs = f64(qb[b:b + 1, kv * g:(kv + 1) * g])
+        ks = f64(kb[b:b + 1, kv:kv + 1])
+        vs = f64(vb[b:b + 1, kv:kv + 1])
+        ms = mask[b:b + 1] if mask is not None else None
+        r = oracle.forward_rows(qs, ks, vs, [(0, hh, i) for (hh, i) in rows], mask=ms,
+                                causal=causal)
+        ref.append(r)
+        got.append(np.stack([out[b, kv * g + hh, i] for (hh, i) in rows]))
+    return np.concatenate(got), np.concatenate(ref)
+
+
+def test_prefill_causal_full_size_sampled(gqa):
+    """B=4, Hq=32, Hkv=8, S=4096, D=128, causal: sampled rows of every kind of tile."""
+    rows = [(hh, i) for hh in range(4) for i in (0, 1, 31, 32, 127, 128, 2047, 2048, 4000, 4095)]
+    got, ref = _sampled(gqa, 4, 4, 32, 8, 4096, 128, True, False,
+                        [(0, 0, rows), (3, 7, rows), (2, 5, rows[::3])])
+    assert_bf16_parity(got, ref, "causal prefill full size")
+
+
+def test_prefill_masked_full_size_sampled(gqa):
+    """B=8, Hq=12, Hkv=2, S=2048, D=64, padding mask len_b ~ U[256, 2048]."""
+    rows = [(hh, i) for hh in range(6) for i in (0, 20, 21, 1000, 2047)]
+    got, ref = _sampled(gqa, 5, 8, 12, 2, 2048, 64, False, True,
+                        [(0, 0, rows), (7, 1, rows), (4, 0, rows)])
+    assert_bf16_parity(got, ref, "masked prefill full size")
