@@ -175,6 +175,41 @@ def _visible_pairs(cfg, mask_host):
 
 # ------------------------------------------------------------------ GPU arm
 
+def _graph_timed(torch, calls, steps, warmup, stream):
+    """Time `steps` launches, launch i being calls[i % len(calls)], each
+    replayed from its own one-launch CUDA graph so that host-side overhead
+    never leaves the GPU idle between launches.  Returns (total_ms,
+    per-launch ms list, host seconds spent enqueuing)."""
+    for i in range(warmup):
+        calls[i % len(calls)]()
+    torch.cuda.synchronize()
+    graphs = []
+    for fn in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs.append(g)
+    for i in range(max(3, len(graphs))):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    e0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        graphs[i % len(graphs)].replay()
+        ev[i][1].record(stream)
+    e1.record(stream)
+    h1 = time.perf_counter()
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in ev]
+    del graphs
+    return e0.elapsed_time(e1), per, h1 - h0
+
+
 def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
     """Device-resident timing of one workload.  Returns a dict of numbers."""
     q, k, v, mask = _host_inputs(cfg, torch)
@@ -188,27 +223,9 @@ def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     plan = gqa.query(qd, ks[0], vs[0], mask=md, causal=cfg["causal"])
     ws = gqa.workspace_for(dev, plan["workspace_bytes"])
     stream = torch.cuda.current_stream(dev)
-    for i in range(warmup):
-        gqa.forward(qd, ks[i % copies], vs[i % copies], mask=md, causal=cfg["causal"], out=out,
-                    workspace=ws)
-    torch.cuda.synchronize(dev)
-    st = gqa.device_status(ws)
-    if st != 0:
-        raise RuntimeError("device status after warm-up: %s" % gqa.status_string(st))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for i in range(steps):
-        ev[i][0].record(stream)
-        gqa.forward(qd, ks[i % copies], vs[i % copies], mask=md, causal=cfg["causal"], out=out,
-                    workspace=ws)
-        ev[i][1].record(stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    total_ms = e0.elapsed_time(e1)
-    per = [a.elapsed_time(b) for a, b in ev]
+    calls = [(lambda i=i: gqa.forward(qd, ks[i], vs[i], mask=md, causal=cfg["causal"], out=out,
+                                      workspace=ws)) for i in range(copies)]
+    total_ms, per, _ = _graph_timed(torch, calls, steps, warmup, stream)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
@@ -300,6 +317,22 @@ def _roofline_prefill(res, tflops, peak_kind, workload):
             "algorithmic_flops_per_launch": fl, "launch_ms": round(res["per_launch_ms"], 5)}
 
 
+WORKLOADS = {c["name"]: c for c in (DECODE, DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED)}
+
+
+def run_profile_case(args):
+    """One workload alone, for profiler captures: warm-up, `steps` timed
+    launches, one JSON line with the launch time."""
+    import torch
+    import grouped_query_attention_fwd_b200 as gqa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = WORKLOADS[args.profile]
+    res = _time_config(gqa, torch, cfg, steps=args.steps, warmup=args.warmup, dev=dev)
+    print(json.dumps({"profile_case": cfg["name"], "launch_ms": res["per_launch_ms"],
+                      "copies": res["copies"], "plan": res["plan"]}), flush=True)
+
+
 def run_gpu(args):
     import torch
     import grouped_query_attention_fwd_b200 as gqa
@@ -336,16 +369,8 @@ def run_gpu(args):
     ws = gqa.workspace_for(dev, plan["workspace_bytes"])
     stream = torch.cuda.current_stream(dev)
 
-    for i in range(args.warmup):
-        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
-    torch.cuda.synchronize(dev)
-    st = gqa.device_status(ws)
-    if st != 0:
-        raise RuntimeError("device status after warm-up: %s" % gqa.status_string(st))
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    calls = [(lambda i=i: gqa.forward(qd, ks[i], vs[i], out=out, workspace=ws))
+             for i in range(copies)]
     sampler = ClockSampler(gpu_id)
     sampler.start()
     time.sleep(0.3)
@@ -353,19 +378,12 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    e0.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
-        ev[i][1].record(stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_ms, per, host_s = _graph_timed(torch, calls, args.steps, args.warmup, stream)
     t_wall1 = time.time()
     if dist is not None:
         dist.barrier()
     sampler.stop()
-    elapsed_ms = e0.elapsed_time(e1)
-    per_launch = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    per_launch = statistics.mean(per)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
@@ -400,6 +418,8 @@ def run_gpu(args):
             "parallelism": "replicas" if world == 1 else "dp%d (independent problems per rank)" % world,
             "l2": "K/V rotated over %d device copies (%.0f MB) so no launch finds its K/V in L2"
                   % (copies, copies * kv_bytes / 1e6),
+            "launch": "one gqa_forward per step, each replayed from a one-launch CUDA graph "
+                      "(host enqueue %.1f us per step)" % (host_s / args.steps * 1e6),
         },
         "gpu_launches": args.steps * plan["launches"],
         "clocks": {k_: v_ for k_, v_ in clocks.items()},
@@ -532,11 +552,15 @@ def main():
     ap.add_argument("--skip-extra", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--profile", default=None, choices=sorted(WORKLOADS),
+                    help="time one workload alone (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.profile:
+        run_profile_case(args)
     else:
         run_gpu(args)
 

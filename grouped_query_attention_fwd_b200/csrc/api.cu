@@ -278,6 +278,11 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     a.Sk = static_cast<int>(p.seq_k);
     a.g = static_cast<int>(g);
     a.scale_log2 = scale_log2;
+    // The ticket counters must start at zero; other calls sharing this
+    // workspace (a prefill's tile classes, a larger problem's partials) may
+    // have left bytes there.
+    if (cudaMemsetAsync(a.counters, 0, static_cast<size_t>(s.groups) * 4, stream) != cudaSuccess)
+      return GQA_ERR_CUDA;
     return launch_decode(p, s, a, tmk, tmv, stream);
   }
 

@@ -26,9 +26,9 @@
 //    one CTA is normalised and written straight to `out`.  A group split over
 //    several CTAs leaves one partial (m, l, O) per head and CTA in the
 //    workspace; each contributor then takes a ticket from the group's counter
-//    and the last one merges all partials, writes bf16 `out` and resets the
-//    counter to zero (so the workspace is left as it was found).  No CTA
-//    ever waits for another one.
+//    and the last one merges all partials and writes bf16 `out` (the counters
+//    are zeroed on the stream before the launch).  No CTA ever waits for
+//    another one.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

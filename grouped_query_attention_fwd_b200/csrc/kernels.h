@@ -41,7 +41,7 @@ struct DecodeArgs {
   int64_t os[4];
   float* part_o;
   float2* part_ml;
-  uint32_t* counters;  // one ticket counter per group; zero between calls
+  uint32_t* counters;  // one ticket counter per group; zeroed before each launch
   uint32_t* err;
   int B, Hq, Hkv, Sk, g;
   float scale_log2;  // scale * log2(e)

@@ -123,15 +123,12 @@ GQA_API int gqa_query(const gqa_problem* p, int sm_count, gqa_plan* plan);
  *   q, k, v, out: device pointers described by `p` (dtype, sizes, strides).
  *   mask:         device uint8 pointer if p->has_mask, else ignored (may be NULL).
  *   workspace:    device scratch of at least plan.workspace_bytes, 256-byte
- *                 aligned, owned by the caller.  It must be all zero before its
- *                 first use.  The parts that must start at zero (the error word
- *                 and the split-merge counters) are back at zero after every
- *                 call that completes without error, and the rest needs no
- *                 particular contents, so zeroing once at allocation is
- *                 enough.  After gqa_device_status reports an error it
- *                 re-zeroes the workspace itself.  Calls that share a
- *                 workspace must be ordered on one stream; calls that overlap
- *                 on the GPU race.
+ *                 aligned, owned by the caller.  Only its first 16 bytes (the
+ *                 error word) must be zero before the first use; each call
+ *                 initialises the rest of what it uses.  gqa_device_status
+ *                 clears the error word after reporting an error.  Calls that
+ *                 share a workspace must be ordered on one stream; calls that
+ *                 overlap on the GPU race.
  *   stream:       cudaStream_t.
  * Returns GQA_OK once the kernels are enqueued, or an error code with nothing
  * enqueued.  Does not synchronise.
@@ -144,8 +141,8 @@ GQA_API int gqa_forward(const gqa_problem* p, const void* q, const void* k, cons
  * gqa_device_status -- synchronise `stream` and read the workspace's error
  * word.  Returns GQA_OK; or GQA_ERR_TIMEOUT if a kernel gave up on a wait (its
  * outputs are then undefined), in which case the first `workspace_bytes` of
- * the workspace are zeroed so that it can be used again; or GQA_ERR_CUDA if
- * the stream reports a CUDA error.
+ * the workspace are zeroed; or GQA_ERR_CUDA if the stream reports a CUDA
+ * error.
  */
 GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream);
 

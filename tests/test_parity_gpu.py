@@ -178,3 +178,27 @@ def test_decode_mistral7b_layer_full(gqa):
 def test_decode_llama70b_layer_sampled(gqa):
     """B=16, Hq=64, Hkv=8, Sk=32768, D=128 (2 GiB of K+V): sampled groups."""
     _full_decode(gqa, 3, 16, 64, 8, 32768, 128, [(0, 0), (7, 3), (15, 7), (9, 5)])
+
+
+def test_decode_after_other_calls_on_one_workspace(gqa):
+    """One workspace shared by a masked prefill, a small decode and a large
+    decode, in that order: leftovers of earlier calls must not leak into the
+    decode's split-merge counters."""
+    shapes = [(3, 12, 2, 300, 300, 64, True), (1, 4, 2, 1, 700, 128, False),
+              (16, 32, 8, 1, 4096, 128, False), (2, 8, 2, 1, 333, 128, False)]
+    cases = []
+    need = 256
+    for i, (B, Hq, Hkv, Sq, Sk, D, masked) in enumerate(shapes):
+        bits, (q, k, v) = bf16_inputs(300 + i, B, Hq, Hkv, Sq, Sk, D)
+        mask = synth.mask_random(301 + i, B, Sq, Sk, 0.4) if masked else None
+        md = torch.from_numpy(mask).cuda() if masked else None
+        need = max(need, gqa.query(q, k, v, mask=md)["workspace_bytes"])
+        cases.append((bits, q, k, v, mask, md))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for bits, q, k, v, mask, md in cases:
+            out = gqa.forward(q, k, v, mask=md, workspace=ws)
+            st = gqa.device_status(ws)
+            assert st == 0, gqa.status_string(st)
+            assert_bf16_parity(to_np(out), oracle_bf16(*bits, mask=mask),
+                               "shared workspace %s" % (tuple(q.shape),))
