@@ -30,10 +30,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQA_OK = 0
 GQA_ERR_NULL, GQA_ERR_SHAPE, GQA_ERR_LAYOUT, GQA_ERR_UNSUPPORTED = 1, 2, 3, 4
 GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 5, 6, 7, 8, 9
+GQA_ERR_SCRATCH_LIMIT = 10
+STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 GQA_DTYPE_BF16, GQA_DTYPE_F32 = 0, 1
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero"}
 
-EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version")
+EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
+           "gqa_forward_decode_noalloc")
 
 
 class Problem(ctypes.Structure):
@@ -74,6 +77,9 @@ _lib.gqa_status_string.argtypes = [ctypes.c_int]
 _lib.gqa_status_string.restype = ctypes.c_char_p
 _lib.gqa_version.argtypes = []
 _lib.gqa_version.restype = ctypes.c_int
+_lib.gqa_forward_decode_noalloc.argtypes = [ctypes.POINTER(Problem), _vp, _vp, _vp, _vp, _vp,
+                                            _vp]
+_lib.gqa_forward_decode_noalloc.restype = ctypes.c_int
 
 
 class GQAError(RuntimeError):

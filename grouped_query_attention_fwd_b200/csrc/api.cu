@@ -182,6 +182,16 @@ bool aligned(const void* ptr, uintptr_t a) {
 }  // namespace
 }  // namespace gqa
 
+namespace gqa {
+// K/V tensor map for the decode tile shape, shared with the static-scratch
+// decode entry point.
+int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& p,
+                         const int64_t st[4]) {
+  return encode_bf16_map(map, base, p.batch, p.heads_kv, p.seq_k, p.head_dim, st,
+                         kDecodeKeysPerTile, 1);
+}
+}  // namespace gqa
+
 using namespace gqa;
 
 extern "C" {
@@ -200,6 +210,7 @@ GQA_API const char* gqa_status_string(int status) {
     case GQA_ERR_TIMEOUT: return "a kernel gave up on an internal wait; outputs are undefined";
     case GQA_ERR_ARG: return "invalid scalar argument (scale must be finite; dtype must be known)";
     case GQA_ERR_DEVICE: return "no usable sm_100 CUDA device";
+    case GQA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the library's static array holds";
     default: return "unknown status";
   }
 }

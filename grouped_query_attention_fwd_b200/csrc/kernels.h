@@ -50,6 +50,10 @@ struct DecodeArgs {
 int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
                   const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream);
 
+// TMA map of a K or V tensor with the decode kernel's box (api.cu).
+int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& p,
+                         const int64_t st[4]);
+
 // ------------------------------------------------------------ prefill
 struct PrefillShape {
   int D;             // 64 or 128

@@ -72,6 +72,8 @@ extern "C" {
 #define GQA_ERR_TIMEOUT 7     /* a kernel's bounded internal wait ran out (gqa_device_status) */
 #define GQA_ERR_ARG 8         /* scale not finite, or an unknown dtype */
 #define GQA_ERR_DEVICE 9      /* no usable CUDA device, or not an sm_100 device */
+#define GQA_ERR_SCRATCH_LIMIT 10 /* gqa_forward_decode_noalloc: the problem needs more scratch
+                                    than GQA_STATIC_SCRATCH_BYTES */
 
 #define GQA_DTYPE_BF16 0
 #define GQA_DTYPE_F32 1
@@ -145,6 +147,39 @@ GQA_API int gqa_forward(const gqa_problem* p, const void* q, const void* k, cons
  * error.
  */
 GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Size of the library's static device scratch array used by
+ * gqa_forward_decode_noalloc: 8 MiB, held on every GPU that loads the library
+ * until the process exits.
+ */
+#define GQA_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/*
+ * gqa_forward_decode_noalloc -- the decode path (bf16, seq_q == 1) without a
+ * caller workspace.  The pages have no counterpart: this is a deployment
+ * variant of gqa_forward for callers that cannot allocate device memory --
+ * code that is only handed the q/k/v/out buffers by a host framework and has
+ * no allocator of its own, or a steady-state loop that must not call
+ * cudaMalloc because it can synchronise the device.
+ *   p, q, k, v, mask, out, stream: as for gqa_forward (device pointers).
+ * Scratch: a file-scope static device array of GQA_STATIC_SCRATCH_BYTES inside
+ * the library.  The first call on each device looks up that array's device
+ * address (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  The call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).  Every call on a device
+ * shares the one array: each call zeroes the part that must start at zero
+ * (with cudaMemsetAsync on `stream`) and leaves the rest as the last call
+ * left it, so calls that overlap on the GPU race -- order them on one stream.
+ * Returns GQA_OK once enqueued; GQA_ERR_UNSUPPORTED for anything but the
+ * decode path; GQA_ERR_SCRATCH_LIMIT when the problem's scratch (the
+ * workspace_bytes gqa_query reports) exceeds GQA_STATIC_SCRATCH_BYTES; the
+ * argument errors of gqa_forward otherwise.  A kernel wait that runs out is
+ * recorded only in the static array and is not reported to the caller.
+ */
+GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const void* q, const void* k,
+                                       const void* v, const uint8_t* mask, void* out,
+                                       void* stream);
 
 /* Static English description of a status code (never NULL). */
 GQA_API const char* gqa_status_string(int status);

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(gqa):
 
 
 def test_status_strings(gqa):
-    for code in range(0, 10):
+    for code in range(0, 11):
         s = gqa.status_string(code)
         assert s and s != "unknown status"
     assert gqa.status_string(1234) == "unknown status"
