@@ -173,6 +173,24 @@ def _visible_pairs(cfg, mask_host):
     return float(cfg["B"] * cfg["Hq"] * cfg["Sq"] * cfg["Sk"])
 
 
+# ------------------------------------------------------------- multi-rank
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest `value` over all ranks (the job is as slow as its slowest
+    rank); `dist` is torch.distributed or None for a single process."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_gbs(bytes_per_step: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job GB/s when every rank runs its own copy of the workload."""
+    return bytes_per_step * steps * world / (elapsed_ms / 1e3) / 1e9
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def _graph_timed(torch, calls, steps, warmup, stream):
@@ -387,15 +405,11 @@ def run_gpu(args):
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     del ks, vs
     torch.cuda.empty_cache()
 
-    total_bytes = plan["algorithmic_bytes"] * args.steps * world
-    value = total_bytes / (elapsed_ms / 1e3) / 1e9
+    value = weak_scaling_gbs(plan["algorithmic_bytes"], args.steps, world, elapsed_ms)
     clocks = sampler.summary(t_wall0 - 0.2, t_wall1 + 0.2)
 
     line = {

@@ -122,7 +122,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
     case GQA_KERNEL_PREFILL: {
       const PrefillShape s = plan_prefill(p, sm_count);
       plan->grid = s.grid;
-      plan->block = 224;
+      plan->block = 352;
       plan->smem_bytes = s.smem_bytes;
       plan->launches = p.has_mask ? 2 : 1;
       plan->work_units = static_cast<int32_t>(s.work);

@@ -267,27 +267,56 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
       if (*last_flag) {
         // Last contributor: every other partial of the group is published.
+        // Stage each contributor's segment index and each head's merged
+        // (max, sum) in shared memory, then accumulate O with 16-byte loads,
+        // several contributors in flight at once.
         __threadfence();
-        for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
-          const int h = idx / D, d = idx % D;
-          if (pass * HP + h >= a.g) continue;
+        const int n = static_cast<int>(c_hi - c_lo + 1);
+        int* sm_seg = reinterpret_cast<int*>(scr_o);          // n ints (scr_o is free now)
+        float* sm_ml = scr_ml;                                 // HP x (M, L)
+        for (int k = threadIdx.x; k < n; k += NCW * 32)
+          sm_seg[k] = static_cast<int>(cur - range_start(c_lo + k, units, P) / tiles_per_group);
+        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+        if (threadIdx.x < HP) {
+          const int h = threadIdx.x;
           float M = -INFINITY;
-          for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
-            const int sg = static_cast<int>(cur - range_start(cc, units, P) / tiles_per_group);
-            M = fmaxf(M, __ldcg(&a.part_ml[(cc * segmax + sg) * HP + h]).x);
-          }
-          float l = 0.f, acc = 0.f;
+#pragma unroll 4
+          for (int k = 0; k < n; ++k)
+            M = fmaxf(M, __ldcg(&a.part_ml[((c_lo + k) * segmax + sm_seg[k]) * HP + h]).x);
+          float Lsum = 0.f;
           if (M != -INFINITY) {
-            for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
-              const int sg = static_cast<int>(cur - range_start(cc, units, P) / tiles_per_group);
-              const int64_t sl = (cc * segmax + sg) * HP + h;
-              const float2 ml = __ldcg(&a.part_ml[sl]);
-              const float sc = fast_exp2(ml.x - M);
-              l += sc * ml.y;
-              acc += sc * __ldcg(&a.part_o[sl * D + d]);
+#pragma unroll 4
+            for (int k = 0; k < n; ++k) {
+              const float2 ml = __ldcg(&a.part_ml[((c_lo + k) * segmax + sm_seg[k]) * HP + h]);
+              Lsum += fast_exp2(ml.x - M) * ml.y;
             }
           }
-          obase[(hq0 + h) * a.os[1] + d] = bf16_bits_rn(acc / l);  // l == 0: NaN
+          sm_ml[2 * h] = M;
+          sm_ml[2 * h + 1] = Lsum;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+        for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
+          const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
+          if (pass * HP + h >= a.g) continue;
+          const float M = sm_ml[2 * h], Lsum = sm_ml[2 * h + 1];
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (M != -INFINITY) {
+#pragma unroll 4
+            for (int k = 0; k < n; ++k) {
+              const int64_t sl = ((c_lo + k) * segmax + sm_seg[k]) * HP + h;
+              const float w = fast_exp2(__ldcg(&a.part_ml[sl]).x - M);
+              const float4 o = __ldcg(reinterpret_cast<const float4*>(&a.part_o[sl * D + d]));
+              acc.x += w * o.x;
+              acc.y += w * o.y;
+              acc.z += w * o.z;
+              acc.w += w * o.w;
+            }
+          }
+          const float inv = 1.f / Lsum;  // Lsum == 0: NaN
+          uint2 pk;
+          pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+          pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+          *reinterpret_cast<uint2*>(obase + (hq0 + h) * a.os[1] + d) = pk;
         }
         if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
       }

@@ -10,16 +10,18 @@
 //
 // Per 128x128 tile:   S = Q K^T       tcgen05.mma, A and B from shared memory,
 //                                     fp32 accumulator in tensor memory (TMEM)
-//                     P = softmax(S)  128 softmax threads, one TMEM lane (row)
-//                                     each: scale, mask, online max / sum
+//                     P = softmax(S)  256 softmax threads, two per TMEM lane
+//                                     (row), 64 keys each: scale, mask,
+//                                     online max / sum
 //                     O += P V        tcgen05.mma, A = P (bf16) from TMEM,
 //                                     B = V from shared memory, O in TMEM
 //
-// Warp roles (224 threads, one CTA per SM, persistent over work tiles):
-//   warps 0-3  softmax, O rescale and epilogue (thread t owns row / lane t)
-//   warp 4     TMA producer of Q tiles and K tiles
-//   warp 5     TMEM allocator and single-thread MMA issuer
-//   warp 6     TMA producer of V tiles
+// Warp roles (352 threads, one CTA per SM, persistent over work tiles):
+//   warps 0-7  softmax, O rescale and epilogue: warp w owns rows 32*(w%4) ..
+//              +31 (TMEM lanes) and column half w/4 of S, P and O
+//   warp 8     TMA producer of Q tiles and K tiles
+//   warp 9     TMEM allocator and single-thread MMA issuer
+//   warp 10    TMA producer of V tiles
 // S is double-buffered in TMEM so that QK^T of tile j+1 runs on the tensor
 // cores while the softmax threads work on tile j, and PV of tile j-1 runs
 // behind it.  The running maximum is rescaled lazily: exponentials use a
@@ -40,15 +42,21 @@ namespace {
 
 constexpr int BM = 128;  // rows per tile = TMEM lanes
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kSoftmaxWarps = 4;
-constexpr int kWarpQK = 4;
-constexpr int kWarpMMA = 5;
-constexpr int kWarpV = 6;
-constexpr int kPrefillThreads = 7 * 32;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kWarpQK = 8;
+constexpr int kWarpMMA = 9;
+constexpr int kWarpV = 10;
+constexpr int kPrefillThreads = 11 * 32;
 constexpr int kStages = 2;  // depth of the K ring and of the V ring
 constexpr int kQBufs = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+// Exponentials of every eight computed on the FMA pipe (exp2_poly) rather
+// than the MUFU unit; the rest use ex2.approx.
+#ifndef GQA_PREFILL_EXP_EMU
+#define GQA_PREFILL_EXP_EMU 0
+#endif
+constexpr int kEmuPerEight = GQA_PREFILL_EXP_EMU;
 
 template <int D>
 struct Layout {
@@ -59,9 +67,10 @@ struct Layout {
   static constexpr int kKOff = kQOff + kQBufs * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 4 * kStages + 2 + 2 + 4;
+  static constexpr int kNumBars = 2 * kQBufs + 4 * kStages + 2 + 2 + 4 + 2 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  static constexpr int kRedOff = kMiscOff + 16;               // row max / sum exchange
+  static constexpr int kBytes = kRedOff + 8 * BM * 4 + 1024;  // + alignment slack
   // TMEM columns.
   static constexpr uint32_t kSCol0 = 0;     // S buffers at 0 and 128
   static constexpr uint32_t kOCol = 256;    // O: D columns
@@ -102,6 +111,42 @@ __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Item& it, 
   return cls;
 }
 
+// Visibility of keys j0 .. j0+127 for query q, one bit per key: inside the
+// sequence (j < Sk), not in the future (causal: j <= q), and allowed by the
+// mask row (nonzero byte), which is read as 16-byte vectors when aligned.
+__device__ __forceinline__ void visible_bits(uint32_t (&vb)[4], const uint8_t* mrow, int j0,
+                                             int Sk, int causal, int q, bool vec) {
+  int n = Sk - j0;  // keys inside the sequence
+  if (causal && q - j0 + 1 < n) n = q - j0 + 1;
+  n = n < 0 ? 0 : (n > BN ? BN : n);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int k = n - 32 * w;
+    vb[w] = k >= 32 ? ~0u : (k <= 0 ? 0u : ((1u << k) - 1u));
+  }
+  if (mrow == nullptr) return;
+  const uint8_t* m = mrow + j0;
+  if (vec && n == BN) {
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 x = *reinterpret_cast<const uint4*>(m + 16 * v);
+      const uint32_t wds[4] = {x.x, x.y, x.z, x.w};
+      uint32_t bits = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        // one bit per nonzero byte: 0xff per nonzero byte, then gather the MSBs
+        const uint32_t ne = __vcmpne4(wds[e], 0u);
+        const uint32_t msb = (ne >> 7) & 0x01010101u;
+        bits |= ((msb * 0x01020408u) >> 24) << (4 * e);  // byte k -> bit k
+      }
+      vb[v >> 1] &= (v & 1) ? ((bits << 16) | 0xFFFFu) : (bits | 0xFFFF0000u);
+    }
+  } else {
+    for (int c = 0; c < n; ++c)
+      if (m[c] == 0) vb[c >> 5] &= ~(1u << (c & 31));
+  }
+}
+
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
   // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; LBO unused (1).
   return smem_desc_sw128(saddr, 16, 1024);
@@ -138,6 +183,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* o_final = o_ready + 1;
   uint64_t* o_free = o_final + 1;
   uint64_t* mma_done = o_free + 1;
+  uint64_t* xchg = mma_done + 1;   // [2]: row-max exchange between column halves
+  uint64_t* lxchg = xchg + 2;      // [2]: row-sum exchange at the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -163,6 +210,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(o_final, 1);
     mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&xchg[i], kSoftmaxWarps);
+      mbar_init(&lxchg[i], kSoftmaxWarps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -342,9 +393,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int row = threadIdx.x;  // TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // Eight warps: warp w serves TMEM lanes 32*(w % 4) .. +31 (its rows) and
+    // column half hf = w / 4 of each S tile (64 keys), of P and of O, so two
+    // warps per SM sub-partition share every row.  The halves exchange their
+    // row maxima through shared memory and an mbarrier once per tile, and
+    // their partial row sums once per work tile.
+    const int quad = warp & 3, hf = warp >> 2;
+    const int row = quad * 32 + lane;  // TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int hh = row / qpt, qi = row % qpt;
+    constexpr int DH = D / 2;  // O columns per half
+    // Mask rows can be read as 16-byte vectors when base and strides allow.
+    const bool mask_vec = a.has_mask && ((reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0) &&
+                          (a.ms[0] % 16 == 0) && (a.ms[1] % 16 == 0);
+    float* red = reinterpret_cast<float*>(smem + L::kRedOff);  // [2 parity][2 halves][BM]
+    float* lred = red + 4 * BM;                                // [2 parity][2 halves][BM]
     uint32_t J = 0;
     int64_t it = 0;
     bool ok = true;
@@ -365,37 +428,57 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           break;
         }
         tc_fence_after();
-        float t[BN];
+        // This half's 64 scores of the row.  Fully visible tiles keep raw
+        // scores and fold the scale into one FMA per element; other tiles go
+        // to the base-2 domain with -inf where a key is hidden.
+        const bool fast = (cls == 2) && (a.scale_log2 >= 0.f);
+        float t[64];
         {
-          uint32_t r[32];
+          uint32_t r[64];
+          const uint32_t sbase = tmem + lane_base + L::kSCol0 + (J & 1) * 128 + hf * 64;
+          tmem_ld32(sbase, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_ld_wait();
+          if (fast) {
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            tmem_ld32(tmem + lane_base + L::kSCol0 + (J & 1) * 128 + c * 32, r);
-            tmem_ld_wait();
+            for (int c = 0; c < 64; ++c) t[c] = __uint_as_float(r[c]);
+          } else {
+            uint32_t vb[4];
+            visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a.Sk, a.causal, q, mask_vec);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) t[c * 32 + e] = __uint_as_float(r[e]) * a.scale_log2;
+            for (int c = 0; c < 64; ++c) {
+              const int cc = hf * 64 + c;
+              t[c] = ((vb[cc >> 5] >> (cc & 31)) & 1u) ? __uint_as_float(r[c]) * a.scale_log2
+                                                       : -INFINITY;
+            }
           }
         }
-        if (cls == 1) {
-          const int j0 = nt * BN;
+        float mx;
+        {
+          float part[8];
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int j = j0 + c;
-            bool vis = j < a.Sk;
-            if (a.causal && j > q) vis = false;
-            if (vis && mrow != nullptr && mrow[j] == 0) vis = false;
-            if (!vis) t[c] = -INFINITY;
-          }
+          for (int e = 0; e < 8; ++e) part[e] = t[e];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) part[c & 7] = fmaxf(part[c & 7], t[c]);
+          mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
+                     fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
+          if (fast) mx *= a.scale_log2;
         }
-        float mx = t[0];
-#pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, t[c]);
+        // Row maximum over both halves.
+        red[((J & 1) * 2 + hf) * BM + row] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xchg[J & 1]);
+        if (!mbar_wait(&xchg[J & 1], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, red[((J & 1) * 2 + (hf ^ 1)) * BM + row]);
         const float m_new = fmaxf(m_ref, mx);
         const bool grow = m_new > m_ref + kRescaleLog2;  // also true for -inf -> finite
         const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         const bool o_live = grow && nloc > 0 && m_ref != -INFINITY;
         if (__any_sync(0xffffffffu, o_live)) {
-          // O holds earlier tiles' P V with the old reference: rescale it.
+          // O holds earlier tiles' P V with the old reference: rescale this half.
           if (!mbar_wait(o_ready, (J - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
             ok = false;
             break;
@@ -403,20 +486,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tc_fence_after();
           const float f = o_live ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < DH / 32; ++c) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_base + L::kOCol + c * 32, r);
+            const uint32_t oa = tmem + lane_base + L::kOCol + hf * DH + c * 32;
+            tmem_ld32(oa, r);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-            uint32_t lo[16], hi[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              lo[e] = r[e];
-              hi[e] = r[16 + e];
-            }
-            tmem_st16(tmem + lane_base + L::kOCol + c * 32, lo);
-            tmem_st16(tmem + lane_base + L::kOCol + c * 32 + 16, hi);
+            tmem_st16(oa, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tmem_st16(oa + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
           }
           tmem_st_wait();
         }
@@ -425,19 +503,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           m_ref = m_new;
         }
         const float ref = exp_ref(m_ref);
-        // P = exp2(t - ref) as bf16 pairs into TMEM (A operand of the PV MMA).
+        // P = 2^(t - ref) as bf16 pairs into TMEM (A operand of the PV MMA);
+        // kEmuPerEight of every eight exponentials run on the FMA pipe.
+        float lp[8];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int e = 0; e < 8; ++e) lp[e] = 0.f;
+        const float sc = fast ? a.scale_log2 : 1.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(t[c * 32 + 2 * e] - ref);
-            const float p1 = fast_exp2(t[c * 32 + 2 * e + 1] - ref);
-            l += p0 + p1;
+            const int c0 = c * 32 + 2 * e, c1 = c0 + 1;
+            const float x0 = fmaf(t[c0], sc, -ref);
+            const float x1 = fmaf(t[c1], sc, -ref);
+            const float p0 = ((c0 & 7) < kEmuPerEight) ? exp2_poly(x0) : fast_exp2(x0);
+            const float p1 = ((c1 & 7) < kEmuPerEight) ? exp2_poly(x1) : fast_exp2(x1);
+            lp[c0 & 7] += p0;
+            lp[c1 & 7] += p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tmem + lane_base + L::kPCol0 + (J & 1) * 64 + c * 16, pk);
+          tmem_st16(tmem + lane_base + L::kPCol0 + (J & 1) * 64 + hf * 32 + c * 16, pk);
         }
+        l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -446,22 +534,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ++nloc;
       }
       if (!ok) break;
-      // Epilogue: out = O / l for this row.
+      // Epilogue: out = O / l for this row and this half of the columns.
       if (!mbar_wait(o_final, static_cast<uint32_t>(it & 1), abort_flag, a.err,
                      kErrPrefillWait)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      lred[((it & 1) * 2 + hf) * BM + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lxchg[it & 1]);
+      if (!mbar_wait(&lxchg[it & 1], static_cast<uint32_t>((it >> 1) & 1), abort_flag, a.err,
+                     kErrPrefillWait)) {
+        ok = false;
+        break;
+      }
+      const float l_row = l + lred[((it & 1) * 2 + (hf ^ 1)) * BM + row];
       uint16_t* orow = a.out + item.b * a.os[0] +
                        static_cast<int64_t>(item.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
-                       static_cast<int64_t>(q) * a.os[2];
-      const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
+                       static_cast<int64_t>(q) * a.os[2] + hf * DH;
+      const float inv_l = 1.f / l_row;  // l == 0: no visible key, NaN output
       if (nloc > 0) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < DH / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem + lane_base + L::kOCol + c * 32, r);
+          tmem_ld32(tmem + lane_base + L::kOCol + hf * DH + c * 32, r);
           tmem_ld_wait();
           if (row_valid) {
 #pragma unroll
@@ -482,7 +579,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else if (row_valid) {
         const float nanv = __int_as_float(0x7fc00000);
         const uint32_t nn = pack_bf16x2(nanv, nanv);
-        for (int d = 0; d < D; d += 8)
+        for (int d = 0; d < DH; d += 8)
           *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
       }
       tc_fence_before();
