@@ -42,6 +42,7 @@ namespace {
 constexpr int KT = kDecodeKeysPerTile;  // keys per tile
 constexpr int NCW = kDecodeConsumerWarps;
 constexpr int CHUNK_BYTES = KT * 128;   // one 64-wide bf16 column chunk of a tile
+constexpr int kFastMerge = 4;           // split groups merged with all loads in flight
 
 __host__ __device__ inline int64_t range_start(int64_t c, int64_t T, int64_t P) {
   return (c * T) / P;
@@ -238,40 +239,94 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
         return;
       }
-      // Split group: publish this CTA's partial, then take a ticket.
+      // Split group: publish this CTA's partial (float4 stores), then take a
+      // ticket: the CTA barrier orders every thread's stores before thread
+      // 0's gpu-scope fence and atomic (release), and thread 0's fence after
+      // the atomic orders the reads of the others' partials (acquire).
       const int64_t slot = (static_cast<int64_t>(blockIdx.x) * segmax + seg) * HP;
-      for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
-        const int h = idx / D, d = idx % D;
+      for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
+        const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
-        float l = 0.f, acc = 0.f;
+        float l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < NCW; ++w) {
             const float sc = fast_exp2(scr_ml[(w * HP + h) * 2] - M);
             l += sc * scr_ml[(w * HP + h) * 2 + 1];
-            acc += sc * scr_o[(w * HP + h) * L::kScrRow + d];
+            const float* src = scr_o + (w * HP + h) * L::kScrRow + d;
+            acc.x += sc * src[0];
+            acc.y += sc * src[1];
+            acc.z += sc * src[2];
+            acc.w += sc * src[3];
           }
         }
-        a.part_o[(slot + h) * D + d] = acc;
+        *reinterpret_cast<float4*>(&a.part_o[(slot + h) * D + d]) = acc;
         if (d == 0) a.part_ml[slot + h] = make_float2(M, l);
       }
-      __threadfence();
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
       if (threadIdx.x == 0) {
         const uint32_t n = static_cast<uint32_t>(c_hi - c_lo + 1);
+        __threadfence();
         const uint32_t old = atomicAdd(&counters[cur], 1u);
+        __threadfence();
         *last_flag = (old == n - 1) ? 1 : 0;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
       if (*last_flag) {
         // Last contributor: every other partial of the group is published.
-        // Stage each contributor's segment index and each head's merged
-        // (max, sum) in shared memory, then accumulate O with 16-byte loads,
-        // several contributors in flight at once.
-        __threadfence();
         const int n = static_cast<int>(c_hi - c_lo + 1);
+        if (n <= kFastMerge) {
+          // Few contributors: every load of a thread's elements in flight at once.
+          int64_t base[kFastMerge];
+#pragma unroll
+          for (int k = 0; k < kFastMerge; ++k) {
+            const int64_t cc = c_lo + (k < n ? k : 0);
+            base[k] = (cc * segmax + (cur - range_start(cc, units, P) / tiles_per_group)) * HP;
+          }
+          for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
+            const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
+            if (pass * HP + h >= a.g) continue;
+            float2 ml[kFastMerge];
+            float4 o[kFastMerge];
+#pragma unroll
+            for (int k = 0; k < kFastMerge; ++k) {
+              if (k < n) {
+                ml[k] = __ldcg(&a.part_ml[base[k] + h]);
+                o[k] = __ldcg(reinterpret_cast<const float4*>(&a.part_o[(base[k] + h) * D + d]));
+              }
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kFastMerge; ++k)
+              if (k < n) M = fmaxf(M, ml[k].x);
+            float Lsum = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (M != -INFINITY) {
+#pragma unroll
+              for (int k = 0; k < kFastMerge; ++k) {
+                if (k < n) {
+                  const float w = fast_exp2(ml[k].x - M);
+                  Lsum += w * ml[k].y;
+                  acc.x += w * o[k].x;
+                  acc.y += w * o[k].y;
+                  acc.z += w * o[k].z;
+                  acc.w += w * o[k].w;
+                }
+              }
+            }
+            const float inv = 1.f / Lsum;  // Lsum == 0: NaN
+            uint2 pk;
+            pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+            pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(obase + (hq0 + h) * a.os[1] + d) = pk;
+          }
+        } else {
+        // Many contributors: stage each one's segment index and each head's
+        // merged (max, sum) in shared memory, then accumulate O with 16-byte
+        // loads, several contributors in flight at once.
         int* sm_seg = reinterpret_cast<int*>(scr_o);          // n ints (scr_o is free now)
         float* sm_ml = scr_ml;                                 // HP x (M, L)
         for (int k = threadIdx.x; k < n; k += NCW * 32)
@@ -317,6 +372,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
           pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
           *reinterpret_cast<uint2*>(obase + (hq0 + h) * a.os[1] + d) = pk;
+        }
         }
         if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
       }

@@ -10,23 +10,33 @@
 //
 // Per 128x128 tile:   S = Q K^T       tcgen05.mma, A and B from shared memory,
 //                                     fp32 accumulator in tensor memory (TMEM)
-//                     P = softmax(S)  256 softmax threads, two per TMEM lane
-//                                     (row), 64 keys each: scale, mask,
-//                                     online max / sum
-//                     O += P V        tcgen05.mma, A = P (bf16) from TMEM,
-//                                     B = V from shared memory, O in TMEM
+//                     P = softmax(S)  128 softmax threads, one TMEM lane (row)
+//                                     each: scale, mask, online max / sum;
+//                                     P (bf16) overwrites the first half of S
+//                     O += P V        tcgen05.mma, A = P from TMEM, B = V from
+//                                     shared memory, O in TMEM
 //
-// Warp roles (352 threads, one CTA per SM, persistent over work tiles):
-//   warps 0-7  softmax, O rescale and epilogue: warp w owns rows 32*(w%4) ..
-//              +31 (TMEM lanes) and column half w/4 of S, P and O
+// Two query tiles (slots A and B: consecutive query blocks of one kv head)
+// share every staged K/V tile, and their work alternates on the tensor core
+// in the order PV_A, QK_A, PV_B, QK_B: while the softmax warps of one slot
+// exponentiate, the tensor core runs the other slot's two products, so the
+// exponential unit and the tensor pipe overlap.  TMEM: S_A, S_B (128 columns
+// each), O_A, O_B (D columns each).  tcgen05.mma instructions from one thread
+// execute in issue order, so QK of a slot may follow the PV that reads the P
+// stored in the same columns.
+//
+// Warp roles (384 threads, one CTA per SM, persistent over pairs of tiles):
+//   warps 0-3  softmax, O rescale and epilogue of slot A (thread t: row t)
+//   warps 4-7  the same for slot B
 //   warp 8     TMA producer of Q tiles and K tiles
 //   warp 9     TMEM allocator and single-thread MMA issuer
-//   warp 10    TMA producer of V tiles
-// S is double-buffered in TMEM so that QK^T of tile j+1 runs on the tensor
-// cores while the softmax threads work on tile j, and PV of tile j-1 runs
-// behind it.  The running maximum is rescaled lazily: exponentials use a
-// reference that may trail the true maximum by up to 2^8, and O and l are
-// rescaled (O in TMEM) only when the maximum grows past that.
+//   warp 10    TMA producer of V tiles (warp 11 idles)
+// The producer / MMA warpgroup gives registers back (setmaxnreg) so that each
+// softmax thread can hold its whole 128-score row in registers and read S
+// from TMEM once per tile.
+// The running maximum is rescaled lazily: exponentials use a reference that
+// may trail the true maximum by up to 2^8, and O and l are rescaled (O in
+// TMEM) only when the maximum grows past that.
 //
 // Causal tiles above the diagonal are never visited; with a bool mask a
 // pre-pass classifies every (query tile, key tile) pair as hidden / mixed /
@@ -42,13 +52,23 @@ namespace {
 
 constexpr int BM = 128;  // rows per tile = TMEM lanes
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kSoftmaxWarps = 8;
 constexpr int kWarpQK = 8;
 constexpr int kWarpMMA = 9;
-constexpr int kWarpV = 10;
-constexpr int kPrefillThreads = 11 * 32;
+constexpr int kWarpV = 10;  // warp 11 idles (it completes the third warpgroup)
+constexpr int kPrefillThreads = 12 * 32;
+// Register split across the three warpgroups (setmaxnreg): the launch gives
+// every thread kLaunchRegs; the producer / MMA warpgroup drops to kIoRegs and
+// the two softmax warpgroups rise to kSoftmaxRegs, which must add up to the
+// launch's total: 128 * kIoRegs + 256 * kSoftmaxRegs <= 384 * kLaunchRegs
+// (setmaxnreg.inc waits for registers that a larger split would never free).
+constexpr int kLaunchRegs = 168;
+constexpr int kIoRegs = 88;
+constexpr int kSoftmaxRegs = 200;
+static_assert(128 * kIoRegs + 256 * kSoftmaxRegs <= kPrefillThreads * kLaunchRegs,
+              "register split must fit in the launch allocation");
 constexpr int kStages = 2;  // depth of the K ring and of the V ring
-constexpr int kQBufs = 2;
+constexpr int kSlots = 2;   // query tiles in flight (A, B)
+static_assert(kStages == 2 && kSlots == 2, "register-packed ring bookkeeping assumes two stages and two slots");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials of every eight computed on the FMA pipe (exp2_poly) rather
@@ -63,50 +83,71 @@ struct Layout {
   static constexpr int CH = D / 64;                  // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 bytes
   static constexpr int kTileBytes = CH * kChunkBytes;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBufs * kTileBytes;
+  static constexpr int kQOff = 0;                    // one Q tile per slot
+  static constexpr int kKOff = kQOff + kSlots * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 4 * kStages + 2 + 2 + 4 + 2 + 2;
+  static constexpr int kNumBars = 2 * kSlots + 4 * kStages + 5 * kSlots + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kRedOff = kMiscOff + 16;               // row max / sum exchange
-  static constexpr int kBytes = kRedOff + 8 * BM * 4 + 1024;  // + alignment slack
-  // TMEM columns.
-  static constexpr uint32_t kSCol0 = 0;     // S buffers at 0 and 128
-  static constexpr uint32_t kOCol = 256;    // O: D columns
-  static constexpr uint32_t kPCol0 = 256 + D;  // P buffers (bf16 pairs): 64 columns each
+  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  // TMEM columns: S of slot s at 128 s (P in its first 64), O at 256 + D s.
+  static constexpr uint32_t kSCol = 128;
+  static constexpr uint32_t kOCol0 = 256;
 };
 
-struct Item {
-  int b, kv, mt, q0, q_last, nt_end;
+struct Pair {
+  int b, kv, mt0, nt_end;
 };
 
-__device__ __forceinline__ Item item_of(int64_t x, const PrefillArgs& a, int m_tiles, int qpt,
-                                        int n_tiles) {
-  Item it;
-  const int64_t bh = static_cast<int64_t>(a.B) * a.Hkv;
-  it.mt = m_tiles - 1 - static_cast<int>(x / bh);  // longest causal rows first
-  const int bk = static_cast<int>(x % bh);
-  it.b = bk / a.Hkv;
-  it.kv = bk % a.Hkv;
-  it.q0 = it.mt * qpt;
-  it.q_last = min(it.q0 + qpt, a.Sq) - 1;
-  it.nt_end = a.causal ? min(n_tiles, it.q_last / BN + 1) : n_tiles;
-  return it;
+struct Slot {  // one query tile of a pair
+  int mt, q0, q_last;
+  bool live;
+};
+
+// Work item x: a pair of consecutive query tiles (2p, 2p+1) of one
+// (batch, kv head); late (long causal) pairs first.
+__device__ __forceinline__ Slot slot_of(const Pair& pr, int s, const PrefillArgs& a,
+                                        int m_tiles, int qpt) {
+  Slot sl;
+  sl.mt = pr.mt0 + s;
+  sl.live = sl.mt < m_tiles;
+  sl.q0 = sl.mt * qpt;
+  sl.q_last = sl.live ? min(sl.q0 + qpt, a.Sq) - 1 : -1;
+  return sl;
 }
 
-// 0: every key hidden from every row (skip), 1: mixed (mask per element),
-// 2: every key visible to every row.
-__device__ __forceinline__ int tile_class(const PrefillArgs& a, const Item& it, int nt,
-                                          int m_tiles, int n_tiles) {
+__device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_tiles, int qpt,
+                                        int n_tiles) {
+  Pair pr;
+  const int64_t bh = static_cast<int64_t>(a.B) * a.Hkv;
+  const int pairs = (m_tiles + 1) / 2;
+  const int p = pairs - 1 - static_cast<int>(x / bh);
+  const int bk = static_cast<int>(x % bh);
+  pr.b = bk / a.Hkv;
+  pr.kv = bk % a.Hkv;
+  pr.mt0 = 2 * p;
+  const int q_hi = max(slot_of(pr, 0, a, m_tiles, qpt).q_last,
+                       slot_of(pr, 1, a, m_tiles, qpt).q_last);
+  pr.nt_end = a.causal ? min(n_tiles, q_hi / BN + 1) : n_tiles;
+  return pr;
+}
+
+// Class of key tile nt for one slot: 0 every key hidden from every row
+// (skip), 1 mixed (mask per element), 2 every key visible to every row.
+__device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, const Slot& sl,
+                                          int nt, int m_tiles, int n_tiles) {
+  if (!sl.live) return 0;
   int cls = 2;
   const int j0 = nt * BN, j1 = j0 + BN - 1;
   if (j1 >= a.Sk) cls = 1;
-  if (a.causal && j1 > it.q0) cls = 1;
+  if (a.causal) {
+    if (j0 > sl.q_last) return 0;
+    if (j1 > sl.q0) cls = 1;
+  }
   if (a.has_mask) {
-    const int s = a.summary[(static_cast<int64_t>(it.b) * m_tiles + it.mt) * n_tiles + nt];
-    if (s == 0) return 0;
-    if (s == 1) cls = 1;
+    const int c = a.summary[(static_cast<int64_t>(pr.b) * m_tiles + sl.mt) * n_tiles + nt];
+    if (c == 0) return 0;
+    if (c == 1) cls = 1;
   }
   return cls;
 }
@@ -171,20 +212,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = q_full + kQBufs;
-  uint64_t* k_full = q_empty + kQBufs;
+  uint64_t* q_full = bars;                   // [slot]
+  uint64_t* q_empty = q_full + kSlots;       // [slot]
+  uint64_t* k_full = q_empty + kSlots;       // [stage]
   uint64_t* k_empty = k_full + kStages;
   uint64_t* v_full = k_empty + kStages;
   uint64_t* v_empty = v_full + kStages;
-  uint64_t* s_full = v_empty + kStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_ready = p_full + 2;
-  uint64_t* o_final = o_ready + 1;
-  uint64_t* o_free = o_final + 1;
-  uint64_t* mma_done = o_free + 1;
-  uint64_t* xchg = mma_done + 1;   // [2]: row-max exchange between column halves
-  uint64_t* lxchg = xchg + 2;      // [2]: row-sum exchange at the epilogue
+  uint64_t* s_full = v_empty + kStages;      // [slot]: S of the slot's next tile is in TMEM
+  uint64_t* p_full = s_full + kSlots;        // [slot]: P written (4 softmax warps)
+  uint64_t* o_ready = p_full + kSlots;       // [slot]: a PV into O has completed
+  uint64_t* o_final = o_ready + kSlots;      // [slot]: the pair's last PV has completed
+  uint64_t* o_free = o_final + kSlots;       // [slot]: epilogue has read O (4 warps)
+  uint64_t* mma_done = o_free + kSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -192,9 +231,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kQBufs; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_ready[i], 1);
+      mbar_init(&o_final[i], 1);
+      mbar_init(&o_free[i], 4);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
@@ -202,24 +246,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kSoftmaxWarps);
-    }
-    mbar_init(o_ready, 1);
-    mbar_init(o_final, 1);
-    mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&xchg[i], kSoftmaxWarps);
-      mbar_init(&lxchg[i], kSoftmaxWarps);
-    }
     *abort_flag = 0;
     fence_mbar_init();
   }
   // Rows past qpt * g of a query tile are never written by TMA: zero them once.
   if (rows < BM && threadIdx.x < BM) {
-    for (int qb = 0; qb < kQBufs; ++qb)
+    for (int qb = 0; qb < kSlots; ++qb)
       for (int c = 0; c < CH; ++c) {
         uint8_t* base = smem + L::kQOff + qb * L::kTileBytes + c * L::kChunkBytes;
         for (int r = rows; r < BM; ++r)
@@ -237,6 +270,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+  // Producer / MMA warpgroup (warps 8-11): every warp drops its registers.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIoRegs));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------- producers
     if (lane == 0) {
@@ -249,28 +285,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (is_qk) prefetch_tmap(&tmq);
       uint32_t kt = 0;
       int64_t it = 0;
-      int32_t last_round[kStages] = {-1, -1};
-      int32_t last_q_round[kQBufs] = {-1, -1};
+      // Last round issued per ring stage / per Q slot (for the unwind drain),
+      // kept in registers: -1 = none.
+      int32_t last_round0 = -1, last_round1 = -1, last_q0 = -1, last_q1 = -1;
       bool ok = true;
       for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
-        const Item item = item_of(x, a, m_tiles, qpt, n_tiles);
+        const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
+        const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
         if (is_qk) {
-          const int qb = static_cast<int>(it & 1);
-          const uint32_t round = static_cast<uint32_t>(it >> 1);
-          if (round > 0 && !mbar_wait(&q_empty[qb], (round - 1) & 1u, abort_flag, a.err,
-                                      kErrPrefillWait)) {
-            ok = false;
-            break;
+#pragma unroll
+          for (int sl = 0; sl < kSlots; ++sl) {
+            if (!ok) break;
+            if (it > 0 && !mbar_wait(&q_empty[sl], static_cast<uint32_t>((it - 1) & 1),
+                                     abort_flag, a.err, kErrPrefillWait)) {
+              ok = false;
+              break;
+            }
+            uint8_t* qdst = smem + L::kQOff + sl * L::kTileBytes;
+            mbar_arrive_expect_tx(&q_full[sl], static_cast<uint32_t>(rows * 128 * CH));
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[sl], c * 64,
+                          (sl == 0 ? s0 : s1).q0, pr.kv * a.g, pr.b);
+            if (sl == 0) last_q0 = static_cast<int32_t>(it); else last_q1 = static_cast<int32_t>(it);
           }
-          uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
-          mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, item.q0,
-                        item.kv * a.g, item.b);
-          last_q_round[qb] = static_cast<int32_t>(round);
+          if (!ok) break;
         }
-        for (int nt = 0; nt < item.nt_end; ++nt) {
-          if (tile_class(a, item, nt, m_tiles, n_tiles) == 0) continue;
+        for (int nt = 0; nt < pr.nt_end; ++nt) {
+          if (tile_class(a, pr, s0, nt, m_tiles, n_tiles) == 0 &&
+              tile_class(a, pr, s1, nt, m_tiles, n_tiles) == 0)
+            continue;
           const int s = static_cast<int>(kt % kStages);
           const uint32_t round = kt / kStages;
           if (round > 0 &&
@@ -281,19 +324,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           uint8_t* dst = ring + s * L::kTileBytes;
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
           for (int c = 0; c < CH; ++c)
-            tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, item.kv,
-                        item.b);
-          last_round[s] = static_cast<int32_t>(round);
+            tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
+          if (s == 0) last_round0 = static_cast<int32_t>(round); else last_round1 = static_cast<int32_t>(round);
           ++kt;
         }
       }
       if (*abort_flag) {  // let every copy in flight land before the CTA exits
-        for (int s = 0; s < kStages; ++s)
-          if (last_round[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(last_round[s]) & 1u);
-        if (is_qk)
-          for (int qb = 0; qb < kQBufs; ++qb)
-            if (last_q_round[qb] >= 0)
-              mbar_wait_drain(&q_full[qb], static_cast<uint32_t>(last_q_round[qb]) & 1u);
+        if (last_round0 >= 0) mbar_wait_drain(&full[0], static_cast<uint32_t>(last_round0) & 1u);
+        if (last_round1 >= 0) mbar_wait_drain(&full[1], static_cast<uint32_t>(last_round1) & 1u);
+        if (is_qk && last_q0 >= 0) mbar_wait_drain(&q_full[0], static_cast<uint32_t>(last_q0) & 1u);
+        if (is_qk && last_q1 >= 0) mbar_wait_drain(&q_full[1], static_cast<uint32_t>(last_q1) & 1u);
       }
     }
   } else if (warp == kWarpMMA) {
@@ -304,197 +344,213 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t q_base = smem_u32(smem + L::kQOff);
       const uint32_t k_base = smem_u32(smem + L::kKOff);
       const uint32_t v_base = smem_u32(smem + L::kVOff);
-      uint32_t kt = 0, J = 0;
+      uint32_t kt = 0;
+      uint32_t J[kSlots] = {0, 0};       // tiles issued per slot, over the whole kernel
+      uint32_t uses = 0;                 // PVs still to read V stage s: bits [8s, 8s+8)
       int64_t it = 0;
       bool ok = true;
 
-      // PV of the tile with global index Jp (K/V ring slot kp): O (+)= P V.
-      auto issue_pv = [&](uint32_t Jp, uint32_t kp, int local, int64_t item_idx) -> bool {
-        if (!mbar_wait(&p_full[Jp & 1], (Jp >> 1) & 1u, abort_flag, a.err, kErrPrefillWait))
-          return false;
+      // O_sl (+)= P_sl V for the slot's tile with per-slot index Jp, K/V tile kp.
+      auto issue_pv = [&](int sl, uint32_t Jp, uint32_t kp, int local) -> bool {
+        if (!mbar_wait(&p_full[sl], Jp & 1u, abort_flag, a.err, kErrPrefillWait)) return false;
         const int s = static_cast<int>(kp % kStages);
         if (!mbar_wait(&v_full[s], (kp / kStages) & 1u, abort_flag, a.err, kErrPrefillWait))
           return false;
-        if (local == 0 && item_idx > 0 &&
-            !mbar_wait(o_free, static_cast<uint32_t>((item_idx - 1) & 1), abort_flag, a.err,
+        if (local == 0 && it > 0 &&
+            !mbar_wait(&o_free[sl], static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
                        kErrPrefillWait))
           return false;
         tc_fence_after();
         const uint32_t vs = v_base + s * L::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint32_t a_tmem = tmem + L::kPCol0 + (Jp & 1) * 64 + ks * 8;
+          const uint32_t a_tmem = tmem + sl * L::kSCol + ks * 8;
           const uint64_t bdesc = mnmajor_desc(vs + ks * 16 * 128, L::kChunkBytes);
-          tc_mma_ts(tmem + L::kOCol, a_tmem, bdesc, idesc_pv, (local > 0 || ks > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + L::kOCol0 + sl * D, a_tmem, bdesc, idesc_pv,
+                    (local > 0 || ks > 0) ? 1u : 0u);
         }
-        tc_commit(&v_empty[s]);
-        tc_commit(o_ready);
+        tc_commit(&o_ready[sl]);
+        uses -= 1u << (8 * s);
+        if (((uses >> (8 * s)) & 0xFFu) == 0) tc_commit(&v_empty[s]);
         return true;
       };
 
       for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
-        const Item item = item_of(x, a, m_tiles, qpt, n_tiles);
-        const int qb = static_cast<int>(it & 1);
-        if (!mbar_wait(&q_full[qb], static_cast<uint32_t>((it >> 1) & 1), abort_flag, a.err,
-                       kErrPrefillWait)) {
-          ok = false;
-          break;
-        }
-        const uint32_t qs = q_base + qb * L::kTileBytes;
-        bool pending = false;
-        uint32_t pJ = 0, pk = 0;
-        int nloc = 0;
-        for (int nt = 0; nt < item.nt_end && ok; ++nt) {
-          if (tile_class(a, item, nt, m_tiles, n_tiles) == 0) continue;
+        const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
+        const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
+#pragma unroll
+        for (int sl = 0; sl < kSlots; ++sl)
+          if (ok && !mbar_wait(&q_full[sl], static_cast<uint32_t>(it & 1), abort_flag, a.err,
+                               kErrPrefillWait))
+            ok = false;
+        if (!ok) break;
+        bool pend[kSlots] = {false, false};
+        uint32_t pJ[kSlots] = {0, 0}, pk[kSlots] = {0, 0};
+        int nloc[kSlots] = {0, 0};
+        for (int nt = 0; nt < pr.nt_end && ok; ++nt) {
+          const int cls0 = tile_class(a, pr, s0, nt, m_tiles, n_tiles);
+          const int cls1 = tile_class(a, pr, s1, nt, m_tiles, n_tiles);
+          if (cls0 == 0 && cls1 == 0) continue;
           const int s = static_cast<int>(kt % kStages);
           if (!mbar_wait(&k_full[s], (kt / kStages) & 1u, abort_flag, a.err, kErrPrefillWait)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          uses = (uses & ~(0xFFu << (8 * s))) |
+                 (static_cast<uint32_t>((cls0 != 0) + (cls1 != 0)) << (8 * s));
           const uint32_t ks_base = k_base + s * L::kTileBytes;
-          const uint32_t d_s = tmem + L::kSCol0 + (J & 1) * 128;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-            tc_mma_ss(d_s, kmajor_desc(qs + off), kmajor_desc(ks_base + off), idesc_qk,
-                      ks > 0 ? 1u : 0u);
+          for (int sl = 0; sl < kSlots; ++sl) {
+            if (!ok) break;
+            const bool act = (sl == 0 ? cls0 : cls1) != 0;
+            // The slot's previous PV goes first: its P lives in the S columns
+            // that this QK overwrites (in-order execution on the tensor core).
+            if (pend[sl]) {
+              if (!issue_pv(sl, pJ[sl], pk[sl], nloc[sl] - 1)) {
+                ok = false;
+                break;
+              }
+              pend[sl] = false;
+            }
+            if (!act) continue;
+            const uint32_t qs = q_base + sl * L::kTileBytes;
+            const uint32_t d_s = tmem + sl * L::kSCol;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+              tc_mma_ss(d_s, kmajor_desc(qs + off), kmajor_desc(ks_base + off), idesc_qk,
+                        ks > 0 ? 1u : 0u);
+            }
+            tc_commit(&s_full[sl]);
+            pend[sl] = true;
+            pJ[sl] = J[sl];
+            pk[sl] = kt;
+            ++nloc[sl];
+            ++J[sl];
           }
-          tc_commit(&s_full[J & 1]);
+          if (!ok) break;
           tc_commit(&k_empty[s]);
-          if (pending && !issue_pv(pJ, pk, nloc - 1, it)) {
-            ok = false;
-            break;
-          }
-          pending = true;
-          pJ = J;
-          pk = kt;
-          ++nloc;
-          ++J;
           ++kt;
         }
         if (!ok) break;
-        if (pending && !issue_pv(pJ, pk, nloc - 1, it)) {
-          ok = false;
-          break;
+#pragma unroll
+        for (int sl = 0; sl < kSlots; ++sl)
+          if (ok && pend[sl] && !issue_pv(sl, pJ[sl], pk[sl], nloc[sl] - 1)) ok = false;
+        if (!ok) break;
+#pragma unroll
+        for (int sl = 0; sl < kSlots; ++sl) {
+          if (!ok) break;
+          tc_commit(&q_empty[sl]);
+          if (nloc[sl] == 0 && it > 0 &&
+              !mbar_wait(&o_free[sl], static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
+                         kErrPrefillWait)) {
+            ok = false;
+            break;
+          }
+          tc_commit(&o_final[sl]);
         }
-        tc_commit(&q_empty[qb]);
-        if (nloc == 0 && it > 0 &&
-            !mbar_wait(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
-                       kErrPrefillWait)) {
-          ok = false;
-          break;
-        }
-        tc_commit(o_final);
       }
       // Every MMA issued so far has completed before TMEM is released.
       tc_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
+  }
   } else {
     // ------------------------------------------------------------- softmax
-    // Eight warps: warp w serves TMEM lanes 32*(w % 4) .. +31 (its rows) and
-    // column half hf = w / 4 of each S tile (64 keys), of P and of O, so two
-    // warps per SM sub-partition share every row.  The halves exchange their
-    // row maxima through shared memory and an mbarrier once per tile, and
-    // their partial row sums once per work tile.
-    const int quad = warp & 3, hf = warp >> 2;
-    const int row = quad * 32 + lane;  // TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // Warps 4 sl .. 4 sl + 3 own slot sl; thread t of the group owns row t
+    // (TMEM lane t) of the slot's tiles.
+    const int sl = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + sl * L::kSCol;
+    const uint32_t o_col = tmem + lane_base + L::kOCol0 + sl * D;
     const int hh = row / qpt, qi = row % qpt;
-    constexpr int DH = D / 2;  // O columns per half
     // Mask rows can be read as 16-byte vectors when base and strides allow.
     const bool mask_vec = a.has_mask && ((reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0) &&
                           (a.ms[0] % 16 == 0) && (a.ms[1] % 16 == 0);
-    float* red = reinterpret_cast<float*>(smem + L::kRedOff);  // [2 parity][2 halves][BM]
-    float* lred = red + 4 * BM;                                // [2 parity][2 halves][BM]
     uint32_t J = 0;
     int64_t it = 0;
     bool ok = true;
     for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
-      const Item item = item_of(x, a, m_tiles, qpt, n_tiles);
-      const int q = item.q0 + qi;
-      const bool row_valid = row < rows && q < a.Sq;
+      const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
+      const Slot me = slot_of(pr, sl, a, m_tiles, qpt);
+      const int q = me.q0 + qi;
+      const bool row_valid = me.live && row < rows && q < a.Sq;
       const uint8_t* mrow =
-          (a.has_mask && row_valid) ? a.mask + item.b * a.ms[0] + static_cast<int64_t>(q) * a.ms[1]
+          (a.has_mask && row_valid) ? a.mask + pr.b * a.ms[0] + static_cast<int64_t>(q) * a.ms[1]
                                     : nullptr;
       float m_ref = -INFINITY, l = 0.f;
       int nloc = 0;
-      for (int nt = 0; nt < item.nt_end; ++nt) {
-        const int cls = tile_class(a, item, nt, m_tiles, n_tiles);
+      for (int nt = 0; nt < pr.nt_end; ++nt) {
+        const int cls = tile_class(a, pr, me, nt, m_tiles, n_tiles);
         if (cls == 0) continue;
-        if (!mbar_wait(&s_full[J & 1], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
+        if (!mbar_wait(&s_full[sl], J & 1u, abort_flag, a.err, kErrPrefillWait)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // This half's 64 scores of the row.  Fully visible tiles keep raw
-        // scores and fold the scale into one FMA per element; other tiles go
-        // to the base-2 domain with -inf where a key is hidden.
+        // Pass 1 over the S row: its maximum.  Fully visible tiles work on raw
+        // scores and fold the scale into one FMA per element in pass 2; other
+        // tiles test each key against the row's visibility bits.
         const bool fast = (cls == 2) && (a.scale_log2 >= 0.f);
-        float t[64];
-        {
-          uint32_t r[64];
-          const uint32_t sbase = tmem + lane_base + L::kSCol0 + (J & 1) * 128 + hf * 64;
-          tmem_ld32(sbase, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          tmem_ld_wait();
-          if (fast) {
+        uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};
+        if (!fast)
+          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a.Sk, a.causal, q, mask_vec);
+        auto masked_t = [&](float sv, int c) -> float {
+          return ((vb[c >> 5] >> (c & 31)) & 1u) ? sv * a.scale_log2 : -INFINITY;
+        };
+        // The whole S row of this thread, read from TMEM once (four loads in
+        // flight), kept in registers for the max and the exponentials.
+        uint32_t r[BN];
+        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        tmem_ld_wait();
+        if (!fast) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) t[c] = __uint_as_float(r[c]);
-          } else {
-            uint32_t vb[4];
-            visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a.Sk, a.causal, q, mask_vec);
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const int cc = hf * 64 + c;
-              t[c] = ((vb[cc >> 5] >> (cc & 31)) & 1u) ? __uint_as_float(r[c]) * a.scale_log2
-                                                       : -INFINITY;
-            }
-          }
+          for (int c = 0; c < BN; ++c) r[c] = __float_as_uint(masked_t(__uint_as_float(r[c]), c));
         }
         float mx;
         {
+          // Eight independent running maxima, two elements per three-input max.
           float part[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) part[e] = t[e];
+          for (int e = 0; e < 8; ++e) part[e] = -INFINITY;
 #pragma unroll
-          for (int c = 8; c < 64; ++c) part[c & 7] = fmaxf(part[c & 7], t[c]);
-          mx = fmaxf(fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3])),
-                     fmaxf(fmaxf(part[4], part[5]), fmaxf(part[6], part[7])));
+          for (int c = 0; c < BN; c += 16)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              part[e] = fmax3(part[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
+          mx = fmax3(fmax3(part[0], part[1], part[2]), fmax3(part[3], part[4], part[5]),
+                     fmaxf(part[6], part[7]));
           if (fast) mx *= a.scale_log2;
         }
-        // Row maximum over both halves.
-        red[((J & 1) * 2 + hf) * BM + row] = mx;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xchg[J & 1]);
-        if (!mbar_wait(&xchg[J & 1], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
-          ok = false;
-          break;
-        }
-        mx = fmaxf(mx, red[((J & 1) * 2 + (hf ^ 1)) * BM + row]);
         const float m_new = fmaxf(m_ref, mx);
         const bool grow = m_new > m_ref + kRescaleLog2;  // also true for -inf -> finite
         const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         const bool o_live = grow && nloc > 0 && m_ref != -INFINITY;
         if (__any_sync(0xffffffffu, o_live)) {
-          // O holds earlier tiles' P V with the old reference: rescale this half.
-          if (!mbar_wait(o_ready, (J - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
+          // O holds earlier tiles' P V with the old reference: rescale it.  The
+          // slot's previous PV was issued before this tile's QK, so it has
+          // completed; the wait returns at once.
+          if (!mbar_wait(&o_ready[sl], (J - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const float f = o_live ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
-            const uint32_t oa = tmem + lane_base + L::kOCol + hf * DH + c * 32;
-            tmem_ld32(oa, r);
+            tmem_ld32(o_col + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-            tmem_st16(oa, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tmem_st16(oa + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+            tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
           }
           tmem_st_wait();
         }
@@ -503,62 +559,54 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           m_ref = m_new;
         }
         const float ref = exp_ref(m_ref);
-        // P = 2^(t - ref) as bf16 pairs into TMEM (A operand of the PV MMA);
-        // kEmuPerEight of every eight exponentials run on the FMA pipe.
+        // P = 2^(t - ref) as bf16 pairs over the first 64 columns of S (A
+        // operand of the PV MMA); S is already in registers.  kEmuPerEight of
+        // every eight exponentials run on the FMA pipe.
         float lp[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) lp[e] = 0.f;
         const float sc = fast ? a.scale_log2 : 1.f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < BN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = c * 32 + 2 * e, c1 = c0 + 1;
-            const float x0 = fmaf(t[c0], sc, -ref);
-            const float x1 = fmaf(t[c1], sc, -ref);
+            const float x0 = fmaf(__uint_as_float(r[c0]), sc, -ref);
+            const float x1 = fmaf(__uint_as_float(r[c1]), sc, -ref);
             const float p0 = ((c0 & 7) < kEmuPerEight) ? exp2_poly(x0) : fast_exp2(x0);
             const float p1 = ((c1 & 7) < kEmuPerEight) ? exp2_poly(x1) : fast_exp2(x1);
             lp[c0 & 7] += p0;
             lp[c1 & 7] += p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tmem + lane_base + L::kPCol0 + (J & 1) * 64 + hf * 32 + c * 16, pk);
+          tmem_st16(s_col + c * 16, pk);
         }
         l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[J & 1]);
+        if (lane == 0) mbar_arrive(&p_full[sl]);
         ++J;
         ++nloc;
       }
       if (!ok) break;
-      // Epilogue: out = O / l for this row and this half of the columns.
-      if (!mbar_wait(o_final, static_cast<uint32_t>(it & 1), abort_flag, a.err,
+      // Epilogue: out = O / l for this row.
+      if (!mbar_wait(&o_final[sl], static_cast<uint32_t>(it & 1), abort_flag, a.err,
                      kErrPrefillWait)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      lred[((it & 1) * 2 + hf) * BM + row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&lxchg[it & 1]);
-      if (!mbar_wait(&lxchg[it & 1], static_cast<uint32_t>((it >> 1) & 1), abort_flag, a.err,
-                     kErrPrefillWait)) {
-        ok = false;
-        break;
-      }
-      const float l_row = l + lred[((it & 1) * 2 + (hf ^ 1)) * BM + row];
-      uint16_t* orow = a.out + item.b * a.os[0] +
-                       static_cast<int64_t>(item.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
-                       static_cast<int64_t>(q) * a.os[2] + hf * DH;
-      const float inv_l = 1.f / l_row;  // l == 0: no visible key, NaN output
+      uint16_t* orow = a.out + pr.b * a.os[0] +
+                       static_cast<int64_t>(pr.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
+                       static_cast<int64_t>(q) * a.os[2];
+      const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
       if (nloc > 0) {
 #pragma unroll
-        for (int c = 0; c < DH / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem + lane_base + L::kOCol + hf * DH + c * 32, r);
+          tmem_ld32(o_col + c * 32, r);
           tmem_ld_wait();
           if (row_valid) {
 #pragma unroll
@@ -579,12 +627,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else if (row_valid) {
         const float nanv = __int_as_float(0x7fc00000);
         const uint32_t nn = pack_bf16x2(nanv, nanv);
-        for (int d = 0; d < DH; d += 8)
+        for (int d = 0; d < D; d += 8)
           *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0) mbar_arrive(&o_free[sl]);
     }
   }
 
@@ -649,7 +697,7 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.rows = static_cast<int>(s.qpt * g);
   s.m_tiles = static_cast<int>((p.seq_q + s.qpt - 1) / s.qpt);
   s.n_tiles = static_cast<int>((p.seq_k + BN - 1) / BN);
-  s.work = p.batch * p.heads_kv * s.m_tiles;
+  s.work = p.batch * p.heads_kv * ((s.m_tiles + 1) / 2);  // pairs of query tiles
   s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
   if (s.grid < 1) s.grid = 1;
   s.smem_bytes = s.D == 128 ? Layout<128>::kBytes : Layout<64>::kBytes;
