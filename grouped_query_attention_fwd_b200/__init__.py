@@ -33,7 +33,7 @@ GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 
 GQA_ERR_SCRATCH_LIMIT = 10
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 GQA_DTYPE_BF16, GQA_DTYPE_F32 = 0, 1
-KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero"}
+KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
 
 EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
            "gqa_forward_decode_noalloc")
@@ -48,6 +48,7 @@ class Problem(ctypes.Structure):
         ("q_stride", ctypes.c_int64 * 4), ("k_stride", ctypes.c_int64 * 4),
         ("v_stride", ctypes.c_int64 * 4), ("o_stride", ctypes.c_int64 * 4),
         ("mask_stride", ctypes.c_int64 * 3),
+        ("causal_offset", ctypes.c_int64), ("window", ctypes.c_int64),
     ]
 
 
@@ -98,11 +99,14 @@ def version() -> int:
 
 def make_problem(dtype: int, B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int,
                  q_stride, k_stride, v_stride, o_stride, mask_stride=None,
-                 causal: bool = False, scale: float | None = None) -> Problem:
+                 causal: bool = False, scale: float | None = None, causal_offset: int = 0,
+                 window: int = 0) -> Problem:
     """Build the C problem descriptor from plain sizes and element strides."""
     p = Problem()
     p.dtype = dtype
     p.causal = int(bool(causal))
+    p.causal_offset = int(causal_offset)
+    p.window = int(window)
     p.has_mask = int(mask_stride is not None)
     p.scale = float((1.0 / math.sqrt(D) if D > 0 else 1.0) if scale is None else scale)
     p.batch, p.heads_q, p.heads_kv, p.seq_q, p.seq_k, p.head_dim = B, Hq, Hkv, Sq, Sk, D
@@ -152,7 +156,26 @@ def _dtype_code(t) -> int:
     raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
 
 
-def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None) -> Problem:
+def _offset(causal, causal_offset, Sq, Sk) -> int:
+    """Causal diagonal: j <= i + offset.  With Sq == Sk the pages' causal
+    attention is offset 0; otherwise the caller must say which alignment it
+    wants ("bottom_right" = Sk - Sq, "top_left" = 0, or an integer)."""
+    if not causal:
+        return 0
+    if causal_offset is None:
+        if Sq != Sk:
+            raise ValueError("causal with seq_q != seq_k needs causal_offset "
+                             "('bottom_right', 'top_left' or an integer)")
+        return 0
+    if causal_offset == "bottom_right":
+        return Sk - Sq
+    if causal_offset == "top_left":
+        return 0
+    return int(causal_offset)
+
+
+def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None, causal_offset=None,
+                window=0) -> Problem:
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, S, D]")
     if not (q.dtype == k.dtype == v.dtype):
@@ -168,11 +191,14 @@ def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None) -> Probl
             raise ValueError("mask must be [B, Sq, Sk]")
         mst = mask.stride()
     return make_problem(_dtype_code(q), B, Hq, Hkv, Sq, Sk, D, q.stride(), k.stride(),
-                        v.stride(), ost, mst, causal=causal, scale=scale)
+                        v.stride(), ost, mst, causal=causal, scale=scale,
+                        causal_offset=_offset(causal, causal_offset, Sq, Sk), window=window)
 
 
-def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0) -> dict:
-    return query_problem(problem_for(q, k, v, mask, causal, scale), sm_count).as_dict()
+def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0, causal_offset=None,
+          window=0) -> dict:
+    return query_problem(problem_for(q, k, v, mask, causal, scale, causal_offset=causal_offset,
+                                     window=window), sm_count).as_dict()
 
 
 def workspace_for(device, nbytes: int):
@@ -188,8 +214,13 @@ def workspace_for(device, nbytes: int):
 
 
 def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=None,
-            stream=None):
-    """out = softmax(mask(q k_{h/g}^T * scale)) v_{h/g} on the GPU."""
+            stream=None, causal_offset=None, window=0):
+    """out = softmax(mask(q k_{h/g}^T * scale)) v_{h/g} on the GPU.
+
+    causal: key j visible to query i iff j <= i + offset (offset 0 for
+    Sq == Sk; pass causal_offset="bottom_right" for a query block at the end
+    of the keys).  window > 0 keeps only the last `window` keys up to the
+    diagonal (sliding-window attention)."""
     torch = _torch()
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors (there is no CPU path)")
@@ -202,7 +233,7 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
             raise TypeError("mask must be bool or uint8")
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
-    p = problem_for(q, k, v, mask, causal, scale, out)
+    p = problem_for(q, k, v, mask, causal, scale, out, causal_offset=causal_offset, window=window)
     plan = query_problem(p)
     if workspace is None:
         workspace = workspace_for(q.device, plan.workspace_bytes)

@@ -35,7 +35,8 @@ int validate(const gqa_problem* pp) {
     if (p.q_stride[d] < 0 || p.k_stride[d] < 0 || p.v_stride[d] < 0 || p.o_stride[d] < 0 ||
         (p.has_mask && p.mask_stride[d] < 0))
       return GQA_ERR_LAYOUT;
-  if (p.causal && p.seq_q != p.seq_k) return GQA_ERR_UNSUPPORTED;
+  if (p.window < 0 || (p.window > 0 && !p.causal)) return GQA_ERR_ARG;
+  if (p.causal_offset <= -lim || p.causal_offset >= lim || p.window >= lim) return GQA_ERR_ARG;
   if (bf16_paths(p)) {
     if (p.head_dim != 64 && p.head_dim != 128) return GQA_ERR_UNSUPPORTED;
     // 16-byte rule of the TMA unit for every stride of a dimension longer than 1.
@@ -55,11 +56,27 @@ int validate(const gqa_problem* pp) {
   return GQA_OK;
 }
 
+// No key is visible to any query under causal / window.
+bool nothing_visible(const gqa_problem& p) {
+  if (!p.causal) return false;
+  // Query i sees keys [i + off - window + 1, i + off] (window > 0) or [0, i + off].
+  const int64_t top = p.seq_q - 1 + p.causal_offset;  // largest upper bound
+  if (top < 0) return true;
+  if (p.window > 0 && p.causal_offset - p.window + 1 > p.seq_k - 1) return true;
+  return false;
+}
+
 int pick_kernel(const gqa_problem& p) {
   if (p.batch == 0 || p.seq_q == 0) return GQA_KERNEL_NONE;
   if (p.seq_k == 0) return GQA_KERNEL_ZERO;
+  if (nothing_visible(p)) return GQA_KERNEL_NAN;
   if (p.dtype == GQA_DTYPE_F32) return GQA_KERNEL_F32;
-  return p.seq_q == 1 ? GQA_KERNEL_DECODE : GQA_KERNEL_PREFILL;
+  // Decode streams K/V once per pass of at most 16 (head, query) rows: one
+  // pass covers every query position when g * seq_q <= 16 (single-token and
+  // short multi-token decode); larger query blocks go to the prefill tiles.
+  const int64_t g = p.heads_q / p.heads_kv;
+  if (p.seq_q == 1 || g * p.seq_q <= kDecodeMaxRowsPerPass) return GQA_KERNEL_DECODE;
+  return GQA_KERNEL_PREFILL;
 }
 
 int device_sm_count(int* out) {
@@ -97,6 +114,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
     case GQA_KERNEL_NONE:
       break;
     case GQA_KERNEL_ZERO:
+    case GQA_KERNEL_NAN:
       plan->grid = 592;
       plan->block = 256;
       plan->launches = 1;
@@ -122,7 +140,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
     case GQA_KERNEL_PREFILL: {
       const PrefillShape s = plan_prefill(p, sm_count);
       plan->grid = s.grid;
-      plan->block = 352;
+      plan->block = kPrefillThreads;
       plan->smem_bytes = s.smem_bytes;
       plan->launches = p.has_mask ? 2 : 1;
       plan->work_units = static_cast<int32_t>(s.work);
@@ -196,7 +214,7 @@ using namespace gqa;
 
 extern "C" {
 
-GQA_API int gqa_version(void) { return 10000; }
+GQA_API int gqa_version(void) { return 10100; }
 
 GQA_API const char* gqa_status_string(int status) {
   switch (status) {
@@ -204,11 +222,11 @@ GQA_API const char* gqa_status_string(int status) {
     case GQA_ERR_NULL: return "a required pointer is NULL";
     case GQA_ERR_SHAPE: return "inconsistent or invalid sizes (heads_q must be a multiple of heads_kv)";
     case GQA_ERR_LAYOUT: return "unsupported memory layout (innermost stride must be 1; bf16 bases and strides must be multiples of 16 bytes)";
-    case GQA_ERR_UNSUPPORTED: return "unsupported combination (bf16 needs head_dim 64 or 128; causal needs seq_q == seq_k)";
+    case GQA_ERR_UNSUPPORTED: return "unsupported combination (bf16 needs head_dim 64 or 128)";
     case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
     case GQA_ERR_CUDA: return "a CUDA runtime call failed";
     case GQA_ERR_TIMEOUT: return "a kernel gave up on an internal wait; outputs are undefined";
-    case GQA_ERR_ARG: return "invalid scalar argument (scale must be finite; dtype must be known)";
+    case GQA_ERR_ARG: return "invalid scalar argument (finite scale, known dtype, window >= 0 and only with causal)";
     case GQA_ERR_DEVICE: return "no usable sm_100 CUDA device";
     case GQA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the library's static array holds";
     default: return "unknown status";
@@ -242,7 +260,8 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   fill_plan(p, sms, &plan);
   if (plan.kernel == GQA_KERNEL_NONE) return GQA_OK;
   if (out == nullptr) return GQA_ERR_NULL;
-  if (plan.kernel == GQA_KERNEL_ZERO) return launch_zero(p, out, stream);
+  if (plan.kernel == GQA_KERNEL_ZERO) return launch_zero(p, out, stream, false);
+  if (plan.kernel == GQA_KERNEL_NAN) return launch_zero(p, out, stream, true);
   if (q == nullptr || k == nullptr || v == nullptr) return GQA_ERR_NULL;
   if (p.has_mask && mask == nullptr) return GQA_ERR_NULL;
   if (workspace == nullptr) return GQA_ERR_WORKSPACE;
@@ -288,6 +307,14 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     a.Hkv = static_cast<int>(p.heads_kv);
     a.Sk = static_cast<int>(p.seq_k);
     a.g = static_cast<int>(g);
+    a.Sq = static_cast<int>(p.seq_q);
+    a.rows = static_cast<int>(g * p.seq_q);
+    a.causal = p.causal;
+    a.causal_offset = p.causal_offset;
+    a.window = p.window;
+    a.t0 = s.t0;
+    a.key_lo = s.key_lo;
+    a.key_hi = s.key_hi;
     a.scale_log2 = scale_log2;
     // The ticket counters must start at zero; other calls sharing this
     // workspace (a prefill's tile classes, a larger problem's partials) may
@@ -321,6 +348,8 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.Sk = static_cast<int>(p.seq_k);
   a.g = static_cast<int>(g);
   a.causal = p.causal;
+  a.causal_offset = p.causal_offset;
+  a.window = p.window;
   a.has_mask = p.has_mask;
   a.scale_log2 = scale_log2;
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);

@@ -68,7 +68,10 @@ struct DecodeSmem {
   }
 };
 
-template <int D, int NT>
+// MQ: several query positions per kv head (seq_q > 1): the rows of a pass
+// are (head, query) pairs, row r = head * seq_q + query, each with its own
+// visible key range and mask row.
+template <int D, int NT, bool MQ>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a,
@@ -128,9 +131,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         mbar_arrive_expect_tx(&full[s], L::kStageBytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
-          tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, t * KT, kv, b);
-          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64, t * KT, kv,
-                      b);
+          tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, (t + a.t0) * KT, kv, b);
+          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64,
+                      (t + a.t0) * KT, kv, b);
         }
       }
       // Unwind: make sure no copy is still landing in this CTA's shared memory.
@@ -162,17 +165,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
     };
 
+    // Visible keys [vlo, vhi) and mask row of the two rows (columns) this
+    // thread's S^T fragments hold in each column tile.
+    int64_t vlo[NT][2], vhi[NT][2];
+    const uint8_t* vmask[NT][2];
+
     auto load_q = [&]() {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int hl = pass * HP + nt * 8 + (lane >> 2);  // head within the group
-        const bool ok = hl < a.g;
-        const uint16_t* qrow = a.q + b * a.qs[0] + (int64_t)(kv * a.g + (ok ? hl : 0)) * a.qs[1];
+        const int hl = pass * HP + nt * 8 + (lane >> 2);  // row within the group
+        const bool ok = hl < a.rows;
+        const int hh = MQ ? (ok ? hl / a.Sq : 0) : (ok ? hl : 0);
+        const int qi = MQ ? (ok ? hl % a.Sq : 0) : 0;
+        const uint16_t* qrow = a.q + b * a.qs[0] + (int64_t)(kv * a.g + hh) * a.qs[1] +
+                               (int64_t)qi * a.qs[2];
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
           const int d0 = ks * 16 + (lane & 3) * 2;
           bq[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
           bq[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (MQ) {
+            const int r = pass * HP + nt * 8 + (lane & 3) * 2 + e;
+            const int i = (r < a.rows ? r : 0) % a.Sq;
+            int64_t lo = 0, hi = a.Sk;
+            if (a.causal) {
+              hi = i + a.causal_offset + 1 < hi ? i + a.causal_offset + 1 : hi;
+              if (a.window > 0 && i + a.causal_offset - a.window + 1 > 0)
+                lo = i + a.causal_offset - a.window + 1;
+            }
+            vlo[nt][e] = lo;
+            vhi[nt][e] = hi;
+            vmask[nt][e] = a.mask ? a.mask + b * a.ms[0] + static_cast<int64_t>(i) * a.ms[1] : nullptr;
+          } else {
+            vlo[nt][e] = a.key_lo;
+            vhi[nt][e] = a.key_hi;
+            vmask[nt][e] = mrow;
+          }
         }
       }
     };
@@ -215,13 +246,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int64_t g_u0 = cur * tiles_per_group, g_u1 = g_u0 + tiles_per_group;
       const int64_t c_lo = cta_of_unit(g_u0, units, P);
       const int64_t c_hi = cta_of_unit(g_u1 - 1, units, P);
-      const int hq0 = kv * a.g + pass * HP;  // first query head of this pass
-      uint16_t* obase = a.out + b * a.os[0];
+      // Output row of row hr of this pass (a head, or a (head, query) pair).
+      auto out_row = [&](int hr) -> uint16_t* {
+        const int r = pass * HP + hr;
+        const int hh = MQ ? r / a.Sq : r;
+        const int qi = MQ ? r % a.Sq : 0;
+        return a.out + b * a.os[0] + static_cast<int64_t>(kv * a.g + hh) * a.os[1] +
+               static_cast<int64_t>(qi) * a.os[2];
+      };
       if (c_lo == c_hi) {
         // The whole group is in this CTA: normalise and write out.
         for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
           const int h = idx / D, d = idx % D;
-          if (pass * HP + h >= a.g) continue;
+          if (pass * HP + h >= a.rows) continue;
           float M = -INFINITY;
 #pragma unroll
           for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
@@ -234,7 +271,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               acc += sc * scr_o[(w * HP + h) * L::kScrRow + d];
             }
           }
-          obase[(hq0 + h) * a.os[1] + d] = bf16_bits_rn(acc / l);  // l == 0: NaN
+          out_row(h)[d] = bf16_bits_rn(acc / l);  // l == 0: NaN
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
         return;
@@ -288,7 +325,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
           for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
             const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
-            if (pass * HP + h >= a.g) continue;
+            if (pass * HP + h >= a.rows) continue;
             float2 ml[kFastMerge];
             float4 o[kFastMerge];
 #pragma unroll
@@ -321,7 +358,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             uint2 pk;
             pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
             pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-            *reinterpret_cast<uint2*>(obase + (hq0 + h) * a.os[1] + d) = pk;
+            *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
           }
         } else {
         // Many contributors: stage each one's segment index and each head's
@@ -352,7 +389,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
         for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
           const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
-          if (pass * HP + h >= a.g) continue;
+          if (pass * HP + h >= a.rows) continue;
           const float M = sm_ml[2 * h], Lsum = sm_ml[2 * h + 1];
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
           if (M != -INFINITY) {
@@ -371,7 +408,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           uint2 pk;
           pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
           pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2*>(obase + (hq0 + h) * a.os[1] + d) = pk;
+          *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
         }
         }
         if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
@@ -429,20 +466,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
 
-      // Visibility of this thread's two keys.
-      const int64_t key0 = static_cast<int64_t>(t) * KT + warp * 16 + (lane >> 2);
+      // Visibility of this thread's two keys for its rows.
+      const int64_t key0 = static_cast<int64_t>(t + a.t0) * KT + warp * 16 + (lane >> 2);
       const int64_t key1 = key0 + 8;
-      const bool vis0 = key0 < a.Sk && key_visible(mrow, key0, 0, 0);
-      const bool vis1 = key1 < a.Sk && key_visible(mrow, key1, 0, 0);
+      auto vis = [&](int64_t key, int nt, int e) -> bool {
+        return key >= vlo[nt][e] && key < vhi[nt][e] && mask_allows(vmask[nt][e], key);
+      };
 
       uint32_t pt0[NT], pt1[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float tv[4];
-        tv[0] = vis0 ? sc[nt][0] * a.scale_log2 : -INFINITY;
-        tv[1] = vis0 ? sc[nt][1] * a.scale_log2 : -INFINITY;
-        tv[2] = vis1 ? sc[nt][2] * a.scale_log2 : -INFINITY;
-        tv[3] = vis1 ? sc[nt][3] * a.scale_log2 : -INFINITY;
+        tv[0] = vis(key0, nt, 0) ? sc[nt][0] * a.scale_log2 : -INFINITY;
+        tv[1] = vis(key0, nt, 1) ? sc[nt][1] * a.scale_log2 : -INFINITY;
+        tv[2] = vis(key1, nt, 0) ? sc[nt][2] * a.scale_log2 : -INFINITY;
+        tv[3] = vis(key1, nt, 1) ? sc[nt][3] * a.scale_log2 : -INFINITY;
         float alpha[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -499,10 +537,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
 }
 
-template <int D, int NT>
+template <int D, int NT, bool MQ>
 int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap& tmk,
                     const CUtensorMap& tmv, cudaStream_t stream) {
-  auto kern = gqa_decode_kernel<D, NT>;
+  auto kern = gqa_decode_kernel<D, NT, MQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_bytes) !=
       cudaSuccess)
     return GQA_ERR_CUDA;
@@ -517,11 +555,22 @@ int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap
 DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
   DecodeShape s{};
   const int64_t g = p.heads_q / p.heads_kv;
+  const int64_t rows = g * p.seq_q;  // (head, query) rows per kv head
   s.D = static_cast<int>(p.head_dim);
-  s.NT = g <= 8 ? 1 : 2;
+  s.NT = rows <= 8 ? 1 : 2;
   s.HP = 8 * s.NT;
-  s.passes = static_cast<int>((g + s.HP - 1) / s.HP);
-  s.tiles_per_group = static_cast<int>((p.seq_k + KT - 1) / KT);
+  s.passes = static_cast<int>((rows + s.HP - 1) / s.HP);
+  // Keys some query can see: [key_lo, key_hi) (query 0's lower limit, the
+  // last query's upper limit).
+  s.key_hi = p.seq_k;
+  s.key_lo = 0;
+  if (p.causal) {
+    if (p.seq_q - 1 + p.causal_offset + 1 < s.key_hi) s.key_hi = p.seq_q + p.causal_offset;
+    if (p.window > 0 && p.causal_offset - p.window + 1 > 0) s.key_lo = p.causal_offset - p.window + 1;
+  }
+  s.t0 = static_cast<int>(s.key_lo / KT);
+  s.tiles_per_group = static_cast<int>((s.key_hi + KT - 1) / KT) - s.t0;
+  if (s.tiles_per_group < 1) s.tiles_per_group = 1;
   s.groups = p.batch * p.heads_kv * s.passes;
   s.units = s.groups * s.tiles_per_group;
   s.grid = static_cast<int>(s.units < sm_count ? s.units : sm_count);
@@ -553,10 +602,19 @@ DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
 int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
                   const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
   (void)p;
-  if (s.D == 128 && s.NT == 1) return launch_decode_t<128, 1>(s, a, tmk, tmv, stream);
-  if (s.D == 128 && s.NT == 2) return launch_decode_t<128, 2>(s, a, tmk, tmv, stream);
-  if (s.D == 64 && s.NT == 1) return launch_decode_t<64, 1>(s, a, tmk, tmv, stream);
-  if (s.D == 64 && s.NT == 2) return launch_decode_t<64, 2>(s, a, tmk, tmv, stream);
+  const bool mq = a.Sq > 1;
+  if (s.D == 128 && s.NT == 1)
+    return mq ? launch_decode_t<128, 1, true>(s, a, tmk, tmv, stream)
+              : launch_decode_t<128, 1, false>(s, a, tmk, tmv, stream);
+  if (s.D == 128 && s.NT == 2)
+    return mq ? launch_decode_t<128, 2, true>(s, a, tmk, tmv, stream)
+              : launch_decode_t<128, 2, false>(s, a, tmk, tmv, stream);
+  if (s.D == 64 && s.NT == 1)
+    return mq ? launch_decode_t<64, 1, true>(s, a, tmk, tmv, stream)
+              : launch_decode_t<64, 1, false>(s, a, tmk, tmv, stream);
+  if (s.D == 64 && s.NT == 2)
+    return mq ? launch_decode_t<64, 2, true>(s, a, tmk, tmv, stream)
+              : launch_decode_t<64, 2, false>(s, a, tmk, tmv, stream);
   return GQA_ERR_UNSUPPORTED;
 }
 

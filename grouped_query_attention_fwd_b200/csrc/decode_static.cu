@@ -113,6 +113,14 @@ extern "C" GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const vo
   a.Hkv = static_cast<int>(p->heads_kv);
   a.Sk = static_cast<int>(p->seq_k);
   a.g = static_cast<int>(p->heads_q / p->heads_kv);
+  a.Sq = static_cast<int>(p->seq_q);
+  a.rows = static_cast<int>(a.g * p->seq_q);
+  a.causal = p->causal;
+  a.causal_offset = p->causal_offset;
+  a.window = p->window;
+  a.t0 = s.t0;
+  a.key_lo = s.key_lo;
+  a.key_hi = s.key_hi;
   a.scale_log2 = static_cast<float>(static_cast<double>(p->scale) * 1.4426950408889634073599);
   return launch_decode(*p, s, a, tmk, tmv, stream);
 }

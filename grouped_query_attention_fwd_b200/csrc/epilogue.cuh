@@ -18,12 +18,10 @@ namespace gqa {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Key j visible from query i under the optional bool mask and causal flag.
-__device__ __forceinline__ bool key_visible(const uint8_t* mask_row, int64_t j, int64_t i,
-                                            int causal) {
-  if (mask_row != nullptr && mask_row[j] == 0) return false;
-  if (causal && j > i) return false;
-  return true;
+// Key j visible from query i under the optional bool mask (causal and window
+// limits are applied by each kernel as a key range).
+__device__ __forceinline__ bool mask_allows(const uint8_t* mask_row, int64_t j) {
+  return mask_row == nullptr || mask_row[j] != 0;
 }
 
 // Exponent reference for a running maximum that may still be -inf.

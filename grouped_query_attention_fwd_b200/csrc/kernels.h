@@ -14,13 +14,16 @@ namespace gqa {
 constexpr int kDecodeKeysPerTile = 64;
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+constexpr int kDecodeMaxRowsPerPass = 16;  // (head, query) rows in the MMA N dimension
 
 struct DecodeShape {
   int D;            // 64 or 128
   int NT;           // 8-head MMA column tiles per pass (1 or 2)
-  int HP;           // heads per pass = 8 * NT
-  int passes;       // ceil(g / HP)
+  int HP;           // rows per pass = 8 * NT (a row: one head, or one (head, query))
+  int passes;       // ceil(g * seq_q / HP)
   int tiles_per_group;
+  int t0;           // first 64-key tile any query can see (window)
+  int64_t key_lo, key_hi;  // keys [key_lo, key_hi) pass the causal / window rules
   int64_t groups;   // batch * heads_kv * passes
   int64_t units;    // groups * tiles_per_group
   int grid;         // CTAs (<= units)
@@ -44,6 +47,11 @@ struct DecodeArgs {
   uint32_t* counters;  // one ticket counter per group; zeroed before each launch
   uint32_t* err;
   int B, Hq, Hkv, Sk, g;
+  int Sq, rows;            // queries per kv head; rows = g * Sq
+  int causal;
+  int64_t causal_offset, window;
+  int t0;                  // tile offset of the streamed key range
+  int64_t key_lo, key_hi;  // keys outside [key_lo, key_hi) are hidden (causal / window)
   float scale_log2;  // scale * log2(e)
 };
 
@@ -55,6 +63,8 @@ int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& 
                          const int64_t st[4]);
 
 // ------------------------------------------------------------ prefill
+constexpr int kPrefillThreads = 12 * 32;  // two softmax warpgroups, load, MMA and V-load warps
+
 struct PrefillShape {
   int D;             // 64 or 128
   int qpt;           // query positions per 128-row tile (rows = qpt * g)
@@ -78,6 +88,7 @@ struct PrefillArgs {
   uint32_t* err;
   int B, Hq, Hkv, Sq, Sk, g;
   int causal, has_mask;
+  int64_t causal_offset, window;
   float scale_log2;
 };
 
@@ -89,7 +100,7 @@ int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArg
 int launch_f32(const gqa_problem& p, const float* q, const float* k, const float* v,
                const uint8_t* mask, float* out, cudaStream_t stream);
 
-// ------------------------------------------------------------ zero fill (seq_k == 0)
-int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream);
+// ------------------------------------------------------------ fill: zeros (seq_k == 0) or NaN
+int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream, bool nan);
 
 }  // namespace gqa

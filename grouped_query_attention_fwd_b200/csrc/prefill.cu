@@ -55,7 +55,7 @@ constexpr int BN = 128;  // keys per K/V tile
 constexpr int kWarpQK = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpV = 10;  // warp 11 idles (it completes the third warpgroup)
-constexpr int kPrefillThreads = 12 * 32;
+
 // Register split across the three warpgroups (setmaxnreg): the launch gives
 // every thread kLaunchRegs; the producer / MMA warpgroup drops to kIoRegs and
 // the two softmax warpgroups rise to kSoftmaxRegs, which must add up to the
@@ -95,13 +95,17 @@ struct Layout {
   static constexpr uint32_t kOCol0 = 256;
 };
 
+__device__ __forceinline__ int64_t imin64(int64_t x, int64_t y) { return x < y ? x : y; }
+__device__ __forceinline__ int64_t imax64(int64_t x, int64_t y) { return x > y ? x : y; }
+
 struct Pair {
-  int b, kv, mt0, nt_end;
+  int b, kv, mt0, nt_beg, nt_end;
 };
 
 struct Slot {  // one query tile of a pair
   int mt, q0, q_last;
   bool live;
+  int64_t key_lo, key_hi;  // keys some row of the tile can see (causal / window)
 };
 
 // Work item x: a pair of consecutive query tiles (2p, 2p+1) of one
@@ -113,7 +117,22 @@ __device__ __forceinline__ Slot slot_of(const Pair& pr, int s, const PrefillArgs
   sl.live = sl.mt < m_tiles;
   sl.q0 = sl.mt * qpt;
   sl.q_last = sl.live ? min(sl.q0 + qpt, a.Sq) - 1 : -1;
+  sl.key_lo = 0;
+  sl.key_hi = a.Sk;
+  if (a.causal) {
+    sl.key_hi = imin64(a.Sk, static_cast<int64_t>(sl.q_last) + a.causal_offset + 1);
+    if (a.window > 0)
+      sl.key_lo = imax64(0, static_cast<int64_t>(sl.q0) + a.causal_offset - a.window + 1);
+  }
+  if (!sl.live || sl.key_hi <= sl.key_lo) sl.key_lo = sl.key_hi = 0;
   return sl;
+}
+
+// Position in the heavy-first list of the r-th pair taken by CTA c: rounds
+// alternate direction (c, then P-1-c, ...) so that every CTA's total causal
+// work comes out nearly equal.
+__device__ __forceinline__ int64_t snake(int64_t r, int64_t c, int64_t P) {
+  return r * P + ((r & 1) ? (P - 1 - c) : c);
 }
 
 __device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_tiles, int qpt,
@@ -126,9 +145,17 @@ __device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_t
   pr.b = bk / a.Hkv;
   pr.kv = bk % a.Hkv;
   pr.mt0 = 2 * p;
-  const int q_hi = max(slot_of(pr, 0, a, m_tiles, qpt).q_last,
-                       slot_of(pr, 1, a, m_tiles, qpt).q_last);
-  pr.nt_end = a.causal ? min(n_tiles, q_hi / BN + 1) : n_tiles;
+  const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
+  // Key tiles either slot can see.
+  int64_t lo = a.Sk, hi = 0;
+  if (s0.key_hi > s0.key_lo) { lo = imin64(lo, s0.key_lo); hi = imax64(hi, s0.key_hi); }
+  if (s1.key_hi > s1.key_lo) { lo = imin64(lo, s1.key_lo); hi = imax64(hi, s1.key_hi); }
+  if (hi <= lo) {
+    pr.nt_beg = pr.nt_end = 0;
+  } else {
+    pr.nt_beg = static_cast<int>(lo / BN);
+    pr.nt_end = min(n_tiles, static_cast<int>((hi + BN - 1) / BN));
+  }
   return pr;
 }
 
@@ -137,12 +164,16 @@ __device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_t
 __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, const Slot& sl,
                                           int nt, int m_tiles, int n_tiles) {
   if (!sl.live) return 0;
+  const int64_t j0 = static_cast<int64_t>(nt) * BN, j1 = j0 + BN - 1;
+  if (j1 < sl.key_lo || j0 >= sl.key_hi) return 0;
   int cls = 2;
-  const int j0 = nt * BN, j1 = j0 + BN - 1;
   if (j1 >= a.Sk) cls = 1;
   if (a.causal) {
-    if (j0 > sl.q_last) return 0;
-    if (j1 > sl.q0) cls = 1;
+    // Every row sees the whole tile iff the first row's upper limit and the
+    // last row's lower limit (window) both enclose it.
+    if (j1 > static_cast<int64_t>(sl.q0) + a.causal_offset) cls = 1;
+    if (a.window > 0 && j0 <= static_cast<int64_t>(sl.q_last) + a.causal_offset - a.window)
+      cls = 1;
   }
   if (a.has_mask) {
     const int c = a.summary[(static_cast<int64_t>(pr.b) * m_tiles + sl.mt) * n_tiles + nt];
@@ -153,17 +184,25 @@ __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, 
 }
 
 // Visibility of keys j0 .. j0+127 for query q, one bit per key: inside the
-// sequence (j < Sk), not in the future (causal: j <= q), and allowed by the
-// mask row (nonzero byte), which is read as 16-byte vectors when aligned.
+// sequence (j < Sk), within the causal limit (j <= q + causal_offset) and the
+// window (j > q + causal_offset - window), and allowed by the mask row
+// (nonzero byte), which is read as 16-byte vectors when aligned.
 __device__ __forceinline__ void visible_bits(uint32_t (&vb)[4], const uint8_t* mrow, int j0,
-                                             int Sk, int causal, int q, bool vec) {
-  int n = Sk - j0;  // keys inside the sequence
-  if (causal && q - j0 + 1 < n) n = q - j0 + 1;
-  n = n < 0 ? 0 : (n > BN ? BN : n);
+                                             const PrefillArgs& a, int q, bool vec) {
+  int64_t hi = a.Sk, lo = 0;  // keys [lo, hi) pass causal and window
+  if (a.causal) {
+    hi = imin64(hi, static_cast<int64_t>(q) + a.causal_offset + 1);
+    if (a.window > 0) lo = static_cast<int64_t>(q) + a.causal_offset - a.window + 1;
+  }
+  const int n = static_cast<int>(imax64(0, imin64(BN, hi - j0)));
+  const int n0 = static_cast<int>(imax64(0, imin64(n, lo - j0)));
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     const int k = n - 32 * w;
-    vb[w] = k >= 32 ? ~0u : (k <= 0 ? 0u : ((1u << k) - 1u));
+    const int k0 = n0 - 32 * w;
+    const uint32_t below_hi = k >= 32 ? ~0u : (k <= 0 ? 0u : ((1u << k) - 1u));
+    const uint32_t below_lo = k0 >= 32 ? ~0u : (k0 <= 0 ? 0u : ((1u << k0) - 1u));
+    vb[w] = below_hi & ~below_lo;
   }
   if (mrow == nullptr) return;
   const uint8_t* m = mrow + j0;
@@ -289,7 +328,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // kept in registers: -1 = none.
       int32_t last_round0 = -1, last_round1 = -1, last_q0 = -1, last_q1 = -1;
       bool ok = true;
-      for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
+      for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
+         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
         const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
         const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
         if (is_qk) {
@@ -310,7 +350,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           if (!ok) break;
         }
-        for (int nt = 0; nt < pr.nt_end; ++nt) {
+        for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
           if (tile_class(a, pr, s0, nt, m_tiles, n_tiles) == 0 &&
               tile_class(a, pr, s1, nt, m_tiles, n_tiles) == 0)
             continue;
@@ -375,7 +415,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return true;
       };
 
-      for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
+      for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
+         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
         const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
         const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
 #pragma unroll
@@ -387,7 +428,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         bool pend[kSlots] = {false, false};
         uint32_t pJ[kSlots] = {0, 0}, pk[kSlots] = {0, 0};
         int nloc[kSlots] = {0, 0};
-        for (int nt = 0; nt < pr.nt_end && ok; ++nt) {
+        // Each slot's last active key tile: its Q buffer is released as soon
+        // as that QK completes, so the producer can fetch the next pair's Q
+        // while this pair's last products and softmax still run.
+        int last0 = -1, last1 = -1;
+        for (int nt = pr.nt_end - 1; nt >= pr.nt_beg && (last0 < 0 || last1 < 0); --nt) {
+          if (last0 < 0 && tile_class(a, pr, s0, nt, m_tiles, n_tiles) != 0) last0 = nt;
+          if (last1 < 0 && tile_class(a, pr, s1, nt, m_tiles, n_tiles) != 0) last1 = nt;
+        }
+        for (int nt = pr.nt_beg; nt < pr.nt_end && ok; ++nt) {
           const int cls0 = tile_class(a, pr, s0, nt, m_tiles, n_tiles);
           const int cls1 = tile_class(a, pr, s1, nt, m_tiles, n_tiles);
           if (cls0 == 0 && cls1 == 0) continue;
@@ -423,6 +472,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         ks > 0 ? 1u : 0u);
             }
             tc_commit(&s_full[sl]);
+            if (nt == (sl == 0 ? last0 : last1)) tc_commit(&q_empty[sl]);
             pend[sl] = true;
             pJ[sl] = J[sl];
             pk[sl] = kt;
@@ -441,7 +491,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int sl = 0; sl < kSlots; ++sl) {
           if (!ok) break;
-          tc_commit(&q_empty[sl]);
+          if (nloc[sl] == 0) tc_commit(&q_empty[sl]);  // no QK used this slot's Q
           if (nloc[sl] == 0 && it > 0 &&
               !mbar_wait(&o_free[sl], static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
                          kErrPrefillWait)) {
@@ -473,7 +523,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t J = 0;
     int64_t it = 0;
     bool ok = true;
-    for (int64_t x = blockIdx.x; x < work && ok; x += gridDim.x, ++it) {
+    for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
+         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
       const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
       const Slot me = slot_of(pr, sl, a, m_tiles, qpt);
       const int q = me.q0 + qi;
@@ -483,7 +534,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                     : nullptr;
       float m_ref = -INFINITY, l = 0.f;
       int nloc = 0;
-      for (int nt = 0; nt < pr.nt_end; ++nt) {
+      for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
         const int cls = tile_class(a, pr, me, nt, m_tiles, n_tiles);
         if (cls == 0) continue;
         if (!mbar_wait(&s_full[sl], J & 1u, abort_flag, a.err, kErrPrefillWait)) {
@@ -497,7 +548,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const bool fast = (cls == 2) && (a.scale_log2 >= 0.f);
         uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};
         if (!fast)
-          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a.Sk, a.causal, q, mask_vec);
+          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a, q, mask_vec);
         auto masked_t = [&](float sv, int c) -> float {
           return ((vb[c >> 5] >> (c & 31)) & 1u) ? sv * a.scale_log2 : -INFINITY;
         };

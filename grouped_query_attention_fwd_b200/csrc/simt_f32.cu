@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(256)
                    int64_t Sk, int64_t D, int64_t qs0, int64_t qs1, int64_t qs2, int64_t ks0,
                    int64_t ks1, int64_t ks2, int64_t vs0, int64_t vs1, int64_t vs2, int64_t os0,
                    int64_t os1, int64_t os2, int64_t ms0, int64_t ms1, int causal,
-                   float scale_log2) {
+                   int64_t causal_offset, int64_t window, float scale_log2) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= B * Hq * Sq) return;
@@ -45,9 +45,14 @@ __global__ void __launch_bounds__(256)
     acc[e] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int64_t jend = causal ? (i + 1 < Sk ? i + 1 : Sk) : Sk;
-  for (int64_t j = 0; j < jend; ++j) {
-    if (!key_visible(mrow, j, i, causal)) continue;
+  // Keys [jbeg, jend) pass the causal and window rules; the mask is per key.
+  int64_t jend = Sk, jbeg = 0;
+  if (causal) {
+    jend = i + causal_offset + 1 < Sk ? i + causal_offset + 1 : Sk;
+    if (window > 0 && i + causal_offset - window + 1 > 0) jbeg = i + causal_offset - window + 1;
+  }
+  for (int64_t j = jbeg; j < jend; ++j) {
+    if (mrow != nullptr && mrow[j] == 0) continue;
     const float* kr = kb + j * ks2;
     float dot = 0.f;
 #pragma unroll
@@ -78,14 +83,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-__global__ void gqa_zero_kernel(uint8_t* out, int64_t B, int64_t Hq, int64_t Sq, int64_t D,
-                                int64_t os0, int64_t os1, int64_t os2, int elem_bytes) {
+// Fills out with zeros (no keys at all: an empty weighted sum) or with NaN
+// (keys exist but causal / window leave none to any query: the softmax of an
+// all -inf row).
+__global__ void gqa_fill_kernel(uint8_t* out, int64_t B, int64_t Hq, int64_t Sq, int64_t D,
+                                int64_t os0, int64_t os1, int64_t os2, int elem_bytes, int nan) {
   const int64_t n = B * Hq * Sq * D;
   for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; x < n;
        x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t d = x % D, i = (x / D) % Sq, h = (x / (D * Sq)) % Hq, b = x / (D * Sq * Hq);
     uint8_t* dst = out + (b * os0 + h * os1 + i * os2 + d) * elem_bytes;
-    for (int e = 0; e < elem_bytes; ++e) dst[e] = 0;
+    if (elem_bytes == 4)
+      *reinterpret_cast<uint32_t*>(dst) = nan ? 0x7FC00000u : 0u;
+    else
+      *reinterpret_cast<uint16_t*>(dst) = nan ? static_cast<uint16_t>(0x7FC0u) : static_cast<uint16_t>(0u);
   }
 }
 
@@ -102,15 +113,16 @@ int launch_f32(const gqa_problem& p, const float* q, const float* k, const float
       q, k, v, p.has_mask ? mask : nullptr, out, p.batch, p.heads_q, p.heads_kv, p.seq_q,
       p.seq_k, p.head_dim, p.q_stride[0], p.q_stride[1], p.q_stride[2], p.k_stride[0],
       p.k_stride[1], p.k_stride[2], p.v_stride[0], p.v_stride[1], p.v_stride[2], p.o_stride[0],
-      p.o_stride[1], p.o_stride[2], p.mask_stride[0], p.mask_stride[1], p.causal, scale_log2);
+      p.o_stride[1], p.o_stride[2], p.mask_stride[0], p.mask_stride[1], p.causal,
+      p.causal_offset, p.window, scale_log2);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
-int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream) {
+int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream, bool nan) {
   const int elem = p.dtype == GQA_DTYPE_F32 ? 4 : 2;
-  gqa_zero_kernel<<<592, 256, 0, stream>>>(static_cast<uint8_t*>(out), p.batch, p.heads_q,
+  gqa_fill_kernel<<<592, 256, 0, stream>>>(static_cast<uint8_t*>(out), p.batch, p.heads_q,
                                            p.seq_q, p.head_dim, p.o_stride[0], p.o_stride[1],
-                                           p.o_stride[2], elem);
+                                           p.o_stride[2], elem, nan ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

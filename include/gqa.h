@@ -26,8 +26,14 @@
  *    [B, H, S, D]), subject to the 16-byte rules below on the bf16 paths.
  *  - dtype: GQA_DTYPE_BF16 (compute in fp32, bf16 in/out, head_dim 64 or 128)
  *    or GQA_DTYPE_F32 (fp32 throughout, head_dim 1..256).
- *  - causal is top-left aligned (key j visible to query i iff j <= i) and
- *    requires seq_q == seq_k.  With has_mask as well, a key must pass both.
+ *  - causal: key j is visible to query i iff j <= i + causal_offset.  The
+ *    pages' causal attention (seq_q == seq_k) is causal_offset = 0 (top-left);
+ *    decoding after a KV cache, bottom-right alignment, is causal_offset =
+ *    seq_k - seq_q.  window > 0 (causal only) also hides keys
+ *    j <= i + causal_offset - window: a sliding window of `window` keys ending
+ *    at the diagonal (the sliding-window attention that "28. Grouped-Query
+ *    Attention (GQA)", "Problem", names for Mistral).  With has_mask as well,
+ *    a key must pass every rule.
  *  - A row whose keys are all hidden yields NaN (the softmax of an all -inf
  *    row).  seq_k == 0 yields zeros (an empty weighted sum).  batch == 0 or
  *    seq_q == 0 is a no-op.
@@ -66,11 +72,11 @@ extern "C" {
 #define GQA_ERR_LAYOUT 3      /* innermost stride != 1, or a base/stride the TMA unit cannot
                                  address (bf16 paths: base and non-innermost strides must be
                                  multiples of 16 bytes) */
-#define GQA_ERR_UNSUPPORTED 4 /* dtype / head_dim combination, or causal with seq_q != seq_k */
+#define GQA_ERR_UNSUPPORTED 4 /* dtype / head_dim combination the kernels do not cover */
 #define GQA_ERR_WORKSPACE 5   /* workspace NULL, too small, or not 256-byte aligned */
 #define GQA_ERR_CUDA 6        /* a CUDA runtime call failed (launch, attribute, encode) */
 #define GQA_ERR_TIMEOUT 7     /* a kernel's bounded internal wait ran out (gqa_device_status) */
-#define GQA_ERR_ARG 8         /* scale not finite, or an unknown dtype */
+#define GQA_ERR_ARG 8         /* scale not finite, unknown dtype, or a window without causal */
 #define GQA_ERR_DEVICE 9      /* no usable CUDA device, or not an sm_100 device */
 #define GQA_ERR_SCRATCH_LIMIT 10 /* gqa_forward_decode_noalloc: the problem needs more scratch
                                     than GQA_STATIC_SCRATCH_BYTES */
@@ -79,10 +85,12 @@ extern "C" {
 #define GQA_DTYPE_F32 1
 
 #define GQA_KERNEL_NONE 0     /* nothing to launch (empty problem) */
-#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1: split-K stream over the KV cache, one launch */
-#define GQA_KERNEL_PREFILL 2  /* bf16, seq_q >= 2: tcgen05 / tensor-memory tiles */
+#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1 or (heads_q/heads_kv) * seq_q <= 16: split-K
+                                 stream over the KV cache, one launch */
+#define GQA_KERNEL_PREFILL 2  /* bf16, longer query blocks: tcgen05 / tensor-memory tiles */
 #define GQA_KERNEL_F32 3      /* fp32 CUDA-core path */
 #define GQA_KERNEL_ZERO 4     /* seq_k == 0: the output is filled with zeros */
+#define GQA_KERNEL_NAN 5      /* causal / window leave no key to any query: NaN (see above) */
 
 /* One attention problem.  Strides are in elements. */
 typedef struct gqa_problem {
@@ -96,6 +104,8 @@ typedef struct gqa_problem {
   int64_t v_stride[4];    /* over (b, h_kv, j, d) */
   int64_t o_stride[4];    /* over (b, h, i, d) */
   int64_t mask_stride[3]; /* over (b, i, j); the j stride must be 1 */
+  int64_t causal_offset;  /* with causal: key j visible to query i iff j <= i + causal_offset */
+  int64_t window;         /* with causal, > 0: keys j <= i + causal_offset - window hidden too */
 } gqa_problem;
 
 /* What gqa_forward will do for a problem on a device. */

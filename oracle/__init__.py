@@ -47,6 +47,12 @@ def _bind(lib):
     lib.oracle_gqa_forward_rows.restype = cint
     lib.oracle_kv_cache_bytes.argtypes = [i64] * 6
     lib.oracle_kv_cache_bytes.restype = i64
+    lib.oracle_gqa_forward_ex.argtypes = ([vp, vp, vp, vp, vp] + [i64] * 6 +
+                                          [cint, i64, i64, dbl, vp])
+    lib.oracle_gqa_forward_ex.restype = cint
+    lib.oracle_gqa_forward_rows_ex.argtypes = ([vp, vp, vp, vp, vp] + [i64] * 6 +
+                                               [cint, i64, i64, dbl, vp, i64, vp])
+    lib.oracle_gqa_forward_rows_ex.restype = cint
     return lib
 
 
@@ -93,8 +99,18 @@ def _mask_arg(mask):
     return m, m.ctypes.data
 
 
-def forward(q, k, v, mask=None, causal=False, scale=None, lib=None) -> np.ndarray:
-    """out [B, Hq, Sq, D] in float64.  ``scale`` defaults to 1/sqrt(D)."""
+def forward(q, k, v, mask=None, causal=False, scale=None, lib=None, causal_offset=None,
+            window=0, kv_lens=None) -> np.ndarray:
+    """out [B, Hq, Sq, D] in float64.  ``scale`` defaults to 1/sqrt(D).
+
+    ``causal_offset`` (with ``causal``): key j is visible to query i iff
+    j <= i + causal_offset; None keeps the pages' form (offset 0, Sq == Sk).
+    ``window`` > 0 (with ``causal``) also hides keys j <= i + offset - window.
+    ``kv_lens`` (int per batch entry): keys j >= kv_lens[b] are hidden and the
+    causal offset moves by kv_lens[b] - Sk."""
+    if causal_offset is not None or window or kv_lens is not None:
+        return _forward_ex(q, k, v, mask, causal, 0 if causal_offset is None else causal_offset,
+                           window, scale, lib, kv_lens)
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Sk, D = _shapes(q, k, v, mask)
     if scale is None:
@@ -125,8 +141,51 @@ def probs(q, k, mask=None, causal=False, scale=None, lib=None) -> np.ndarray:
     return out
 
 
-def forward_rows(q, k, v, rows, mask=None, causal=False, scale=None, lib=None) -> np.ndarray:
+def _lens_arg(kv_lens, B):
+    if kv_lens is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(kv_lens, dtype=np.int32).reshape(-1))
+    if a.shape[0] != B:
+        raise OracleError("kv_lens must have one entry per batch entry")
+    return a, a.ctypes.data
+
+
+def _forward_ex(q, k, v, mask, causal, causal_offset, window, scale, lib, kv_lens=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Sk, D = _shapes(q, k, v, mask)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    m, mp = _mask_arg(mask)
+    la, lp = _lens_arg(kv_lens, B)
+    out = np.empty((B, Hq, Sq, D), dtype=np.float64)
+    rc = (lib or _load()).oracle_gqa_forward_ex(q.ctypes.data, k.ctypes.data, v.ctypes.data, mp,
+                                                lp, B, Hq, Hkv, Sq, Sk, D, int(bool(causal)),
+                                                int(causal_offset), int(window), float(scale),
+                                                out.ctypes.data)
+    if rc != 0:
+        raise OracleError("invalid problem for the oracle")
+    return out
+
+
+def forward_rows(q, k, v, rows, mask=None, causal=False, scale=None, lib=None,
+                 causal_offset=None, window=0, kv_lens=None) -> np.ndarray:
     """Only the rows ``rows`` = [(b, h, i), ...]; returns [n, D] float64."""
+    if causal_offset is not None or window or kv_lens is not None:
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Hq, Hkv, Sq, Sk, D = _shapes(q, k, v, mask)
+        if scale is None:
+            scale = 1.0 / np.sqrt(D)
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        m, mp = _mask_arg(mask)
+        la, lp = _lens_arg(kv_lens, B)
+        out = np.empty((r.shape[0], D), dtype=np.float64)
+        rc = (lib or _load()).oracle_gqa_forward_rows_ex(
+            q.ctypes.data, k.ctypes.data, v.ctypes.data, mp, lp, B, Hq, Hkv, Sq, Sk, D,
+            int(bool(causal)), int(0 if causal_offset is None else causal_offset), int(window),
+            float(scale), r.ctypes.data, r.shape[0], out.ctypes.data)
+        if rc != 0:
+            raise OracleError("invalid problem or row index for the oracle")
+        return out
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Sk, D = _shapes(q, k, v, mask)
     if scale is None:

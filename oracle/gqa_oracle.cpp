@@ -38,7 +38,17 @@
 //  * mask and causal together: a key is visible only if both allow it;
 //  * a row in which every key is hidden has max = -inf, so its weights and its
 //    output are NaN, as in the reference solution's softmax of an all -inf row;
-//  * causal is top-left aligned (j <= i) and is only defined here for Sq == Sk.
+//  * causal is top-left aligned (j <= i) and, in the plain entry points, only
+//    defined for Sq == Sk.  The "_ex" entry points take an explicit offset:
+//    key j is visible to query i iff j <= i + causal_offset (bottom-right
+//    alignment is causal_offset = Sk - Sq), and an optional sliding window of
+//    `window` keys ending at that diagonal (Mistral's sliding-window attention,
+//    named on "28. Grouped-Query Attention (GQA)", "Problem"): key j is also
+//    hidden when j <= i + causal_offset - window.
+//  * a ragged KV cache (the "_ex" entry points' kv_lens, one length per batch
+//    entry, NULL = all seq_k): keys j >= kv_lens[b] are hidden, and the causal
+//    diagonal of batch entry b moves with its length: causal_offset is given
+//    for a full cache and becomes causal_offset + kv_lens[b] - seq_k.
 //
 // Layout: every array is contiguous, Q and out [B, Hq, Sq, D], K and V
 // [B, Hkv, Sk, D], probs [B, Hq, Sq, Sk], mask [B, Sq, Sk] (uint8, nonzero =
@@ -59,12 +69,17 @@ struct Problem {
   int64_t B, Hq, Hkv, Sq, Sk, D;
   int causal;
   double scale;
+  int64_t causal_offset;  // key j visible to query i iff j <= i + causal_offset
+  int64_t window;         // > 0: also hidden iff j <= i + causal_offset - window
+  bool explicit_offset;   // false: the pages' causal, Sq == Sk required
+  const int32_t* kv_lens = nullptr;  // per batch entry: keys j >= kv_lens[b] hidden
 };
 
 bool valid(const Problem& p) {
   if (p.B < 0 || p.Hq <= 0 || p.Hkv <= 0 || p.Sq < 0 || p.Sk < 0 || p.D <= 0) return false;
   if (p.Hq % p.Hkv != 0) return false;
-  if (p.causal && p.Sq != p.Sk) return false;
+  if (p.causal && !p.explicit_offset && p.Sq != p.Sk) return false;
+  if (p.window < 0 || (p.window > 0 && !p.causal)) return false;
   return true;
 }
 
@@ -75,6 +90,8 @@ void row_weights(const Problem& p, int64_t b, int64_t h, int64_t i, double* w) {
   const double* qrow = p.q + ((b * p.Hq + h) * p.Sq + i) * p.D;
   const double* kbase = p.k + ((b * p.Hkv + kv) * p.Sk) * p.D;
   const double neg_inf = -std::numeric_limits<double>::infinity();
+  const int64_t len = p.kv_lens ? p.kv_lens[b] : p.Sk;
+  const int64_t off = p.causal_offset + (len - p.Sk);
 
   // Pass 1: scores and their maximum.
   double m = neg_inf;
@@ -84,7 +101,9 @@ void row_weights(const Problem& p, int64_t b, int64_t h, int64_t i, double* w) {
     for (int64_t d = 0; d < p.D; ++d) dot += qrow[d] * krow[d];
     double s = p.scale * dot;
     if (p.mask != nullptr && p.mask[(b * p.Sq + i) * p.Sk + j] == 0) s = neg_inf;
-    if (p.causal && j > i) s = neg_inf;
+    if (j >= len) s = neg_inf;
+    if (p.causal && j > i + off) s = neg_inf;
+    if (p.window > 0 && j <= i + off - p.window) s = neg_inf;
     w[j] = s;
     if (s > m) m = s;
   }
@@ -117,7 +136,7 @@ extern "C" {
 int oracle_gqa_probs(const double* q, const double* k, const uint8_t* mask, int64_t B,
                      int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Sk, int64_t D, int causal,
                      double scale, double* probs) {
-  Problem p{q, k, nullptr, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  Problem p{q, k, nullptr, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale, 0, 0, false};
   if (!valid(p)) return -1;
   for (int64_t b = 0; b < B; ++b)
     for (int64_t h = 0; h < Hq; ++h)
@@ -130,7 +149,7 @@ int oracle_gqa_probs(const double* q, const double* k, const uint8_t* mask, int6
 int oracle_gqa_forward(const double* q, const double* k, const double* v, const uint8_t* mask,
                        int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Sk, int64_t D,
                        int causal, double scale, double* out) {
-  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale, 0, 0, false};
   if (!valid(p)) return -1;
   std::vector<double> w(static_cast<size_t>(Sk > 0 ? Sk : 1));
   for (int64_t b = 0; b < B; ++b)
@@ -147,7 +166,7 @@ int oracle_gqa_forward_rows(const double* q, const double* k, const double* v,
                             const uint8_t* mask, int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq,
                             int64_t Sk, int64_t D, int causal, double scale, const int64_t* rows,
                             int64_t n, double* out) {
-  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale, 0, 0, false};
   if (!valid(p)) return -1;
   for (int64_t r = 0; r < n; ++r) {
     const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
@@ -159,6 +178,51 @@ int oracle_gqa_forward_rows(const double* q, const double* k, const double* v,
     row_weights(p, b, h, i, w.data());
     row_output(p, b, h, i, w.data(), out + r * D);
   }
+  return 0;
+}
+
+// Selected rows with an explicit causal offset and sliding window (see the
+// header); rows[3*r .. 3*r+2] = (b, h, i); out is [n, D].
+int oracle_gqa_forward_rows_ex(const double* q, const double* k, const double* v,
+                               const uint8_t* mask, const int32_t* kv_lens, int64_t B, int64_t Hq,
+                               int64_t Hkv, int64_t Sq, int64_t Sk, int64_t D, int causal,
+                               int64_t causal_offset, int64_t window, double scale,
+                               const int64_t* rows, int64_t n, double* out) {
+  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale, causal_offset, window, true,
+            kv_lens};
+  if (!valid(p)) return -1;
+  for (int64_t b = 0; kv_lens != nullptr && b < B; ++b)
+    if (kv_lens[b] < 0 || kv_lens[b] > Sk) return -1;
+  for (int64_t r = 0; r < n; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= Sq) return -1;
+  }
+  std::vector<double> w(static_cast<size_t>(Sk > 0 ? Sk : 1));
+  for (int64_t r = 0; r < n; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    row_weights(p, b, h, i, w.data());
+    row_output(p, b, h, i, w.data(), out + r * D);
+  }
+  return 0;
+}
+
+// Full output with an explicit causal offset and sliding window.
+int oracle_gqa_forward_ex(const double* q, const double* k, const double* v, const uint8_t* mask,
+                          const int32_t* kv_lens, int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq,
+                          int64_t Sk, int64_t D, int causal, int64_t causal_offset,
+                          int64_t window, double scale, double* out) {
+  Problem p{q, k, v, mask, B, Hq, Hkv, Sq, Sk, D, causal, scale, causal_offset, window, true,
+            kv_lens};
+  if (!valid(p)) return -1;
+  for (int64_t b = 0; kv_lens != nullptr && b < B; ++b)
+    if (kv_lens[b] < 0 || kv_lens[b] > Sk) return -1;
+  std::vector<double> w(static_cast<size_t>(Sk > 0 ? Sk : 1));
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t h = 0; h < Hq; ++h)
+      for (int64_t i = 0; i < Sq; ++i) {
+        row_weights(p, b, h, i, w.data());
+        row_output(p, b, h, i, w.data(), out + ((b * Hq + h) * Sq + i) * D);
+      }
   return 0;
 }
 

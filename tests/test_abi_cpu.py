@@ -65,7 +65,8 @@ def _rc(gqa, p, sms=148):
     (dict(Hkv=0), 2),
     (dict(D=96), 4),                              # bf16 needs 64 or 128
     (dict(D=300, dtype=1), 4),                    # fp32 path: D <= 256
-    (dict(Sq=3, Sk=5, causal=True), 4),           # causal needs Sq == Sk
+    (dict(window=4), 8),                          # a window needs causal
+    (dict(causal=True, window=-1), 8),
     (dict(scale=float("nan")), 8),
     (dict(scale=float("inf")), 8),
     (dict(dtype=7), 8),
@@ -112,6 +113,14 @@ def test_plans_for_the_five_workloads(gqa):
     assert pl.algorithmic_bytes == 2 * 8 * 12 * 2048 * 64 * 2 + 2 * 8 * 2 * 2048 * 64 * 2 + 8 * 2048 * 2048
 
 
+def test_short_query_blocks_decode(gqa):
+    # g * Sq rows per kv head: up to 16 run on the decode stream in one pass.
+    for (Hq, Hkv, Sq, kind) in ((8, 2, 4, "decode"), (8, 1, 2, "decode"), (4, 4, 16, "decode"),
+                                (8, 2, 5, "prefill"), (16, 1, 2, "prefill")):
+        rc, pl = _rc(gqa, _p(gqa, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=300))
+        assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == kind, (Hq, Hkv, Sq)
+
+
 def test_decode_grid_small_problem(gqa):
     # Fewer 64-key tiles than SMs: one tile per CTA.
     rc, pl = _rc(gqa, _p(gqa, B=1, Hq=4, Hkv=1, Sq=1, Sk=130, D=64))
@@ -119,6 +128,34 @@ def test_decode_grid_small_problem(gqa):
     # g > 8 uses 16-head passes.
     rc, pl = _rc(gqa, _p(gqa, B=1, Hq=40, Hkv=1, Sq=1, Sk=64, D=128))
     assert rc == 0 and pl.work_units == 3  # ceil(40 / 16) passes x 1 tile
+
+
+def test_causal_offset_and_window_plans(gqa):
+    # Causal with Sq != Sk is defined by the offset (bottom-right here); a short
+    # query block (g * Sq <= 16 rows) stays on the decode stream.
+    rc, pl = _rc(gqa, _p(gqa, Sq=3, Sk=5, causal=True, causal_offset=2))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "decode"
+    rc, pl = _rc(gqa, _p(gqa, Sq=5, Sk=9, causal=True, causal_offset=4))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "prefill"
+    # No query sees any key: NaN fill, no attention kernel.
+    rc, pl = _rc(gqa, _p(gqa, Sq=4, Sk=8, causal=True, causal_offset=-4))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "nan"
+    rc, pl = _rc(gqa, _p(gqa, Sq=1, Sk=8, causal=True, causal_offset=20, window=4))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "nan"
+    # Decode with a sliding window streams only the window's tiles.
+    rc, full = _rc(gqa, _p(gqa, B=1, Hq=8, Hkv=2, Sq=1, Sk=4096, causal=True, causal_offset=4095))
+    rc2, win = _rc(gqa, _p(gqa, B=1, Hq=8, Hkv=2, Sq=1, Sk=4096, causal=True, causal_offset=4095,
+                           window=256))
+    assert rc == rc2 == 0 and full.work_units == 2 * 64 and win.work_units == 2 * 4
+
+
+def test_binding_offset_rules(gqa):
+    assert gqa._offset(False, None, 3, 5) == 0
+    assert gqa._offset(True, None, 4, 4) == 0
+    assert gqa._offset(True, "bottom_right", 3, 5) == 2
+    assert gqa._offset(True, "top_left", 3, 5) == 0
+    with pytest.raises(ValueError):
+        gqa._offset(True, None, 3, 5)
 
 
 def test_empty_problems(gqa):

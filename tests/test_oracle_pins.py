@@ -29,7 +29,7 @@ def _sdpa(q, k, v, mask=None, causal=False, scale=None, gqa=True):
     tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x)) for x in (q, k, v))
     am = None
     if mask is not None:
-        am = torch.from_numpy(np.asarray(mask, dtype=bool))[:, None, :, :]
+        am = torch.from_numpy(np.array(mask, dtype=bool))[:, None, :, :]
     if causal:
         Sq, Sk = q.shape[2], k.shape[2]
         cm = torch.ones(Sq, Sk, dtype=torch.bool).tril()
@@ -308,12 +308,121 @@ def test_invalid_shapes_rejected(oracle_mod):
                            causal=True)
 
 
+# ------------------------------------------- causal offset and sliding window
+
+def _offset_window_mask(Sq, Sk, off, window):
+    i = np.arange(Sq)[:, None]
+    j = np.arange(Sk)[None, :]
+    vis = j <= i + off
+    if window:
+        vis &= j > i + off - window
+    return vis
+
+
+OFFSET_CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, offset, window
+    (2, 8, 2, 5, 12, 8, 7, 0),      # bottom-right causal, Sq < Sk
+    (1, 6, 3, 9, 9, 4, 0, 3),       # sliding window of 3 keys
+    (2, 4, 1, 4, 20, 8, 16, 5),     # bottom-right + window
+    (1, 4, 2, 6, 6, 8, -2, 0),      # diagonal shifted down: first rows fully hidden
+]
+
+
+def _offset_window_ref(q, k, v, off, window, mask=None):
+    B, Sq, Sk = q.shape[0], q.shape[2], k.shape[2]
+    vis = np.broadcast_to(_offset_window_mask(Sq, Sk, off, window), (B, Sq, Sk))
+    if mask is not None:
+        vis = vis & mask
+    return _sdpa(q, k, v, mask=vis, scale=1.0 / np.sqrt(q.shape[-1])), vis
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,off,window", OFFSET_CASES)
+def test_causal_offset_and_window_match_torch(oracle_mod, B, Hq, Hkv, Sq, Sk, D, off, window):
+    rng = np.random.default_rng(Sq * 31 + Sk)
+    q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+    ours = oracle_mod.forward(q, k, v, causal=True, causal_offset=off, window=window)
+    ref, vis = _offset_window_ref(q, k, v, off, window)
+    hidden_rows = ~vis.any(axis=-1)  # [B, Sq]
+    for b in range(B):
+        for i in range(Sq):
+            if hidden_rows[b, i]:
+                assert np.all(np.isnan(ours[b, :, i]))
+            else:
+                np.testing.assert_allclose(ours[b, :, i], ref[b, :, i], rtol=1e-11, atol=1e-12)
+
+
+def test_offset_zero_is_the_pages_causal(oracle_mod):
+    rng = np.random.default_rng(41)
+    q, k, v = _rand(rng, 2, 4, 7, 8), _rand(rng, 2, 2, 7, 8), _rand(rng, 2, 2, 7, 8)
+    assert np.array_equal(oracle_mod.forward(q, k, v, causal=True),
+                          oracle_mod.forward(q, k, v, causal=True, causal_offset=0))
+    # A window covering every visible key changes nothing.
+    assert np.array_equal(oracle_mod.forward(q, k, v, causal=True),
+                          oracle_mod.forward(q, k, v, causal=True, causal_offset=0, window=7))
+
+
+def test_window_of_one_selects_the_diagonal_value(oracle_mod):
+    rng = np.random.default_rng(42)
+    q, k, v = _rand(rng, 1, 4, 5, 8), _rand(rng, 1, 2, 9, 8), _rand(rng, 1, 2, 9, 8)
+    out = oracle_mod.forward(q, k, v, causal=True, causal_offset=4, window=1)
+    for h in range(4):
+        for i in range(5):
+            assert np.array_equal(out[0, h, i], v[0, h // 2, i + 4])
+
+
+def test_bottom_right_decode_sees_everything(oracle_mod):
+    rng = np.random.default_rng(43)
+    q, k, v = _rand(rng, 2, 8, 1, 8), _rand(rng, 2, 2, 33, 8), _rand(rng, 2, 2, 33, 8)
+    np.testing.assert_array_equal(oracle_mod.forward(q, k, v, causal=True, causal_offset=32),
+                                  oracle_mod.forward(q, k, v))
+
+
+def test_window_needs_causal(oracle_mod):
+    rng = np.random.default_rng(44)
+    q, k = _rand(rng, 1, 2, 3, 4), _rand(rng, 1, 1, 3, 4)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.forward(q, k, k, causal=False, causal_offset=0, window=2)
+
+
+# ---------------------------------------------------------- ragged KV cache
+
+def test_kv_lens_equal_truncated_cache(oracle_mod):
+    """Batch entry b with kv_lens[b] = n gives what the pages' function gives on
+    the first n keys alone (bottom-right causal included)."""
+    rng = np.random.default_rng(45)
+    B, Hq, Hkv, Sq, Sk, D = 3, 8, 2, 3, 20, 8
+    q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+    lens = np.array([20, 7, 12], dtype=np.int32)
+    for causal in (False, True):
+        out = oracle_mod.forward(q, k, v, causal=causal,
+                                 causal_offset=(Sk - Sq) if causal else None, kv_lens=lens)
+        for b in range(B):
+            n = int(lens[b])
+            ref, _ = _offset_window_ref(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n],
+                                        n - Sq if causal else n, 0)
+            np.testing.assert_allclose(out[b:b + 1], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_kv_lens_bounds(oracle_mod):
+    rng = np.random.default_rng(46)
+    q, k = _rand(rng, 2, 2, 1, 4), _rand(rng, 2, 1, 5, 4)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.forward(q, k, k, kv_lens=[5, 6])
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.forward(q, k, k, kv_lens=[5])
+
+
 # ---------------------------------------------------------- planted mistakes
 
 MUTANTS = {
     "tiling head map": ("const int64_t kv = h / g;", "const int64_t kv = h % p.Hkv;"),
     "scale dropped": ("double s = p.scale * dot;", "double s = dot;"),
-    "causal off by one": ("if (p.causal && j > i)", "if (p.causal && j >= i)"),
+    "causal off by one": ("if (p.causal && j > i + off)", "if (p.causal && j >= i + off)"),
+    "causal offset ignored": ("if (p.causal && j > i + off)", "if (p.causal && j > i)"),
+    "window off by one": ("j <= i + off - p.window", "j < i + off - p.window"),
+    "kv length off by one": ("if (j >= len) s = neg_inf;", "if (j > len) s = neg_inf;"),
+    "kv length ignored by causal": ("const int64_t off = p.causal_offset + (len - p.Sk);",
+                                    "const int64_t off = p.causal_offset;"),
     "mask polarity": ("p.mask[(b * p.Sq + i) * p.Sk + j] == 0", "p.mask[(b * p.Sq + i) * p.Sk + j] != 0"),
     "max not subtracted": ("w[j] = std::exp(w[j] - m);", "w[j] = std::exp(w[j]);"),
     "no normalisation": ("for (int64_t j = 0; j < p.Sk; ++j) w[j] = w[j] / l;", ""),
@@ -337,6 +446,25 @@ def _pins_hold(oracle_mod, lib):
             return False
         ref = _sdpa(q, k, v, mask=mask, causal=causal, scale=1.0 / np.sqrt(D))
         ok &= bool(np.allclose(ours, ref, rtol=1e-11, atol=1e-12))
+    for (B, Hq, Hkv, Sq, Sk, D, off, window) in OFFSET_CASES[:3]:
+        q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+        try:
+            ours = oracle_mod.forward(q, k, v, causal=True, causal_offset=off, window=window, lib=lib)
+        except oracle_mod.OracleError:
+            return False
+        ref, _ = _offset_window_ref(q, k, v, off, window)
+        ok &= bool(np.allclose(ours, ref, rtol=1e-11, atol=1e-12))
+    q, k, v = _rand(rng, 2, 4, 2, 8), _rand(rng, 2, 2, 9, 8), _rand(rng, 2, 2, 9, 8)
+    try:
+        ragged = oracle_mod.forward(q, k, v, causal=True, causal_offset=7, kv_lens=[9, 5], lib=lib)
+    except oracle_mod.OracleError:
+        return False
+    plain = oracle_mod.forward(q, k, v, kv_lens=[9, 5], lib=lib)
+    for b, n in ((0, 9), (1, 5)):
+        ref, _ = _offset_window_ref(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], n - 2, 0)
+        ok &= bool(np.allclose(ragged[b:b + 1], ref, rtol=1e-11, atol=1e-12))
+        ref, _ = _offset_window_ref(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], n, 0)
+        ok &= bool(np.allclose(plain[b:b + 1], ref, rtol=1e-11, atol=1e-12))
     q, k, v = _rand(rng, 1, 4, 5, 8) * 60.0, _rand(rng, 1, 2, 7, 8) * 60.0, _rand(rng, 1, 2, 7, 8)
     big = oracle_mod.forward(q, k, v, scale=1.0, lib=lib)
     ok &= bool(np.allclose(big, _sdpa(q, k, v, scale=1.0), rtol=1e-11, atol=1e-12))

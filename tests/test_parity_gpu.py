@@ -202,3 +202,79 @@ def test_decode_after_other_calls_on_one_workspace(gqa):
             assert st == 0, gqa.status_string(st)
             assert_bf16_parity(to_np(out), oracle_bf16(*bits, mask=mask),
                                "shared workspace %s" % (tuple(q.shape),))
+
+
+# ----------------------------------------------- causal offset and sliding window
+
+def _nan_rows_match(got, ref):
+    """Rows the oracle leaves NaN (no visible key) must be NaN on the GPU too;
+    returns the boolean array of the other rows."""
+    nan_ref = np.isnan(ref).all(axis=-1)
+    assert np.array_equal(np.isnan(got).all(axis=-1), nan_ref)
+    return ~nan_ref
+
+
+@pytest.mark.parametrize("Sq,Sk,off,window", [(5, 40, 35, 0), (5, 40, 35, 7), (6, 6, -2, 0),
+                                              (4, 30, 10, 3)])
+def test_f32_offset_window(gqa, Sq, Sk, off, window):
+    q, k, v = synth.qkv_f32(Sq * 7 + Sk, 2, 8, 2, Sq, Sk, 32)
+    out = gqa.forward(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(),
+                      torch.from_numpy(v).cuda(), causal=True, causal_offset=off, window=window)
+    ref = oracle.forward(q, k, v, causal=True, causal_offset=off, window=window)
+    got = out.cpu().numpy().astype(np.float64)
+    ok = _nan_rows_match(got, ref)
+    assert np.abs(got[ok] - ref[ok]).max() <= F32_ABS
+
+
+@pytest.mark.parametrize("Sk,off,window,masked", [
+    (1000, 999, 0, False),     # bottom-right: the one query sees every key
+    (4096, 4095, 256, False),  # sliding window over the last 256 keys
+    (1000, 500, 200, True),    # keys 301..500, with a mask
+    (777, 700, 65, False),     # window straddling tile edges
+])
+def test_decode_offset_window(gqa, Sk, off, window, masked):
+    B, Hq, Hkv, D = 3, 16, 4, 128
+    bits, (q, k, v) = bf16_inputs(Sk + window, B, Hq, Hkv, 1, Sk, D)
+    mask = synth.mask_random(9, B, 1, Sk, 0.5) if masked else None
+    if masked:  # keep a visible key inside the window
+        mask[:, :, off] = 1
+    out = gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda() if masked else None,
+                      causal=True, causal_offset=off, window=window)
+    _status_ok(gqa)
+    ref = oracle.forward(f64(bits[0]), f64(bits[1]), f64(bits[2]), mask=mask, causal=True,
+                         causal_offset=off, window=window)
+    assert_bf16_parity(to_np(out), ref, "decode offset/window")
+
+
+def test_nothing_visible_is_nan(gqa):
+    bits, (q, k, v) = bf16_inputs(12, 2, 8, 2, 4, 64, 128)
+    out = to_np(gqa.forward(q, k, v, causal=True, causal_offset=-4))
+    assert np.all(np.isnan(out))
+
+
+# ------------------------------------------------ short multi-query decode
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,off,window,masked", [
+    (2, 8, 2, 4, 1000, 128, "br", 0, False),   # 4 heads x 4 queries = 16 rows, bottom-right
+    (3, 8, 1, 2, 517, 64, None, 0, False),     # 8 heads x 2 queries, no causal
+    (1, 4, 4, 16, 300, 128, "br", 50, False),  # MHA, 16 queries, sliding window
+    (2, 8, 2, 3, 400, 128, "br", 0, True),     # 12 rows with a mask
+    (2, 6, 2, 5, 129, 64, "br", 0, False),     # g = 3: 15 rows
+])
+def test_short_query_block_decode(gqa, B, Hq, Hkv, Sq, Sk, D, off, window, masked):
+    bits, (q, k, v) = bf16_inputs(Sq * 100 + Sk, B, Hq, Hkv, Sq, Sk, D)
+    plan = gqa.query(q, k, v, causal=off is not None,
+                     causal_offset="bottom_right" if off else None, window=window)
+    assert plan["kernel_name"] == "decode"
+    mask = synth.mask_random(31, B, Sq, Sk, 0.5) if masked else None
+    if masked:
+        for i in range(Sq):
+            mask[:, i, Sk - Sq + i] = 1
+    out = gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda() if masked else None,
+                      causal=off is not None, causal_offset="bottom_right" if off else None,
+                      window=window)
+    _status_ok(gqa)
+    ref = oracle.forward(f64(bits[0]), f64(bits[1]), f64(bits[2]), mask=mask,
+                         causal=off is not None, causal_offset=(Sk - Sq) if off else None,
+                         window=window)
+    assert_bf16_parity(to_np(out), ref, "short query decode")

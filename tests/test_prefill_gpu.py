@@ -159,3 +159,30 @@ def test_prefill_masked_full_size_sampled(gqa):
     got, ref = _sampled(gqa, 5, 8, 12, 2, 2048, 64, False, True,
                         [(0, 0, rows), (7, 1, rows), (4, 0, rows)])
     assert_bf16_parity(got, ref, "masked prefill full size")
+
+
+# ----------------------------------------------- causal offset and sliding window
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,off,window,mask_kind", [
+    (1, 8, 2, 200, 700, 128, 500, 0, None),       # bottom-right causal, query block at the end
+    (2, 8, 2, 600, 600, 128, 0, 256, None),       # sliding window of 256 keys
+    (1, 12, 2, 300, 900, 64, 600, 130, "random"), # bottom-right + window + mask, g = 6
+    (1, 8, 2, 130, 130, 128, -3, 0, None),        # first three rows see nothing: NaN
+    (2, 32, 8, 256, 2048, 128, 1792, 1000, None), # several key tiles, window > tile
+])
+def test_prefill_offset_window(gqa, B, Hq, Hkv, Sq, Sk, D, off, window, mask_kind):
+    seed = 2000 + Sq + Sk + window
+    bits, (q, k, v) = bf16_inputs(seed, B, Hq, Hkv, Sq, Sk, D)
+    mask = synth.mask_random(seed, B, Sq, Sk, 0.6) if mask_kind else None
+    if mask is not None:  # keep the diagonal key visible
+        for i in range(Sq):
+            if 0 <= i + off < Sk:
+                mask[:, i, i + off] = 1
+    out = to_np(gqa.forward(q, k, v, mask=torch.from_numpy(mask).cuda() if mask is not None else None,
+                            causal=True, causal_offset=off, window=window))
+    _status_ok(gqa)
+    ref = oracle.forward(f64(bits[0]), f64(bits[1]), f64(bits[2]), mask=mask, causal=True,
+                         causal_offset=off, window=window)
+    nan_ref = np.isnan(ref).all(axis=-1)
+    assert np.array_equal(np.isnan(out).all(axis=-1), nan_ref)
+    assert_bf16_parity(out[~nan_ref], ref[~nan_ref], "prefill offset/window")
