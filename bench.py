@@ -50,6 +50,13 @@ PREFILL_CAUSAL = dict(name="prefill_causal", B=4, Hq=32, Hkv=8, Sq=4096, Sk=4096
                       causal=True, mask=False, seed=4)
 PREFILL_MASKED = dict(name="prefill_padded_mask", B=8, Hq=12, Hkv=2, Sq=2048, Sk=2048, D=64,
                       causal=False, mask=True, seed=5)
+# Ragged KV cache: 4096-key capacity, entry b holds len_b ~ U[256, 4096] keys.
+DECODE_RAGGED = dict(name="decode_ragged_cache", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128,
+                     causal=False, mask=False, seed=6, lens=(256, 4096), append=0)
+# One generation step: append one token per sequence, then attend over the
+# grown cache (bottom-right causal); capacity leaves room for the appends.
+DECODE_STEP = dict(name="decode_step_append", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096 + 512, D=128,
+                   causal=True, mask=False, seed=7, lens=(256, 4096), append=1)
 
 L2_BYTES = 126 * 1024 * 1024
 
@@ -255,6 +262,63 @@ def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     return res
 
 
+def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
+    """Device-resident timing of a ragged-cache workload: per step an optional
+    gqa_kv_append of one token per sequence, then gqa_forward with kv_lens."""
+    import numpy as np
+    B, Hkv, Sk, D = cfg["B"], cfg["Hkv"], cfg["Sk"], cfg["D"]
+    q, k, v, _ = _host_inputs(cfg, torch)
+    lo, hi = cfg["lens"]
+    lens0 = synth.uniform_int(cfg["seed"], synth.STREAM_MASK, B, lo, hi).astype(np.int32)
+    valid_bytes = int(lens0.sum()) * Hkv * D * 2 * 2
+    copies = max(3, math.ceil(rotate_to_bytes / valid_bytes))
+    qd = q.to(dev)
+    ks = [k.to(dev) for _ in range(copies)]
+    vs = [v.to(dev) for _ in range(copies)]
+    lens = [torch.from_numpy(lens0.copy()).to(dev) for _ in range(copies)]
+    n_new = cfg["append"]
+    kn = vn = None
+    if n_new:
+        kn = ks[0][:, :, :n_new].clone()
+        vn = vs[0][:, :, :n_new].clone()
+    out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
+    off = "bottom_right" if cfg["causal"] else None
+    plan = gqa.query(qd, ks[0], vs[0], causal=cfg["causal"], causal_offset=off, kv_lens=lens[0])
+    ws = gqa.workspace_for(dev, plan["workspace_bytes"])
+    stream = torch.cuda.current_stream(dev)
+
+    def call(i):
+        if n_new:
+            gqa.kv_append(ks[i], vs[i], kn, vn, lens[i], workspace=ws)
+        gqa.forward(qd, ks[i], vs[i], out=out, workspace=ws, causal=cfg["causal"],
+                    causal_offset=off, kv_lens=lens[i])
+
+    calls = [(lambda i=i: call(i)) for i in range(copies)]
+    if n_new:  # every call of a copy appends n_new tokens: they must fit the capacity
+        calls_per_copy = math.ceil((warmup + max(3, copies) + steps) / copies)
+        if hi + calls_per_copy * n_new > Sk:
+            raise ValueError("%d steps overflow the %d-key cache; use fewer" % (steps, Sk))
+    total_ms, per, _ = _graph_timed(torch, calls, steps, warmup, stream)
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
+    # Keys read per step: the lengths grow by n_new per call of a copy, so the
+    # mean of each copy's first and last lengths is the mean over its calls.
+    final = [int(x.sum().item()) for x in lens]
+    mean_keys = statistics.mean((int(lens0.sum()) + f) / 2.0 for f in final)
+    if n_new:
+        mean_keys += n_new * B  # the appended token is read too
+    step_bytes = (mean_keys * Hkv * D * 2 * 2 + 2 * qd.numel() * 2 +
+                  (4 * B * Hkv * n_new * D * 2 if n_new else 0))
+    res = dict(total_ms=total_ms, per_launch_ms=statistics.mean(per),
+               per_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
+               step_bytes=step_bytes, launches=plan["launches"] + (1 if n_new else 0),
+               mean_len=mean_keys / B)
+    del ks, vs, qd, out, lens
+    torch.cuda.empty_cache()
+    return res
+
+
 def _e2e(gqa, torch, cfg, steps, dev):
     """Through the public call with host buffers: pinned host -> device copy
     of the step's inputs, the forward, and a device -> host read of out."""
@@ -335,7 +399,18 @@ def _roofline_prefill(res, tflops, peak_kind, workload):
             "algorithmic_flops_per_launch": fl, "launch_ms": round(res["per_launch_ms"], 5)}
 
 
-WORKLOADS = {c["name"]: c for c in (DECODE, DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED)}
+def _roofline_ragged(res, hbm, peak_kind, workload):
+    achieved = res["step_bytes"] / (res["per_launch_ms"] / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
+            "traffic": _traffic_for("decode.cu", workload),
+            "algorithmic_bytes_per_step": int(res["step_bytes"]),
+            "mean_len": round(res["mean_len"], 1), "kernels_per_step": res["launches"],
+            "step_ms": round(res["per_launch_ms"], 5)}
+
+
+WORKLOADS = {c["name"]: c for c in (DECODE, DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED,
+                                    DECODE_RAGGED, DECODE_STEP)}
 
 
 def run_profile_case(args):
@@ -346,7 +421,8 @@ def run_profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     cfg = WORKLOADS[args.profile]
-    res = _time_config(gqa, torch, cfg, steps=args.steps, warmup=args.warmup, dev=dev)
+    timer = _time_ragged if "lens" in cfg else _time_config
+    res = timer(gqa, torch, cfg, steps=args.steps, warmup=args.warmup, dev=dev)
     print(json.dumps({"profile_case": cfg["name"], "launch_ms": res["per_launch_ms"],
                       "copies": res["copies"], "plan": res["plan"]}), flush=True)
 
@@ -445,7 +521,7 @@ def run_gpu(args):
             "frac": round(plan["algorithmic_bytes"] / (per_launch / 1e3) / 1e9 / hbm, 4),
             "traffic": _traffic_for("decode.cu", DECODE["name"]),
             "peak_source": peak_kind,
-            "kernel": "gqa_decode_kernel + gqa_decode_combine_kernel (timed together per call)",
+            "kernel": "gqa_decode_kernel (split merge fused; the counter memset is in the same graph)",
             "algorithmic_bytes_per_launch": plan["algorithmic_bytes"],
             "launch_ms": round(per_launch, 5),
         },
@@ -453,14 +529,18 @@ def run_gpu(args):
 
     if rank == 0 and world == 1 and not args.skip_extra:
         extra = {}
-        for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED):
+        for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED, DECODE_RAGGED, DECODE_STEP):
+            timer = _time_ragged if "lens" in c else _time_config
             try:
-                res = _time_config(gqa, torch, c, steps=max(3, min(args.steps, 50)),
-                                   warmup=max(3, min(args.warmup, 10)), dev=dev)
+                res = timer(gqa, torch, c, steps=max(3, min(args.steps, 50)),
+                            warmup=max(3, min(args.warmup, 10)), dev=dev)
             except Exception as e:  # report, keep the primary line
                 extra[c["name"]] = {"unavailable": "%s: %s" % (type(e).__name__, e)}
                 continue
-            if c["Sq"] == 1:
+            if "lens" in c:
+                rf = _roofline_ragged(res, hbm, peak_kind, c["name"])
+                extra[c["name"]] = {"value": rf["achieved"], "unit": "GB/s", "roofline": rf}
+            elif c["Sq"] == 1:
                 rf = _roofline_decode(res, hbm, peak_kind, c["name"])
                 extra[c["name"]] = {"value": rf["achieved"], "unit": "GB/s", "roofline": rf}
             else:

@@ -6,10 +6,12 @@ runs in the CUDA kernels of ``libgqa_b200.so``.  There is no CPU or PyTorch
 fallback: if the library is missing this module raises at import time.
 
     out = forward(q, k, v, mask=None, causal=False, scale=None)
+    kv_append(cache_k, cache_v, k_new, v_new, kv_lens)
 
 q [B, Hq, Sq, D], k and v [B, Hkv, Sk, D] (CUDA tensors, bf16 or fp32, last
 dim contiguous), mask bool/uint8 [B, Sq, Sk] (True = attend, shared by all
-heads), ``scale`` defaults to 1/sqrt(D).
+heads), ``scale`` defaults to 1/sqrt(D).  ``kv_lens`` (int32 CUDA [B]) makes
+k and v a cache of capacity Sk whose entry b holds kv_lens[b] keys.
 """
 from __future__ import annotations
 
@@ -30,13 +32,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQA_OK = 0
 GQA_ERR_NULL, GQA_ERR_SHAPE, GQA_ERR_LAYOUT, GQA_ERR_UNSUPPORTED = 1, 2, 3, 4
 GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 5, 6, 7, 8, 9
-GQA_ERR_SCRATCH_LIMIT = 10
+GQA_ERR_SCRATCH_LIMIT, GQA_ERR_KV_LENGTH = 10, 11
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 GQA_DTYPE_BF16, GQA_DTYPE_F32 = 0, 1
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
 
 EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
-           "gqa_forward_decode_noalloc")
+           "gqa_forward_decode_noalloc", "gqa_kv_append")
 
 
 class Problem(ctypes.Structure):
@@ -49,6 +51,17 @@ class Problem(ctypes.Structure):
         ("v_stride", ctypes.c_int64 * 4), ("o_stride", ctypes.c_int64 * 4),
         ("mask_stride", ctypes.c_int64 * 3),
         ("causal_offset", ctypes.c_int64), ("window", ctypes.c_int64),
+        ("kv_lens", ctypes.c_void_p),
+    ]
+
+
+class AppendDesc(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("batch", ctypes.c_int64), ("heads_kv", ctypes.c_int64), ("capacity", ctypes.c_int64),
+        ("head_dim", ctypes.c_int64), ("n_new", ctypes.c_int64),
+        ("cache_k_stride", ctypes.c_int64 * 4), ("cache_v_stride", ctypes.c_int64 * 4),
+        ("k_new_stride", ctypes.c_int64 * 4), ("v_new_stride", ctypes.c_int64 * 4),
     ]
 
 
@@ -81,6 +94,9 @@ _lib.gqa_version.restype = ctypes.c_int
 _lib.gqa_forward_decode_noalloc.argtypes = [ctypes.POINTER(Problem), _vp, _vp, _vp, _vp, _vp,
                                             _vp]
 _lib.gqa_forward_decode_noalloc.restype = ctypes.c_int
+_lib.gqa_kv_append.argtypes = [ctypes.POINTER(AppendDesc), _vp, _vp, _vp, _vp, _vp, _vp,
+                               ctypes.c_size_t, _vp]
+_lib.gqa_kv_append.restype = ctypes.c_int
 
 
 class GQAError(RuntimeError):
@@ -100,9 +116,11 @@ def version() -> int:
 def make_problem(dtype: int, B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int,
                  q_stride, k_stride, v_stride, o_stride, mask_stride=None,
                  causal: bool = False, scale: float | None = None, causal_offset: int = 0,
-                 window: int = 0) -> Problem:
-    """Build the C problem descriptor from plain sizes and element strides."""
+                 window: int = 0, kv_lens_ptr: int | None = None) -> Problem:
+    """Build the C problem descriptor from plain sizes and element strides
+    (``kv_lens_ptr``: device address of int32 [B] cache lengths, or None)."""
     p = Problem()
+    p.kv_lens = kv_lens_ptr
     p.dtype = dtype
     p.causal = int(bool(causal))
     p.causal_offset = int(causal_offset)
@@ -174,8 +192,18 @@ def _offset(causal, causal_offset, Sq, Sk) -> int:
     return int(causal_offset)
 
 
+def _lens_ptr(kv_lens, B):
+    if kv_lens is None:
+        return None
+    torch = _torch()
+    if not kv_lens.is_cuda or kv_lens.dtype != torch.int32 or tuple(kv_lens.shape) != (B,) or \
+            not kv_lens.is_contiguous():
+        raise ValueError("kv_lens must be a contiguous int32 CUDA tensor of shape [B]")
+    return kv_lens.data_ptr()
+
+
 def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None, causal_offset=None,
-                window=0) -> Problem:
+                window=0, kv_lens=None) -> Problem:
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, S, D]")
     if not (q.dtype == k.dtype == v.dtype):
@@ -192,13 +220,14 @@ def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None, causal_o
         mst = mask.stride()
     return make_problem(_dtype_code(q), B, Hq, Hkv, Sq, Sk, D, q.stride(), k.stride(),
                         v.stride(), ost, mst, causal=causal, scale=scale,
-                        causal_offset=_offset(causal, causal_offset, Sq, Sk), window=window)
+                        causal_offset=_offset(causal, causal_offset, Sq, Sk), window=window,
+                        kv_lens_ptr=_lens_ptr(kv_lens, B))
 
 
 def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0, causal_offset=None,
-          window=0) -> dict:
+          window=0, kv_lens=None) -> dict:
     return query_problem(problem_for(q, k, v, mask, causal, scale, causal_offset=causal_offset,
-                                     window=window), sm_count).as_dict()
+                                     window=window, kv_lens=kv_lens), sm_count).as_dict()
 
 
 def workspace_for(device, nbytes: int):
@@ -214,13 +243,15 @@ def workspace_for(device, nbytes: int):
 
 
 def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=None,
-            stream=None, causal_offset=None, window=0):
+            stream=None, causal_offset=None, window=0, kv_lens=None):
     """out = softmax(mask(q k_{h/g}^T * scale)) v_{h/g} on the GPU.
 
     causal: key j visible to query i iff j <= i + offset (offset 0 for
     Sq == Sk; pass causal_offset="bottom_right" for a query block at the end
     of the keys).  window > 0 keeps only the last `window` keys up to the
-    diagonal (sliding-window attention)."""
+    diagonal (sliding-window attention).  kv_lens (int32 CUDA [B]): entry b
+    holds kv_lens[b] keys of the Sk-long cache; the offset is given for a
+    full cache and moves by kv_lens[b] - Sk."""
     torch = _torch()
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors (there is no CPU path)")
@@ -233,7 +264,8 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
             raise TypeError("mask must be bool or uint8")
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
-    p = problem_for(q, k, v, mask, causal, scale, out, causal_offset=causal_offset, window=window)
+    p = problem_for(q, k, v, mask, causal, scale, out, causal_offset=causal_offset, window=window,
+                    kv_lens=kv_lens)
     plan = query_problem(p)
     if workspace is None:
         workspace = workspace_for(q.device, plan.workspace_bytes)
@@ -243,6 +275,54 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
                  mask.data_ptr() if mask is not None else None, out.data_ptr(),
                  workspace.data_ptr(), workspace.numel(), stream)
     return out
+
+
+def append_desc(dtype: int, B: int, Hkv: int, capacity: int, D: int, n_new: int,
+                cache_k_stride, cache_v_stride, k_new_stride, v_new_stride) -> AppendDesc:
+    d = AppendDesc()
+    d.dtype, d.reserved = dtype, 0
+    d.batch, d.heads_kv, d.capacity, d.head_dim, d.n_new = B, Hkv, capacity, D, n_new
+    for i in range(4):
+        d.cache_k_stride[i], d.cache_v_stride[i] = int(cache_k_stride[i]), int(cache_v_stride[i])
+        d.k_new_stride[i], d.v_new_stride[i] = int(k_new_stride[i]), int(v_new_stride[i])
+    return d
+
+
+def kv_append_ptrs(d: AppendDesc, cache_k: int, cache_v: int, k_new: int, v_new: int,
+                   kv_lens: int, workspace: int, workspace_bytes: int, stream: int) -> None:
+    """Raw pointer form of gqa_kv_append (all device pointers)."""
+    rc = _lib.gqa_kv_append(ctypes.byref(d), cache_k, cache_v, k_new, v_new, kv_lens, workspace,
+                            workspace_bytes, stream)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_kv_append")
+
+
+def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=None):
+    """Write k_new / v_new [B, Hkv, n_new, D] into rows kv_lens[b] .. kv_lens[b] + n_new
+    of cache_k / cache_v [B, Hkv, capacity, D], then advance kv_lens (int32 CUDA [B])
+    in place.  An entry that does not fit is left as it was and device_status()
+    reports GQA_ERR_KV_LENGTH."""
+    torch = _torch()
+    for t in (cache_k, cache_v, k_new, v_new, kv_lens):
+        if not t.is_cuda:
+            raise ValueError("kv_append takes CUDA tensors only")
+    if cache_k.dim() != 4 or tuple(cache_v.shape) != tuple(cache_k.shape):
+        raise ValueError("cache_k and cache_v must be [B, Hkv, capacity, D]")
+    B, Hkv, cap, D = cache_k.shape
+    if k_new.dim() != 4 or tuple(v_new.shape) != tuple(k_new.shape) or \
+            k_new.shape[0] != B or k_new.shape[1] != Hkv or k_new.shape[3] != D:
+        raise ValueError("k_new and v_new must be [B, Hkv, n_new, D]")
+    if not (cache_k.dtype == cache_v.dtype == k_new.dtype == v_new.dtype):
+        raise TypeError("cache and new rows must share a dtype")
+    d = append_desc(_dtype_code(cache_k), B, Hkv, cap, D, k_new.shape[2], cache_k.stride(),
+                    cache_v.stride(), k_new.stride(), v_new.stride())
+    lp = _lens_ptr(kv_lens, B)
+    if workspace is None:
+        workspace = workspace_for(cache_k.device, 256)
+    if stream is None:
+        stream = torch.cuda.current_stream(cache_k.device).cuda_stream
+    kv_append_ptrs(d, cache_k.data_ptr(), cache_v.data_ptr(), k_new.data_ptr(),
+                   v_new.data_ptr(), lp, workspace.data_ptr(), workspace.numel(), stream)
 
 
 def device_status(workspace=None, stream=None) -> int:

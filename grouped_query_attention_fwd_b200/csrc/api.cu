@@ -9,6 +9,7 @@
 
 #include "gqa.h"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace gqa {
 namespace {
@@ -52,6 +53,14 @@ int validate(const gqa_problem* pp) {
     }
   } else {
     if (p.head_dim > 256) return GQA_ERR_UNSUPPORTED;
+  }
+  if (p.kv_lens != nullptr) {
+    // The decode kernel keeps the lengths and their prefix sums in shared
+    // memory and counts tiles in 32 bits.
+    if (p.batch > kMaxRaggedBatch) return GQA_ERR_UNSUPPORTED;
+    const int64_t tiles = (p.seq_k + kDecodeKeysPerTile - 1) / kDecodeKeysPerTile;
+    if (p.batch * p.heads_kv * ((p.heads_q / p.heads_kv) * p.seq_q + 7) / 8 * tiles >= lim)
+      return GQA_ERR_UNSUPPORTED;
   }
   return GQA_OK;
 }
@@ -129,6 +138,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
     }
     case GQA_KERNEL_DECODE: {
       const DecodeShape s = plan_decode(p, sm_count);
+      if (s.units >= (int64_t(1) << 31)) return GQA_ERR_UNSUPPORTED;  // 32-bit unit indices
       plan->grid = s.grid;
       plan->block = kDecodeThreads;
       plan->smem_bytes = s.smem_bytes;
@@ -214,7 +224,7 @@ using namespace gqa;
 
 extern "C" {
 
-GQA_API int gqa_version(void) { return 10100; }
+GQA_API int gqa_version(void) { return 10200; }
 
 GQA_API const char* gqa_status_string(int status) {
   switch (status) {
@@ -229,6 +239,7 @@ GQA_API const char* gqa_status_string(int status) {
     case GQA_ERR_ARG: return "invalid scalar argument (finite scale, known dtype, window >= 0 and only with causal)";
     case GQA_ERR_DEVICE: return "no usable sm_100 CUDA device";
     case GQA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the library's static array holds";
+    case GQA_ERR_KV_LENGTH: return "a kv length was outside [0, capacity], or an append did not fit the cache";
     default: return "unknown status";
   }
 }
@@ -257,7 +268,8 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     const int drc = device_sm_count(&sms);
     if (drc != GQA_OK) return drc;
   }
-  fill_plan(p, sms, &plan);
+  const int prc = fill_plan(p, sms, &plan);
+  if (prc != GQA_OK) return prc;
   if (plan.kernel == GQA_KERNEL_NONE) return GQA_OK;
   if (out == nullptr) return GQA_ERR_NULL;
   if (plan.kernel == GQA_KERNEL_ZERO) return launch_zero(p, out, stream, false);
@@ -274,7 +286,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(out, 4))
       return GQA_ERR_LAYOUT;
     return launch_f32(p, static_cast<const float*>(q), static_cast<const float*>(k),
-                      static_cast<const float*>(v), mask, static_cast<float*>(out), stream);
+                      static_cast<const float*>(v), mask, static_cast<float*>(out), err, stream);
   }
 
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
@@ -292,30 +304,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     erc = encode_bf16_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride,
                           kDecodeKeysPerTile, 1);
     if (erc != GQA_OK) return erc;
-    DecodeArgs a{};
-    a.q = static_cast<const uint16_t*>(q);
-    for (int d = 0; d < 4; ++d) a.qs[d] = p.q_stride[d], a.os[d] = p.o_stride[d];
-    a.mask = p.has_mask ? mask : nullptr;
-    for (int d = 0; d < 3; ++d) a.ms[d] = p.mask_stride[d];
-    a.out = static_cast<uint16_t*>(out);
-    a.part_ml = reinterpret_cast<float2*>(ws + s.part_ml_offset);
-    a.part_o = reinterpret_cast<float*>(ws + s.part_o_offset);
-    a.counters = reinterpret_cast<uint32_t*>(ws + s.counters_offset);
-    a.err = err;
-    a.B = static_cast<int>(p.batch);
-    a.Hq = static_cast<int>(p.heads_q);
-    a.Hkv = static_cast<int>(p.heads_kv);
-    a.Sk = static_cast<int>(p.seq_k);
-    a.g = static_cast<int>(g);
-    a.Sq = static_cast<int>(p.seq_q);
-    a.rows = static_cast<int>(g * p.seq_q);
-    a.causal = p.causal;
-    a.causal_offset = p.causal_offset;
-    a.window = p.window;
-    a.t0 = s.t0;
-    a.key_lo = s.key_lo;
-    a.key_hi = s.key_hi;
-    a.scale_log2 = scale_log2;
+    const DecodeArgs a = make_decode_args(p, s, q, mask, out, ws);
     // The ticket counters must start at zero; other calls sharing this
     // workspace (a prefill's tile classes, a larger problem's partials) may
     // have left bytes there.
@@ -351,8 +340,63 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.causal_offset = p.causal_offset;
   a.window = p.window;
   a.has_mask = p.has_mask;
+  a.lens = p.kv_lens;
   a.scale_log2 = scale_log2;
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
+}
+
+GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cache_v,
+                          const void* k_new, const void* v_new, int32_t* kv_lens,
+                          void* workspace, size_t workspace_bytes, void* stream_ptr) {
+  if (d == nullptr) return GQA_ERR_NULL;
+  if (d->dtype != GQA_DTYPE_BF16 && d->dtype != GQA_DTYPE_F32) return GQA_ERR_ARG;
+  if (d->reserved != 0) return GQA_ERR_ARG;
+  const int64_t lim = int64_t(1) << 31;
+  if (d->batch < 0 || d->heads_kv <= 0 || d->capacity < 0 || d->head_dim <= 0 || d->n_new < 0 ||
+      d->batch >= lim || d->heads_kv >= lim || d->capacity >= lim || d->head_dim > 4096)
+    return GQA_ERR_SHAPE;
+  if (d->n_new > d->capacity) return GQA_ERR_SHAPE;
+  const int64_t* st[4] = {d->cache_k_stride, d->cache_v_stride, d->k_new_stride, d->v_new_stride};
+  for (const int64_t* x : st) {
+    if (x[3] != 1) return GQA_ERR_LAYOUT;
+    if (x[0] < 0 || x[1] < 0 || x[2] < 0) return GQA_ERR_LAYOUT;
+  }
+  if (d->batch == 0 || d->n_new == 0) return GQA_OK;
+  if (cache_k == nullptr || cache_v == nullptr || k_new == nullptr || v_new == nullptr ||
+      kv_lens == nullptr)
+    return GQA_ERR_NULL;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < 256)
+    return GQA_ERR_WORKSPACE;
+  const int eb = d->dtype == GQA_DTYPE_F32 ? 4 : 2;
+  if (!aligned(cache_k, eb) || !aligned(cache_v, eb) || !aligned(k_new, eb) ||
+      !aligned(v_new, eb) || !aligned(kv_lens, 4))
+    return GQA_ERR_LAYOUT;
+  AppendArgs a{};
+  a.ck = static_cast<uint8_t*>(cache_k);
+  a.cv = static_cast<uint8_t*>(cache_v);
+  a.kn = static_cast<const uint8_t*>(k_new);
+  a.vn = static_cast<const uint8_t*>(v_new);
+  a.lens = kv_lens;
+  a.err = static_cast<uint32_t*>(workspace);
+  a.ticket = static_cast<uint32_t*>(workspace) + 1;
+  for (int i = 0; i < 3; ++i) {
+    a.cks[i] = d->cache_k_stride[i] * eb;
+    a.cvs[i] = d->cache_v_stride[i] * eb;
+    a.kns[i] = d->k_new_stride[i] * eb;
+    a.vns[i] = d->v_new_stride[i] * eb;
+  }
+  a.B = static_cast<int>(d->batch);
+  a.H = static_cast<int>(d->heads_kv);
+  a.cap = d->capacity;
+  a.n_new = d->n_new;
+  a.row_bytes = static_cast<int>(d->head_dim * eb);
+  // 16-byte pieces when every row start is 16-byte aligned, else elements.
+  bool v16 = a.row_bytes % 16 == 0 && aligned(cache_k, 16) && aligned(cache_v, 16) &&
+             aligned(k_new, 16) && aligned(v_new, 16);
+  for (int i = 0; i < 3 && v16; ++i)
+    v16 = a.cks[i] % 16 == 0 && a.cvs[i] % 16 == 0 && a.kns[i] % 16 == 0 && a.vns[i] % 16 == 0;
+  a.vec = v16 ? 16 : eb;
+  return launch_kv_append(a, static_cast<cudaStream_t>(stream_ptr));
 }
 
 GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream_ptr) {
@@ -368,6 +412,17 @@ GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* str
       cudaStreamSynchronize(stream) != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_CUDA;
+  }
+  if (word[0] == kErrKvLength) {
+    // Only a length was out of range: the kernels finished normally.
+    const uint32_t zero = 0;
+    if (cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    return GQA_ERR_KV_LENGTH;
   }
   if (word[0] != 0) {
     // A kernel gave up part-way: its split counters may be off.  Return the

@@ -6,7 +6,7 @@
 // Explained Simply", "Why it matters").  The kernel is built around that
 // bound:
 //
-//  * Work unit = one 64-key tile of one (batch, kv head, head pass).  All units
+//  * Work unit = one 128-key tile of one (batch, kv head, head pass).  All units
 //    of the problem are laid end to end and cut into one contiguous range per
 //    CTA (a persistent grid of one CTA per SM), so every SM streams the same
 //    number of bytes whatever B * Hkv is; a range may start or end inside a
@@ -14,21 +14,26 @@
 //  * A producer warp streams K and V tiles with TMA (128-byte swizzled boxes,
 //    so the ldmatrix reads below are bank-conflict free) into a ring of
 //    shared-memory stages guarded by mbarriers; each tile crosses HBM once.
-//  * Four consumer warps take 16 keys each of every staged tile and serve all
-//    g query heads of the group from it: the kv head is never expanded
+//  * Eight consumer warps (two per SM sub-partition, so that one hides the
+//    other's MMA and shuffle latency) take 16 keys each of every staged
+//    128-key tile and serve all g query heads of the group from it: the kv head is never expanded
 //    ("Multi-Query Attention": a zero stride over the head dimension).  The
 //    dot products run on the tensor cores as S^T = K Q^T with keys in the MMA
 //    M dimension and the group's heads in N (g <= 8 fills one 8-wide column
 //    tile), then O^T += V^T P^T; at g = 8 a CUDA-core version would need about
 //    as many FMA issue slots as the HBM time allows, the MMA needs a few %.
 //  * Online softmax in fp32 with warp-shuffle max/sum reductions; at the end
-//    of a range the four warps merge in shared memory.  A group handled by
+//    of a group the eight warps merge in shared memory.  A group handled by
 //    one CTA is normalised and written straight to `out`.  A group split over
 //    several CTAs leaves one partial (m, l, O) per head and CTA in the
 //    workspace; each contributor then takes a ticket from the group's counter
 //    and the last one merges all partials and writes bf16 `out` (the counters
 //    are zeroed on the stream before the launch).  No CTA ever waits for
 //    another one.
+//  * Per-sequence cache lengths (kv_lens): each CTA reads the B lengths,
+//    counts the tiles every batch entry needs and prefix-sums them in shared
+//    memory, so the units -- and the cut into CTA ranges -- cover only keys
+//    that exist, and the split stays even however ragged the batch is.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,17 +46,18 @@ namespace {
 
 constexpr int KT = kDecodeKeysPerTile;  // keys per tile
 constexpr int NCW = kDecodeConsumerWarps;
+constexpr int kMergeWarps = NCW / 2;    // warps whose states are merged per element
 constexpr int CHUNK_BYTES = KT * 128;   // one 64-wide bf16 column chunk of a tile
 constexpr int kFastMerge = 4;           // split groups merged with all loads in flight
 
-__host__ __device__ inline int64_t range_start(int64_t c, int64_t T, int64_t P) {
-  return (c * T) / P;
+__host__ __device__ inline int range_start(int c, int T, int P) {
+  return static_cast<int>((static_cast<int64_t>(c) * T) / P);
 }
 
 // The CTA whose range [range_start(c), range_start(c + 1)) holds unit u:
 // the largest c with floor(c T / P) <= u, i.e. ceil((u + 1) P / T) - 1.
-__host__ __device__ inline int64_t cta_of_unit(int64_t u, int64_t T, int64_t P) {
-  return ((u + 1) * P + T - 1) / T - 1;
+__host__ __device__ inline int cta_of_unit(int u, int T, int P) {
+  return static_cast<int>(((static_cast<int64_t>(u) + 1) * P + T - 1) / T) - 1;
 }
 
 template <int D, int NT>
@@ -59,14 +65,65 @@ struct DecodeSmem {
   static constexpr int kTileBytes = KT * D * 2;        // K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
   static constexpr int HP = 8 * NT;
-  static constexpr int kScrRow = D + 4;                // padded head row (floats)
-  static constexpr int kScrOBytes = NCW * HP * kScrRow * 4;
-  static constexpr int kScrMLBytes = NCW * HP * 2 * 4;
-  static int bytes(int stages) {
-    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + kScrMLBytes +
-           2 * stages * 8 + 16;
+  static constexpr int kScrRow = D + 4;  // one row's O, then (m, l), padded (floats)
+  static constexpr int kScrOBytes = kMergeWarps * HP * kScrRow * 4;
+  // Ragged launches keep the B lengths and B + 1 prefix sums after the flags.
+  static int bytes(int stages, int ragged_batch) {
+    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + 2 * stages * 8 + 16 +
+           (ragged_batch > 0 ? ((8 * ragged_batch + 4 + 15) / 16) * 16 : 0);
   }
 };
+
+// Unit layout of one launch.  Units run over batch entries, then kv heads,
+// then head passes, then key tiles; every group (one kv head and pass of one
+// batch entry) of entry b has the same number of tiles, so the units of b
+// start at pre[b] (ragged) or b * per_b.
+struct Sched {
+  const int* pre;  // ragged: B + 1 prefix sums (shared memory), else nullptr
+  const int* len;  // ragged: cache length per entry (shared memory), else nullptr
+  int per_b;       // uniform: units per batch entry
+  int gpb;         // groups per batch entry = Hkv * passes
+  int B;
+  int total;       // units of the launch (< 2^31, checked by the planner)
+  int P;           // CTAs that get units: min(grid, total)
+
+  __device__ int batch_of(int u) const {
+    if (pre == nullptr) return u / per_b;
+    int lo = 0, hi = B - 1;  // largest b with pre[b] <= u (pre is strictly increasing)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= u)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    return lo;
+  }
+  __device__ int start_of(int b) const { return pre ? pre[b] : b * per_b; }
+};
+
+// Batch entry of the unit last looked up, with its key range.
+struct Cursor {
+  int b = -1;
+  int beg = 0, end = 0;  // units [beg, end) belong to entry b
+  KeyRange kr{};
+};
+
+__device__ __forceinline__ void seek(Cursor& c, int u, const Sched& sc, const DecodeArgs& a) {
+  if (c.b >= 0 && u >= c.beg && u < c.end) return;
+  c.b = sc.batch_of(u);
+  c.beg = sc.start_of(c.b);
+  c.kr = decode_key_range(sc.len ? sc.len[c.b] : a.Sk, a.Sk, a.Sq, a.causal, a.causal_offset,
+                          a.window);
+  c.end = c.beg + sc.gpb * c.kr.tiles;
+}
+
+// Group of unit u (its index over the whole launch).
+__device__ __forceinline__ int group_of(int u, const Sched& sc, const DecodeArgs& a) {
+  Cursor c;
+  seek(c, u, sc, a);
+  return c.b * sc.gpb + (u - c.beg) / c.kr.tiles;
+}
 
 // MQ: several query positions per kv head (seq_q > 1): the rows of a pass
 // are (head, query) pairs, row r = head * seq_q + query, each with its own
@@ -75,8 +132,8 @@ template <int D, int NT, bool MQ>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a,
-                      const int tiles_per_group, const int passes, const int64_t units,
-                      const int segmax, const int stages, uint32_t* __restrict__ counters) {
+                      const int tiles_per_group, const int passes, const int units,
+                      const int stages, uint32_t* __restrict__ counters) {
   using L = DecodeSmem<D, NT>;
   constexpr int HP = L::HP;
   constexpr int KSTEPS = D / 16;
@@ -87,19 +144,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
   float* scr_o = reinterpret_cast<float*>(ring + stages * L::kStageBytes);
-  float* scr_ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scr_o) + L::kScrOBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scr_ml) +
-                                               L::kScrMLBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scr_o) + L::kScrOBytes);
   uint64_t* empty = full + stages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  uint8_t* tail = reinterpret_cast<uint8_t*>(empty + stages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tail);
   volatile int* last_flag = abort_flag + 1;
+  int* len_s = reinterpret_cast<int*>(tail + 16);
+  int* pre_s = len_s + a.B;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t P = gridDim.x;
-  const int64_t u_begin = range_start(blockIdx.x, units, P);
-  const int64_t u_end = range_start(blockIdx.x + 1, units, P);
+  const bool ragged = a.lens != nullptr;
+  const int gpb = a.Hkv * passes;
 
+  if (ragged) {
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+      int len = a.lens[b];
+      if (len < 0 || len > a.Sk) {
+        if (blockIdx.x == 0) atomicOr(a.err, kErrKvLength);
+        len = len < 0 ? 0 : a.Sk;
+      }
+      len_s[b] = len;
+    }
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
@@ -109,37 +176,73 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  if (ragged) {
+    if (warp == 0) {
+      // pre[b + 1] = sum over entries <= b of (groups per entry) x (tiles of the entry).
+      int carry = 0;
+      for (int b0 = 0; b0 < a.B; b0 += 32) {
+        const int b = b0 + lane;
+        int v = 0;
+        if (b < a.B)
+          v = gpb * decode_key_range(len_s[b], a.Sk, a.Sq, a.causal, a.causal_offset, a.window)
+                        .tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += n;
+        }
+        if (b < a.B) pre_s[b + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) pre_s[0] = 0;
+    }
+    __syncthreads();
+  }
+  Sched sc;
+  sc.pre = ragged ? pre_s : nullptr;
+  sc.len = ragged ? len_s : nullptr;
+  sc.per_b = gpb * tiles_per_group;
+  sc.gpb = gpb;
+  sc.B = a.B;
+  sc.total = ragged ? pre_s[a.B] : units;
+  sc.P = static_cast<int>(gridDim.x) < sc.total ? static_cast<int>(gridDim.x) : sc.total;
+  // CTAs past P (a ragged batch with fewer units than CTAs) get no range; a
+  // split group counts only CTAs that hold some of its units.
+  const bool has_range = static_cast<int>(blockIdx.x) < sc.P;
+  const int u_begin = has_range ? range_start(blockIdx.x, sc.total, sc.P) : 0;
+  const int u_end = has_range ? range_start(blockIdx.x + 1, sc.total, sc.P) : 0;
 
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
-      int64_t it = 0;
-      for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-        const int s = static_cast<int>(it % stages);
+      int it = 0;
+      Cursor cu;
+      for (int u = u_begin; u < u_end; ++u, ++it) {
+        const int s = it % stages;
         const uint32_t round = static_cast<uint32_t>(it / stages);
         if (round > 0 &&
             !mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, a.err, kErrDecodeWait))
           break;
-        const int64_t grp = u / tiles_per_group;
-        const int t = static_cast<int>(u % tiles_per_group);
-        const int64_t bk = grp / passes;  // b * Hkv + kv
-        const int kv = static_cast<int>(bk % a.Hkv);
-        const int b = static_cast<int>(bk / a.Hkv);
+        seek(cu, u, sc, a);
+        const int r = u - cu.beg;
+        const int gi = r / cu.kr.tiles;  // group within the entry: kv * passes + pass
+        const int key0 = (r - gi * cu.kr.tiles + cu.kr.t0) * KT;
+        const int kv = gi / passes;
+        const int b = cu.b;
         uint8_t* st = ring + s * L::kStageBytes;
         mbar_arrive_expect_tx(&full[s], L::kStageBytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
-          tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, (t + a.t0) * KT, kv, b);
-          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64,
-                      (t + a.t0) * KT, kv, b);
+          tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, key0, kv, b);
+          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64, key0, kv, b);
         }
       }
       // Unwind: make sure no copy is still landing in this CTA's shared memory.
       if (*abort_flag) {
-        const int64_t issued = it;
-        for (int64_t j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+        const int issued = it;
+        for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
           mbar_wait_drain(&full[j % stages], static_cast<uint32_t>((j / stages) & 1));
       }
     }
@@ -148,10 +251,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     uint32_t bq[NT][KSTEPS][2];
     float o[NT][KSTEPS][4];
     float m_run[NT][2], l_run[NT][2];
-    int64_t cur = -1;
-    int seg = 0;
+    int cur = -1;                // group being accumulated
+    int cur_beg = 0;             // its first unit
+    int cur_tiles = 1;           // its units
+    int cur_lo = 0, cur_hi = 0, cur_len = 0;  // its key range and cache length
     int b = 0, kv = 0, pass = 0;
     const uint8_t* mrow = nullptr;
+    const int first_grp = u_begin < u_end ? group_of(u_begin, sc, a) : -1;
 
     auto reset_state = [&]() {
 #pragma unroll
@@ -167,7 +273,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
     // Visible keys [vlo, vhi) and mask row of the two rows (columns) this
     // thread's S^T fragments hold in each column tile.
-    int64_t vlo[NT][2], vhi[NT][2];
+    int vlo[NT][2], vhi[NT][2];
     const uint8_t* vmask[NT][2];
 
     auto load_q = [&]() {
@@ -190,26 +296,31 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           if (MQ) {
             const int r = pass * HP + nt * 8 + (lane & 3) * 2 + e;
             const int i = (r < a.rows ? r : 0) % a.Sq;
-            int64_t lo = 0, hi = a.Sk;
+            const int64_t lim = i + a.causal_offset + (cur_len - a.Sk);  // query i's diagonal
+            int64_t lo = 0, hi = cur_len;
             if (a.causal) {
-              hi = i + a.causal_offset + 1 < hi ? i + a.causal_offset + 1 : hi;
-              if (a.window > 0 && i + a.causal_offset - a.window + 1 > 0)
-                lo = i + a.causal_offset - a.window + 1;
+              hi = lim + 1 < hi ? lim + 1 : hi;
+              if (a.window > 0 && lim - a.window + 1 > 0) lo = lim - a.window + 1;
             }
-            vlo[nt][e] = lo;
-            vhi[nt][e] = hi;
+            vlo[nt][e] = static_cast<int>(lo < cur_len ? lo : cur_len);  // within [0, len]
+            vhi[nt][e] = static_cast<int>(hi > 0 ? hi : 0);
             vmask[nt][e] = a.mask ? a.mask + b * a.ms[0] + static_cast<int64_t>(i) * a.ms[1] : nullptr;
           } else {
-            vlo[nt][e] = a.key_lo;
-            vhi[nt][e] = a.key_hi;
+            vlo[nt][e] = cur_lo;
+            vhi[nt][e] = cur_hi;
             vmask[nt][e] = mrow;
           }
         }
       }
     };
 
-    // Merge the four warps' states of the finished range and write one partial.
+    // Merge the eight warps' states of the finished group and write it out
+    // (whole in this CTA) or publish one partial (split).  Warps w and w + 4
+    // hold the same fragment positions of different keys: w + 4 hands its
+    // state over, then the four merged states combine per output element.
+    // The scratch rows keep (m, l) in the padding after the D values.
     auto flush = [&]() {
+      constexpr int R = L::kScrRow;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -220,32 +331,69 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           l += __shfl_xor_sync(0xffffffffu, l, 16);
           l_run[nt][e] = l;
         }
-      float* my_o = scr_o + warp * HP * L::kScrRow;
-      float* my_ml = scr_ml + warp * HP * 2;
+      float* my_rows = scr_o + (warp & 3) * HP * R;
+      auto put_state = [&]() {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt)
+          for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int h = nt * 8 + (lane & 3) * 2 + (c & 1);
-            const int d = mt * 16 + (lane >> 2) + ((c & 2) ? 8 : 0);
-            my_o[h * L::kScrRow + d] = o[nt][mt][c];
-          }
-        if (lane < 4) {
+            for (int c = 0; c < 4; ++c) {
+              const int h = nt * 8 + (lane & 3) * 2 + (c & 1);
+              const int d = mt * 16 + (lane >> 2) + ((c & 2) ? 8 : 0);
+              my_rows[h * R + d] = o[nt][mt][c];
+            }
+          if (lane < 4) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = nt * 8 + lane * 2 + e;
-            my_ml[h * 2 + 0] = m_run[nt][e];
-            my_ml[h * 2 + 1] = l_run[nt][e];
+            for (int e = 0; e < 2; ++e) {
+              const int h = nt * 8 + lane * 2 + e;
+              my_rows[h * R + D] = m_run[nt][e];
+              my_rows[h * R + D + 1] = l_run[nt][e];
+            }
           }
         }
+      };
+      if (warp >= kMergeWarps) put_state();
+      asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      if (warp < kMergeWarps) {
+        float wa[NT][2], wb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = nt * 8 + (lane & 3) * 2 + e;
+            const float mp = my_rows[h * R + D], lp = my_rows[h * R + D + 1];
+            const float M = fmaxf(m_run[nt][e], mp);
+            wa[nt][e] = M == -INFINITY ? 0.f : fast_exp2(m_run[nt][e] - M);
+            wb[nt][e] = M == -INFINITY ? 0.f : fast_exp2(mp - M);
+            l_run[nt][e] = l_run[nt][e] * wa[nt][e] + lp * wb[nt][e];
+            m_run[nt][e] = M;
+          }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int h = nt * 8 + (lane & 3) * 2 + (c & 1);
+              const int d = mt * 16 + (lane >> 2) + ((c & 2) ? 8 : 0);
+              o[nt][mt][c] = o[nt][mt][c] * wa[nt][c & 1] + my_rows[h * R + d] * wb[nt][c & 1];
+            }
+        __syncwarp();
+        put_state();
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
-      // Which CTAs share this group?  Ranges are static, so every CTA can tell.
-      const int64_t g_u0 = cur * tiles_per_group, g_u1 = g_u0 + tiles_per_group;
-      const int64_t c_lo = cta_of_unit(g_u0, units, P);
-      const int64_t c_hi = cta_of_unit(g_u1 - 1, units, P);
+      auto m_of = [&](int w, int h) { return scr_o[(w * HP + h) * R + D]; };
+      auto l_of = [&](int w, int h) { return scr_o[(w * HP + h) * R + D + 1]; };
+      // Which CTAs share this group?  Every CTA computes the same ranges.
+      const int c_lo = cta_of_unit(cur_beg, sc.total, sc.P);
+      const int c_hi = cta_of_unit(cur_beg + cur_tiles - 1, sc.total, sc.P);
+      // Partial slot of CTA cc for this group: only a range's first and last
+      // groups can be split, so two slots per CTA suffice.
+      auto slot_of = [&](int cc) -> int {
+        const int first = group_of(range_start(cc, sc.total, sc.P), sc, a);
+        return (cc * 2 + (first == cur ? 0 : 1)) * HP;
+      };
       // Output row of row hr of this pass (a head, or a (head, query) pair).
       auto out_row = [&](int hr) -> uint16_t* {
         const int r = pass * HP + hr;
@@ -255,23 +403,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                static_cast<int64_t>(qi) * a.os[2];
       };
       if (c_lo == c_hi) {
-        // The whole group is in this CTA: normalise and write out.
-        for (int idx = threadIdx.x; idx < HP * D; idx += NCW * 32) {
-          const int h = idx / D, d = idx % D;
+        // The whole group is in this CTA: normalise and write out, two
+        // elements per thread.
+        for (int idx = threadIdx.x; idx < HP * D / 2; idx += NCW * 32) {
+          const int h = idx / (D / 2), d = (idx % (D / 2)) * 2;
           if (pass * HP + h >= a.rows) continue;
           float M = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
-          float l = 0.f, acc = 0.f;
+          for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, m_of(w, h));
+          float l = 0.f, acc0 = 0.f, acc1 = 0.f;
           if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < NCW; ++w) {
-              const float sc = fast_exp2(scr_ml[(w * HP + h) * 2] - M);
-              l += sc * scr_ml[(w * HP + h) * 2 + 1];
-              acc += sc * scr_o[(w * HP + h) * L::kScrRow + d];
+            for (int w = 0; w < kMergeWarps; ++w) {
+              const float sc = fast_exp2(m_of(w, h) - M);
+              l += sc * l_of(w, h);
+              const float2 ov = *reinterpret_cast<const float2*>(&scr_o[(w * HP + h) * R + d]);
+              acc0 += sc * ov.x;
+              acc1 += sc * ov.y;
             }
           }
-          out_row(h)[d] = bf16_bits_rn(acc / l);  // l == 0: NaN
+          const float inv = 1.f / l;  // l == 0: NaN
+          *reinterpret_cast<uint32_t*>(out_row(h) + d) = pack_bf16x2(acc0 * inv, acc1 * inv);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
         return;
@@ -280,24 +432,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // ticket: the CTA barrier orders every thread's stores before thread
       // 0's gpu-scope fence and atomic (release), and thread 0's fence after
       // the atomic orders the reads of the others' partials (acquire).
-      const int64_t slot = (static_cast<int64_t>(blockIdx.x) * segmax + seg) * HP;
+      const int slot = (static_cast<int>(blockIdx.x) * 2 + (cur == first_grp ? 0 : 1)) * HP;
       for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
         const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NCW; ++w) M = fmaxf(M, scr_ml[(w * HP + h) * 2]);
+        for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, m_of(w, h));
         float l = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY) {
 #pragma unroll
-          for (int w = 0; w < NCW; ++w) {
-            const float sc = fast_exp2(scr_ml[(w * HP + h) * 2] - M);
-            l += sc * scr_ml[(w * HP + h) * 2 + 1];
-            const float* src = scr_o + (w * HP + h) * L::kScrRow + d;
-            acc.x += sc * src[0];
-            acc.y += sc * src[1];
-            acc.z += sc * src[2];
-            acc.w += sc * src[3];
+          for (int w = 0; w < kMergeWarps; ++w) {
+            const float sc = fast_exp2(m_of(w, h) - M);
+            l += sc * l_of(w, h);
+            const float4 ov = *reinterpret_cast<const float4*>(&scr_o[(w * HP + h) * R + d]);
+            acc.x += sc * ov.x;
+            acc.y += sc * ov.y;
+            acc.z += sc * ov.z;
+            acc.w += sc * ov.w;
           }
         }
         *reinterpret_cast<float4*>(&a.part_o[(slot + h) * D + d]) = acc;
@@ -317,22 +469,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int n = static_cast<int>(c_hi - c_lo + 1);
         if (n <= kFastMerge) {
           // Few contributors: every load of a thread's elements in flight at once.
-          int64_t base[kFastMerge];
+          int base[kFastMerge];
 #pragma unroll
-          for (int k = 0; k < kFastMerge; ++k) {
-            const int64_t cc = c_lo + (k < n ? k : 0);
-            base[k] = (cc * segmax + (cur - range_start(cc, units, P) / tiles_per_group)) * HP;
-          }
+          for (int k = 0; k < kFastMerge; ++k) base[k] = slot_of(c_lo + (k < n ? k : 0));
           for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
             const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
             if (pass * HP + h >= a.rows) continue;
             float2 ml[kFastMerge];
-            float4 o[kFastMerge];
+            float4 ov[kFastMerge];
 #pragma unroll
             for (int k = 0; k < kFastMerge; ++k) {
               if (k < n) {
                 ml[k] = __ldcg(&a.part_ml[base[k] + h]);
-                o[k] = __ldcg(reinterpret_cast<const float4*>(&a.part_o[(base[k] + h) * D + d]));
+                ov[k] = __ldcg(reinterpret_cast<const float4*>(&a.part_o[(base[k] + h) * D + d]));
               }
             }
             float M = -INFINITY;
@@ -347,10 +496,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 if (k < n) {
                   const float w = fast_exp2(ml[k].x - M);
                   Lsum += w * ml[k].y;
-                  acc.x += w * o[k].x;
-                  acc.y += w * o[k].y;
-                  acc.z += w * o[k].z;
-                  acc.w += w * o[k].w;
+                  acc.x += w * ov[k].x;
+                  acc.y += w * ov[k].y;
+                  acc.z += w * ov[k].z;
+                  acc.w += w * ov[k].w;
                 }
               }
             }
@@ -361,81 +510,85 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
           }
         } else {
-        // Many contributors: stage each one's segment index and each head's
-        // merged (max, sum) in shared memory, then accumulate O with 16-byte
-        // loads, several contributors in flight at once.
-        int* sm_seg = reinterpret_cast<int*>(scr_o);          // n ints (scr_o is free now)
-        float* sm_ml = scr_ml;                                 // HP x (M, L)
-        for (int k = threadIdx.x; k < n; k += NCW * 32)
-          sm_seg[k] = static_cast<int>(cur - range_start(c_lo + k, units, P) / tiles_per_group);
-        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
-        if (threadIdx.x < HP) {
-          const int h = threadIdx.x;
-          float M = -INFINITY;
+          // Many contributors: stage each one's slot and each row's merged
+          // (max, sum) in shared memory (the scratch rows are free now), then
+          // accumulate O with 16-byte loads.
+          int* sm_slot = reinterpret_cast<int*>(scr_o);
+          float* sm_ml = scr_o + kMergeWarps * HP * R / 2;  // HP x (M, L), past the slots
+          for (int k = threadIdx.x; k < n; k += NCW * 32)
+            sm_slot[k] = slot_of(c_lo + k);
+          asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+          if (threadIdx.x < HP) {
+            const int h = threadIdx.x;
+            float M = -INFINITY;
 #pragma unroll 4
-          for (int k = 0; k < n; ++k)
-            M = fmaxf(M, __ldcg(&a.part_ml[((c_lo + k) * segmax + sm_seg[k]) * HP + h]).x);
-          float Lsum = 0.f;
-          if (M != -INFINITY) {
+            for (int k = 0; k < n; ++k) M = fmaxf(M, __ldcg(&a.part_ml[sm_slot[k] + h]).x);
+            float Lsum = 0.f;
+            if (M != -INFINITY) {
 #pragma unroll 4
-            for (int k = 0; k < n; ++k) {
-              const float2 ml = __ldcg(&a.part_ml[((c_lo + k) * segmax + sm_seg[k]) * HP + h]);
-              Lsum += fast_exp2(ml.x - M) * ml.y;
+              for (int k = 0; k < n; ++k) {
+                const float2 ml = __ldcg(&a.part_ml[sm_slot[k] + h]);
+                Lsum += fast_exp2(ml.x - M) * ml.y;
+              }
             }
+            sm_ml[2 * h] = M;
+            sm_ml[2 * h + 1] = Lsum;
           }
-          sm_ml[2 * h] = M;
-          sm_ml[2 * h + 1] = Lsum;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
-        for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
-          const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
-          if (pass * HP + h >= a.rows) continue;
-          const float M = sm_ml[2 * h], Lsum = sm_ml[2 * h + 1];
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (M != -INFINITY) {
+          asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+          for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
+            const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
+            if (pass * HP + h >= a.rows) continue;
+            const float M = sm_ml[2 * h], Lsum = sm_ml[2 * h + 1];
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (M != -INFINITY) {
 #pragma unroll 4
-            for (int k = 0; k < n; ++k) {
-              const int64_t sl = ((c_lo + k) * segmax + sm_seg[k]) * HP + h;
-              const float w = fast_exp2(__ldcg(&a.part_ml[sl]).x - M);
-              const float4 o = __ldcg(reinterpret_cast<const float4*>(&a.part_o[sl * D + d]));
-              acc.x += w * o.x;
-              acc.y += w * o.y;
-              acc.z += w * o.z;
-              acc.w += w * o.w;
+              for (int k = 0; k < n; ++k) {
+                const int sl = sm_slot[k] + h;
+                const float w = fast_exp2(__ldcg(&a.part_ml[sl]).x - M);
+                const float4 ov = __ldcg(reinterpret_cast<const float4*>(&a.part_o[sl * D + d]));
+                acc.x += w * ov.x;
+                acc.y += w * ov.y;
+                acc.z += w * ov.z;
+                acc.w += w * ov.w;
+              }
             }
+            const float inv = 1.f / Lsum;  // Lsum == 0: NaN
+            uint2 pk;
+            pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+            pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
           }
-          const float inv = 1.f / Lsum;  // Lsum == 0: NaN
-          uint2 pk;
-          pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-          pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
-        }
         }
         if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
     };
 
-    int64_t it = 0;
+    int it = 0;
     bool ok = true;
-    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-      const int64_t grp = u / tiles_per_group;
-      const int t = static_cast<int>(u % tiles_per_group);
+    Cursor cu;
+    for (int u = u_begin; u < u_end; ++u, ++it) {
+      seek(cu, u, sc, a);
+      const int r = u - cu.beg;
+      const int gi = r / cu.kr.tiles;
+      const int grp = cu.b * gpb + gi;
+      const int tile = r - gi * cu.kr.tiles + cu.kr.t0;
       if (grp != cur) {
-        if (cur >= 0) {
-          flush();
-          ++seg;
-        }
+        if (cur >= 0) flush();
         cur = grp;
-        const int64_t bk = grp / passes;
-        pass = static_cast<int>(grp % passes);
-        kv = static_cast<int>(bk % a.Hkv);
-        b = static_cast<int>(bk / a.Hkv);
+        cur_beg = cu.beg + gi * cu.kr.tiles;
+        cur_tiles = cu.kr.tiles;
+        cur_lo = cu.kr.lo;
+        cur_hi = cu.kr.hi;
+        cur_len = sc.len ? sc.len[cu.b] : a.Sk;
+        pass = gi % passes;
+        kv = gi / passes;
+        b = cu.b;
         mrow = a.mask ? a.mask + b * a.ms[0] : nullptr;
         load_q();
         reset_state();
       }
-      const int s = static_cast<int>(it % stages);
+      const int s = it % stages;
       const uint32_t round = static_cast<uint32_t>(it / stages);
       if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
         ok = false;
@@ -444,12 +597,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const uint32_t kbase = smem_u32(ring + s * L::kStageBytes);
       const uint32_t vbase = kbase + L::kTileBytes;
 
-      // S^T[16 keys x 8 heads] = K[16 x D] Q^T[D x 8] per column tile.
-      float sc[NT][4];
+      // S^T[16 keys x 8 heads] = K[16 x D] Q^T[D x 8] per column tile.  With
+      // one column tile, even and odd k-steps go to two accumulators (half the
+      // dependent MMA chain); two column tiles already interleave two chains.
+      constexpr bool kSplit = NT == 1;
+      float sc[NT][4], sc2[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
+        for (int c = 0; c < 4; ++c) sc[nt][c] = sc2[nt][c] = 0.f;
       {
         const int mi = lane >> 3;
         const int r = warp * 16 + (mi & 1) * 8 + (lane & 7);
@@ -462,14 +618,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           ldmatrix_x4(a0, a1, a2, a3, addr);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(sc[nt], a0, a1, a2, a3, bq[nt][ks][0], bq[nt][ks][1]);
+            mma_bf16_16816((kSplit && (ks & 1)) ? sc2[nt] : sc[nt], a0, a1, a2, a3,
+                           bq[nt][ks][0], bq[nt][ks][1]);
+        }
+        if (kSplit) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sc[nt][c] += sc2[nt][c];
         }
       }
 
       // Visibility of this thread's two keys for its rows.
-      const int64_t key0 = static_cast<int64_t>(t + a.t0) * KT + warp * 16 + (lane >> 2);
-      const int64_t key1 = key0 + 8;
-      auto vis = [&](int64_t key, int nt, int e) -> bool {
+      const int key0 = tile * KT + warp * 16 + (lane >> 2);
+      const int key1 = key0 + 8;
+      auto vis = [&](int key, int nt, int e) -> bool {
         return key >= vlo[nt][e] && key < vhi[nt][e] && mask_allows(vmask[nt][e], key);
       };
 
@@ -545,8 +708,8 @@ int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap
       cudaSuccess)
     return GQA_ERR_CUDA;
   kern<<<s.grid, kDecodeThreads, s.smem_bytes, stream>>>(tmk, tmv, a, s.tiles_per_group,
-                                                          s.passes, s.units, s.segmax, s.stages,
-                                                          a.counters);
+                                                          s.passes, static_cast<int>(s.units),
+                                                          s.stages, a.counters);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -560,43 +723,65 @@ DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
   s.NT = rows <= 8 ? 1 : 2;
   s.HP = 8 * s.NT;
   s.passes = static_cast<int>((rows + s.HP - 1) / s.HP);
-  // Keys some query can see: [key_lo, key_hi) (query 0's lower limit, the
-  // last query's upper limit).
-  s.key_hi = p.seq_k;
-  s.key_lo = 0;
-  if (p.causal) {
-    if (p.seq_q - 1 + p.causal_offset + 1 < s.key_hi) s.key_hi = p.seq_q + p.causal_offset;
-    if (p.window > 0 && p.causal_offset - p.window + 1 > 0) s.key_lo = p.causal_offset - p.window + 1;
-  }
-  s.t0 = static_cast<int>(s.key_lo / KT);
-  s.tiles_per_group = static_cast<int>((s.key_hi + KT - 1) / KT) - s.t0;
+  s.ragged = p.kv_lens != nullptr;
+  // Without kv_lens every group streams the same tiles; with them a group
+  // needs at most the tiles of the whole capacity.
+  s.tiles_per_group =
+      s.ragged ? static_cast<int>((p.seq_k + KT - 1) / KT)
+               : decode_key_range(p.seq_k, p.seq_k, p.seq_q, p.causal, p.causal_offset, p.window)
+                     .tiles;
   if (s.tiles_per_group < 1) s.tiles_per_group = 1;
   s.groups = p.batch * p.heads_kv * s.passes;
   s.units = s.groups * s.tiles_per_group;
   s.grid = static_cast<int>(s.units < sm_count ? s.units : sm_count);
   if (s.grid < 1) s.grid = 1;
-  const int64_t per_cta = (s.units + s.grid - 1) / s.grid;
-  s.segmax = static_cast<int>((per_cta + s.tiles_per_group - 1) / s.tiles_per_group + 1);
-  const int stage_bytes = 2 * KT * s.D * 2;
-  if (s.D == 128)
-    s.stages = s.NT == 1 ? 6 : 5;
-  else
-    s.stages = 8;
-  if (s.D == 128 && s.NT == 1)
-    s.smem_bytes = DecodeSmem<128, 1>::bytes(s.stages);
-  else if (s.D == 128)
-    s.smem_bytes = DecodeSmem<128, 2>::bytes(s.stages);
-  else if (s.NT == 1)
-    s.smem_bytes = DecodeSmem<64, 1>::bytes(s.stages);
-  else
-    s.smem_bytes = DecodeSmem<64, 2>::bytes(s.stages);
-  (void)stage_bytes;
-  const int64_t slots = static_cast<int64_t>(s.grid) * s.segmax * s.HP;
+  const int rb = s.ragged ? static_cast<int>(p.batch) : 0;
+  s.stages = s.D == 128 ? 3 : 6;  // 192 KB of K/V in flight per SM
+  for (;; --s.stages) {
+    if (s.D == 128 && s.NT == 1)
+      s.smem_bytes = DecodeSmem<128, 1>::bytes(s.stages, rb);
+    else if (s.D == 128)
+      s.smem_bytes = DecodeSmem<128, 2>::bytes(s.stages, rb);
+    else if (s.NT == 1)
+      s.smem_bytes = DecodeSmem<64, 1>::bytes(s.stages, rb);
+    else
+      s.smem_bytes = DecodeSmem<64, 2>::bytes(s.stages, rb);
+    if (s.smem_bytes <= kDecodeMaxSmem || s.stages <= 2) break;
+  }
+  // Two partial slots per CTA: its first and its last group.
+  const int64_t slots = static_cast<int64_t>(s.grid) * 2 * s.HP;
   s.counters_offset = 256;
   s.part_ml_offset = s.counters_offset + ((s.groups * 4 + 255) / 256) * 256;
   s.part_o_offset = s.part_ml_offset + ((slots * 8 + 255) / 256) * 256;
   s.part_bytes = (s.part_o_offset - 256) + slots * s.D * 4;
   return s;
+}
+
+DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const void* q,
+                            const uint8_t* mask, void* out, uint8_t* ws) {
+  DecodeArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  for (int d = 0; d < 4; ++d) a.qs[d] = p.q_stride[d], a.os[d] = p.o_stride[d];
+  a.mask = p.has_mask ? mask : nullptr;
+  for (int d = 0; d < 3; ++d) a.ms[d] = p.mask_stride[d];
+  a.out = static_cast<uint16_t*>(out);
+  a.part_ml = reinterpret_cast<float2*>(ws + s.part_ml_offset);
+  a.part_o = reinterpret_cast<float*>(ws + s.part_o_offset);
+  a.counters = reinterpret_cast<uint32_t*>(ws + s.counters_offset);
+  a.err = reinterpret_cast<uint32_t*>(ws);
+  a.lens = p.kv_lens;
+  a.B = static_cast<int>(p.batch);
+  a.Hq = static_cast<int>(p.heads_q);
+  a.Hkv = static_cast<int>(p.heads_kv);
+  a.Sk = static_cast<int>(p.seq_k);
+  a.g = static_cast<int>(p.heads_q / p.heads_kv);
+  a.Sq = static_cast<int>(p.seq_q);
+  a.rows = static_cast<int>(a.g * p.seq_q);
+  a.causal = p.causal;
+  a.causal_offset = p.causal_offset;
+  a.window = p.window;
+  a.scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634073599);
+  return a;
 }
 
 int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,

@@ -98,29 +98,6 @@ extern "C" GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const vo
   erc = encode_decode_kv_map(&tmv, v, *p, p->v_stride);
   if (erc != GQA_OK) return erc;
 
-  DecodeArgs a{};
-  a.q = static_cast<const uint16_t*>(q);
-  for (int d = 0; d < 4; ++d) a.qs[d] = p->q_stride[d], a.os[d] = p->o_stride[d];
-  a.mask = p->has_mask ? mask : nullptr;
-  for (int d = 0; d < 3; ++d) a.ms[d] = p->mask_stride[d];
-  a.out = static_cast<uint16_t*>(out);
-  a.part_ml = reinterpret_cast<float2*>(ws + s.part_ml_offset);
-  a.part_o = reinterpret_cast<float*>(ws + s.part_o_offset);
-  a.counters = reinterpret_cast<uint32_t*>(ws + s.counters_offset);
-  a.err = reinterpret_cast<uint32_t*>(ws);
-  a.B = static_cast<int>(p->batch);
-  a.Hq = static_cast<int>(p->heads_q);
-  a.Hkv = static_cast<int>(p->heads_kv);
-  a.Sk = static_cast<int>(p->seq_k);
-  a.g = static_cast<int>(p->heads_q / p->heads_kv);
-  a.Sq = static_cast<int>(p->seq_q);
-  a.rows = static_cast<int>(a.g * p->seq_q);
-  a.causal = p->causal;
-  a.causal_offset = p->causal_offset;
-  a.window = p->window;
-  a.t0 = s.t0;
-  a.key_lo = s.key_lo;
-  a.key_hi = s.key_hi;
-  a.scale_log2 = static_cast<float>(static_cast<double>(p->scale) * 1.4426950408889634073599);
+  const DecodeArgs a = make_decode_args(*p, s, q, mask, out, ws);
   return launch_decode(*p, s, a, tmk, tmv, stream);
 }

@@ -11,25 +11,57 @@ namespace gqa {
 
 // ------------------------------------------------------------ decode
 // Keys per streamed tile and consumer warps per CTA of the decode kernel.
-constexpr int kDecodeKeysPerTile = 64;
-constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeKeysPerTile = 128;
+constexpr int kDecodeConsumerWarps = 8;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kDecodeMaxRowsPerPass = 16;  // (head, query) rows in the MMA N dimension
+constexpr int kDecodeMaxSmem = 227 * 1024;  // dynamic shared memory one CTA may take
+constexpr int64_t kMaxRaggedBatch = 16384;  // batch entries with per-sequence lengths
+
+// Keys [lo, hi) of one batch entry that some query of the block can see,
+// and the decode key tiles [t0, t0 + tiles) that hold them.  `len` is the entry's
+// cache length (seq_k without per-sequence lengths); the causal diagonal
+// moves with it by len - seq_k.  A range with no visible key still gets one
+// tile, streamed fully hidden, so that its rows come out NaN.
+struct KeyRange {
+  int lo, hi;
+  int t0, tiles;
+};
+
+__host__ __device__ inline KeyRange decode_key_range(int64_t len, int64_t Sk, int64_t Sq,
+                                                     int causal, int64_t off, int64_t window) {
+  const int64_t shift = len - Sk;
+  int64_t lo = 0, hi = len;
+  if (causal) {
+    if (Sq + off + shift < hi) hi = Sq + off + shift;  // last query: j <= Sq - 1 + off + shift
+    if (window > 0 && off + shift - window + 1 > 0) lo = off + shift - window + 1;  // query 0
+  }
+  KeyRange r;
+  if (hi <= lo) {
+    r.lo = r.hi = 0;
+    r.t0 = 0;
+    r.tiles = 1;
+  } else {  // 0 <= lo < hi <= len <= Sk < 2^31
+    r.lo = static_cast<int>(lo);
+    r.hi = static_cast<int>(hi);
+    r.t0 = r.lo / kDecodeKeysPerTile;
+    r.tiles = (r.hi + kDecodeKeysPerTile - 1) / kDecodeKeysPerTile - r.t0;
+  }
+  return r;
+}
 
 struct DecodeShape {
   int D;            // 64 or 128
   int NT;           // 8-head MMA column tiles per pass (1 or 2)
   int HP;           // rows per pass = 8 * NT (a row: one head, or one (head, query))
   int passes;       // ceil(g * seq_q / HP)
-  int tiles_per_group;
-  int t0;           // first 64-key tile any query can see (window)
-  int64_t key_lo, key_hi;  // keys [key_lo, key_hi) pass the causal / window rules
+  int tiles_per_group;  // without kv_lens; with them, the most any group can need
   int64_t groups;   // batch * heads_kv * passes
-  int64_t units;    // groups * tiles_per_group
+  int64_t units;    // groups * tiles_per_group (an upper bound with kv_lens)
   int grid;         // CTAs (<= units)
-  int segmax;       // partial segments per CTA
   int stages;       // shared-memory ring depth
   int smem_bytes;
+  bool ragged;      // per-sequence kv_lens: the partition is computed on the device
   int64_t counters_offset, part_o_offset, part_ml_offset, part_bytes;
 };
 
@@ -46,14 +78,18 @@ struct DecodeArgs {
   float2* part_ml;
   uint32_t* counters;  // one ticket counter per group; zeroed before each launch
   uint32_t* err;
+  const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
   int B, Hq, Hkv, Sk, g;
   int Sq, rows;            // queries per kv head; rows = g * Sq
   int causal;
   int64_t causal_offset, window;
-  int t0;                  // tile offset of the streamed key range
-  int64_t key_lo, key_hi;  // keys outside [key_lo, key_hi) are hidden (causal / window)
   float scale_log2;  // scale * log2(e)
 };
+
+// Arguments of one decode launch; the workspace `ws` holds the error word at
+// offset 0 and the plan's counters and partials.
+DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const void* q,
+                            const uint8_t* mask, void* out, uint8_t* ws);
 
 int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
                   const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream);
@@ -86,6 +122,7 @@ struct PrefillArgs {
   int64_t os[4];
   uint8_t* summary;  // [B][m_tiles][n_tiles]: 0 all hidden, 1 mixed, 2 all visible
   uint32_t* err;
+  const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
   int B, Hq, Hkv, Sq, Sk, g;
   int causal, has_mask;
   int64_t causal_offset, window;
@@ -98,7 +135,25 @@ int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArg
 
 // ------------------------------------------------------------ fp32 path
 int launch_f32(const gqa_problem& p, const float* q, const float* k, const float* v,
-               const uint8_t* mask, float* out, cudaStream_t stream);
+               const uint8_t* mask, float* out, uint32_t* err, cudaStream_t stream);
+
+// ------------------------------------------------------------ KV-cache append
+struct AppendArgs {
+  uint8_t* ck;          // cache_k, cache_v (bytes)
+  uint8_t* cv;
+  const uint8_t* kn;    // k_new, v_new (bytes)
+  const uint8_t* vn;
+  int32_t* lens;        // read, then advanced by n_new by the last CTA
+  uint32_t* err;
+  uint32_t* ticket;     // CTAs done; zero between launches
+  int64_t cks[3], cvs[3], kns[3], vns[3];  // byte strides over (b, h, row)
+  int B, H;
+  int64_t cap, n_new;
+  int row_bytes;        // head_dim * element bytes
+  int vec;              // bytes per copied vector: 16, 4 or 2
+};
+
+int launch_kv_append(const AppendArgs& a, cudaStream_t stream);
 
 // ------------------------------------------------------------ fill: zeros (seq_k == 0) or NaN
 int launch_zero(const gqa_problem& p, void* out, cudaStream_t stream, bool nan);

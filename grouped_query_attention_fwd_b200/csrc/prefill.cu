@@ -100,7 +100,13 @@ __device__ __forceinline__ int64_t imax64(int64_t x, int64_t y) { return x > y ?
 
 struct Pair {
   int b, kv, mt0, nt_beg, nt_end;
+  int len;  // cache length of entry b (seq_k without per-sequence lengths)
 };
+
+// Causal offset of the pair's entry: the diagonal moves with its length.
+__device__ __forceinline__ int64_t pair_off(const PrefillArgs& a, const Pair& pr) {
+  return a.causal_offset + (static_cast<int64_t>(pr.len) - a.Sk);
+}
 
 struct Slot {  // one query tile of a pair
   int mt, q0, q_last;
@@ -118,11 +124,11 @@ __device__ __forceinline__ Slot slot_of(const Pair& pr, int s, const PrefillArgs
   sl.q0 = sl.mt * qpt;
   sl.q_last = sl.live ? min(sl.q0 + qpt, a.Sq) - 1 : -1;
   sl.key_lo = 0;
-  sl.key_hi = a.Sk;
+  sl.key_hi = pr.len;
   if (a.causal) {
-    sl.key_hi = imin64(a.Sk, static_cast<int64_t>(sl.q_last) + a.causal_offset + 1);
-    if (a.window > 0)
-      sl.key_lo = imax64(0, static_cast<int64_t>(sl.q0) + a.causal_offset - a.window + 1);
+    const int64_t off = pair_off(a, pr);
+    sl.key_hi = imin64(pr.len, static_cast<int64_t>(sl.q_last) + off + 1);
+    if (a.window > 0) sl.key_lo = imax64(0, static_cast<int64_t>(sl.q0) + off - a.window + 1);
   }
   if (!sl.live || sl.key_hi <= sl.key_lo) sl.key_lo = sl.key_hi = 0;
   return sl;
@@ -145,9 +151,14 @@ __device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_t
   pr.b = bk / a.Hkv;
   pr.kv = bk % a.Hkv;
   pr.mt0 = 2 * p;
+  pr.len = a.Sk;
+  if (a.lens != nullptr) {  // out-of-range lengths are clamped (and reported at kernel start)
+    const int len = a.lens[pr.b];
+    pr.len = len < 0 ? 0 : (len > a.Sk ? a.Sk : len);
+  }
   const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
   // Key tiles either slot can see.
-  int64_t lo = a.Sk, hi = 0;
+  int64_t lo = pr.len, hi = 0;
   if (s0.key_hi > s0.key_lo) { lo = imin64(lo, s0.key_lo); hi = imax64(hi, s0.key_hi); }
   if (s1.key_hi > s1.key_lo) { lo = imin64(lo, s1.key_lo); hi = imax64(hi, s1.key_hi); }
   if (hi <= lo) {
@@ -167,13 +178,13 @@ __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, 
   const int64_t j0 = static_cast<int64_t>(nt) * BN, j1 = j0 + BN - 1;
   if (j1 < sl.key_lo || j0 >= sl.key_hi) return 0;
   int cls = 2;
-  if (j1 >= a.Sk) cls = 1;
+  if (j1 >= pr.len) cls = 1;
   if (a.causal) {
     // Every row sees the whole tile iff the first row's upper limit and the
     // last row's lower limit (window) both enclose it.
-    if (j1 > static_cast<int64_t>(sl.q0) + a.causal_offset) cls = 1;
-    if (a.window > 0 && j0 <= static_cast<int64_t>(sl.q_last) + a.causal_offset - a.window)
-      cls = 1;
+    const int64_t off = pair_off(a, pr);
+    if (j1 > static_cast<int64_t>(sl.q0) + off) cls = 1;
+    if (a.window > 0 && j0 <= static_cast<int64_t>(sl.q_last) + off - a.window) cls = 1;
   }
   if (a.has_mask) {
     const int c = a.summary[(static_cast<int64_t>(pr.b) * m_tiles + sl.mt) * n_tiles + nt];
@@ -184,15 +195,17 @@ __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, 
 }
 
 // Visibility of keys j0 .. j0+127 for query q, one bit per key: inside the
-// sequence (j < Sk), within the causal limit (j <= q + causal_offset) and the
-// window (j > q + causal_offset - window), and allowed by the mask row
-// (nonzero byte), which is read as 16-byte vectors when aligned.
+// entry's cache (j < len), within the causal limit (j <= q + off) and the
+// window (j > q + off - window), and allowed by the mask row (nonzero byte),
+// which is read as 16-byte vectors when aligned.
 __device__ __forceinline__ void visible_bits(uint32_t (&vb)[4], const uint8_t* mrow, int j0,
-                                             const PrefillArgs& a, int q, bool vec) {
-  int64_t hi = a.Sk, lo = 0;  // keys [lo, hi) pass causal and window
+                                             const PrefillArgs& a, const Pair& pr, int q,
+                                             bool vec) {
+  int64_t hi = pr.len, lo = 0;  // keys [lo, hi) pass the length, causal and window rules
   if (a.causal) {
-    hi = imin64(hi, static_cast<int64_t>(q) + a.causal_offset + 1);
-    if (a.window > 0) lo = static_cast<int64_t>(q) + a.causal_offset - a.window + 1;
+    const int64_t off = pair_off(a, pr);
+    hi = imin64(hi, static_cast<int64_t>(q) + off + 1);
+    if (a.window > 0) lo = static_cast<int64_t>(q) + off - a.window + 1;
   }
   const int n = static_cast<int>(imax64(0, imin64(BN, hi - j0)));
   const int n0 = static_cast<int>(imax64(0, imin64(n, lo - j0)));
@@ -288,6 +301,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (a.lens != nullptr && blockIdx.x == 0) {
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+      const int len = a.lens[b];
+      if (len < 0 || len > a.Sk) atomicOr(a.err, kErrKvLength);
+    }
   }
   // Rows past qpt * g of a query tile are never written by TMA: zero them once.
   if (rows < BM && threadIdx.x < BM) {
@@ -548,7 +567,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const bool fast = (cls == 2) && (a.scale_log2 >= 0.f);
         uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};
         if (!fast)
-          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a, q, mask_vec);
+          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a, pr, q, mask_vec);
         auto masked_t = [&](float sv, int c) -> float {
           return ((vb[c >> 5] >> (c & 31)) & 1u) ? sv * a.scale_log2 : -INFINITY;
         };

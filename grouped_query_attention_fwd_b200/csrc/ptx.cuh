@@ -91,6 +91,7 @@ enum : uint32_t {
   kErrDecodeWait = 1u << 0,
   kErrPrefillWait = 1u << 1,
   kErrBadArgs = 1u << 2,
+  kErrKvLength = 1u << 3,  // a kv_lens entry outside [0, capacity]: clamped, result undefined
 };
 
 // Bounded wait on `bar` reaching phase `parity`.  Returns false if the limit

@@ -9,6 +9,7 @@
 
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace gqa {
 namespace {
@@ -22,7 +23,8 @@ __global__ void __launch_bounds__(256)
                    int64_t Sk, int64_t D, int64_t qs0, int64_t qs1, int64_t qs2, int64_t ks0,
                    int64_t ks1, int64_t ks2, int64_t vs0, int64_t vs1, int64_t vs2, int64_t os0,
                    int64_t os1, int64_t os2, int64_t ms0, int64_t ms1, int causal,
-                   int64_t causal_offset, int64_t window, float scale_log2) {
+                   int64_t causal_offset, int64_t window, const int32_t* __restrict__ lens,
+                   uint32_t* __restrict__ err, float scale_log2) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= B * Hq * Sq) return;
@@ -45,11 +47,21 @@ __global__ void __launch_bounds__(256)
     acc[e] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  // Keys [jbeg, jend) pass the causal and window rules; the mask is per key.
-  int64_t jend = Sk, jbeg = 0;
+  // Entry b holds len keys; its diagonal sits at i + off.
+  int64_t len = Sk;
+  if (lens != nullptr) {
+    len = lens[b];
+    if (len < 0 || len > Sk) {
+      if (h == 0 && i == 0 && lane == 0) atomicOr(err, kErrKvLength);
+      len = len < 0 ? 0 : Sk;
+    }
+  }
+  const int64_t off = causal_offset + (len - Sk);
+  // Keys [jbeg, jend) pass the length, causal and window rules; the mask is per key.
+  int64_t jend = len, jbeg = 0;
   if (causal) {
-    jend = i + causal_offset + 1 < Sk ? i + causal_offset + 1 : Sk;
-    if (window > 0 && i + causal_offset - window + 1 > 0) jbeg = i + causal_offset - window + 1;
+    jend = i + off + 1 < len ? i + off + 1 : len;
+    if (window > 0 && i + off - window + 1 > 0) jbeg = i + off - window + 1;
   }
   for (int64_t j = jbeg; j < jend; ++j) {
     if (mrow != nullptr && mrow[j] == 0) continue;
@@ -103,7 +115,7 @@ __global__ void gqa_fill_kernel(uint8_t* out, int64_t B, int64_t Hq, int64_t Sq,
 }  // namespace
 
 int launch_f32(const gqa_problem& p, const float* q, const float* k, const float* v,
-               const uint8_t* mask, float* out, cudaStream_t stream) {
+               const uint8_t* mask, float* out, uint32_t* err, cudaStream_t stream) {
   const int64_t rows = p.batch * p.heads_q * p.seq_q;
   const int warps_per_block = 8;
   const int64_t blocks = (rows + warps_per_block - 1) / warps_per_block;
@@ -114,7 +126,7 @@ int launch_f32(const gqa_problem& p, const float* q, const float* k, const float
       p.seq_k, p.head_dim, p.q_stride[0], p.q_stride[1], p.q_stride[2], p.k_stride[0],
       p.k_stride[1], p.k_stride[2], p.v_stride[0], p.v_stride[1], p.v_stride[2], p.o_stride[0],
       p.o_stride[1], p.o_stride[2], p.mask_stride[0], p.mask_stride[1], p.causal,
-      p.causal_offset, p.window, scale_log2);
+      p.causal_offset, p.window, p.kv_lens, err, scale_log2);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

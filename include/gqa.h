@@ -34,6 +34,16 @@
  *    at the diagonal (the sliding-window attention that "28. Grouped-Query
  *    Attention (GQA)", "Problem", names for Mistral).  With has_mask as well,
  *    a key must pass every rule.
+ *  - kv_lens (optional, device int32 [batch]): a KV cache of capacity seq_k
+ *    whose entry b holds kv_lens[b] valid keys.  Keys j >= kv_lens[b] are
+ *    hidden, and the causal diagonal moves with the length: entry b uses
+ *    causal_offset + kv_lens[b] - seq_k, so the offset is given for a full
+ *    cache (bottom-right: seq_k - seq_q).  This is the GQA cache of shape
+ *    (B, num_kv_groups, T, head_dim) that "Grouped-Query Attention vs
+ *    Multi-Head Attention: Understanding GQA Implementation", "Memory
+ *    Footprint and KV-Cache Optimization", describes, with a per-sequence T.
+ *    A length outside [0, seq_k] is clamped and reported by gqa_device_status
+ *    as GQA_ERR_KV_LENGTH.
  *  - A row whose keys are all hidden yields NaN (the softmax of an all -inf
  *    row).  seq_k == 0 yields zeros (an empty weighted sum).  batch == 0 or
  *    seq_q == 0 is a no-op.
@@ -80,6 +90,8 @@ extern "C" {
 #define GQA_ERR_DEVICE 9      /* no usable CUDA device, or not an sm_100 device */
 #define GQA_ERR_SCRATCH_LIMIT 10 /* gqa_forward_decode_noalloc: the problem needs more scratch
                                     than GQA_STATIC_SCRATCH_BYTES */
+#define GQA_ERR_KV_LENGTH 11  /* gqa_device_status: a kv_lens entry was outside [0, seq_k], or an
+                                 append did not fit the cache (that entry was left unchanged) */
 
 #define GQA_DTYPE_BF16 0
 #define GQA_DTYPE_F32 1
@@ -106,6 +118,7 @@ typedef struct gqa_problem {
   int64_t mask_stride[3]; /* over (b, i, j); the j stride must be 1 */
   int64_t causal_offset;  /* with causal: key j visible to query i iff j <= i + causal_offset */
   int64_t window;         /* with causal, > 0: keys j <= i + causal_offset - window hidden too */
+  const int32_t* kv_lens; /* NULL, or device [batch]: valid keys per entry (see above) */
 } gqa_problem;
 
 /* What gqa_forward will do for a problem on a device. */
@@ -115,7 +128,7 @@ typedef struct gqa_plan {
   int32_t block;             /* threads per CTA of the main kernel */
   int32_t smem_bytes;        /* dynamic shared memory per CTA of the main kernel */
   int32_t launches;          /* kernels enqueued per call */
-  int32_t work_units;        /* decode: 64-key tiles streamed; prefill: 128-row tiles */
+  int32_t work_units;        /* decode: 128-key tiles streamed; prefill: 128-row tiles */
   int64_t workspace_bytes;   /* bytes of device scratch gqa_forward needs (>= 256) */
   int64_t algorithmic_bytes; /* bytes of q, k, v, out (and mask) the call must move once */
   double algorithmic_flops;  /* 4*B*Hq*Sq*Sk*D, halved when causal */
@@ -153,7 +166,8 @@ GQA_API int gqa_forward(const gqa_problem* p, const void* q, const void* k, cons
  * gqa_device_status -- synchronise `stream` and read the workspace's error
  * word.  Returns GQA_OK; or GQA_ERR_TIMEOUT if a kernel gave up on a wait (its
  * outputs are then undefined), in which case the first `workspace_bytes` of
- * the workspace are zeroed; or GQA_ERR_CUDA if the stream reports a CUDA
+ * the workspace are zeroed; or GQA_ERR_KV_LENGTH if a length was out of range
+ * (the error word is cleared); or GQA_ERR_CUDA if the stream reports a CUDA
  * error.
  */
 GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream);
@@ -190,6 +204,43 @@ GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* str
 GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const void* q, const void* k,
                                        const void* v, const uint8_t* mask, void* out,
                                        void* stream);
+
+/*
+ * KV-cache append: the step before each decode or prefill chunk, writing the
+ * new tokens' keys and values after the ones a sequence already holds (the
+ * cache_k / cache_v buffers of "Grouped-Query Attention vs Multi-Head
+ * Attention: Understanding GQA Implementation", "GroupedQueryAttention Class
+ * Structure", grown in place per sequence instead of concatenated).
+ */
+typedef struct gqa_kv_append_desc {
+  int32_t dtype;                /* GQA_DTYPE_BF16 or GQA_DTYPE_F32 (cache and new rows alike) */
+  int32_t reserved;             /* must be 0 */
+  int64_t batch, heads_kv, capacity, head_dim, n_new;
+  int64_t cache_k_stride[4];    /* over (b, h_kv, j, d), j < capacity; d stride 1 */
+  int64_t cache_v_stride[4];
+  int64_t k_new_stride[4];      /* over (b, h_kv, t, d), t < n_new; d stride 1 */
+  int64_t v_new_stride[4];
+} gqa_kv_append_desc;
+
+/*
+ * gqa_kv_append -- for every entry b with L = kv_lens[b] and
+ * 0 <= L <= capacity - n_new: cache_k[b, :, L + t, :] = k_new[b, :, t, :] and
+ * the same for v, for t < n_new, then kv_lens[b] = L + n_new.  An entry that
+ * does not fit is left unchanged (cache and length) and gqa_device_status
+ * then returns GQA_ERR_KV_LENGTH.
+ *   cache_k, cache_v, k_new, v_new: device pointers described by `d`; the new
+ *                 rows must not overlap the cache.
+ *   kv_lens:      device int32 [batch], read and updated in place.
+ *   workspace:    the same kind of device scratch as gqa_forward's (at least
+ *                 256 bytes, 256-byte aligned, first 16 bytes zero before the
+ *                 first use); one launch, no cross-CTA wait.
+ * Returns GQA_OK once enqueued, or an argument error with nothing enqueued.
+ * The pages have no counterpart for the in-place length update: the pages
+ * concatenate along the sequence and keep one length for the whole batch.
+ */
+GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cache_v,
+                          const void* k_new, const void* v_new, int32_t* kv_lens,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static English description of a status code (never NULL). */
 GQA_API const char* gqa_status_string(int status);

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(gqa):
 
 
 def test_status_strings(gqa):
-    for code in range(0, 11):
+    for code in range(0, 12):
         s = gqa.status_string(code)
         assert s and s != "unknown status"
     assert gqa.status_string(1234) == "unknown status"
@@ -96,7 +96,7 @@ def test_plans_for_the_five_workloads(gqa):
     rc, pl = _rc(gqa, _p(gqa, B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128))
     assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "decode"
     assert pl.algorithmic_bytes == 268697600
-    assert pl.grid == 148 and pl.work_units == 16 * 8 * 64 and pl.launches == 1
+    assert pl.grid == 148 and pl.work_units == 16 * 8 * 32 and pl.launches == 1
     assert pl.workspace_bytes > 256 and pl.workspace_bytes % 256 == 0
     assert pl.smem_bytes <= 227 * 1024
     # long-context decode, Llama-2-70B-shaped layer
@@ -122,8 +122,8 @@ def test_short_query_blocks_decode(gqa):
 
 
 def test_decode_grid_small_problem(gqa):
-    # Fewer 64-key tiles than SMs: one tile per CTA.
-    rc, pl = _rc(gqa, _p(gqa, B=1, Hq=4, Hkv=1, Sq=1, Sk=130, D=64))
+    # Fewer 128-key tiles than SMs: one tile per CTA.
+    rc, pl = _rc(gqa, _p(gqa, B=1, Hq=4, Hkv=1, Sq=1, Sk=300, D=64))
     assert rc == 0 and pl.work_units == 3 and pl.grid == 3
     # g > 8 uses 16-head passes.
     rc, pl = _rc(gqa, _p(gqa, B=1, Hq=40, Hkv=1, Sq=1, Sk=64, D=128))
@@ -146,7 +146,7 @@ def test_causal_offset_and_window_plans(gqa):
     rc, full = _rc(gqa, _p(gqa, B=1, Hq=8, Hkv=2, Sq=1, Sk=4096, causal=True, causal_offset=4095))
     rc2, win = _rc(gqa, _p(gqa, B=1, Hq=8, Hkv=2, Sq=1, Sk=4096, causal=True, causal_offset=4095,
                            window=256))
-    assert rc == rc2 == 0 and full.work_units == 2 * 64 and win.work_units == 2 * 4
+    assert rc == rc2 == 0 and full.work_units == 2 * 32 and win.work_units == 2 * 2
 
 
 def test_binding_offset_rules(gqa):
@@ -178,3 +178,73 @@ def test_no_device_is_an_error_not_a_fallback(gqa):
     assert ei.value.status == gqa.GQA_ERR_DEVICE
     with pytest.raises(ValueError):
         gqa.forward(torch.zeros(1, 2, 1, 64), torch.zeros(1, 1, 3, 64), torch.zeros(1, 1, 3, 64))
+
+
+# ------------------------------------------------------------ ragged caches and append
+
+def test_ragged_plans(gqa):
+    """With kv_lens the decode plan covers the whole capacity (the kernel cuts
+    the real units on the device) and reserves shared memory for the lengths."""
+    fake = 1 << 20  # never dereferenced by gqa_query
+    rc, uni = _rc(gqa, _p(gqa, B=16, Hq=32, Hkv=8, Sq=1, Sk=4096))
+    rc2, rag = _rc(gqa, _p(gqa, B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, kv_lens=fake))
+    assert rc == rc2 == 0
+    assert gqa.KERNEL_NAMES[rag.kernel] == "decode"
+    assert rag.work_units == uni.work_units == 16 * 8 * 32
+    assert rag.smem_bytes >= uni.smem_bytes + 8 * 16
+    assert rag.smem_bytes <= 227 * 1024
+    # Many sequences: the ring gives up stages to keep the lengths resident.
+    rc, big = _rc(gqa, _p(gqa, B=8000, Hq=8, Hkv=1, Sq=1, Sk=256, kv_lens=fake))
+    assert rc == 0 and big.smem_bytes <= 227 * 1024
+    rc, _ = _rc(gqa, _p(gqa, B=20000, Hq=8, Hkv=1, Sq=1, Sk=256, kv_lens=fake))
+    assert rc == gqa.GQA_ERR_UNSUPPORTED
+    # Prefill and fp32 take lengths too.
+    rc, pf = _rc(gqa, _p(gqa, B=2, Hq=8, Hkv=2, Sq=300, Sk=1000, causal=True,
+                         causal_offset=700, kv_lens=fake))
+    assert rc == 0 and gqa.KERNEL_NAMES[pf.kernel] == "prefill"
+    rc, f = _rc(gqa, _p(gqa, dtype=1, D=40, kv_lens=fake))
+    assert rc == 0 and gqa.KERNEL_NAMES[f.kernel] == "f32"
+
+
+def _append(gqa, B=2, H=2, cap=100, D=128, n=1, dtype=0, **over):
+    c = (H * cap * D, cap * D, D, 1)
+    nw = (H * n * D, n * D, D, 1)
+    d = gqa.append_desc(dtype, B, H, cap, D, n, over.pop("ck", c), over.pop("cv", c),
+                        over.pop("kn", nw), over.pop("vn", nw))
+    for k, v in over.items():
+        setattr(d, k, v)
+    return d
+
+
+def _append_rc(gqa, d, ptr=256, lens=256, ws=256, wsb=256):
+    import ctypes
+    return gqa._lib.gqa_kv_append(ctypes.byref(d), ptr, ptr, ptr, ptr, lens, ws, wsb, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dtype=7), 8),
+    (dict(reserved=1), 8),
+    (dict(batch=-1), 2),
+    (dict(heads_kv=0), 2),
+    (dict(head_dim=0), 2),
+    (dict(n_new=-1), 2),
+    (dict(n_new=101), 2),
+    (dict(ck=(100 * 2 * 128, 100 * 128, 128, 2)), 3),
+    (dict(vn=(-1, 128, 128, 1)), 3),
+])
+def test_append_validation(gqa, over, code):
+    assert _append_rc(gqa, _append(gqa, **over)) == code
+
+
+def test_append_nulls_and_workspace(gqa):
+    d = _append(gqa)
+    assert _append_rc(gqa, d, lens=None) == gqa.GQA_ERR_NULL
+    assert _append_rc(gqa, d, ptr=None) == gqa.GQA_ERR_NULL
+    assert _append_rc(gqa, d, ws=None) == gqa.GQA_ERR_WORKSPACE
+    assert _append_rc(gqa, d, ws=128) == gqa.GQA_ERR_WORKSPACE
+    assert _append_rc(gqa, d, wsb=64) == gqa.GQA_ERR_WORKSPACE
+    assert _append_rc(gqa, d, ptr=257) == gqa.GQA_ERR_LAYOUT  # bf16 rows need 2-byte alignment
+    assert _append_rc(gqa, _append(gqa, dtype=1), ptr=258) == gqa.GQA_ERR_LAYOUT
+    # Nothing to append: OK without touching the device.
+    assert _append_rc(gqa, _append(gqa, B=0)) == gqa.GQA_OK
+    assert _append_rc(gqa, _append(gqa, n=0)) == gqa.GQA_OK

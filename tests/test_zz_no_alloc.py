@@ -59,11 +59,14 @@ def test_noalloc_matches_workspace_entry_point_twice(gqa, shape):
 
 
 def test_noalloc_rejects_what_it_cannot_hold(gqa):
-    # More scratch than the static array holds: many short 16-head groups give
-    # every CTA many partial slots.
-    big_q = torch.zeros(1, 16 * 2048, 1, 128, dtype=torch.bfloat16, device="cuda")
-    big_out = torch.empty_like(big_q)
-    big_k = torch.zeros(1, 2048, 64, 128, dtype=torch.bfloat16, device="cuda")
+    # More scratch than the static array holds: one ticket counter per kv
+    # head, 2.2 M heads.  Zero-stride views: the call is refused before it
+    # reads or writes any of them.
+    H = 2200000
+    one = torch.zeros(1, 1, 1, 64, dtype=torch.bfloat16, device="cuda")
+    big_q = one.expand(1, H, 1, 64)
+    big_k = one.expand(1, H, 1, 64)
+    big_out = torch.zeros(1, 1, 1, 64, dtype=torch.bfloat16, device="cuda").expand(1, H, 1, 64)
     plan = gqa.query(big_q, big_k, big_k)
     assert plan["workspace_bytes"] > gqa.STATIC_SCRATCH_BYTES
     assert _noalloc(gqa, big_q, big_k, big_k, big_out) == gqa.GQA_ERR_SCRATCH_LIMIT
