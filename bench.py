@@ -72,6 +72,18 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+TRAFFIC_SOURCES = ("kernels.h", "ptx.cuh", "epilogue.cuh")
+
+
+def kernel_source_sha256(kernel_file: str) -> str:
+    """Hash of a kernel's source and the headers it includes."""
+    h = hashlib.sha256()
+    for name in (kernel_file,) + TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "grouped_query_attention_fwd_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _traffic_for(kernel_file: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel
     source is unchanged since it was captured; else None."""
@@ -80,10 +92,7 @@ def _traffic_for(kernel_file: str, workload: str):
         with open(path) as f:
             rec = json.load(f)
         ent = rec[workload]
-        src = os.path.join(ROOT, "grouped_query_attention_fwd_b200", "csrc", kernel_file)
-        with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
-        if ent.get("source_sha256") != h:
+        if ent.get("source_sha256") != kernel_source_sha256(kernel_file):
             return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:
@@ -200,39 +209,60 @@ def weak_scaling_gbs(bytes_per_step: int, steps: int, world: int, elapsed_ms: fl
 
 # ------------------------------------------------------------------ GPU arm
 
-def _graph_timed(torch, calls, steps, warmup, stream):
-    """Time `steps` launches, launch i being calls[i % len(calls)], each
-    replayed from its own one-launch CUDA graph so that host-side overhead
-    never leaves the GPU idle between launches.  Returns (total_ms,
-    per-launch ms list, host seconds spent enqueuing)."""
+def _graph_timed(torch, calls, steps, warmup, stream, per_launch_samples=200):
+    """Time exactly `steps` launches, launch i being calls[i % len(calls)].
+
+    Whole run: the launches are captured into CUDA graphs of many launches
+    each (one host call per ~32 launches, so the host never starves the GPU)
+    and the run is bracketed by two events.  Per launch: a separate pass
+    replays one-launch graphs with an event pair around each.  Returns
+    (total_ms for the `steps` launches, per-launch ms list, host seconds per
+    launch spent enqueuing the whole run)."""
     for i in range(warmup):
         calls[i % len(calls)]()
     torch.cuda.synchronize()
-    graphs = []
-    for fn in calls:
+    n = len(calls)
+    reps = max(1, 32 // n)
+
+    def capture(count, start):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn()
-        graphs.append(g)
-    for i in range(max(3, len(graphs))):
-        graphs[i % len(graphs)].replay()
+            for j in range(count):
+                calls[(start + j) % n]()
+        return g
+
+    chain = capture(n * reps, 0)            # a whole number of rounds over the copies
+    tail = capture(steps % (n * reps), 0) if steps % (n * reps) else None
+    singles = [capture(1, i) for i in range(n)]
+    chain.replay()
+    for g in singles:
+        g.replay()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
+
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     h0 = time.perf_counter()
     e0.record(stream)
-    for i in range(steps):
-        ev[i][0].record(stream)
-        graphs[i % len(graphs)].replay()
-        ev[i][1].record(stream)
+    for _ in range(steps // (n * reps)):
+        chain.replay()
+    if tail is not None:
+        tail.replay()
     e1.record(stream)
     h1 = time.perf_counter()
     torch.cuda.synchronize()
+    total_ms = e0.elapsed_time(e1)
+
+    k = min(steps, per_launch_samples)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(k)]
+    for i in range(k):
+        ev[i][0].record(stream)
+        singles[i % n].replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
     per = [a.elapsed_time(b) for a, b in ev]
-    del graphs
-    return e0.elapsed_time(e1), per, h1 - h0
+    del chain, tail, singles
+    return total_ms, per, (h1 - h0) / steps
 
 
 def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
@@ -295,7 +325,9 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
 
     calls = [(lambda i=i: call(i)) for i in range(copies)]
     if n_new:  # every call of a copy appends n_new tokens: they must fit the capacity
-        calls_per_copy = math.ceil((warmup + max(3, copies) + steps) / copies)
+        rounds = max(1, 32 // copies) * copies  # warm replay of the many-launch graph
+        executed = warmup + rounds + copies + steps + min(steps, 200)
+        calls_per_copy = math.ceil(executed / copies)
         if hi + calls_per_copy * n_new > Sk:
             raise ValueError("%d steps overflow the %d-key cache; use fewer" % (steps, Sk))
     total_ms, per, _ = _graph_timed(torch, calls, steps, warmup, stream)
@@ -508,8 +540,10 @@ def run_gpu(args):
             "parallelism": "replicas" if world == 1 else "dp%d (independent problems per rank)" % world,
             "l2": "K/V rotated over %d device copies (%.0f MB) so no launch finds its K/V in L2"
                   % (copies, copies * kv_bytes / 1e6),
-            "launch": "one gqa_forward per step, each replayed from a one-launch CUDA graph "
-                      "(host enqueue %.1f us per step)" % (host_s / args.steps * 1e6),
+            "launch": "one gqa_forward per step; the steps are replayed from CUDA graphs of "
+                      "%d launches (host enqueue %.2f us per step); per-launch times from a "
+                      "separate pass of one-launch graphs" % (max(1, 32 // copies) * copies,
+                                                              host_s * 1e6),
         },
         "gpu_launches": args.steps * plan["launches"],
         "clocks": {k_: v_ for k_, v_ in clocks.items()},

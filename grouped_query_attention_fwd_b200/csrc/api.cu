@@ -14,7 +14,7 @@
 namespace gqa {
 namespace {
 
-constexpr int64_t kErrWordBytes = 256;  // workspace head reserved for the error word
+constexpr int64_t kErrWordBytes = kWorkspaceHeadBytes;  // error word, append ticket
 
 bool bf16_paths(const gqa_problem& p) { return p.dtype == GQA_DTYPE_BF16; }
 
@@ -142,9 +142,9 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       plan->grid = s.grid;
       plan->block = kDecodeThreads;
       plan->smem_bytes = s.smem_bytes;
-      plan->launches = 1;
+      plan->launches = s.zero_counters ? 2 : 1;  // (+ a counter memset for huge problems)
       plan->work_units = static_cast<int32_t>(s.units);
-      plan->workspace_bytes = kErrWordBytes + s.part_bytes;
+      plan->workspace_bytes = s.workspace_end;
       break;
     }
     case GQA_KERNEL_PREFILL: {
@@ -154,7 +154,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       plan->smem_bytes = s.smem_bytes;
       plan->launches = p.has_mask ? 2 : 1;
       plan->work_units = static_cast<int32_t>(s.work);
-      plan->workspace_bytes = kErrWordBytes + s.summary_bytes;
+      plan->workspace_bytes = s.workspace_end;
       break;
     }
   }
@@ -308,7 +308,8 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
     // The ticket counters must start at zero; other calls sharing this
     // workspace (a prefill's tile classes, a larger problem's partials) may
     // have left bytes there.
-    if (cudaMemsetAsync(a.counters, 0, static_cast<size_t>(s.groups) * 4, stream) != cudaSuccess)
+    if (s.zero_counters &&
+        cudaMemsetAsync(a.counters, 0, static_cast<size_t>(s.groups) * 4, stream) != cudaSuccess)
       return GQA_ERR_CUDA;
     return launch_decode(p, s, a, tmk, tmv, stream);
   }

@@ -69,7 +69,7 @@ struct DecodeSmem {
   static constexpr int kScrOBytes = kMergeWarps * HP * kScrRow * 4;
   // Ragged launches keep the B lengths and B + 1 prefix sums after the flags.
   static int bytes(int stages, int ragged_batch) {
-    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + 2 * stages * 8 + 16 +
+    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + 3 * stages * 8 + 16 +
            (ragged_batch > 0 ? ((8 * ragged_batch + 4 + 15) / 16) * 16 : 0);
   }
 };
@@ -145,7 +145,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* ring = smem;
   float* scr_o = reinterpret_cast<float*>(ring + stages * L::kStageBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scr_o) + L::kScrOBytes);
-  uint64_t* empty = full + stages;
+  uint64_t* full_v = full + stages;  // full: the stage's K tile landed; full_v: its V tile
+  uint64_t* empty = full_v + stages;
   uint8_t* tail = reinterpret_cast<uint8_t*>(empty + stages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tail);
   volatile int* last_flag = abort_flag + 1;
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&full_v[s], 1);
       mbar_init(&empty[s], NCW);
     }
     *abort_flag = 0;
@@ -232,23 +234,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int kv = gi / passes;
         const int b = cu.b;
         uint8_t* st = ring + s * L::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+        mbar_arrive_expect_tx(&full[s], L::kTileBytes);
 #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
+        for (int c = 0; c < CHUNKS; ++c)
           tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, key0, kv, b);
-          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full[s], c * 64, key0, kv, b);
-        }
+        mbar_arrive_expect_tx(&full_v[s], L::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c)
+          tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full_v[s], c * 64, key0, kv, b);
       }
       // Unwind: make sure no copy is still landing in this CTA's shared memory.
       if (*abort_flag) {
         const int issued = it;
-        for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+        for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j) {
           mbar_wait_drain(&full[j % stages], static_cast<uint32_t>((j / stages) & 1));
+          mbar_wait_drain(&full_v[j % stages], static_cast<uint32_t>((j / stages) & 1));
+        }
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    uint32_t bq[NT][KSTEPS][2];
+    // Q as MMA B fragments: in registers for one column tile; for two, in
+    // shared memory (head rows padded to D * 2 + 16 bytes, conflict-free for
+    // ldmatrix), aliasing the flush scratch, to stay within the registers
+    // that 288 threads may hold.
+    constexpr bool kQSmem = NT == 2;
+    constexpr int kQRow = D * 2 + 16;
+    static_assert(!kQSmem || HP * kQRow <= L::kScrOBytes, "Q rows must fit the scratch");
+    uint32_t bq[kQSmem ? 1 : NT][kQSmem ? 1 : KSTEPS][2];
+    uint8_t* q_smem = reinterpret_cast<uint8_t*>(scr_o);
     float o[NT][KSTEPS][4];
     float m_run[NT][2], l_run[NT][2];
     int cur = -1;                // group being accumulated
@@ -276,20 +290,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     int vlo[NT][2], vhi[NT][2];
     const uint8_t* vmask[NT][2];
 
+    // Global address of row hl (a head, or a (head, query) pair) of this pass.
+    auto q_row = [&](int hl) -> const uint16_t* {
+      const int hh = MQ ? hl / a.Sq : hl;
+      const int qi = MQ ? hl % a.Sq : 0;
+      return a.q + b * a.qs[0] + (int64_t)(kv * a.g + hh) * a.qs[1] + (int64_t)qi * a.qs[2];
+    };
+
     auto load_q = [&]() {
+      if (kQSmem) {
+        // 16-byte pieces of the pass's HP rows; rows past the group are zero.
+        for (int x = threadIdx.x; x < HP * (D / 8); x += NCW * 32) {
+          const int r = x / (D / 8), c = x % (D / 8);
+          const int hl = pass * HP + r;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (hl < a.rows) v = *reinterpret_cast<const uint4*>(q_row(hl) + c * 8);
+          *reinterpret_cast<uint4*>(q_smem + r * kQRow + c * 16) = v;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int hl = pass * HP + nt * 8 + (lane >> 2);  // row within the group
-        const bool ok = hl < a.rows;
-        const int hh = MQ ? (ok ? hl / a.Sq : 0) : (ok ? hl : 0);
-        const int qi = MQ ? (ok ? hl % a.Sq : 0) : 0;
-        const uint16_t* qrow = a.q + b * a.qs[0] + (int64_t)(kv * a.g + hh) * a.qs[1] +
-                               (int64_t)qi * a.qs[2];
+        if (!kQSmem) {
+          const int hl = pass * HP + nt * 8 + (lane >> 2);  // row within the group
+          const bool ok = hl < a.rows;
+          const uint16_t* qrow = q_row(ok ? hl : 0);
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) {
-          const int d0 = ks * 16 + (lane & 3) * 2;
-          bq[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
-          bq[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            const int d0 = ks * 16 + (lane & 3) * 2;
+            bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][0] =
+                ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+            bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][1] =
+                ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+          }
         }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -332,6 +365,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           l_run[nt][e] = l;
         }
       float* my_rows = scr_o + (warp & 3) * HP * R;
+      // Q lives in the scratch: every warp must be done with its last S first.
+      if (kQSmem) asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
       auto put_state = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -429,9 +464,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         return;
       }
       // Split group: publish this CTA's partial (float4 stores), then take a
-      // ticket: the CTA barrier orders every thread's stores before thread
-      // 0's gpu-scope fence and atomic (release), and thread 0's fence after
-      // the atomic orders the reads of the others' partials (acquire).
+      // ticket on the group's counter.
       const int slot = (static_cast<int>(blockIdx.x) * 2 + (cur == first_grp ? 0 : 1)) * HP;
       for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
         const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
@@ -457,10 +490,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
       if (threadIdx.x == 0) {
+        // The barrier above makes every thread's partial visible to thread 0;
+        // its acquire-release add at gpu scope publishes them (release) and,
+        // for the last arriver, makes the others' partials visible (acquire).
         const uint32_t n = static_cast<uint32_t>(c_hi - c_lo + 1);
-        __threadfence();
-        const uint32_t old = atomicAdd(&counters[cur], 1u);
-        __threadfence();
+        const uint32_t old = atom_add_acq_rel_gpu(&counters[cur], 1u);
         *last_flag = (old == n - 1) ? 1 : 0;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
@@ -565,7 +599,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     };
 
     int it = 0;
-    bool ok = true;
     Cursor cu;
     for (int u = u_begin; u < u_end; ++u, ++it) {
       seek(cu, u, sc, a);
@@ -590,9 +623,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       const int s = it % stages;
       const uint32_t round = static_cast<uint32_t>(it / stages);
+      // A wait that gives up sets the abort flag; from then on every wait
+      // fails at once and the warps skip the arithmetic but keep walking the
+      // units, so that all eight reach the same flush() barriers.
       if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
-        ok = false;
-        break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
       }
       const uint32_t kbase = smem_u32(ring + s * L::kStageBytes);
       const uint32_t vbase = kbase + L::kTileBytes;
@@ -616,10 +653,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               kbase + (ks >> 2) * CHUNK_BYTES + r * 128 + ((u16 ^ (r & 7)) << 4);
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4(a0, a1, a2, a3, addr);
+          if (kQSmem) {
+            // B fragments of both column tiles: matrices (rows 0-7 | 8-15) x
+            // (d ks*16 + 0-7 | + 8-15), row and half picked by the lane.
+            const int qr = ((lane >> 4) << 3) + (lane & 7);
+            const uint32_t qaddr =
+                smem_u32(q_smem) + qr * kQRow + ks * 32 + ((lane >> 3) & 1) * 16;
+            uint32_t q0, q1, q2, q3;
+            ldmatrix_x4(q0, q1, q2, q3, qaddr);
+            mma_bf16_16816(sc[0], a0, a1, a2, a3, q0, q1);
+            mma_bf16_16816(sc[NT - 1], a0, a1, a2, a3, q2, q3);
+          } else {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816((kSplit && (ks & 1)) ? sc2[nt] : sc[nt], a0, a1, a2, a3,
-                           bq[nt][ks][0], bq[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt)
+              mma_bf16_16816((kSplit && (ks & 1)) ? sc2[nt] : sc[nt], a0, a1, a2, a3,
+                             bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][0],
+                             bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][1]);
+          }
         }
         if (kSplit) {
 #pragma unroll
@@ -671,7 +721,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         pt1[nt] = movmatrix_trans(pack_bf16x2(tv[2], tv[3]));
       }
 
-      // O^T[D x 8] += V^T[D x 16 keys] P^T[16 keys x 8].
+      // O^T[D x 8] += V^T[D x 16 keys] P^T[16 keys x 8], once the V tile is in.
+      if (!mbar_wait(&full_v[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
+      }
       {
         const int mi = lane >> 3;
         const int key = warp * 16 + (mi >> 1) * 8 + (lane & 7);
@@ -691,11 +746,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (ok && cur >= 0) flush();
-    if (!ok) {
-      // Keep the named barrier count consistent for warps still in flush():
-      // nothing else to do, the error word is already set.
-    }
+    if (cur >= 0) flush();  // after an abort too (its output is undefined, the error word set)
   }
   __syncthreads();
 }
@@ -748,12 +799,21 @@ DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
       s.smem_bytes = DecodeSmem<64, 2>::bytes(s.stages, rb);
     if (s.smem_bytes <= kDecodeMaxSmem || s.stages <= 2) break;
   }
-  // Two partial slots per CTA: its first and its last group.
+  // Two partial slots per CTA: its first and its last group.  The ticket
+  // counters sit in the workspace's counter region, which stays zero between
+  // calls; a launch with more groups keeps them past it and zeroes them.
   const int64_t slots = static_cast<int64_t>(s.grid) * 2 * s.HP;
-  s.counters_offset = 256;
-  s.part_ml_offset = s.counters_offset + ((s.groups * 4 + 255) / 256) * 256;
+  int64_t at = kScratchOffset;
+  s.zero_counters = s.groups * 4 > kCounterRegionBytes;
+  if (s.zero_counters) {
+    s.counters_offset = at;
+    at += ((s.groups * 4 + 255) / 256) * 256;
+  } else {
+    s.counters_offset = kWorkspaceHeadBytes;
+  }
+  s.part_ml_offset = at;
   s.part_o_offset = s.part_ml_offset + ((slots * 8 + 255) / 256) * 256;
-  s.part_bytes = (s.part_o_offset - 256) + slots * s.D * 4;
+  s.workspace_end = s.part_o_offset + slots * s.D * 4;
   return s;
 }
 

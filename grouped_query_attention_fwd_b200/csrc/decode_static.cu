@@ -88,7 +88,10 @@ extern "C" GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const vo
 
   const DecodeShape s = plan_decode(*p, sms);
   // Error word and ticket counters must start at zero; partials need not.
-  if (cudaMemsetAsync(ws, 0, static_cast<size_t>(s.part_ml_offset), stream) != cudaSuccess) {
+  // Nothing reports a wait that gave up here, so the counters are zeroed on
+  // every call instead of trusting the last one to have left them zero.
+  const int64_t zero_end = s.counters_offset + s.groups * 4;
+  if (cudaMemsetAsync(ws, 0, static_cast<size_t>(zero_end), stream) != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_CUDA;
   }

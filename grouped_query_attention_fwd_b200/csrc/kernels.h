@@ -18,6 +18,15 @@ constexpr int kDecodeMaxRowsPerPass = 16;  // (head, query) rows in the MMA N di
 constexpr int kDecodeMaxSmem = 227 * 1024;  // dynamic shared memory one CTA may take
 constexpr int64_t kMaxRaggedBatch = 16384;  // batch entries with per-sequence lengths
 
+// Workspace layout shared by every call: bytes [0, 256) hold the error word
+// (and the append ticket), [256, 256 + kCounterRegionBytes) the decode ticket
+// counters, which each group's last contributor resets, so the region stays
+// zero between calls; other scratch (decode partials, prefill tile classes)
+// starts after it and never touches it.
+constexpr int64_t kWorkspaceHeadBytes = 256;
+constexpr int64_t kCounterRegionBytes = 64 * 1024;
+constexpr int64_t kScratchOffset = kWorkspaceHeadBytes + kCounterRegionBytes;
+
 // Keys [lo, hi) of one batch entry that some query of the block can see,
 // and the decode key tiles [t0, t0 + tiles) that hold them.  `len` is the entry's
 // cache length (seq_k without per-sequence lengths); the causal diagonal
@@ -62,7 +71,9 @@ struct DecodeShape {
   int stages;       // shared-memory ring depth
   int smem_bytes;
   bool ragged;      // per-sequence kv_lens: the partition is computed on the device
-  int64_t counters_offset, part_o_offset, part_ml_offset, part_bytes;
+  bool zero_counters;  // more groups than the counter region holds: zero them per call
+  int64_t counters_offset, part_o_offset, part_ml_offset;
+  int64_t workspace_end;  // bytes of workspace the launch uses
 };
 
 DecodeShape plan_decode(const gqa_problem& p, int sm_count);
@@ -110,7 +121,7 @@ struct PrefillShape {
   int64_t work;      // batch * heads_kv * m_tiles
   int grid;
   int smem_bytes;
-  int64_t summary_offset, summary_bytes;
+  int64_t summary_offset, workspace_end;
 };
 
 PrefillShape plan_prefill(const gqa_problem& p, int sm_count);

@@ -771,8 +771,8 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
   if (s.grid < 1) s.grid = 1;
   s.smem_bytes = s.D == 128 ? Layout<128>::kBytes : Layout<64>::kBytes;
-  s.summary_offset = 256;
-  s.summary_bytes = p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0;
+  s.summary_offset = kScratchOffset;
+  s.workspace_end = s.summary_offset + (p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0);
   return s;
 }
 

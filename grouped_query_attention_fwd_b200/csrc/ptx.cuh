@@ -62,6 +62,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
       : "memory");
 }
 
+// Atomic add with acquire-release semantics at gpu scope; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .b64 st;\n\t"
@@ -94,11 +104,12 @@ enum : uint32_t {
   kErrKvLength = 1u << 3,  // a kv_lens entry outside [0, capacity]: clamped, result undefined
 };
 
-// Bounded wait on `bar` reaching phase `parity`.  Returns false if the limit
-// ran out or another role already aborted (`*abort` nonzero); in that case the
-// error word gets `err_bit` and `*abort` is set.
+// Bounded wait on `bar` reaching phase `parity`.  Returns false if another
+// role already aborted (`*abort` nonzero), or if the limit ran out, in which
+// case the error word gets `err_bit` and `*abort` is set.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err_word, uint32_t err_bit) {
+  if (*abort) return false;  // another role gave up: unwind in step with it
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;

@@ -148,12 +148,14 @@ GQA_API int gqa_query(const gqa_problem* p, int sm_count, gqa_plan* plan);
  *   q, k, v, out: device pointers described by `p` (dtype, sizes, strides).
  *   mask:         device uint8 pointer if p->has_mask, else ignored (may be NULL).
  *   workspace:    device scratch of at least plan.workspace_bytes, 256-byte
- *                 aligned, owned by the caller.  Only its first 16 bytes (the
- *                 error word) must be zero before the first use; each call
- *                 initialises the rest of what it uses.  gqa_device_status
- *                 clears the error word after reporting an error.  Calls that
- *                 share a workspace must be ordered on one stream; calls that
- *                 overlap on the GPU race.
+ *                 aligned, owned by the caller, ZERO-FILLED before its first
+ *                 use.  Its head holds the error word and the decode ticket
+ *                 counters (bytes [256, 256 + 64 KiB)); every call leaves that
+ *                 head as it found it, so one workspace serves any sequence
+ *                 of calls of any shapes without being cleared again.  After
+ *                 an error gqa_device_status re-zeroes it.  Calls that share a
+ *                 workspace must be ordered on one stream; calls that overlap
+ *                 on the GPU race.
  *   stream:       cudaStream_t.
  * Returns GQA_OK once the kernels are enqueued, or an error code with nothing
  * enqueued.  Does not synchronise.
@@ -231,9 +233,10 @@ typedef struct gqa_kv_append_desc {
  *   cache_k, cache_v, k_new, v_new: device pointers described by `d`; the new
  *                 rows must not overlap the cache.
  *   kv_lens:      device int32 [batch], read and updated in place.
- *   workspace:    the same kind of device scratch as gqa_forward's (at least
- *                 256 bytes, 256-byte aligned, first 16 bytes zero before the
- *                 first use); one launch, no cross-CTA wait.
+ *   workspace:    a gqa_forward workspace (zero-filled before its first use,
+ *                 256-byte aligned, at least 256 bytes); the append uses only
+ *                 its first 16 bytes and leaves them as it found them.  One
+ *                 launch, no cross-CTA wait.
  * Returns GQA_OK once enqueued, or an argument error with nothing enqueued.
  * The pages have no counterpart for the in-place length update: the pages
  * concatenate along the sequence and keep one length for the whole batch.

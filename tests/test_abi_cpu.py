@@ -248,3 +248,17 @@ def test_append_nulls_and_workspace(gqa):
     # Nothing to append: OK without touching the device.
     assert _append_rc(gqa, _append(gqa, B=0)) == gqa.GQA_OK
     assert _append_rc(gqa, _append(gqa, n=0)) == gqa.GQA_OK
+
+
+def test_workspace_layout_keeps_counters_apart(gqa):
+    """Decode counters live in a fixed region after the 256-byte head; every
+    other scratch starts past it, so a workspace shared by calls of any shape
+    never needs clearing.  Huge decode problems keep their counters past the
+    region and zero them per call (one extra launch)."""
+    region = 256 + 64 * 1024
+    rc, dec = _rc(gqa, _p(gqa, B=16, Hq=32, Hkv=8, Sq=1, Sk=4096))
+    assert rc == 0 and dec.workspace_bytes > region and dec.launches == 1
+    rc, pre = _rc(gqa, _p(gqa, B=2, Hq=8, Hkv=2, Sq=300, Sk=300, mask=True))
+    assert rc == 0 and pre.workspace_bytes == (region + 2 * 3 * 3 + 255) // 256 * 256  # classes after it
+    rc, huge = _rc(gqa, _p(gqa, B=2100, Hq=32, Hkv=8, Sq=1, Sk=100))
+    assert rc == 0 and huge.launches == 2 and huge.workspace_bytes > region + 2100 * 8 * 4

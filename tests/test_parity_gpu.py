@@ -73,6 +73,11 @@ DECODE_CASES = [
     (1, 24, 2, 700, 128),     # g = 12: two 8-wide column tiles
     (1, 40, 1, 300, 64),      # g = 40: three 16-head passes
     (5, 32, 8, 4096, 128),
+    (2, 8, 2, 127, 128),      # one key short of a 128-key tile
+    (2, 8, 2, 128, 128),      # exactly one tile
+    (2, 8, 2, 129, 128),      # one key into the second tile
+    (2, 32, 2, 1025, 128),    # g = 16: Q fragments from shared memory
+    (3, 64, 4, 2000, 64),     # g = 16, D = 64
 ]
 
 
@@ -278,3 +283,18 @@ def test_short_query_block_decode(gqa, B, Hq, Hkv, Sq, Sk, D, off, window, maske
                          causal=off is not None, causal_offset=(Sk - Sq) if off else None,
                          window=window)
     assert_bf16_parity(to_np(out), ref, "short query decode")
+
+
+def test_decode_many_groups_zeroes_its_counters(gqa):
+    """16800 (batch, kv head) groups: more ticket counters than the workspace's
+    counter region holds, so the call zeroes its own; sampled rows checked."""
+    B, Hq, Hkv, Sk, D = 2100, 32, 8, 100, 128
+    assert gqa.query(*(torch.empty(s, dtype=torch.bfloat16, device="cuda") for s in
+                       ((B, Hq, 1, D), (B, Hkv, Sk, D), (B, Hkv, Sk, D))))["launches"] == 2
+    bits, (q, k, v) = bf16_inputs(4400, B, Hq, Hkv, 1, Sk, D)
+    for _ in range(2):  # twice: the counters must be clean for the second call too
+        out = to_np(gqa.forward(q, k, v))
+        _status_ok(gqa)
+    for b in (0, 777, 2099):
+        ref = oracle_bf16(bits[0][b:b + 1], bits[1][b:b + 1], bits[2][b:b + 1])
+        assert_bf16_parity(out[b:b + 1], ref, "many groups b=%d" % b)
