@@ -34,7 +34,7 @@ GQA_ERR_NULL, GQA_ERR_SHAPE, GQA_ERR_LAYOUT, GQA_ERR_UNSUPPORTED = 1, 2, 3, 4
 GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 5, 6, 7, 8, 9
 GQA_ERR_SCRATCH_LIMIT, GQA_ERR_KV_LENGTH = 10, 11
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
-GQA_DTYPE_BF16, GQA_DTYPE_F32 = 0, 1
+GQA_DTYPE_BF16, GQA_DTYPE_F32, GQA_DTYPE_F16 = 0, 1, 2
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
 
 EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
@@ -171,7 +171,9 @@ def _dtype_code(t) -> int:
         return GQA_DTYPE_BF16
     if t.dtype == torch.float32:
         return GQA_DTYPE_F32
-    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+    if t.dtype == torch.float16:
+        return GQA_DTYPE_F16
+    raise TypeError("q/k/v must be bfloat16, float16 or float32, got %s" % t.dtype)
 
 
 def _offset(causal, causal_offset, Sq, Sk) -> int:

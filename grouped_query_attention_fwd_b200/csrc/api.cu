@@ -16,12 +16,16 @@ namespace {
 
 constexpr int64_t kErrWordBytes = kWorkspaceHeadBytes;  // error word, append ticket
 
-bool bf16_paths(const gqa_problem& p) { return p.dtype == GQA_DTYPE_BF16; }
+// bf16 and fp16 share the tensor-core paths.
+bool half_paths(const gqa_problem& p) {
+  return p.dtype == GQA_DTYPE_BF16 || p.dtype == GQA_DTYPE_F16;
+}
 
 int validate(const gqa_problem* pp) {
   if (pp == nullptr) return GQA_ERR_NULL;
   const gqa_problem& p = *pp;
-  if (p.dtype != GQA_DTYPE_BF16 && p.dtype != GQA_DTYPE_F32) return GQA_ERR_ARG;
+  if (p.dtype != GQA_DTYPE_BF16 && p.dtype != GQA_DTYPE_F32 && p.dtype != GQA_DTYPE_F16)
+    return GQA_ERR_ARG;
   if (!std::isfinite(p.scale)) return GQA_ERR_ARG;
   if (p.batch < 0 || p.seq_q < 0 || p.seq_k < 0) return GQA_ERR_SHAPE;
   if (p.heads_q <= 0 || p.heads_kv <= 0 || p.head_dim <= 0) return GQA_ERR_SHAPE;
@@ -38,8 +42,10 @@ int validate(const gqa_problem* pp) {
       return GQA_ERR_LAYOUT;
   if (p.window < 0 || (p.window > 0 && !p.causal)) return GQA_ERR_ARG;
   if (p.causal_offset <= -lim || p.causal_offset >= lim || p.window >= lim) return GQA_ERR_ARG;
-  if (bf16_paths(p)) {
-    if (p.head_dim != 64 && p.head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (half_paths(p)) {
+    // Multiples of 8 up to 128: the kernels run at 64 or 128 wide, TMA
+    // filling the columns past head_dim with zeros.
+    if (p.head_dim % 8 != 0 || p.head_dim > 128) return GQA_ERR_UNSUPPORTED;
     // 16-byte rule of the TMA unit for every stride of a dimension longer than 1.
     const int64_t qsz[3] = {p.batch, p.heads_q, p.seq_q};
     const int64_t ksz[3] = {p.batch, p.heads_kv, p.seq_k};
@@ -182,8 +188,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 
 // 4-D bf16 map over (d, s, h, b) of a tensor with element strides st[0..2]
 // for (b, h, s); box {64, box_s, box_h, 1} with 128-byte swizzle.
-int encode_bf16_map(CUtensorMap* map, const void* base, int64_t B, int64_t H, int64_t S,
-                    int64_t D, const int64_t st[4], uint32_t box_s, uint32_t box_h) {
+int encode_half_map(CUtensorMap* map, const void* base, int64_t B, int64_t H, int64_t S,
+                    int64_t D, const int64_t st[4], uint32_t box_s, uint32_t box_h, bool f16) {
   auto enc = get_encoder();
   if (enc == nullptr) return GQA_ERR_CUDA;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
@@ -197,7 +203,8 @@ int encode_bf16_map(CUtensorMap* map, const void* base, int64_t B, int64_t H, in
                            static_cast<cuuint64_t>(bb)};
   cuuint32_t box[4] = {64, box_s, box_h, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   4, const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_LAYOUT;
@@ -215,8 +222,8 @@ namespace gqa {
 // decode entry point.
 int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& p,
                          const int64_t st[4]) {
-  return encode_bf16_map(map, base, p.batch, p.heads_kv, p.seq_k, p.head_dim, st,
-                         kDecodeKeysPerTile, 1);
+  return encode_half_map(map, base, p.batch, p.heads_kv, p.seq_k, p.head_dim, st,
+                         kDecodeKeysPerTile, 1, p.dtype == GQA_DTYPE_F16);
 }
 }  // namespace gqa
 
@@ -224,7 +231,7 @@ using namespace gqa;
 
 extern "C" {
 
-GQA_API int gqa_version(void) { return 10200; }
+GQA_API int gqa_version(void) { return 10300; }
 
 GQA_API const char* gqa_status_string(int status) {
   switch (status) {
@@ -232,7 +239,7 @@ GQA_API const char* gqa_status_string(int status) {
     case GQA_ERR_NULL: return "a required pointer is NULL";
     case GQA_ERR_SHAPE: return "inconsistent or invalid sizes (heads_q must be a multiple of heads_kv)";
     case GQA_ERR_LAYOUT: return "unsupported memory layout (innermost stride must be 1; bf16 bases and strides must be multiples of 16 bytes)";
-    case GQA_ERR_UNSUPPORTED: return "unsupported combination (bf16 needs head_dim 64 or 128)";
+    case GQA_ERR_UNSUPPORTED: return "unsupported combination (bf16/fp16 need head_dim a multiple of 8, at most 128)";
     case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
     case GQA_ERR_CUDA: return "a CUDA runtime call failed";
     case GQA_ERR_TIMEOUT: return "a kernel gave up on an internal wait; outputs are undefined";
@@ -298,11 +305,9 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   if (plan.kernel == GQA_KERNEL_DECODE) {
     const DecodeShape s = plan_decode(p, sms);
     CUtensorMap tmk, tmv;
-    int erc = encode_bf16_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride,
-                              kDecodeKeysPerTile, 1);
+    int erc = encode_decode_kv_map(&tmk, k, p, p.k_stride);
     if (erc != GQA_OK) return erc;
-    erc = encode_bf16_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride,
-                          kDecodeKeysPerTile, 1);
+    erc = encode_decode_kv_map(&tmv, v, p, p.v_stride);
     if (erc != GQA_OK) return erc;
     const DecodeArgs a = make_decode_args(p, s, q, mask, out, ws);
     // The ticket counters must start at zero; other calls sharing this
@@ -317,12 +322,15 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   // Prefill.
   const PrefillShape s = plan_prefill(p, sms);
   CUtensorMap tmq, tmk, tmv;
-  int erc = encode_bf16_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
-                            static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g));
+  const bool f16 = p.dtype == GQA_DTYPE_F16;
+  int erc = encode_half_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
+                            static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g), f16);
   if (erc != GQA_OK) return erc;
-  erc = encode_bf16_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 128, 1);
+  erc = encode_half_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 128, 1,
+                        f16);
   if (erc != GQA_OK) return erc;
-  erc = encode_bf16_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128, 1);
+  erc = encode_half_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128, 1,
+                        f16);
   if (erc != GQA_OK) return erc;
   PrefillArgs a{};
   a.mask = p.has_mask ? mask : nullptr;
@@ -342,6 +350,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.window = p.window;
   a.has_mask = p.has_mask;
   a.lens = p.kv_lens;
+  a.Dv = static_cast<int>(p.head_dim);
   a.scale_log2 = scale_log2;
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
 }
@@ -350,7 +359,8 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
                           const void* k_new, const void* v_new, int32_t* kv_lens,
                           void* workspace, size_t workspace_bytes, void* stream_ptr) {
   if (d == nullptr) return GQA_ERR_NULL;
-  if (d->dtype != GQA_DTYPE_BF16 && d->dtype != GQA_DTYPE_F32) return GQA_ERR_ARG;
+  if (d->dtype != GQA_DTYPE_BF16 && d->dtype != GQA_DTYPE_F32 && d->dtype != GQA_DTYPE_F16)
+    return GQA_ERR_ARG;
   if (d->reserved != 0) return GQA_ERR_ARG;
   const int64_t lim = int64_t(1) << 31;
   if (d->batch < 0 || d->heads_kv <= 0 || d->capacity < 0 || d->head_dim <= 0 || d->n_new < 0 ||

@@ -128,7 +128,10 @@ __device__ __forceinline__ int group_of(int u, const Sched& sc, const DecodeArgs
 // MQ: several query positions per kv head (seq_q > 1): the rows of a pass
 // are (head, query) pairs, row r = head * seq_q + query, each with its own
 // visible key range and mask row.
-template <int D, int NT, bool MQ>
+// D: the padded head dim the kernel is built for (64 or 128); columns past
+// a.Dv (the problem's head dim, a multiple of 8) arrive as zeros from TMA and
+// are never written.  F16: fp16 operands instead of bf16.
+template <int D, int NT, bool MQ, bool F16>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const DecodeArgs a,
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const int r = x / (D / 8), c = x % (D / 8);
           const int hl = pass * HP + r;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (hl < a.rows) v = *reinterpret_cast<const uint4*>(q_row(hl) + c * 8);
+          if (hl < a.rows && c * 8 < a.Dv) v = *reinterpret_cast<const uint4*>(q_row(hl) + c * 8);
           *reinterpret_cast<uint4*>(q_smem + r * kQRow + c * 16) = v;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
@@ -319,9 +322,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           for (int ks = 0; ks < KSTEPS; ++ks) {
             const int d0 = ks * 16 + (lane & 3) * 2;
             bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][0] =
-                ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+                (ok && d0 < a.Dv) ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
             bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][1] =
-                ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+                (ok && d0 + 8 < a.Dv) ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
           }
         }
 #pragma unroll
@@ -442,7 +445,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // elements per thread.
         for (int idx = threadIdx.x; idx < HP * D / 2; idx += NCW * 32) {
           const int h = idx / (D / 2), d = (idx % (D / 2)) * 2;
-          if (pass * HP + h >= a.rows) continue;
+          if (pass * HP + h >= a.rows || d >= a.Dv) continue;
           float M = -INFINITY;
 #pragma unroll
           for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, m_of(w, h));
@@ -458,7 +461,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
           }
           const float inv = 1.f / l;  // l == 0: NaN
-          *reinterpret_cast<uint32_t*>(out_row(h) + d) = pack_bf16x2(acc0 * inv, acc1 * inv);
+          *reinterpret_cast<uint32_t*>(out_row(h) + d) = pack2<F16>(acc0 * inv, acc1 * inv);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
         return;
@@ -508,7 +511,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           for (int k = 0; k < kFastMerge; ++k) base[k] = slot_of(c_lo + (k < n ? k : 0));
           for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
             const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
-            if (pass * HP + h >= a.rows) continue;
+            if (pass * HP + h >= a.rows || d >= a.Dv) continue;
             float2 ml[kFastMerge];
             float4 ov[kFastMerge];
 #pragma unroll
@@ -539,8 +542,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
             const float inv = 1.f / Lsum;  // Lsum == 0: NaN
             uint2 pk;
-            pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-            pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            pk.x = pack2<F16>(acc.x * inv, acc.y * inv);
+            pk.y = pack2<F16>(acc.z * inv, acc.w * inv);
             *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
           }
         } else {
@@ -571,7 +574,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
           for (int idx = threadIdx.x; idx < HP * D / 4; idx += NCW * 32) {
             const int h = idx / (D / 4), d = (idx % (D / 4)) * 4;
-            if (pass * HP + h >= a.rows) continue;
+            if (pass * HP + h >= a.rows || d >= a.Dv) continue;
             const float M = sm_ml[2 * h], Lsum = sm_ml[2 * h + 1];
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             if (M != -INFINITY) {
@@ -588,8 +591,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
             const float inv = 1.f / Lsum;  // Lsum == 0: NaN
             uint2 pk;
-            pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-            pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+            pk.x = pack2<F16>(acc.x * inv, acc.y * inv);
+            pk.y = pack2<F16>(acc.z * inv, acc.w * inv);
             *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
           }
         }
@@ -661,12 +664,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 smem_u32(q_smem) + qr * kQRow + ks * 32 + ((lane >> 3) & 1) * 16;
             uint32_t q0, q1, q2, q3;
             ldmatrix_x4(q0, q1, q2, q3, qaddr);
-            mma_bf16_16816(sc[0], a0, a1, a2, a3, q0, q1);
-            mma_bf16_16816(sc[NT - 1], a0, a1, a2, a3, q2, q3);
+            mma_16816<F16>(sc[0], a0, a1, a2, a3, q0, q1);
+            mma_16816<F16>(sc[NT - 1], a0, a1, a2, a3, q2, q3);
           } else {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              mma_bf16_16816((kSplit && (ks & 1)) ? sc2[nt] : sc[nt], a0, a1, a2, a3,
+              mma_16816<F16>((kSplit && (ks & 1)) ? sc2[nt] : sc[nt], a0, a1, a2, a3,
                              bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][0],
                              bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][1]);
           }
@@ -717,8 +720,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           o[nt][mt][3] *= alpha[1];
         }
         // P^T as the B operand: transpose the two 8x8 (keys x heads) blocks.
-        pt0[nt] = movmatrix_trans(pack_bf16x2(tv[0], tv[1]));
-        pt1[nt] = movmatrix_trans(pack_bf16x2(tv[2], tv[3]));
+        pt0[nt] = movmatrix_trans(pack2<F16>(tv[0], tv[1]));
+        pt1[nt] = movmatrix_trans(pack2<F16>(tv[2], tv[3]));
       }
 
       // O^T[D x 8] += V^T[D x 16 keys] P^T[16 keys x 8], once the V tile is in.
@@ -740,7 +743,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           ldmatrix_x4_trans(a0, a1, a2, a3, addr);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, pt0[nt], pt1[nt]);
+            mma_16816<F16>(o[nt][mt], a0, a1, a2, a3, pt0[nt], pt1[nt]);
         }
       }
       __syncwarp();
@@ -751,10 +754,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
 }
 
-template <int D, int NT, bool MQ>
+template <int D, int NT, bool MQ, bool F16>
 int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap& tmk,
                     const CUtensorMap& tmv, cudaStream_t stream) {
-  auto kern = gqa_decode_kernel<D, NT, MQ>;
+  auto kern = gqa_decode_kernel<D, NT, MQ, F16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_bytes) !=
       cudaSuccess)
     return GQA_ERR_CUDA;
@@ -770,7 +773,7 @@ DecodeShape plan_decode(const gqa_problem& p, int sm_count) {
   DecodeShape s{};
   const int64_t g = p.heads_q / p.heads_kv;
   const int64_t rows = g * p.seq_q;  // (head, query) rows per kv head
-  s.D = static_cast<int>(p.head_dim);
+  s.D = p.head_dim <= 64 ? 64 : 128;  // padded: TMA fills the columns past head_dim with zeros
   s.NT = rows <= 8 ? 1 : 2;
   s.HP = 8 * s.NT;
   s.passes = static_cast<int>((rows + s.HP - 1) / s.HP);
@@ -830,6 +833,7 @@ DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const vo
   a.counters = reinterpret_cast<uint32_t*>(ws + s.counters_offset);
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.lens = p.kv_lens;
+  a.Dv = static_cast<int>(p.head_dim);
   a.B = static_cast<int>(p.batch);
   a.Hq = static_cast<int>(p.heads_q);
   a.Hkv = static_cast<int>(p.heads_kv);
@@ -844,22 +848,24 @@ DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const vo
   return a;
 }
 
+template <int D, int NT>
+int launch_decode_dt(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap& tmk,
+                     const CUtensorMap& tmv, cudaStream_t stream, bool mq, bool f16) {
+  if (f16)
+    return mq ? launch_decode_t<D, NT, true, true>(s, a, tmk, tmv, stream)
+              : launch_decode_t<D, NT, false, true>(s, a, tmk, tmv, stream);
+  return mq ? launch_decode_t<D, NT, true, false>(s, a, tmk, tmv, stream)
+            : launch_decode_t<D, NT, false, false>(s, a, tmk, tmv, stream);
+}
+
 int launch_decode(const gqa_problem& p, const DecodeShape& s, const DecodeArgs& a,
                   const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
-  (void)p;
   const bool mq = a.Sq > 1;
-  if (s.D == 128 && s.NT == 1)
-    return mq ? launch_decode_t<128, 1, true>(s, a, tmk, tmv, stream)
-              : launch_decode_t<128, 1, false>(s, a, tmk, tmv, stream);
-  if (s.D == 128 && s.NT == 2)
-    return mq ? launch_decode_t<128, 2, true>(s, a, tmk, tmv, stream)
-              : launch_decode_t<128, 2, false>(s, a, tmk, tmv, stream);
-  if (s.D == 64 && s.NT == 1)
-    return mq ? launch_decode_t<64, 1, true>(s, a, tmk, tmv, stream)
-              : launch_decode_t<64, 1, false>(s, a, tmk, tmv, stream);
-  if (s.D == 64 && s.NT == 2)
-    return mq ? launch_decode_t<64, 2, true>(s, a, tmk, tmv, stream)
-              : launch_decode_t<64, 2, false>(s, a, tmk, tmv, stream);
+  const bool f16 = p.dtype == GQA_DTYPE_F16;
+  if (s.D == 128 && s.NT == 1) return launch_decode_dt<128, 1>(s, a, tmk, tmv, stream, mq, f16);
+  if (s.D == 128 && s.NT == 2) return launch_decode_dt<128, 2>(s, a, tmk, tmv, stream, mq, f16);
+  if (s.D == 64 && s.NT == 1) return launch_decode_dt<64, 1>(s, a, tmk, tmv, stream, mq, f16);
+  if (s.D == 64 && s.NT == 2) return launch_decode_dt<64, 2>(s, a, tmk, tmv, stream, mq, f16);
   return GQA_ERR_UNSUPPORTED;
 }
 

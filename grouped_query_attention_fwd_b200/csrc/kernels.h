@@ -60,7 +60,7 @@ __host__ __device__ inline KeyRange decode_key_range(int64_t len, int64_t Sk, in
 }
 
 struct DecodeShape {
-  int D;            // 64 or 128
+  int D;            // 64 or 128: head_dim rounded up (the kernel's width)
   int NT;           // 8-head MMA column tiles per pass (1 or 2)
   int HP;           // rows per pass = 8 * NT (a row: one head, or one (head, query))
   int passes;       // ceil(g * seq_q / HP)
@@ -90,6 +90,7 @@ struct DecodeArgs {
   uint32_t* counters;  // one ticket counter per group; zeroed before each launch
   uint32_t* err;
   const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
+  int Dv;                  // head_dim (<= the kernel's D; a multiple of 8)
   int B, Hq, Hkv, Sk, g;
   int Sq, rows;            // queries per kv head; rows = g * Sq
   int causal;
@@ -134,6 +135,7 @@ struct PrefillArgs {
   uint8_t* summary;  // [B][m_tiles][n_tiles]: 0 all hidden, 1 mixed, 2 all visible
   uint32_t* err;
   const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
+  int Dv;               // head_dim (<= the kernel's D; a multiple of 8)
   int B, Hq, Hkv, Sq, Sk, g;
   int causal, has_mask;
   int64_t causal_offset, window;

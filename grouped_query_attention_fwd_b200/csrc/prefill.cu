@@ -251,7 +251,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t chunk_
   return smem_desc_sw128(saddr, chunk_bytes, 1024);
 }
 
-template <int D>
+// D: the padded head dim (64 or 128); columns past a.Dv arrive as zeros from
+// TMA and are never written.  F16: fp16 operands instead of bf16.
+template <int D, bool F16>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
@@ -398,8 +400,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+      constexpr uint32_t idesc_qk = F16 ? idesc_f16_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idesc_pv = F16 ? idesc_f16_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t q_base = smem_u32(smem + L::kQOff);
       const uint32_t k_base = smem_u32(smem + L::kKOff);
       const uint32_t v_base = smem_u32(smem + L::kVOff);
@@ -648,7 +650,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const float p1 = ((c1 & 7) < kEmuPerEight) ? exp2_poly(x1) : fast_exp2(x1);
             lp[c0 & 7] += p0;
             lp[c1 & 7] += p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            pk[e] = pack2<F16>(p0, p1);
           }
           tmem_st16(s_col + c * 16, pk);
         }
@@ -681,14 +683,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (row_valid) {
 #pragma unroll
             for (int v8 = 0; v8 < 4; ++v8) {
+              if (c * 32 + v8 * 8 >= a.Dv) break;
               uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
+              w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
                                 __uint_as_float(r[v8 * 8 + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l,
+              w.y = pack2<F16>(__uint_as_float(r[v8 * 8 + 2]) * inv_l,
                                 __uint_as_float(r[v8 * 8 + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l,
+              w.z = pack2<F16>(__uint_as_float(r[v8 * 8 + 4]) * inv_l,
                                 __uint_as_float(r[v8 * 8 + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l,
+              w.w = pack2<F16>(__uint_as_float(r[v8 * 8 + 6]) * inv_l,
                                 __uint_as_float(r[v8 * 8 + 7]) * inv_l);
               reinterpret_cast<uint4*>(orow + c * 32)[v8] = w;
             }
@@ -696,8 +699,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       } else if (row_valid) {
         const float nanv = __int_as_float(0x7fc00000);
-        const uint32_t nn = pack_bf16x2(nanv, nanv);
-        for (int d = 0; d < D; d += 8)
+        const uint32_t nn = pack2<F16>(nanv, nanv);
+        for (int d = 0; d < a.Dv; d += 8)
           *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
       }
       tc_fence_before();
@@ -740,7 +743,7 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-template <int D>
+template <int D, bool F16>
 int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
                      const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
   if (a.has_mask) {
@@ -748,7 +751,7 @@ int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensor
         a.mask, a.ms[0], a.ms[1], a.summary, a.Sq, a.Sk, s.qpt, s.m_tiles, s.n_tiles);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
-  auto kern = gqa_prefill_kernel<D>;
+  auto kern = gqa_prefill_kernel<D, F16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Layout<D>::kBytes) != cudaSuccess)
     return GQA_ERR_CUDA;
@@ -762,7 +765,7 @@ int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensor
 PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   PrefillShape s{};
   const int64_t g = p.heads_q / p.heads_kv;
-  s.D = static_cast<int>(p.head_dim);
+  s.D = p.head_dim <= 64 ? 64 : 128;  // padded: TMA fills the columns past head_dim with zeros
   s.qpt = static_cast<int>(BM / g);
   s.rows = static_cast<int>(s.qpt * g);
   s.m_tiles = static_cast<int>((p.seq_q + s.qpt - 1) / s.qpt);
@@ -779,9 +782,13 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
 int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
                    const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                    cudaStream_t stream) {
-  (void)p;
-  if (s.D == 128) return launch_prefill_t<128>(s, a, tmq, tmk, tmv, stream);
-  if (s.D == 64) return launch_prefill_t<64>(s, a, tmq, tmk, tmv, stream);
+  const bool f16 = p.dtype == GQA_DTYPE_F16;
+  if (s.D == 128)
+    return f16 ? launch_prefill_t<128, true>(s, a, tmq, tmk, tmv, stream)
+               : launch_prefill_t<128, false>(s, a, tmq, tmk, tmv, stream);
+  if (s.D == 64)
+    return f16 ? launch_prefill_t<64, true>(s, a, tmq, tmk, tmv, stream)
+               : launch_prefill_t<64, false>(s, a, tmq, tmk, tmv, stream);
   return GQA_ERR_UNSUPPORTED;
 }
 

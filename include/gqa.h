@@ -24,8 +24,9 @@
  *    mask is uint8 [batch, seq_q, seq_k], nonzero = attend, shared by every
  *    head.  Any other strides are allowed (e.g. a [B, S, H, D] buffer viewed as
  *    [B, H, S, D]), subject to the 16-byte rules below on the bf16 paths.
- *  - dtype: GQA_DTYPE_BF16 (compute in fp32, bf16 in/out, head_dim 64 or 128)
- *    or GQA_DTYPE_F32 (fp32 throughout, head_dim 1..256).
+ *  - dtype: GQA_DTYPE_BF16 or GQA_DTYPE_F16 (16-bit in/out, fp32 accumulation
+ *    and softmax, head_dim a multiple of 8 up to 128) or GQA_DTYPE_F32 (fp32
+ *    throughout, head_dim 1..256).
  *  - causal: key j is visible to query i iff j <= i + causal_offset.  The
  *    pages' causal attention (seq_q == seq_k) is causal_offset = 0 (top-left);
  *    decoding after a KV cache, bottom-right alignment, is causal_offset =
@@ -95,18 +96,19 @@ extern "C" {
 
 #define GQA_DTYPE_BF16 0
 #define GQA_DTYPE_F32 1
+#define GQA_DTYPE_F16 2
 
 #define GQA_KERNEL_NONE 0     /* nothing to launch (empty problem) */
-#define GQA_KERNEL_DECODE 1   /* bf16, seq_q == 1 or (heads_q/heads_kv) * seq_q <= 16: split-K
-                                 stream over the KV cache, one launch */
-#define GQA_KERNEL_PREFILL 2  /* bf16, longer query blocks: tcgen05 / tensor-memory tiles */
+#define GQA_KERNEL_DECODE 1   /* bf16 / fp16, seq_q == 1 or (heads_q/heads_kv) * seq_q <= 16:
+                                 split-K stream over the KV cache, one launch */
+#define GQA_KERNEL_PREFILL 2  /* bf16 / fp16, longer query blocks: tcgen05 / tensor-memory tiles */
 #define GQA_KERNEL_F32 3      /* fp32 CUDA-core path */
 #define GQA_KERNEL_ZERO 4     /* seq_k == 0: the output is filled with zeros */
 #define GQA_KERNEL_NAN 5      /* causal / window leave no key to any query: NaN (see above) */
 
 /* One attention problem.  Strides are in elements. */
 typedef struct gqa_problem {
-  int32_t dtype;          /* GQA_DTYPE_BF16 or GQA_DTYPE_F32, for q, k, v and out */
+  int32_t dtype;          /* GQA_DTYPE_BF16, GQA_DTYPE_F16 or GQA_DTYPE_F32, for q, k, v, out */
   int32_t causal;         /* nonzero: key j hidden from query i when j > i */
   int32_t has_mask;       /* nonzero: a mask pointer is passed to gqa_forward */
   float scale;            /* multiplies q.k; 1/sqrt(head_dim) reproduces the pages */
@@ -215,7 +217,7 @@ GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const void* q, cons
  * Structure", grown in place per sequence instead of concatenated).
  */
 typedef struct gqa_kv_append_desc {
-  int32_t dtype;                /* GQA_DTYPE_BF16 or GQA_DTYPE_F32 (cache and new rows alike) */
+  int32_t dtype;                /* GQA_DTYPE_BF16, F16 or F32 (cache and new rows alike) */
   int32_t reserved;             /* must be 0 */
   int64_t batch, heads_kv, capacity, head_dim, n_new;
   int64_t cache_k_stride[4];    /* over (b, h_kv, j, d), j < capacity; d stride 1 */

@@ -50,3 +50,11 @@ def to_np(t: torch.Tensor) -> np.ndarray:
 def oracle_bf16(bits_q, bits_k, bits_v, mask=None, causal=False, scale=None):
     return oracle.forward(f64(bits_q), f64(bits_k), f64(bits_v), mask=mask, causal=causal,
                           scale=scale)
+
+
+def f16_inputs(seed, B, Hq, Hkv, Sq, Sk, D, device="cuda"):
+    """Seeded N(0,1) q, k, v rounded to fp16: (float64 copies for the oracle,
+    fp16 device tensors)."""
+    q, k, v = synth.qkv_f32(seed, B, Hq, Hkv, Sq, Sk, D)
+    h = [x.astype(np.float16) for x in (q, k, v)]
+    return tuple(x.astype(np.float64) for x in h), tuple(torch.from_numpy(x).to(device) for x in h)

@@ -63,7 +63,9 @@ def _rc(gqa, p, sms=148):
     (dict(B=-1), 2),
     (dict(D=0), 2),
     (dict(Hkv=0), 2),
-    (dict(D=96), 4),                              # bf16 needs 64 or 128
+    (dict(D=100), 4),                             # bf16 / fp16: a multiple of 8
+    (dict(D=136), 4),                             # bf16 / fp16: at most 128
+    (dict(D=136, dtype=2), 4),
     (dict(D=300, dtype=1), 4),                    # fp32 path: D <= 256
     (dict(window=4), 8),                          # a window needs causal
     (dict(causal=True, window=-1), 8),
@@ -262,3 +264,17 @@ def test_workspace_layout_keeps_counters_apart(gqa):
     assert rc == 0 and pre.workspace_bytes == (region + 2 * 3 * 3 + 255) // 256 * 256  # classes after it
     rc, huge = _rc(gqa, _p(gqa, B=2100, Hq=32, Hkv=8, Sq=1, Sk=100))
     assert rc == 0 and huge.launches == 2 and huge.workspace_bytes > region + 2100 * 8 * 4
+
+
+def test_half_dtypes_and_head_dims(gqa):
+    """fp16 takes the bf16 kernels; any multiple of 8 up to 128 is accepted and
+    planned at the padded width (64 or 128)."""
+    for dtype in (0, 2):
+        for D in (8, 24, 64, 72, 96, 128):
+            rc, pl = _rc(gqa, _p(gqa, D=D, dtype=dtype))
+            assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "decode", (dtype, D)
+            rc, pl = _rc(gqa, _p(gqa, D=D, dtype=dtype, Sq=300, Sk=300, causal=True))
+            assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "prefill", (dtype, D)
+            # algorithmic bytes count the real head dim
+            rc, pl = _rc(gqa, _p(gqa, B=1, Hq=2, Hkv=1, Sq=1, Sk=10, D=D, dtype=dtype))
+            assert pl.algorithmic_bytes == 2 * (2 * D * 2) + 2 * (10 * D * 2)
