@@ -32,7 +32,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GQA_OK = 0
 GQA_ERR_NULL, GQA_ERR_SHAPE, GQA_ERR_LAYOUT, GQA_ERR_UNSUPPORTED = 1, 2, 3, 4
 GQA_ERR_WORKSPACE, GQA_ERR_CUDA, GQA_ERR_TIMEOUT, GQA_ERR_ARG, GQA_ERR_DEVICE = 5, 6, 7, 8, 9
-GQA_ERR_SCRATCH_LIMIT, GQA_ERR_KV_LENGTH = 10, 11
+GQA_ERR_SCRATCH_LIMIT, GQA_ERR_KV_LENGTH, GQA_ERR_PAGE = 10, 11, 12
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 GQA_DTYPE_BF16, GQA_DTYPE_F32, GQA_DTYPE_F16 = 0, 1, 2
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
@@ -52,6 +52,8 @@ class Problem(ctypes.Structure):
         ("mask_stride", ctypes.c_int64 * 3),
         ("causal_offset", ctypes.c_int64), ("window", ctypes.c_int64),
         ("kv_lens", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("block_table_stride", ctypes.c_int64),
+        ("page_size", ctypes.c_int64), ("num_pages", ctypes.c_int64),
     ]
 
 
@@ -62,6 +64,8 @@ class AppendDesc(ctypes.Structure):
         ("head_dim", ctypes.c_int64), ("n_new", ctypes.c_int64),
         ("cache_k_stride", ctypes.c_int64 * 4), ("cache_v_stride", ctypes.c_int64 * 4),
         ("k_new_stride", ctypes.c_int64 * 4), ("v_new_stride", ctypes.c_int64 * 4),
+        ("block_table", ctypes.c_void_p), ("block_table_stride", ctypes.c_int64),
+        ("page_size", ctypes.c_int64), ("num_pages", ctypes.c_int64),
     ]
 
 
@@ -204,15 +208,33 @@ def _lens_ptr(kv_lens, B):
     return kv_lens.data_ptr()
 
 
+def _table(block_table, B):
+    torch = _torch()
+    if not block_table.is_cuda or block_table.dtype != torch.int32 or block_table.dim() != 2 or \
+            block_table.shape[0] != B or block_table.stride(1) != 1:
+        raise ValueError("block_table must be an int32 CUDA tensor [B, pages per sequence] "
+                         "with unit stride along the pages")
+    return block_table.data_ptr(), block_table.stride(0), block_table.shape[1]
+
+
 def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None, causal_offset=None,
-                window=0, kv_lens=None) -> Problem:
+                window=0, kv_lens=None, block_table=None) -> Problem:
+    """With block_table, k and v are page pools [num_pages, Hkv, page_size, D]
+    and a sequence holds up to block_table.shape[1] * page_size keys."""
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, S, D]")
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
     B, Hq, Sq, D = q.shape
     Bk, Hkv, Sk, Dk = k.shape
-    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+    paged = block_table is not None
+    if paged:
+        num_pages, page_size = Bk, Sk
+        bt_ptr, bt_stride, per_seq = _table(block_table, B)
+        Sk = per_seq * page_size
+        if tuple(v.shape) != tuple(k.shape) or Dk != D:
+            raise ValueError("paged k and v must be [num_pages, Hkv, page_size, D] with q's D")
+    elif tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
         raise ValueError("k and v must be [B, Hkv, Sk, D] with q's B and D")
     ost = out.stride() if out is not None else (Hq * Sq * D, Sq * D, D, 1)
     mst = None
@@ -220,16 +242,21 @@ def problem_for(q, k, v, mask=None, causal=False, scale=None, out=None, causal_o
         if tuple(mask.shape) != (B, Sq, Sk):
             raise ValueError("mask must be [B, Sq, Sk]")
         mst = mask.stride()
-    return make_problem(_dtype_code(q), B, Hq, Hkv, Sq, Sk, D, q.stride(), k.stride(),
-                        v.stride(), ost, mst, causal=causal, scale=scale,
-                        causal_offset=_offset(causal, causal_offset, Sq, Sk), window=window,
-                        kv_lens_ptr=_lens_ptr(kv_lens, B))
+    p = make_problem(_dtype_code(q), B, Hq, Hkv, Sq, Sk, D, q.stride(), k.stride(),
+                     v.stride(), ost, mst, causal=causal, scale=scale,
+                     causal_offset=_offset(causal, causal_offset, Sq, Sk), window=window,
+                     kv_lens_ptr=_lens_ptr(kv_lens, B))
+    if paged:
+        p.block_table, p.block_table_stride = bt_ptr, bt_stride
+        p.page_size, p.num_pages = page_size, num_pages
+    return p
 
 
 def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0, causal_offset=None,
-          window=0, kv_lens=None) -> dict:
+          window=0, kv_lens=None, block_table=None) -> dict:
     return query_problem(problem_for(q, k, v, mask, causal, scale, causal_offset=causal_offset,
-                                     window=window, kv_lens=kv_lens), sm_count).as_dict()
+                                     window=window, kv_lens=kv_lens, block_table=block_table),
+                         sm_count).as_dict()
 
 
 def workspace_for(device, nbytes: int):
@@ -245,7 +272,7 @@ def workspace_for(device, nbytes: int):
 
 
 def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=None,
-            stream=None, causal_offset=None, window=0, kv_lens=None):
+            stream=None, causal_offset=None, window=0, kv_lens=None, block_table=None):
     """out = softmax(mask(q k_{h/g}^T * scale)) v_{h/g} on the GPU.
 
     causal: key j visible to query i iff j <= i + offset (offset 0 for
@@ -253,7 +280,10 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
     of the keys).  window > 0 keeps only the last `window` keys up to the
     diagonal (sliding-window attention).  kv_lens (int32 CUDA [B]): entry b
     holds kv_lens[b] keys of the Sk-long cache; the offset is given for a
-    full cache and moves by kv_lens[b] - Sk."""
+    full cache and moves by kv_lens[b] - Sk.  block_table (int32 CUDA
+    [B, pages per sequence]): k and v are page pools [num_pages, Hkv,
+    page_size, D] (page_size a multiple of 64) and Sk = pages per sequence *
+    page_size."""
     torch = _torch()
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors (there is no CPU path)")
@@ -267,7 +297,7 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
     p = problem_for(q, k, v, mask, causal, scale, out, causal_offset=causal_offset, window=window,
-                    kv_lens=kv_lens)
+                    kv_lens=kv_lens, block_table=block_table)
     plan = query_problem(p)
     if workspace is None:
         workspace = workspace_for(q.device, plan.workspace_bytes)
@@ -299,11 +329,13 @@ def kv_append_ptrs(d: AppendDesc, cache_k: int, cache_v: int, k_new: int, v_new:
         raise GQAError(rc, "gqa_kv_append")
 
 
-def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=None):
+def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=None,
+              block_table=None):
     """Write k_new / v_new [B, Hkv, n_new, D] into rows kv_lens[b] .. kv_lens[b] + n_new
     of cache_k / cache_v [B, Hkv, capacity, D], then advance kv_lens (int32 CUDA [B])
     in place.  An entry that does not fit is left as it was and device_status()
-    reports GQA_ERR_KV_LENGTH."""
+    reports GQA_ERR_KV_LENGTH.  With block_table the caches are page pools
+    [num_pages, Hkv, page_size, D] and capacity = pages per sequence * page_size."""
     torch = _torch()
     for t in (cache_k, cache_v, k_new, v_new, kv_lens):
         if not t.is_cuda:
@@ -311,6 +343,11 @@ def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=No
     if cache_k.dim() != 4 or tuple(cache_v.shape) != tuple(cache_k.shape):
         raise ValueError("cache_k and cache_v must be [B, Hkv, capacity, D]")
     B, Hkv, cap, D = cache_k.shape
+    if block_table is not None:
+        num_pages, page_size = B, cap
+        B = k_new.shape[0]
+        bt_ptr, bt_stride, per_seq = _table(block_table, B)
+        cap = per_seq * page_size
     if k_new.dim() != 4 or tuple(v_new.shape) != tuple(k_new.shape) or \
             k_new.shape[0] != B or k_new.shape[1] != Hkv or k_new.shape[3] != D:
         raise ValueError("k_new and v_new must be [B, Hkv, n_new, D]")
@@ -318,6 +355,9 @@ def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=No
         raise TypeError("cache and new rows must share a dtype")
     d = append_desc(_dtype_code(cache_k), B, Hkv, cap, D, k_new.shape[2], cache_k.stride(),
                     cache_v.stride(), k_new.stride(), v_new.stride())
+    if block_table is not None:
+        d.block_table, d.block_table_stride = bt_ptr, bt_stride
+        d.page_size, d.num_pages = page_size, num_pages
     lp = _lens_ptr(kv_lens, B)
     if workspace is None:
         workspace = workspace_for(cache_k.device, 256)

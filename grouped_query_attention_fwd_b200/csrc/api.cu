@@ -47,8 +47,10 @@ int validate(const gqa_problem* pp) {
     // filling the columns past head_dim with zeros.
     if (p.head_dim % 8 != 0 || p.head_dim > 128) return GQA_ERR_UNSUPPORTED;
     // 16-byte rule of the TMA unit for every stride of a dimension longer than 1.
+    // A paged k / v runs over (page, kv head, key in page).
     const int64_t qsz[3] = {p.batch, p.heads_q, p.seq_q};
-    const int64_t ksz[3] = {p.batch, p.heads_kv, p.seq_k};
+    const int64_t ksz[3] = {p.block_table ? p.num_pages : p.batch, p.heads_kv,
+                            p.block_table ? p.page_size : p.seq_k};
     for (int d = 0; d < 3; ++d) {
       if (qsz[d] > 1 && (p.q_stride[d] % 8 != 0 || p.o_stride[d] % 8 != 0)) return GQA_ERR_LAYOUT;
       if (ksz[d] > 1 && (p.k_stride[d] % 8 != 0 || p.v_stride[d] % 8 != 0)) return GQA_ERR_LAYOUT;
@@ -59,6 +61,13 @@ int validate(const gqa_problem* pp) {
     }
   } else {
     if (p.head_dim > 256) return GQA_ERR_UNSUPPORTED;
+  }
+  if (p.block_table != nullptr) {
+    // Pages hold whole 64-key halves of the decode kernel's 128-key tiles.
+    if (p.page_size < 64 || p.page_size % 64 != 0 || p.page_size >= lim) return GQA_ERR_SHAPE;
+    if (p.block_table_stride < 1 || p.block_table_stride >= lim) return GQA_ERR_SHAPE;
+    if (p.num_pages < 1 || p.num_pages >= lim) return GQA_ERR_SHAPE;
+    if (p.seq_k > p.block_table_stride * p.page_size) return GQA_ERR_SHAPE;
   }
   if (p.kv_lens != nullptr) {
     // The decode kernel keeps the lengths and their prefix sums in shared
@@ -154,6 +163,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       break;
     }
     case GQA_KERNEL_PREFILL: {
+      if (p.block_table != nullptr) return GQA_ERR_UNSUPPORTED;  // paged: decode and fp32 only
       const PrefillShape s = plan_prefill(p, sm_count);
       plan->grid = s.grid;
       plan->block = kPrefillThreads;
@@ -222,8 +232,12 @@ namespace gqa {
 // decode entry point.
 int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& p,
                          const int64_t st[4]) {
+  const bool f16 = p.dtype == GQA_DTYPE_F16;
+  if (p.block_table != nullptr)  // (d, key in page, kv head, page), 64-key boxes
+    return encode_half_map(map, base, p.num_pages, p.heads_kv, p.page_size, p.head_dim, st,
+                           kDecodePageBox, 1, f16);
   return encode_half_map(map, base, p.batch, p.heads_kv, p.seq_k, p.head_dim, st,
-                         kDecodeKeysPerTile, 1, p.dtype == GQA_DTYPE_F16);
+                         kDecodeKeysPerTile, 1, f16);
 }
 }  // namespace gqa
 
@@ -247,6 +261,7 @@ GQA_API const char* gqa_status_string(int status) {
     case GQA_ERR_DEVICE: return "no usable sm_100 CUDA device";
     case GQA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the library's static array holds";
     case GQA_ERR_KV_LENGTH: return "a kv length was outside [0, capacity], or an append did not fit the cache";
+    case GQA_ERR_PAGE: return "a block-table entry in use was outside [0, num_pages)";
     default: return "unknown status";
   }
 }
@@ -367,6 +382,10 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
       d->batch >= lim || d->heads_kv >= lim || d->capacity >= lim || d->head_dim > 4096)
     return GQA_ERR_SHAPE;
   if (d->n_new > d->capacity) return GQA_ERR_SHAPE;
+  if (d->block_table != nullptr &&
+      (d->page_size < 1 || d->block_table_stride < 1 || d->num_pages < 1 ||
+       d->capacity > d->block_table_stride * d->page_size))
+    return GQA_ERR_SHAPE;
   const int64_t* st[4] = {d->cache_k_stride, d->cache_v_stride, d->k_new_stride, d->v_new_stride};
   for (const int64_t* x : st) {
     if (x[3] != 1) return GQA_ERR_LAYOUT;
@@ -407,6 +426,10 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
   for (int i = 0; i < 3 && v16; ++i)
     v16 = a.cks[i] % 16 == 0 && a.cvs[i] % 16 == 0 && a.kns[i] % 16 == 0 && a.vns[i] % 16 == 0;
   a.vec = v16 ? 16 : eb;
+  a.bt = d->block_table;
+  a.bt_stride = d->block_table_stride;
+  a.page_size = d->page_size;
+  a.num_pages = d->num_pages;
   return launch_kv_append(a, static_cast<cudaStream_t>(stream_ptr));
 }
 
@@ -424,8 +447,9 @@ GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* str
     cudaGetLastError();
     return GQA_ERR_CUDA;
   }
-  if (word[0] == kErrKvLength) {
-    // Only a length was out of range: the kernels finished normally.
+  if (word[0] != 0 && (word[0] & ~(kErrKvLength | kErrPage)) == 0) {
+    // Only a length or a page index was out of range: the kernels finished.
+    const int status = (word[0] & kErrKvLength) ? GQA_ERR_KV_LENGTH : GQA_ERR_PAGE;
     const uint32_t zero = 0;
     if (cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, stream) !=
             cudaSuccess ||
@@ -433,7 +457,7 @@ GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* str
       cudaGetLastError();
       return GQA_ERR_CUDA;
     }
-    return GQA_ERR_KV_LENGTH;
+    return status;
   }
   if (word[0] != 0) {
     // A kernel gave up part-way: its split counters may be off.  Return the

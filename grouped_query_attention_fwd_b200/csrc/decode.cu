@@ -224,6 +224,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       prefetch_tmap(&tmv);
       int it = 0;
       Cursor cu;
+      // Paged cache: each 128-key tile is two 64-key boxes, each in one page.
+      // The block-table entries of the next unit are loaded one iteration
+      // ahead, so their latency overlaps the wait for a free stage.  A box
+      // past the sequence's length takes page index num_pages, out of range:
+      // TMA fills it with zeros and reads nothing.
+      const bool paged = a.bt != nullptr;
+      Cursor cn;
+      int npage[2] = {0, 0}, nrow[2] = {0, 0};
+      bool nuse[2] = {false, false};
+      auto fetch_pages = [&](int u) {
+        seek(cn, u, sc, a);
+        const int r = u - cn.beg;
+        const int gi = r / cn.kr.tiles;
+        const int key0 = (r - gi * cn.kr.tiles + cn.kr.t0) * KT;
+        const int len = sc.len ? sc.len[cn.b] : a.Sk;
+#pragma unroll
+        for (int h = 0; h < KT / kDecodePageBox; ++h) {
+          const int key = key0 + h * kDecodePageBox;
+          nuse[h] = key < len;
+          nrow[h] = key % a.page_size;
+          npage[h] = nuse[h] ? __ldg(a.bt + cn.b * a.bt_stride + key / a.page_size) : a.num_pages;
+        }
+      };
+      if (paged && u_begin < u_end) fetch_pages(u_begin);
       for (int u = u_begin; u < u_end; ++u, ++it) {
         const int s = it % stages;
         const uint32_t round = static_cast<uint32_t>(it / stages);
@@ -237,6 +261,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int kv = gi / passes;
         const int b = cu.b;
         uint8_t* st = ring + s * L::kStageBytes;
+        if (paged) {
+          int page[2], prow[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            page[h] = npage[h];
+            prow[h] = nrow[h];
+            if (nuse[h] && (page[h] < 0 || page[h] >= a.num_pages)) {
+              atomicOr(a.err, kErrPage);
+              page[h] = a.num_pages;  // read as zeros
+            }
+          }
+          if (u + 1 < u_end) fetch_pages(u + 1);
+          mbar_arrive_expect_tx(&full[s], L::kTileBytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = 0; c < CHUNKS; ++c)
+              tma_load_4d(st + c * CHUNK_BYTES + h * kDecodePageBox * 128, &tmk, &full[s], c * 64,
+                          prow[h], kv, page[h]);
+          mbar_arrive_expect_tx(&full_v[s], L::kTileBytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = 0; c < CHUNKS; ++c)
+              tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES + h * kDecodePageBox * 128, &tmv,
+                          &full_v[s], c * 64, prow[h], kv, page[h]);
+          continue;
+        }
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c)
@@ -730,6 +782,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
         continue;
       }
+      if ((tile + 1) * KT > cur_len) {
+        // Cache rows past the sequence's length may hold anything (NaN
+        // included), and zero weights would not cancel them: clear this
+        // warp's V rows for those keys before its PV reads them.
+        const int row0 = warp * 16;
+        for (int x = lane; x < 16 * CHUNKS * 8; x += 32) {
+          const int rr = x / (CHUNKS * 8), c = (x / 8) % CHUNKS, q16 = x % 8;
+          if (tile * KT + row0 + rr >= cur_len)
+            *reinterpret_cast<uint4*>(ring + s * L::kStageBytes + L::kTileBytes + c * CHUNK_BYTES +
+                                      (row0 + rr) * 128 + q16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // before the stage's next TMA write
+        __syncwarp();
+      }
       {
         const int mi = lane >> 3;
         const int key = warp * 16 + (mi >> 1) * 8 + (lane & 7);
@@ -834,6 +900,10 @@ DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const vo
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.lens = p.kv_lens;
   a.Dv = static_cast<int>(p.head_dim);
+  a.bt = p.block_table;
+  a.bt_stride = p.block_table_stride;
+  a.page_size = static_cast<int>(p.page_size);
+  a.num_pages = static_cast<int>(p.num_pages);
   a.B = static_cast<int>(p.batch);
   a.Hq = static_cast<int>(p.heads_q);
   a.Hkv = static_cast<int>(p.heads_kv);

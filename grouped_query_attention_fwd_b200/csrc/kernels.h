@@ -16,6 +16,7 @@ constexpr int kDecodeConsumerWarps = 8;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kDecodeMaxRowsPerPass = 16;  // (head, query) rows in the MMA N dimension
 constexpr int kDecodeMaxSmem = 227 * 1024;  // dynamic shared memory one CTA may take
+constexpr int kDecodePageBox = 64;          // keys per TMA box of a paged cache
 constexpr int64_t kMaxRaggedBatch = 16384;  // batch entries with per-sequence lengths
 
 // Workspace layout shared by every call: bytes [0, 256) hold the error word
@@ -91,6 +92,9 @@ struct DecodeArgs {
   uint32_t* err;
   const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
   int Dv;                  // head_dim (<= the kernel's D; a multiple of 8)
+  const int32_t* bt;       // paged cache: block table, or nullptr (contiguous k / v)
+  int64_t bt_stride;
+  int page_size, num_pages;
   int B, Hq, Hkv, Sk, g;
   int Sq, rows;            // queries per kv head; rows = g * Sq
   int causal;
@@ -164,6 +168,8 @@ struct AppendArgs {
   int64_t cap, n_new;
   int row_bytes;        // head_dim * element bytes
   int vec;              // bytes per copied vector: 16, 4 or 2
+  const int32_t* bt;    // paged cache: block table, or nullptr
+  int64_t bt_stride, page_size, num_pages;
 };
 
 int launch_kv_append(const AppendArgs& a, cudaStream_t stream);

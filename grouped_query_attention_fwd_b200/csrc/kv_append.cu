@@ -39,8 +39,16 @@ __global__ void __launch_bounds__(256) gqa_kv_append_kernel(const AppendArgs a) 
     const int64_t* cs = is_v ? a.cvs : a.cks;
     const uint8_t* src = (is_v ? a.vn : a.kn) + b * ns[0] + h * ns[1] + t * ns[2] +
                          static_cast<int64_t>(c) * sizeof(V);
-    uint8_t* dst = (is_v ? a.cv : a.ck) + b * cs[0] + h * cs[1] + (len + t) * cs[2] +
-                   static_cast<int64_t>(c) * sizeof(V);
+    int64_t row_off = b * cs[0] + (len + t) * cs[2];
+    if (a.bt != nullptr) {  // paged: row len + t of entry b lives in a page of the pool
+      const int64_t page = a.bt[b * a.bt_stride + (len + t) / a.page_size];
+      if (page < 0 || page >= a.num_pages) {
+        if (!is_v && h == 0 && c == 0) atomicOr(a.err, kErrPage);
+        continue;
+      }
+      row_off = page * cs[0] + ((len + t) % a.page_size) * cs[2];
+    }
+    uint8_t* dst = (is_v ? a.cv : a.ck) + row_off + h * cs[1] + static_cast<int64_t>(c) * sizeof(V);
     *reinterpret_cast<V*>(dst) = *reinterpret_cast<const V*>(src);
   }
 
@@ -56,7 +64,15 @@ __global__ void __launch_bounds__(256) gqa_kv_append_kernel(const AppendArgs a) 
     __threadfence();
     for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
       const int64_t len = a.lens[b];
-      if (len >= 0 && len <= a.cap - a.n_new) a.lens[b] = static_cast<int32_t>(len + a.n_new);
+      if (len < 0 || len > a.cap - a.n_new) continue;
+      bool pages_ok = true;  // every page the new rows went to was in the pool
+      if (a.bt != nullptr) {
+        for (int64_t pg = len / a.page_size; pg <= (len + a.n_new - 1) / a.page_size; ++pg) {
+          const int64_t page = a.bt[b * a.bt_stride + pg];
+          pages_ok = pages_ok && page >= 0 && page < a.num_pages;
+        }
+      }
+      if (pages_ok) a.lens[b] = static_cast<int32_t>(len + a.n_new);
     }
     if (threadIdx.x == 0) atomicExch(a.ticket, 0u);
   }

@@ -103,6 +103,7 @@ enum : uint32_t {
   kErrPrefillWait = 1u << 1,
   kErrBadArgs = 1u << 2,
   kErrKvLength = 1u << 3,  // a kv_lens entry outside [0, capacity]: clamped, result undefined
+  kErrPage = 1u << 4,      // a block-table entry in use outside [0, num_pages): read as zeros
 };
 
 // Bounded wait on `bar` reaching phase `parity`.  Returns false if another

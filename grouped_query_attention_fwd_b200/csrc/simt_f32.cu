@@ -24,7 +24,8 @@ __global__ void __launch_bounds__(256)
                    int64_t ks1, int64_t ks2, int64_t vs0, int64_t vs1, int64_t vs2, int64_t os0,
                    int64_t os1, int64_t os2, int64_t ms0, int64_t ms1, int causal,
                    int64_t causal_offset, int64_t window, const int32_t* __restrict__ lens,
-                   uint32_t* __restrict__ err, float scale_log2) {
+                   const int32_t* __restrict__ bt, int64_t bt_stride, int64_t page_size,
+                   int64_t num_pages, uint32_t* __restrict__ err, float scale_log2) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= B * Hq * Sq) return;
@@ -35,8 +36,10 @@ __global__ void __launch_bounds__(256)
   const int64_t kv = h / g;
 
   const float* qr = q + b * qs0 + h * qs1 + i * qs2;
-  const float* kb = k + b * ks0 + kv * ks1;
-  const float* vb = v + b * vs0 + kv * vs1;
+  // Contiguous: key j of entry b at b * s0 + kv * s1 + j * s2.  Paged: at
+  // page * s0 + kv * s1 + (j % page_size) * s2, page from the block table.
+  const float* kb = k + (bt ? 0 : b * ks0) + kv * ks1;
+  const float* vb = v + (bt ? 0 : b * vs0) + kv * vs1;
   const uint8_t* mrow = mask ? mask + b * ms0 + i * ms1 : nullptr;
 
   float qv[kMaxDPerLane], acc[kMaxDPerLane];
@@ -65,7 +68,17 @@ __global__ void __launch_bounds__(256)
   }
   for (int64_t j = jbeg; j < jend; ++j) {
     if (mrow != nullptr && mrow[j] == 0) continue;
-    const float* kr = kb + j * ks2;
+    int64_t koff = j * ks2, voff = j * vs2;
+    if (bt != nullptr) {
+      const int64_t page = bt[b * bt_stride + j / page_size];
+      if (page < 0 || page >= num_pages) {
+        if (lane == 0) atomicOr(err, kErrPage);
+        continue;  // the result is undefined once this is reported; skip the key
+      }
+      koff = page * ks0 + (j % page_size) * ks2;
+      voff = page * vs0 + (j % page_size) * vs2;
+    }
+    const float* kr = kb + koff;
     float dot = 0.f;
 #pragma unroll
     for (int e = 0; e < kMaxDPerLane; ++e) {
@@ -79,7 +92,7 @@ __global__ void __launch_bounds__(256)
     const float alpha = exp2f(m - m_new);
     const float p = exp2f(t - m_new);
     l = l * alpha + p;
-    const float* vr = vb + j * vs2;
+    const float* vr = vb + voff;
 #pragma unroll
     for (int e = 0; e < kMaxDPerLane; ++e) {
       const int64_t d = lane + 32 * e;
@@ -126,7 +139,8 @@ int launch_f32(const gqa_problem& p, const float* q, const float* k, const float
       p.seq_k, p.head_dim, p.q_stride[0], p.q_stride[1], p.q_stride[2], p.k_stride[0],
       p.k_stride[1], p.k_stride[2], p.v_stride[0], p.v_stride[1], p.v_stride[2], p.o_stride[0],
       p.o_stride[1], p.o_stride[2], p.mask_stride[0], p.mask_stride[1], p.causal,
-      p.causal_offset, p.window, p.kv_lens, err, scale_log2);
+      p.causal_offset, p.window, p.kv_lens, p.block_table, p.block_table_stride, p.page_size,
+      p.num_pages, err, scale_log2);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

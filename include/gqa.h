@@ -44,7 +44,18 @@
  *    Multi-Head Attention: Understanding GQA Implementation", "Memory
  *    Footprint and KV-Cache Optimization", describes, with a per-sequence T.
  *    A length outside [0, seq_k] is clamped and reported by gqa_device_status
- *    as GQA_ERR_KV_LENGTH.
+ *    as GQA_ERR_KV_LENGTH.  The decode path never lets cache rows past a
+ *    length reach the result; the prefill path multiplies them by zero
+ *    weights, so there they must hold finite values (zeros, or old keys).
+ *  - Paged cache (block_table != NULL; decode and fp32 paths): k and v point
+ *    to a pool of num_pages pages, each [heads_kv, page_size, head_dim],
+ *    described by k_stride / v_stride over (page, h_kv, key in page, d).  Key
+ *    j of batch entry b lives in page block_table[b * block_table_stride +
+ *    j / page_size], row j % page_size.  page_size is a multiple of 64;
+ *    seq_k <= block_table_stride * page_size is the capacity of a sequence.
+ *    Pages past a sequence's length are never read, so their table entries
+ *    may hold anything; a page index outside [0, num_pages) for a key below
+ *    the length reads zeros and is reported as GQA_ERR_PAGE.
  *  - A row whose keys are all hidden yields NaN (the softmax of an all -inf
  *    row).  seq_k == 0 yields zeros (an empty weighted sum).  batch == 0 or
  *    seq_q == 0 is a no-op.
@@ -93,6 +104,8 @@ extern "C" {
                                     than GQA_STATIC_SCRATCH_BYTES */
 #define GQA_ERR_KV_LENGTH 11  /* gqa_device_status: a kv_lens entry was outside [0, seq_k], or an
                                  append did not fit the cache (that entry was left unchanged) */
+#define GQA_ERR_PAGE 12       /* gqa_device_status: a block-table entry used for a key below
+                                 the length was outside [0, num_pages) */
 
 #define GQA_DTYPE_BF16 0
 #define GQA_DTYPE_F32 1
@@ -121,6 +134,10 @@ typedef struct gqa_problem {
   int64_t causal_offset;  /* with causal: key j visible to query i iff j <= i + causal_offset */
   int64_t window;         /* with causal, > 0: keys j <= i + causal_offset - window hidden too */
   const int32_t* kv_lens; /* NULL, or device [batch]: valid keys per entry (see above) */
+  const int32_t* block_table; /* NULL (contiguous k / v), or device [batch, block_table_stride] */
+  int64_t block_table_stride; /* entries per batch row of block_table */
+  int64_t page_size;          /* keys per page, a multiple of 64 */
+  int64_t num_pages;          /* pages in the k / v pools */
 } gqa_problem;
 
 /* What gqa_forward will do for a problem on a device. */
@@ -224,6 +241,11 @@ typedef struct gqa_kv_append_desc {
   int64_t cache_v_stride[4];
   int64_t k_new_stride[4];      /* over (b, h_kv, t, d), t < n_new; d stride 1 */
   int64_t v_new_stride[4];
+  /* Paged cache (block_table != NULL): cache_k / cache_v are page pools and
+   * their strides run over (page, h_kv, key in page, d), as for gqa_forward;
+   * capacity is then the largest length a sequence may reach. */
+  const int32_t* block_table;
+  int64_t block_table_stride, page_size, num_pages;
 } gqa_kv_append_desc;
 
 /*
@@ -231,7 +253,10 @@ typedef struct gqa_kv_append_desc {
  * 0 <= L <= capacity - n_new: cache_k[b, :, L + t, :] = k_new[b, :, t, :] and
  * the same for v, for t < n_new, then kv_lens[b] = L + n_new.  An entry that
  * does not fit is left unchanged (cache and length) and gqa_device_status
- * then returns GQA_ERR_KV_LENGTH.
+ * then returns GQA_ERR_KV_LENGTH.  With a block table, row L + t of entry b is
+ * row (L + t) % page_size of page block_table[b * stride + (L + t) /
+ * page_size]; an entry whose new rows would use a page index outside
+ * [0, num_pages) is left unchanged and reported as GQA_ERR_PAGE.
  *   cache_k, cache_v, k_new, v_new: device pointers described by `d`; the new
  *                 rows must not overlap the cache.
  *   kv_lens:      device int32 [batch], read and updated in place.

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(gqa):
 
 
 def test_status_strings(gqa):
-    for code in range(0, 12):
+    for code in range(0, 13):
         s = gqa.status_string(code)
         assert s and s != "unknown status"
     assert gqa.status_string(1234) == "unknown status"
@@ -278,3 +278,31 @@ def test_half_dtypes_and_head_dims(gqa):
             # algorithmic bytes count the real head dim
             rc, pl = _rc(gqa, _p(gqa, B=1, Hq=2, Hkv=1, Sq=1, Sk=10, D=D, dtype=dtype))
             assert pl.algorithmic_bytes == 2 * (2 * D * 2) + 2 * (10 * D * 2)
+
+
+def test_paged_validation(gqa):
+    fake = 1 << 20
+    base = dict(B=4, Hq=32, Hkv=8, Sq=1, Sk=1024, block_table=fake, block_table_stride=8,
+                num_pages=100, kv_lens=fake)
+    # pool strides over (page, kv head, key in page, d)
+    pool = (8 * 128 * 128, 128 * 128, 128, 1)
+    rc, pl = _rc(gqa, _p(gqa, **base, page_size=128, k_stride=pool, v_stride=pool))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "decode"
+    assert _rc(gqa, _p(gqa, **base, page_size=96, k_stride=pool, v_stride=pool))[0] == 2
+    assert _rc(gqa, _p(gqa, **dict(base, Sk=1025), page_size=128, k_stride=pool,
+                       v_stride=pool))[0] == 2        # more keys than the table can address
+    assert _rc(gqa, _p(gqa, **dict(base, num_pages=0), page_size=128, k_stride=pool,
+                       v_stride=pool))[0] == 2
+    # the prefill path takes contiguous caches only
+    rc, _ = _rc(gqa, _p(gqa, **dict(base, Sq=300, causal=True, causal_offset=724),
+                        page_size=128, k_stride=pool, v_stride=pool))
+    assert rc == gqa.GQA_ERR_UNSUPPORTED
+    # fp32 gathers through the table too
+    rc, pl = _rc(gqa, _p(gqa, **base, page_size=128, dtype=1, k_stride=pool, v_stride=pool))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "f32"
+
+
+def test_paged_append_validation(gqa):
+    d = _append(gqa, cap=1024)
+    d.block_table, d.block_table_stride, d.page_size, d.num_pages = 256, 4, 128, 16
+    assert _append_rc(gqa, d) == gqa.GQA_ERR_SHAPE   # 4 pages of 128 < capacity 1024
