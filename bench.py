@@ -57,6 +57,12 @@ DECODE_RAGGED = dict(name="decode_ragged_cache", B=16, Hq=32, Hkv=8, Sq=1, Sk=40
 # grown cache (bottom-right causal); capacity leaves room for the appends.
 DECODE_STEP = dict(name="decode_step_append", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096 + 512, D=128,
                    causal=True, mask=False, seed=7, lens=(256, 4096), append=1)
+# The ragged cache held in 64-key pages of a shuffled pool (block table per sequence).
+DECODE_PAGED = dict(name="decode_paged_cache", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128,
+                    causal=False, mask=False, seed=6, lens=(256, 4096), append=0, page=64)
+# The Mistral-7B-shaped decode with fp16 operands, and with head dim 96.
+DECODE_F16 = dict(DECODE, name="decode_mistral7b_layer_fp16", dtype="f16", seed=8)
+DECODE_D96 = dict(DECODE, name="decode_head_dim_96", D=96, seed=9)
 
 L2_BYTES = 126 * 1024 * 1024
 
@@ -159,11 +165,19 @@ class ClockSampler:
 # ------------------------------------------------------------------ inputs
 
 def _host_inputs(cfg, torch, pin=False):
-    """Seeded q, k, v (bf16) and mask as host tensors."""
+    """Seeded q, k, v (bf16, or fp16 when cfg["dtype"] says so) and mask as
+    host tensors."""
     B, Hq, Hkv, Sq, Sk, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sq", "Sk", "D"))
     seed = cfg["seed"]
+    f16 = cfg.get("dtype") == "f16"
 
     def gen(stream, shape):
+        if f16:
+            n = 1
+            for x in shape:
+                n *= x
+            t = torch.from_numpy(synth.normal_f32(seed, stream, n).reshape(shape)).half()
+            return t.pin_memory() if pin else t
         t = torch.empty(shape, dtype=torch.bfloat16, pin_memory=pin)
         synth.normal_bf16_into(seed, stream, t.data_ptr(), t.numel())
         return t
@@ -284,8 +298,8 @@ def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
-    res = dict(total_ms=total_ms, per_launch_ms=statistics.mean(per),
-               per_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
+    res = dict(total_ms=total_ms, per_launch_ms=total_ms / steps,
+               single_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
                visible_pairs=_visible_pairs(cfg, mask))
     del ks, vs, qd, md, out
     torch.cuda.empty_cache()
@@ -311,9 +325,25 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     if n_new:
         kn = ks[0][:, :, :n_new].clone()
         vn = vs[0][:, :, :n_new].clone()
+    tables = [None] * copies
+    ps = cfg.get("page")
+    if ps:
+        # Every (sequence, page) of the cache goes to a random slot of a pool.
+        per_seq = Sk // ps
+        gen = torch.Generator().manual_seed(cfg["seed"])
+        for i in range(copies):
+            perm = torch.randperm(B * per_seq, generator=gen)
+            inv = torch.empty_like(perm)
+            inv[perm] = torch.arange(B * per_seq)
+            def pool(x):
+                return x.view(B, Hkv, per_seq, ps, D).permute(0, 2, 1, 3, 4).reshape(
+                    B * per_seq, Hkv, ps, D)[perm.to(dev)].contiguous()
+            ks[i], vs[i] = pool(ks[i]), pool(vs[i])
+            tables[i] = inv.view(B, per_seq).to(torch.int32).to(dev)
     out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
     off = "bottom_right" if cfg["causal"] else None
-    plan = gqa.query(qd, ks[0], vs[0], causal=cfg["causal"], causal_offset=off, kv_lens=lens[0])
+    plan = gqa.query(qd, ks[0], vs[0], causal=cfg["causal"], causal_offset=off, kv_lens=lens[0],
+                     block_table=tables[0])
     ws = gqa.workspace_for(dev, plan["workspace_bytes"])
     stream = torch.cuda.current_stream(dev)
 
@@ -321,7 +351,7 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
         if n_new:
             gqa.kv_append(ks[i], vs[i], kn, vn, lens[i], workspace=ws)
         gqa.forward(qd, ks[i], vs[i], out=out, workspace=ws, causal=cfg["causal"],
-                    causal_offset=off, kv_lens=lens[i])
+                    causal_offset=off, kv_lens=lens[i], block_table=tables[i])
 
     calls = [(lambda i=i: call(i)) for i in range(copies)]
     if n_new:  # every call of a copy appends n_new tokens: they must fit the capacity
@@ -342,8 +372,8 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
         mean_keys += n_new * B  # the appended token is read too
     step_bytes = (mean_keys * Hkv * D * 2 * 2 + 2 * qd.numel() * 2 +
                   (4 * B * Hkv * n_new * D * 2 if n_new else 0))
-    res = dict(total_ms=total_ms, per_launch_ms=statistics.mean(per),
-               per_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
+    res = dict(total_ms=total_ms, per_launch_ms=total_ms / steps,
+               single_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
                step_bytes=step_bytes, launches=plan["launches"] + (1 if n_new else 0),
                mean_len=mean_keys / B)
     del ks, vs, qd, out, lens
@@ -442,7 +472,8 @@ def _roofline_ragged(res, hbm, peak_kind, workload):
 
 
 WORKLOADS = {c["name"]: c for c in (DECODE, DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED,
-                                    DECODE_RAGGED, DECODE_STEP)}
+                                    DECODE_RAGGED, DECODE_STEP, DECODE_PAGED, DECODE_F16,
+                                    DECODE_D96)}
 
 
 def run_profile_case(args):
@@ -509,7 +540,10 @@ def run_gpu(args):
     if dist is not None:
         dist.barrier()
     sampler.stop()
-    per_launch = statistics.mean(per)
+    # Average launch duration over the timed region (graphs of many launches);
+    # the one-launch-graph pass adds the graph launch to every launch.
+    per_launch = elapsed_ms / args.steps
+    single_launch = statistics.median(per)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
@@ -558,12 +592,15 @@ def run_gpu(args):
             "kernel": "gqa_decode_kernel (split merge fused; the counter memset is in the same graph)",
             "algorithmic_bytes_per_launch": plan["algorithmic_bytes"],
             "launch_ms": round(per_launch, 5),
+            "launch_ms_basis": "timed region / steps (CUDA events around the graphs of launches)",
+            "single_launch_graph_median_ms": round(single_launch, 5),
         },
     }
 
     if rank == 0 and world == 1 and not args.skip_extra:
         extra = {}
-        for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED, DECODE_RAGGED, DECODE_STEP):
+        for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED, DECODE_RAGGED, DECODE_STEP,
+                  DECODE_PAGED, DECODE_F16, DECODE_D96):
             timer = _time_ragged if "lens" in c else _time_config
             try:
                 res = timer(gqa, torch, c, steps=max(3, min(args.steps, 50)),

@@ -782,19 +782,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
         continue;
       }
+      // Cache rows past the sequence's length may hold anything (NaN
+      // included), and zero weights would not cancel them: their V values
+      // are cleared in the A fragments.  Fragments a0 / a1 hold keys
+      // 2 (lane % 4) + {0, 1} of this warp's 16, a2 / a3 the same + 8, one
+      // key per 16-bit half.
+      uint32_t vm_lo = ~0u, vm_hi = ~0u;
       if ((tile + 1) * KT > cur_len) {
-        // Cache rows past the sequence's length may hold anything (NaN
-        // included), and zero weights would not cancel them: clear this
-        // warp's V rows for those keys before its PV reads them.
-        const int row0 = warp * 16;
-        for (int x = lane; x < 16 * CHUNKS * 8; x += 32) {
-          const int rr = x / (CHUNKS * 8), c = (x / 8) % CHUNKS, q16 = x % 8;
-          if (tile * KT + row0 + rr >= cur_len)
-            *reinterpret_cast<uint4*>(ring + s * L::kStageBytes + L::kTileBytes + c * CHUNK_BYTES +
-                                      (row0 + rr) * 128 + q16 * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();  // before the stage's next TMA write
-        __syncwarp();
+        const int kb = tile * KT + warp * 16 + (lane & 3) * 2;
+        vm_lo = (kb < cur_len ? 0xFFFFu : 0u) | (kb + 1 < cur_len ? 0xFFFF0000u : 0u);
+        vm_hi = (kb + 8 < cur_len ? 0xFFFFu : 0u) | (kb + 9 < cur_len ? 0xFFFF0000u : 0u);
       }
       {
         const int mi = lane >> 3;
@@ -807,6 +804,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               vbase + (dcol >> 6) * CHUNK_BYTES + key * 128 + ((u16 ^ (key & 7)) << 4);
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4_trans(a0, a1, a2, a3, addr);
+          a0 &= vm_lo;
+          a1 &= vm_lo;
+          a2 &= vm_hi;
+          a3 &= vm_hi;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
             mma_16816<F16>(o[nt][mt], a0, a1, a2, a3, pt0[nt], pt1[nt]);

@@ -680,10 +680,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           uint32_t r[32];
           tmem_ld32(o_col + c * 32, r);
           tmem_ld_wait();
-          if (row_valid) {
+          if (row_valid && c * 32 < a.Dv) {
 #pragma unroll
             for (int v8 = 0; v8 < 4; ++v8) {
-              if (c * 32 + v8 * 8 >= a.Dv) break;
+              if (a.Dv < D && c * 32 + v8 * 8 >= a.Dv) break;
               uint4 w;
               w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
                                 __uint_as_float(r[v8 * 8 + 1]) * inv_l);
