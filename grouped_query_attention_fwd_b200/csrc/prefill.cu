@@ -675,26 +675,30 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                        static_cast<int64_t>(q) * a.os[2];
       const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
       if (nloc > 0) {
+        // The whole O row in registers: every TMEM load in flight, one wait.
+        uint32_t r[D];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(o_col + c * 32, r);
-          tmem_ld_wait();
-          if (row_valid && c * 32 < a.Dv) {
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+        tmem_ld_wait();
+        // O is in registers: the next pair's first PV may overwrite it now.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[sl]);
+        if (row_valid) {
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) {
-              if (a.Dv < D && c * 32 + v8 * 8 >= a.Dv) break;
-              uint4 w;
-              w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
-                                __uint_as_float(r[v8 * 8 + 1]) * inv_l);
-              w.y = pack2<F16>(__uint_as_float(r[v8 * 8 + 2]) * inv_l,
-                                __uint_as_float(r[v8 * 8 + 3]) * inv_l);
-              w.z = pack2<F16>(__uint_as_float(r[v8 * 8 + 4]) * inv_l,
-                                __uint_as_float(r[v8 * 8 + 5]) * inv_l);
-              w.w = pack2<F16>(__uint_as_float(r[v8 * 8 + 6]) * inv_l,
-                                __uint_as_float(r[v8 * 8 + 7]) * inv_l);
-              reinterpret_cast<uint4*>(orow + c * 32)[v8] = w;
-            }
+          for (int v8 = 0; v8 < D / 8; ++v8) {
+            if (a.Dv < D && v8 * 8 >= a.Dv) break;
+            uint4 w;
+            w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 1]) * inv_l);
+            w.y = pack2<F16>(__uint_as_float(r[v8 * 8 + 2]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 3]) * inv_l);
+            w.z = pack2<F16>(__uint_as_float(r[v8 * 8 + 4]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 5]) * inv_l);
+            w.w = pack2<F16>(__uint_as_float(r[v8 * 8 + 6]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+            reinterpret_cast<uint4*>(orow)[v8] = w;
           }
         }
       } else if (row_valid) {
@@ -703,9 +707,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int d = 0; d < a.Dv; d += 8)
           *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[sl]);
+      if (nloc == 0) {  // no PV wrote O for this pair: release it as it is
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[sl]);
+      }
     }
   }
 
@@ -716,30 +722,50 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 }
 
 // summary[b][mt][nt] = 0 (all hidden), 1 (mixed) or 2 (all visible) over
-// mask[b, q0 : q0 + qpt, nt*128 : nt*128 + 128].
+// mask[b, q0 : q0 + qpt, nt*BN : nt*BN + BN].  Each thread owns a 16-byte
+// column piece and reads it down the tile's rows (one 16-byte load per row
+// when the rows are 16-byte aligned); the BN / 16 threads of a key tile then
+// combine their flags with warp shuffles.
 __global__ void __launch_bounds__(128)
     gqa_mask_summary_kernel(const uint8_t* __restrict__ mask, int64_t ms0, int64_t ms1,
                             uint8_t* __restrict__ summary, int Sq, int Sk, int qpt, int m_tiles,
-                            int n_tiles) {
+                            int n_tiles, int BN, int vec) {
   const int mt = blockIdx.x, b = blockIdx.y;
   const int q0 = mt * qpt;
   const int qn = min(qpt, Sq - q0);
-  const uint8_t* base = mask + b * ms0;
-  for (int nt = 0; nt < n_tiles; ++nt) {
-    const int j = nt * BN + threadIdx.x;
+  const uint8_t* base = mask + b * ms0 + static_cast<int64_t>(q0) * ms1;
+  const int pieces = (Sk + 15) / 16;
+  const int per_tile = BN / 16;  // 4 or 8: divides the warp, and 128 divides by it
+  for (int c0 = 0; c0 < pieces; c0 += 128) {
+    const int c = c0 + threadIdx.x;
     bool any1 = false, any0 = false;
-    if (threadIdx.x < BN && j < Sk) {
-      for (int r = 0; r < qn; ++r) {
-        const uint8_t v = base[static_cast<int64_t>(q0 + r) * ms1 + j];
-        any1 |= v != 0;
-        any0 |= v == 0;
+    if (c < pieces) {
+      const int j0 = c * 16;
+      const int nv = min(16, Sk - j0);
+      if (vec && nv == 16) {
+#pragma unroll 4
+        for (int r = 0; r < qn; ++r) {
+          const uint4 x = *reinterpret_cast<const uint4*>(base + r * ms1 + j0);
+          any1 |= (x.x | x.y | x.z | x.w) != 0u;
+          any0 |= (__vcmpeq4(x.x, 0u) | __vcmpeq4(x.y, 0u) | __vcmpeq4(x.z, 0u) |
+                   __vcmpeq4(x.w, 0u)) != 0u;
+        }
+      } else {
+        for (int r = 0; r < qn; ++r)
+          for (int e = 0; e < nv; ++e) {
+            const uint8_t v = base[r * ms1 + j0 + e];
+            any1 |= v != 0;
+            any0 |= v == 0;
+          }
       }
     }
-    const int o1 = __syncthreads_or(any1);
-    const int o0 = __syncthreads_or(any0);
-    if (threadIdx.x == 0)
-      summary[(static_cast<int64_t>(b) * m_tiles + mt) * n_tiles + nt] =
-          static_cast<uint8_t>(o1 ? (o0 ? 1 : 2) : 0);
+    for (int o = 1; o < per_tile; o <<= 1) {
+      any1 |= __shfl_xor_sync(0xffffffffu, any1, o) != 0;
+      any0 |= __shfl_xor_sync(0xffffffffu, any0, o) != 0;
+    }
+    if (c < pieces && threadIdx.x % per_tile == 0)
+      summary[(static_cast<int64_t>(b) * m_tiles + mt) * n_tiles + c / per_tile] =
+          static_cast<uint8_t>(any1 ? (any0 ? 1 : 2) : 0);
   }
 }
 
@@ -747,8 +773,11 @@ template <int D, bool F16>
 int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
                      const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
   if (a.has_mask) {
+    const bool vec = (reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0 && a.ms[0] % 16 == 0 &&
+                     a.ms[1] % 16 == 0;
     gqa_mask_summary_kernel<<<dim3(s.m_tiles, a.B), 128, 0, stream>>>(
-        a.mask, a.ms[0], a.ms[1], a.summary, a.Sq, a.Sk, s.qpt, s.m_tiles, s.n_tiles);
+        a.mask, a.ms[0], a.ms[1], a.summary, a.Sq, a.Sk, s.qpt, s.m_tiles, s.n_tiles, BN,
+        vec ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
   auto kern = gqa_prefill_kernel<D, F16>;
