@@ -1,4 +1,4 @@
-// Prefill kernel (seq_q >= 2) on the 5th-generation tensor cores.
+// Prefill kernel (longer query blocks) on the 5th-generation tensor cores.
 //
 // The g query heads that share a kv head are packed into the 128 rows (M) of
 // one tcgen05 tile: row r holds head h0 + r / qpt at query position
@@ -8,32 +8,39 @@
 // is read once and broadcast); the expanded K/V of the reference solution's
 // repeat_interleave never exists.
 //
-// Per 128x128 tile:   S = Q K^T       tcgen05.mma, A and B from shared memory,
-//                                     fp32 accumulator in tensor memory (TMEM)
-//                     P = softmax(S)  128 softmax threads, one TMEM lane (row)
-//                                     each: scale, mask, online max / sum;
-//                                     P (bf16) overwrites the first half of S
+// Per 128x128 tile:   S = Q K^T       tcgen05.mma, A = Q from TMEM (copied
+//                                     in once per query tile), B = K from
+//                                     shared memory, fp32 accumulator in TMEM
+//                     P = softmax(S)  256 softmax threads, two per TMEM lane
+//                                     (row), 64 keys each: scale, mask, online
+//                                     max / sum; P (bf16) overwrites the first
+//                                     half of S
 //                     O += P V        tcgen05.mma, A = P from TMEM, B = V from
 //                                     shared memory, O in TMEM
+// Both products read one operand from shared memory: with Q and K both there
+// the QK product ran at about half the rate of the PV product, the shared
+// memory operand bytes per FLOP being the limit.
 //
-// Two query tiles (slots A and B: consecutive query blocks of one kv head)
-// share every staged K/V tile, and their work alternates on the tensor core
-// in the order PV_A, QK_A, PV_B, QK_B: while the softmax warps of one slot
-// exponentiate, the tensor core runs the other slot's two products, so the
-// exponential unit and the tensor pipe overlap.  TMEM: S_A, S_B (128 columns
-// each), O_A, O_B (D columns each).  tcgen05.mma instructions from one thread
-// execute in issue order, so QK of a slot may follow the PV that reads the P
-// stored in the same columns.
+// S is double-buffered in TMEM, so the tensor core computes the next tile's
+// S (and the previous tile's PV) while the softmax threads work on this one:
+// the order on the tensor core is QK(0), QK(1), PV(0), QK(2), PV(1), QK(3),
+// ...; tcgen05 MMAs and copies from one thread execute in issue order, so
+// QK(j + 2) may follow the PV(j) that reads the P stored in the same columns,
+// and the next query tile's Q may be copied in after the last QK of this one.
+// TMEM (512 columns): S0, S1 (128 each), Q (D / 2: bf16 pairs), O (D).
 //
-// Warp roles (384 threads, one CTA per SM, persistent over pairs of tiles):
-//   warps 0-3  softmax, O rescale and epilogue of slot A (thread t: row t)
-//   warps 4-7  the same for slot B
+// Warp roles (384 threads, one CTA per SM, persistent over query tiles):
+//   warps 0-3  softmax, O rescale and epilogue for keys 0-63 of each S tile
+//              and the first half of the O columns (thread t: row t)
+//   warps 4-7  the same for keys 64-127 and the second half of O
 //   warp 8     TMA producer of Q tiles and K tiles
 //   warp 9     TMEM allocator and single-thread MMA issuer
 //   warp 10    TMA producer of V tiles (warp 11 idles)
-// The producer / MMA warpgroup gives registers back (setmaxnreg) so that each
-// softmax thread can hold its whole 128-score row in registers and read S
-// from TMEM once per tile.
+// One warpgroup alone spent about 1 us of every 1.3 us tile on the softmax
+// while the two products need about 0.75 us at the tensor cores' measured
+// rate; two halves bring the softmax under the tensor-core time.  The two
+// threads of a row trade their partial maxima every tile, so both pick the
+// same reference, and their row sums once per query tile.
 // The running maximum is rescaled lazily: exponentials use a reference that
 // may trail the true maximum by up to 2^8, and O and l are rescaled (O in
 // TMEM) only when the maximum grows past that.
@@ -52,23 +59,27 @@ namespace {
 
 constexpr int BM = 128;  // rows per tile = TMEM lanes
 constexpr int BN = 128;  // keys per K/V tile
+constexpr int kSoftmaxWarps = 8;  // two warpgroups, one half of the key columns each
 constexpr int kWarpQK = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpV = 10;  // warp 11 idles (it completes the third warpgroup)
-
+constexpr int kKStages = 3;  // depth of the K ring
+constexpr int kVStages = 2;  // depth of the V ring
+// One Q landing buffer: it is free again as soon as Q has been copied into
+// TMEM at the start of a query tile, long before the next tile's Q is due.
+constexpr int kQBufs = 1;
+constexpr int HK = BN / 2;  // keys of an S tile per softmax warpgroup
 // Register split across the three warpgroups (setmaxnreg): the launch gives
 // every thread kLaunchRegs; the producer / MMA warpgroup drops to kIoRegs and
 // the two softmax warpgroups rise to kSoftmaxRegs, which must add up to the
-// launch's total: 128 * kIoRegs + 256 * kSoftmaxRegs <= 384 * kLaunchRegs
-// (setmaxnreg.inc waits for registers that a larger split would never free).
+// launch's total (setmaxnreg.inc waits for registers that a larger split
+// would never free).
 constexpr int kLaunchRegs = 168;
-constexpr int kIoRegs = 88;
-constexpr int kSoftmaxRegs = 200;
+constexpr int kIoRegs = 152;
+constexpr int kSoftmaxRegs = 176;
 static_assert(128 * kIoRegs + 256 * kSoftmaxRegs <= kPrefillThreads * kLaunchRegs,
               "register split must fit in the launch allocation");
-constexpr int kStages = 2;  // depth of the K ring and of the V ring
-constexpr int kSlots = 2;   // query tiles in flight (A, B)
-static_assert(kStages == 2 && kSlots == 2, "register-packed ring bookkeeping assumes two stages and two slots");
+static_assert(kPrefillThreads == 12 * 32, "two softmax warpgroups and one producer / MMA warpgroup");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials of every eight computed on the FMA pipe (exp2_poly) rather
@@ -83,46 +94,45 @@ struct Layout {
   static constexpr int CH = D / 64;                  // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 bytes
   static constexpr int kTileBytes = CH * kChunkBytes;
-  static constexpr int kQOff = 0;                    // one Q tile per slot
-  static constexpr int kKOff = kQOff + kSlots * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kSlots + 4 * kStages + 5 * kSlots + 1;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kQBufs * kTileBytes;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + alignment slack
-  // TMEM columns: S of slot s at 128 s (P in its first 64), O at 256 + D s.
-  static constexpr uint32_t kSCol = 128;
-  static constexpr uint32_t kOCol0 = 256;
+  static constexpr int kXOff = kMiscOff + 16;  // float [2][2][128]: per-row values the halves trade
+  static constexpr int kBytes = kXOff + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
+  static constexpr uint32_t kSCol = 0;     // S buffer s at 128 s (P in its first 64 columns)
+  static constexpr uint32_t kQCol = 256;   // D / 2 columns
+  static constexpr uint32_t kOCol = 384;   // D columns
 };
 
 __device__ __forceinline__ int64_t imin64(int64_t x, int64_t y) { return x < y ? x : y; }
 __device__ __forceinline__ int64_t imax64(int64_t x, int64_t y) { return x > y ? x : y; }
 
+// Work item: one query tile of one (batch, kv head).
 struct Pair {
   int b, kv, mt0, nt_beg, nt_end;
   int len;  // cache length of entry b (seq_k without per-sequence lengths)
 };
 
-// Causal offset of the pair's entry: the diagonal moves with its length.
+// Causal offset of the item's entry: the diagonal moves with its length.
 __device__ __forceinline__ int64_t pair_off(const PrefillArgs& a, const Pair& pr) {
   return a.causal_offset + (static_cast<int64_t>(pr.len) - a.Sk);
 }
 
-struct Slot {  // one query tile of a pair
+struct Slot {  // the item's query tile
   int mt, q0, q_last;
   bool live;
   int64_t key_lo, key_hi;  // keys some row of the tile can see (causal / window)
 };
 
-// Work item x: a pair of consecutive query tiles (2p, 2p+1) of one
-// (batch, kv head); late (long causal) pairs first.
-__device__ __forceinline__ Slot slot_of(const Pair& pr, int s, const PrefillArgs& a,
-                                        int m_tiles, int qpt) {
+__device__ __forceinline__ Slot slot_of(const Pair& pr, const PrefillArgs& a, int qpt) {
   Slot sl;
-  sl.mt = pr.mt0 + s;
-  sl.live = sl.mt < m_tiles;
+  sl.mt = pr.mt0;
+  sl.live = true;
   sl.q0 = sl.mt * qpt;
-  sl.q_last = sl.live ? min(sl.q0 + qpt, a.Sq) - 1 : -1;
+  sl.q_last = min(sl.q0 + qpt, a.Sq) - 1;
   sl.key_lo = 0;
   sl.key_hi = pr.len;
   if (a.causal) {
@@ -130,48 +140,43 @@ __device__ __forceinline__ Slot slot_of(const Pair& pr, int s, const PrefillArgs
     sl.key_hi = imin64(pr.len, static_cast<int64_t>(sl.q_last) + off + 1);
     if (a.window > 0) sl.key_lo = imax64(0, static_cast<int64_t>(sl.q0) + off - a.window + 1);
   }
-  if (!sl.live || sl.key_hi <= sl.key_lo) sl.key_lo = sl.key_hi = 0;
+  if (sl.key_hi <= sl.key_lo) sl.key_lo = sl.key_hi = 0;
   return sl;
 }
 
-// Position in the heavy-first list of the r-th pair taken by CTA c: rounds
+// Position in the heavy-first list of the r-th item taken by CTA c: rounds
 // alternate direction (c, then P-1-c, ...) so that every CTA's total causal
 // work comes out nearly equal.
 __device__ __forceinline__ int64_t snake(int64_t r, int64_t c, int64_t P) {
   return r * P + ((r & 1) ? (P - 1 - c) : c);
 }
 
+// Item x: late (long causal) query tiles first.
 __device__ __forceinline__ Pair pair_of(int64_t x, const PrefillArgs& a, int m_tiles, int qpt,
                                         int n_tiles) {
   Pair pr;
   const int64_t bh = static_cast<int64_t>(a.B) * a.Hkv;
-  const int pairs = (m_tiles + 1) / 2;
-  const int p = pairs - 1 - static_cast<int>(x / bh);
   const int bk = static_cast<int>(x % bh);
   pr.b = bk / a.Hkv;
   pr.kv = bk % a.Hkv;
-  pr.mt0 = 2 * p;
+  pr.mt0 = m_tiles - 1 - static_cast<int>(x / bh);
   pr.len = a.Sk;
   if (a.lens != nullptr) {  // out-of-range lengths are clamped (and reported at kernel start)
     const int len = a.lens[pr.b];
     pr.len = len < 0 ? 0 : (len > a.Sk ? a.Sk : len);
   }
-  const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
-  // Key tiles either slot can see.
-  int64_t lo = pr.len, hi = 0;
-  if (s0.key_hi > s0.key_lo) { lo = imin64(lo, s0.key_lo); hi = imax64(hi, s0.key_hi); }
-  if (s1.key_hi > s1.key_lo) { lo = imin64(lo, s1.key_lo); hi = imax64(hi, s1.key_hi); }
-  if (hi <= lo) {
+  const Slot s0 = slot_of(pr, a, qpt);
+  if (s0.key_hi <= s0.key_lo) {
     pr.nt_beg = pr.nt_end = 0;
   } else {
-    pr.nt_beg = static_cast<int>(lo / BN);
-    pr.nt_end = min(n_tiles, static_cast<int>((hi + BN - 1) / BN));
+    pr.nt_beg = static_cast<int>(s0.key_lo / BN);
+    pr.nt_end = min(n_tiles, static_cast<int>((s0.key_hi + BN - 1) / BN));
   }
   return pr;
 }
 
-// Class of key tile nt for one slot: 0 every key hidden from every row
-// (skip), 1 mixed (mask per element), 2 every key visible to every row.
+// Class of key tile nt for the item's query tile: 0 every key hidden from
+// every row (skip), 1 mixed (mask per element), 2 every key visible to every row.
 __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, const Slot& sl,
                                           int nt, int m_tiles, int n_tiles) {
   if (!sl.live) return 0;
@@ -194,23 +199,25 @@ __device__ __forceinline__ int tile_class(const PrefillArgs& a, const Pair& pr, 
   return cls;
 }
 
-// Visibility of keys j0 .. j0+127 for query q, one bit per key: inside the
+// Visibility of keys j0 .. j0 + 32 NW - 1 for query q, one bit per key: inside the
 // entry's cache (j < len), within the causal limit (j <= q + off) and the
 // window (j > q + off - window), and allowed by the mask row (nonzero byte),
 // which is read as 16-byte vectors when aligned.
-__device__ __forceinline__ void visible_bits(uint32_t (&vb)[4], const uint8_t* mrow, int j0,
+template <int NW>
+__device__ __forceinline__ void visible_bits(uint32_t (&vb)[NW], const uint8_t* mrow, int j0,
                                              const PrefillArgs& a, const Pair& pr, int q,
                                              bool vec) {
+  constexpr int W = 32 * NW;
   int64_t hi = pr.len, lo = 0;  // keys [lo, hi) pass the length, causal and window rules
   if (a.causal) {
     const int64_t off = pair_off(a, pr);
     hi = imin64(hi, static_cast<int64_t>(q) + off + 1);
     if (a.window > 0) lo = static_cast<int64_t>(q) + off - a.window + 1;
   }
-  const int n = static_cast<int>(imax64(0, imin64(BN, hi - j0)));
+  const int n = static_cast<int>(imax64(0, imin64(W, hi - j0)));
   const int n0 = static_cast<int>(imax64(0, imin64(n, lo - j0)));
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const int k = n - 32 * w;
     const int k0 = n0 - 32 * w;
     const uint32_t below_hi = k >= 32 ? ~0u : (k <= 0 ? 0u : ((1u << k) - 1u));
@@ -219,9 +226,9 @@ __device__ __forceinline__ void visible_bits(uint32_t (&vb)[4], const uint8_t* m
   }
   if (mrow == nullptr) return;
   const uint8_t* m = mrow + j0;
-  if (vec && n == BN) {
+  if (vec && n == W) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
+    for (int v = 0; v < 2 * NW; ++v) {
       const uint4 x = *reinterpret_cast<const uint4*>(m + 16 * v);
       const uint32_t wds[4] = {x.x, x.y, x.z, x.w};
       uint32_t bits = 0;
@@ -251,8 +258,7 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t chunk_
   return smem_desc_sw128(saddr, chunk_bytes, 1024);
 }
 
-// D: the padded head dim (64 or 128); columns past a.Dv arrive as zeros from
-// TMA and are never written.  F16: fp16 operands instead of bf16.
+
 template <int D, bool F16>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tmq,
@@ -266,18 +272,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;                   // [slot]
-  uint64_t* q_empty = q_full + kSlots;       // [slot]
-  uint64_t* k_full = q_empty + kSlots;       // [stage]
-  uint64_t* k_empty = k_full + kStages;
-  uint64_t* v_full = k_empty + kStages;
-  uint64_t* v_empty = v_full + kStages;
-  uint64_t* s_full = v_empty + kStages;      // [slot]: S of the slot's next tile is in TMEM
-  uint64_t* p_full = s_full + kSlots;        // [slot]: P written (4 softmax warps)
-  uint64_t* o_ready = p_full + kSlots;       // [slot]: a PV into O has completed
-  uint64_t* o_final = o_ready + kSlots;      // [slot]: the pair's last PV has completed
-  uint64_t* o_free = o_final + kSlots;       // [slot]: epilogue has read O (4 warps)
-  uint64_t* mma_done = o_free + kSlots;
+  uint64_t* q_full = bars;                   // [Q buffer]
+  uint64_t* q_empty = q_full + kQBufs;       // [Q buffer]: copied into TMEM
+  uint64_t* k_full = q_empty + kQBufs;       // [stage]
+  uint64_t* k_empty = k_full + kKStages;
+  uint64_t* v_full = k_empty + kKStages;
+  uint64_t* v_empty = v_full + kVStages;
+  // Per-tile barriers come in pairs indexed by the tile's parity: QK runs two
+  // tiles ahead of PV, so the softmax may finish P(J + 1) before the MMA
+  // thread has looked at P(J), and one barrier would then have moved two
+  // phases past it.
+  uint64_t* s_full = v_empty + kVStages;     // [J & 1]: QK(J) done
+  uint64_t* p_full = s_full + 2;             // [J & 1]: P(J) written (8 warps)
+  uint64_t* o_ready = p_full + 2;            // [J & 1]: PV(J) into O has completed
+  uint64_t* o_final = o_ready + 2;           // the item's last PV has completed
+  uint64_t* o_free = o_final + 1;            // the epilogue has read O (8 warps)
+  uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -285,21 +295,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < kQBufs; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&o_ready[i], 1);
-      mbar_init(&o_final[i], 1);
-      mbar_init(&o_free[i], 4);
     }
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kSoftmaxWarps);
+      mbar_init(&o_ready[i], 1);
+    }
+    mbar_init(o_final, 1);
+    mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -312,7 +326,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
   // Rows past qpt * g of a query tile are never written by TMA: zero them once.
   if (rows < BM && threadIdx.x < BM) {
-    for (int qb = 0; qb < kSlots; ++qb)
+    for (int qb = 0; qb < kQBufs; ++qb)
       for (int c = 0; c < CH; ++c) {
         uint8_t* base = smem + L::kQOff + qb * L::kTileBytes + c * L::kChunkBytes;
         for (int r = rows; r < BM; ++r)
@@ -330,7 +344,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 8) {
+  if (warp >= kSoftmaxWarps) {
   // Producer / MMA warpgroup (warps 8-11): every warp drops its registers.
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIoRegs));
   if (warp == kWarpQK || warp == kWarpV) {
@@ -341,42 +355,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint64_t* full = is_qk ? k_full : v_full;
       uint64_t* empty = is_qk ? k_empty : v_empty;
       uint8_t* ring = smem + (is_qk ? L::kKOff : L::kVOff);
+      const int stages = is_qk ? kKStages : kVStages;
       prefetch_tmap(map);
       if (is_qk) prefetch_tmap(&tmq);
       uint32_t kt = 0;
-      int64_t it = 0;
-      // Last round issued per ring stage / per Q slot (for the unwind drain),
-      // kept in registers: -1 = none.
-      int32_t last_round0 = -1, last_round1 = -1, last_q0 = -1, last_q1 = -1;
+      int64_t it = 0, q_issued = 0;
       bool ok = true;
       for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
-         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
+           ++it, x = snake(it, blockIdx.x, gridDim.x)) {
         const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
-        const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
+        const Slot me = slot_of(pr, a, qpt);
         if (is_qk) {
-#pragma unroll
-          for (int sl = 0; sl < kSlots; ++sl) {
-            if (!ok) break;
-            if (it > 0 && !mbar_wait(&q_empty[sl], static_cast<uint32_t>((it - 1) & 1),
-                                     abort_flag, a.err, kErrPrefillWait)) {
-              ok = false;
-              break;
-            }
-            uint8_t* qdst = smem + L::kQOff + sl * L::kTileBytes;
-            mbar_arrive_expect_tx(&q_full[sl], static_cast<uint32_t>(rows * 128 * CH));
-            for (int c = 0; c < CH; ++c)
-              tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[sl], c * 64,
-                          (sl == 0 ? s0 : s1).q0, pr.kv * a.g, pr.b);
-            if (sl == 0) last_q0 = static_cast<int32_t>(it); else last_q1 = static_cast<int32_t>(it);
+          const int qb = static_cast<int>(it % kQBufs);
+          if (it >= kQBufs &&
+              !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), abort_flag,
+                         a.err, kErrPrefillWait)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
+          uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
+          mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, me.q0,
+                        pr.kv * a.g, pr.b);
+          ++q_issued;
         }
         for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
-          if (tile_class(a, pr, s0, nt, m_tiles, n_tiles) == 0 &&
-              tile_class(a, pr, s1, nt, m_tiles, n_tiles) == 0)
-            continue;
-          const int s = static_cast<int>(kt % kStages);
-          const uint32_t round = kt / kStages;
+          if (tile_class(a, pr, me, nt, m_tiles, n_tiles) == 0) continue;
+          const int s = static_cast<int>(kt % stages);
+          const uint32_t round = kt / stages;
           if (round > 0 &&
               !mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
             ok = false;
@@ -386,15 +393,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
           for (int c = 0; c < CH; ++c)
             tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
-          if (s == 0) last_round0 = static_cast<int32_t>(round); else last_round1 = static_cast<int32_t>(round);
           ++kt;
         }
       }
       if (*abort_flag) {  // let every copy in flight land before the CTA exits
-        if (last_round0 >= 0) mbar_wait_drain(&full[0], static_cast<uint32_t>(last_round0) & 1u);
-        if (last_round1 >= 0) mbar_wait_drain(&full[1], static_cast<uint32_t>(last_round1) & 1u);
-        if (is_qk && last_q0 >= 0) mbar_wait_drain(&q_full[0], static_cast<uint32_t>(last_q0) & 1u);
-        if (is_qk && last_q1 >= 0) mbar_wait_drain(&q_full[1], static_cast<uint32_t>(last_q1) & 1u);
+        for (uint32_t j = kt > static_cast<uint32_t>(stages) ? kt - stages : 0; j < kt; ++j)
+          mbar_wait_drain(&full[j % stages], (j / stages) & 1u);
+        if (is_qk)
+          for (int64_t j = q_issued > kQBufs ? q_issued - kQBufs : 0; j < q_issued; ++j)
+            mbar_wait_drain(&q_full[j % kQBufs], static_cast<uint32_t>((j / kQBufs) & 1));
       }
     }
   } else if (warp == kWarpMMA) {
@@ -403,124 +410,99 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_qk = F16 ? idesc_f16_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = F16 ? idesc_f16_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t q_base = smem_u32(smem + L::kQOff);
-      const uint32_t k_base = smem_u32(smem + L::kKOff);
-      const uint32_t v_base = smem_u32(smem + L::kVOff);
-      uint32_t kt = 0;
-      uint32_t J[kSlots] = {0, 0};       // tiles issued per slot, over the whole kernel
-      uint32_t uses = 0;                 // PVs still to read V stage s: bits [8s, 8s+8)
+      const uint32_t t_q = tmem + L::kQCol, t_o = tmem + L::kOCol;
+      // Descriptors of stage 0, k-step 0; every other (stage, k-step) adds a
+      // constant to the 16-byte address field (shared memory stays below
+      // 256 KB, so the 14-bit field never carries).
+      const uint64_t dk0 = kmajor_desc(smem_u32(smem + L::kKOff));
+      const uint64_t dv0 = mnmajor_desc(smem_u32(smem + L::kVOff), L::kChunkBytes);
+      constexpr uint32_t kStageStep = L::kTileBytes >> 4;
+      uint32_t Jq = 0, Jp = 0;  // tiles whose QK / PV have been issued, over the whole kernel
       int64_t it = 0;
       bool ok = true;
+      // This thread issues every MMA of the CTA, one dependent instruction
+      // every few cycles: its path per tile is kept to the waits, the
+      // MMAs and the commits.
 
-      // O_sl (+)= P_sl V for the slot's tile with per-slot index Jp, K/V tile kp.
-      auto issue_pv = [&](int sl, uint32_t Jp, uint32_t kp, int local) -> bool {
-        if (!mbar_wait(&p_full[sl], Jp & 1u, abort_flag, a.err, kErrPrefillWait)) return false;
-        const int s = static_cast<int>(kp % kStages);
-        if (!mbar_wait(&v_full[s], (kp / kStages) & 1u, abort_flag, a.err, kErrPrefillWait))
-          return false;
-        if (local == 0 && it > 0 &&
-            !mbar_wait(&o_free[sl], static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
-                       kErrPrefillWait))
+      // S(J & 1) = Q K(J)^T; the K stage is released when the MMA completes.
+      auto issue_qk = [&](uint32_t J) -> bool {
+        const uint32_t s = J % kKStages;
+        if (!mbar_wait_hot(&k_full[s], (J / kKStages) & 1u, abort_flag, a.err, kErrPrefillWait))
           return false;
         tc_fence_after();
-        const uint32_t vs = v_base + s * L::kTileBytes;
+        const uint64_t dk = dk0 + s * kStageStep;
+        const uint32_t d_s = tmem + L::kSCol + (J & 1u) * BN;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint32_t a_tmem = tmem + sl * L::kSCol + ks * 8;
-          const uint64_t bdesc = mnmajor_desc(vs + ks * 16 * 128, L::kChunkBytes);
-          tc_mma_ts(tmem + L::kOCol0 + sl * D, a_tmem, bdesc, idesc_pv,
-                    (local > 0 || ks > 0) ? 1u : 0u);
-        }
-        tc_commit(&o_ready[sl]);
-        uses -= 1u << (8 * s);
-        if (((uses >> (8 * s)) & 0xFFu) == 0) tc_commit(&v_empty[s]);
+        for (int ks = 0; ks < D / 16; ++ks)
+          tc_mma_ts(d_s, t_q + ks * 8, dk + (((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4),
+                    idesc_qk, ks > 0 ? 1u : 0u);
+        tc_commit(&s_full[J & 1u]);
+        tc_commit(&k_empty[s]);
+        return true;
+      };
+      // O (+)= P(J) V(J); `first`: the item's first PV overwrites O.
+      auto issue_pv = [&](uint32_t J, bool first) -> bool {
+        const uint32_t s = J % kVStages;
+        if (!mbar_wait_hot(&p_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait) ||
+            !mbar_wait_hot(&v_full[s], (J / kVStages) & 1u, abort_flag, a.err, kErrPrefillWait))
+          return false;
+        if (first && it > 0 &&
+            !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
+                           kErrPrefillWait))
+          return false;
+        tc_fence_after();
+        const uint64_t dv = dv0 + s * kStageStep;
+        const uint32_t p_t = tmem + L::kSCol + (J & 1u) * BN;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks)
+          tc_mma_ts(t_o, p_t + ks * 8, dv + ((ks * 16 * 128) >> 4), idesc_pv,
+                    (!first || ks > 0) ? 1u : 0u);
+        tc_commit(&o_ready[J & 1u]);
+        tc_commit(&v_empty[s]);
         return true;
       };
 
       for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
-         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
+           ++it, x = snake(it, blockIdx.x, gridDim.x)) {
         const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
-        const Slot s0 = slot_of(pr, 0, a, m_tiles, qpt), s1 = slot_of(pr, 1, a, m_tiles, qpt);
-#pragma unroll
-        for (int sl = 0; sl < kSlots; ++sl)
-          if (ok && !mbar_wait(&q_full[sl], static_cast<uint32_t>(it & 1), abort_flag, a.err,
-                               kErrPrefillWait))
-            ok = false;
-        if (!ok) break;
-        bool pend[kSlots] = {false, false};
-        uint32_t pJ[kSlots] = {0, 0}, pk[kSlots] = {0, 0};
-        int nloc[kSlots] = {0, 0};
-        // Each slot's last active key tile: its Q buffer is released as soon
-        // as that QK completes, so the producer can fetch the next pair's Q
-        // while this pair's last products and softmax still run.
-        int last0 = -1, last1 = -1;
-        for (int nt = pr.nt_end - 1; nt >= pr.nt_beg && (last0 < 0 || last1 < 0); --nt) {
-          if (last0 < 0 && tile_class(a, pr, s0, nt, m_tiles, n_tiles) != 0) last0 = nt;
-          if (last1 < 0 && tile_class(a, pr, s1, nt, m_tiles, n_tiles) != 0) last1 = nt;
+        // Key tiles the query tile visits: without a mask every tile of
+        // [nt_beg, nt_end) holds a key some row may see.
+        int n = pr.nt_end - pr.nt_beg;
+        if (a.has_mask) {
+          const Slot me = slot_of(pr, a, qpt);
+          n = 0;
+          for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt)
+            n += tile_class(a, pr, me, nt, m_tiles, n_tiles) != 0;
         }
-        for (int nt = pr.nt_beg; nt < pr.nt_end && ok; ++nt) {
-          const int cls0 = tile_class(a, pr, s0, nt, m_tiles, n_tiles);
-          const int cls1 = tile_class(a, pr, s1, nt, m_tiles, n_tiles);
-          if (cls0 == 0 && cls1 == 0) continue;
-          const int s = static_cast<int>(kt % kStages);
-          if (!mbar_wait(&k_full[s], (kt / kStages) & 1u, abort_flag, a.err, kErrPrefillWait)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uses = (uses & ~(0xFFu << (8 * s))) |
-                 (static_cast<uint32_t>((cls0 != 0) + (cls1 != 0)) << (8 * s));
-          const uint32_t ks_base = k_base + s * L::kTileBytes;
+        // Q from its landing buffer into TMEM (the A operand of every QK of
+        // this query tile); the copy follows the previous tile's last QK on
+        // the tensor core, and the buffer is released when the copy is done.
+        const int qb = static_cast<int>(it % kQBufs);
+        if (!mbar_wait_hot(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1), abort_flag,
+                           a.err, kErrPrefillWait)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qs = q_base + qb * L::kTileBytes;
 #pragma unroll
-          for (int sl = 0; sl < kSlots; ++sl) {
-            if (!ok) break;
-            const bool act = (sl == 0 ? cls0 : cls1) != 0;
-            // The slot's previous PV goes first: its P lives in the S columns
-            // that this QK overwrites (in-order execution on the tensor core).
-            if (pend[sl]) {
-              if (!issue_pv(sl, pJ[sl], pk[sl], nloc[sl] - 1)) {
-                ok = false;
-                break;
-              }
-              pend[sl] = false;
-            }
-            if (!act) continue;
-            const uint32_t qs = q_base + sl * L::kTileBytes;
-            const uint32_t d_s = tmem + sl * L::kSCol;
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-              tc_mma_ss(d_s, kmajor_desc(qs + off), kmajor_desc(ks_base + off), idesc_qk,
-                        ks > 0 ? 1u : 0u);
-            }
-            tc_commit(&s_full[sl]);
-            if (nt == (sl == 0 ? last0 : last1)) tc_commit(&q_empty[sl]);
-            pend[sl] = true;
-            pJ[sl] = J[sl];
-            pk[sl] = kt;
-            ++nloc[sl];
-            ++J[sl];
-          }
-          if (!ok) break;
-          tc_commit(&k_empty[s]);
-          ++kt;
+        for (int ks = 0; ks < D / 16; ++ks)
+          tc_cp_128x256b(t_q + ks * 8, kmajor_desc(qs + (ks >> 2) * L::kChunkBytes + (ks & 3) * 32));
+        tc_commit(&q_empty[qb]);
+        // QK runs two tiles ahead of PV: QK(0), QK(1), PV(0), QK(2), PV(1), ...
+        for (int i = 0; i < 2 && i < n && ok; ++i) ok = issue_qk(Jq++);
+        for (int i = 0; i < n && ok; ++i) {
+          ok = issue_pv(Jp++, i == 0);
+          if (ok && i + 2 < n) ok = issue_qk(Jq++);
         }
         if (!ok) break;
-#pragma unroll
-        for (int sl = 0; sl < kSlots; ++sl)
-          if (ok && pend[sl] && !issue_pv(sl, pJ[sl], pk[sl], nloc[sl] - 1)) ok = false;
-        if (!ok) break;
-#pragma unroll
-        for (int sl = 0; sl < kSlots; ++sl) {
-          if (!ok) break;
-          if (nloc[sl] == 0) tc_commit(&q_empty[sl]);  // no QK used this slot's Q
-          if (nloc[sl] == 0 && it > 0 &&
-              !mbar_wait(&o_free[sl], static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
-                         kErrPrefillWait)) {
-            ok = false;
-            break;
-          }
-          tc_commit(&o_final[sl]);
+        if (n == 0 && it > 0 &&  // no PV: O is left as it is, but the epilogue must be done
+            !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
+                           kErrPrefillWait)) {
+          ok = false;
+          break;
         }
+        tc_commit(o_final);
       }
       // Every MMA issued so far has completed before TMEM is released.
       tc_commit(mma_done);
@@ -530,69 +512,83 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ------------------------------------------------------------- softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    // Warps 4 sl .. 4 sl + 3 own slot sl; thread t of the group owns row t
-    // (TMEM lane t) of the slot's tiles.
-    const int sl = warp >> 2;
+    // Two warpgroups.  Thread t of warpgroup h owns row t (TMEM lane t), the
+    // keys [64 h, 64 h + 64) of every S tile and the O columns
+    // [h D / 2, (h + 1) D / 2).  The two threads of a row trade their partial
+    // maxima (every tile) and row sums (every query tile) through shared
+    // memory, under a named barrier per pair of warps that share TMEM lanes.
+    constexpr int HD = D / 2;
+    const int h = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + sl * L::kSCol;
-    const uint32_t o_col = tmem + lane_base + L::kOCol0 + sl * D;
+    const uint32_t o_col = tmem + lane_base + L::kOCol + h * HD;
+    const int pair_bar = 1 + (warp & 3);
+    float* xch = reinterpret_cast<float*>(smem + L::kXOff);  // [X & 1][half][row]
+    uint32_t X = 0;  // values traded so far (identical in both threads of a row)
+    // Publish v, meet the partner, return its value; `flag` becomes the AND
+    // of both threads' flags (and of the other 62 threads of the two warps).
+    auto trade = [&](float v, bool& flag) -> float {
+      float* slot = xch + (X & 1u) * 256;
+      slot[h * 128 + row] = v;
+      flag = bar_and(pair_bar, 64, flag);
+      const float other = slot[(h ^ 1) * 128 + row];
+      ++X;
+      return other;
+    };
     const int hh = row / qpt, qi = row % qpt;
     // Mask rows can be read as 16-byte vectors when base and strides allow.
     const bool mask_vec = a.has_mask && ((reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0) &&
                           (a.ms[0] % 16 == 0) && (a.ms[1] % 16 == 0);
     uint32_t J = 0;
     int64_t it = 0;
-    bool ok = true;
-    for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && ok;
+    // `ok`: nothing this thread waited on has failed.  `live`: both threads
+    // of the pair of warps still agree to go on; failures only end the loops
+    // right after a trade, so the partner is never left at a named barrier.
+    bool ok = true, live = true;
+    for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < work && live;
          ++it, x = snake(it, blockIdx.x, gridDim.x)) {
       const Pair pr = pair_of(x, a, m_tiles, qpt, n_tiles);
-      const Slot me = slot_of(pr, sl, a, m_tiles, qpt);
+      const Slot me = slot_of(pr, a, qpt);
       const int q = me.q0 + qi;
-      const bool row_valid = me.live && row < rows && q < a.Sq;
+      const bool row_valid = row < rows && q < a.Sq;
       const uint8_t* mrow =
           (a.has_mask && row_valid) ? a.mask + pr.b * a.ms[0] + static_cast<int64_t>(q) * a.ms[1]
                                     : nullptr;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f;  // m_ref is the same in both threads of the row
       int nloc = 0;
       for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
         const int cls = tile_class(a, pr, me, nt, m_tiles, n_tiles);
         if (cls == 0) continue;
-        if (!mbar_wait(&s_full[sl], J & 1u, abort_flag, a.err, kErrPrefillWait)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // Pass 1 over the S row: its maximum.  Fully visible tiles work on raw
-        // scores and fold the scale into one FMA per element in pass 2; other
+        const uint32_t s_col = tmem + lane_base + L::kSCol + (J & 1u) * BN;
+        bool okt = ok && mbar_wait(&s_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err,
+                                   kErrPrefillWait);
+        // This half of the S row: its maximum.  Fully visible tiles work on
+        // raw scores and fold the scale into one FMA per element below; other
         // tiles test each key against the row's visibility bits.
         const bool fast = (cls == 2) && (a.scale_log2 >= 0.f);
-        uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};
-        if (!fast)
-          visible_bits(vb, row_valid ? mrow : nullptr, nt * BN, a, pr, q, mask_vec);
-        auto masked_t = [&](float sv, int c) -> float {
-          return ((vb[c >> 5] >> (c & 31)) & 1u) ? sv * a.scale_log2 : -INFINITY;
-        };
-        // The whole S row of this thread, read from TMEM once (four loads in
-        // flight), kept in registers for the max and the exponentials.
-        uint32_t r[BN];
-        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-        tmem_ld_wait();
-        if (!fast) {
+        uint32_t r[HK];
+        float mx = -INFINITY;
+        if (okt) {
+          tc_fence_after();
+          uint32_t vb[2] = {~0u, ~0u};
+          if (!fast)
+            visible_bits<2>(vb, row_valid ? mrow : nullptr, nt * BN + h * HK, a, pr, q, mask_vec);
+          tmem_ld32(s_col + h * HK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(s_col + h * HK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_ld_wait();
+          if (!fast) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c) r[c] = __float_as_uint(masked_t(__uint_as_float(r[c]), c));
-        }
-        float mx;
-        {
+            for (int c = 0; c < HK; ++c)
+              r[c] = __float_as_uint(((vb[c >> 5] >> (c & 31)) & 1u)
+                                         ? __uint_as_float(r[c]) * a.scale_log2
+                                         : -INFINITY);
+          }
           // Eight independent running maxima, two elements per three-input max.
           float part[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) part[e] = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < BN; c += 16)
+          for (int c = 0; c < HK; c += 16)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               part[e] = fmax3(part[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
@@ -600,46 +596,54 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                      fmaxf(part[6], part[7]));
           if (fast) mx *= a.scale_log2;
         }
-        const float m_new = fmaxf(m_ref, mx);
+        // Both halves of S are in registers once the trade is done: P may then
+        // overwrite the first 64 columns, half of which the other warpgroup read.
+        tc_fence_before();
+        const float mx_other = trade(mx, okt);
+        tc_fence_after();
+        if (!okt) {
+          live = false;
+          break;
+        }
+        const float m_new = fmaxf(m_ref, fmaxf(mx, mx_other));
         const bool grow = m_new > m_ref + kRescaleLog2;  // also true for -inf -> finite
         const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         const bool o_live = grow && nloc > 0 && m_ref != -INFINITY;
         if (__any_sync(0xffffffffu, o_live)) {
-          // O holds earlier tiles' P V with the old reference: rescale it.  The
-          // slot's previous PV was issued before this tile's QK, so it has
-          // completed; the wait returns at once.
-          if (!mbar_wait(&o_ready[sl], (J - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float f = o_live ? alpha : 1.f;
+          // O holds the earlier tiles' P V with the old reference: rescale this
+          // half once the previous tile's PV has completed.
+          if (mbar_wait(&o_ready[(J - 1) & 1u], ((J - 1) >> 1) & 1u, abort_flag, a.err,
+                        kErrPrefillWait)) {
+            tc_fence_after();
+            const float f = o_live ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(o_col + c * 32, r);
-            tmem_ld_wait();
+            for (int c = 0; c < HD / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(o_col + c * 32, o);
+              tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-            tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+              tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+            }
+            tmem_st_wait();
+          } else {
+            ok = false;  // carried to the next trade
           }
-          tmem_st_wait();
         }
         if (grow) {
           l *= alpha;
           m_ref = m_new;
         }
         const float ref = exp_ref(m_ref);
-        // P = 2^(t - ref) as bf16 pairs over the first 64 columns of S (A
-        // operand of the PV MMA); S is already in registers.  kEmuPerEight of
-        // every eight exponentials run on the FMA pipe.
+        // P = 2^(t - ref) as 16-bit pairs: keys [64 h, 64 h + 64) land in the
+        // P columns [32 h, 32 h + 32) of S (A operand of the PV MMA).
         float lp[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) lp[e] = 0.f;
         const float sc = fast ? a.scale_log2 : 1.f;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HK / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -652,43 +656,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             lp[c1 & 7] += p1;
             pk[e] = pack2<F16>(p0, p1);
           }
-          tmem_st16(s_col + c * 16, pk);
+          tmem_st16(s_col + h * (HK / 2) + c * 16, pk);
         }
         l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sl]);
+        if (lane == 0) mbar_arrive(&p_full[J & 1u]);
         ++J;
         ++nloc;
       }
-      if (!ok) break;
-      // Epilogue: out = O / l for this row.
-      if (!mbar_wait(&o_final[sl], static_cast<uint32_t>(it & 1), abort_flag, a.err,
-                     kErrPrefillWait)) {
-        ok = false;
+      if (!live) break;
+      // Epilogue: out = O / l for this half row, l being both halves' sum.
+      bool oke = ok && mbar_wait(o_final, static_cast<uint32_t>(it & 1), abort_flag, a.err,
+                                 kErrPrefillWait);
+      const float l_other = trade(l, oke);
+      if (!oke) {
+        live = false;
         break;
       }
       tc_fence_after();
       uint16_t* orow = a.out + pr.b * a.os[0] +
                        static_cast<int64_t>(pr.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
-                       static_cast<int64_t>(q) * a.os[2];
-      const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
+                       static_cast<int64_t>(q) * a.os[2] + h * HD;
+      const int dv = a.Dv - h * HD;        // columns of this half inside head_dim_v
+      const float inv_l = 1.f / (l + l_other);  // l == 0: no visible key, NaN output
       if (nloc > 0) {
-        // The whole O row in registers: every TMEM load in flight, one wait.
-        uint32_t r[D];
+        // The half O row in registers: every TMEM load in flight, one wait.
+        uint32_t r[HD];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c)
+        for (int c = 0; c < HD / 32; ++c)
           tmem_ld32(o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
         tmem_ld_wait();
-        // O is in registers: the next pair's first PV may overwrite it now.
+        // O is in registers: the next tile's first PV may overwrite it now.
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[sl]);
+        if (lane == 0) mbar_arrive(o_free);
         if (row_valid) {
 #pragma unroll
-          for (int v8 = 0; v8 < D / 8; ++v8) {
-            if (a.Dv < D && v8 * 8 >= a.Dv) break;
+          for (int v8 = 0; v8 < HD / 8; ++v8) {
+            if (v8 * 8 >= dv) break;
             uint4 w;
             w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
                              __uint_as_float(r[v8 * 8 + 1]) * inv_l);
@@ -701,16 +708,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             reinterpret_cast<uint4*>(orow)[v8] = w;
           }
         }
-      } else if (row_valid) {
-        const float nanv = __int_as_float(0x7fc00000);
-        const uint32_t nn = pack2<F16>(nanv, nanv);
-        for (int d = 0; d < a.Dv; d += 8)
-          *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
-      }
-      if (nloc == 0) {  // no PV wrote O for this pair: release it as it is
+      } else {
+        if (row_valid) {
+          const float nanv = __int_as_float(0x7fc00000);
+          const uint32_t nn = pack2<F16>(nanv, nanv);
+          for (int d = 0; d < dv && d < HD; d += 8)
+            *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[sl]);
+        if (lane == 0) mbar_arrive(o_free);
       }
     }
   }
@@ -784,6 +791,11 @@ int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensor
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Layout<D>::kBytes) != cudaSuccess)
     return GQA_ERR_CUDA;
+  // The register split assumes the launch allocation it was sized for: with
+  // fewer registers per thread, setmaxnreg.inc could never be granted.
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQA_ERR_CUDA;
+  if (fa.numRegs != kLaunchRegs) return GQA_ERR_CUDA;
   kern<<<s.grid, kPrefillThreads, Layout<D>::kBytes, stream>>>(tmq, tmk, tmv, a, s.qpt, s.rows,
                                                                 s.m_tiles, s.n_tiles, s.work);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
@@ -799,7 +811,7 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.rows = static_cast<int>(s.qpt * g);
   s.m_tiles = static_cast<int>((p.seq_q + s.qpt - 1) / s.qpt);
   s.n_tiles = static_cast<int>((p.seq_k + BN - 1) / BN);
-  s.work = p.batch * p.heads_kv * ((s.m_tiles + 1) / 2);  // pairs of query tiles
+  s.work = p.batch * p.heads_kv * s.m_tiles;  // query tiles
   s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
   if (s.grid < 1) s.grid = 1;
   s.smem_bytes = s.D == 128 ? Layout<128>::kBytes : Layout<64>::kBytes;

@@ -128,12 +128,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait for a thread whose waits are usually satisfied already (the
+// single MMA issuer): the barrier is tried before anything else.
+__device__ __forceinline__ bool mbar_wait_hot(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint32_t* err_word, uint32_t err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort, err_word, err_bit);
+}
+
 // Bounded wait used while unwinding: no error is recorded, the limit is short.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs / 4) return;
   }
+}
+
+// Named barrier `id` over `nthreads` threads (a multiple of 32) that also
+// ANDs a flag across them; shared-memory writes before it are visible to all
+// participants after it.
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -275,6 +299,13 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]; one thread issues.
+// Copy a 128-row x 256-bit matrix (16 16-bit values per row) described by a
+// shared-memory matrix descriptor into 8 TMEM columns of 128 lanes; ordered
+// with this thread's other tcgen05 MMAs and copies.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
