@@ -88,6 +88,18 @@ constexpr float kRescaleLog2 = 8.0f;
 #define GQA_PREFILL_EXP_EMU 0
 #endif
 constexpr int kEmuPerEight = GQA_PREFILL_EXP_EMU;
+#ifndef GQA_PREFILL_INT_PACK
+#define GQA_PREFILL_INT_PACK 1
+#endif
+
+// P as a 16-bit pair, `lo` in the low half.  For bf16, P being finite and
+// non-negative, rounding to nearest (ties away from zero) is an integer add
+// of half a unit in the last place and a byte permute.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+  if (F16 || !GQA_PREFILL_INT_PACK) return pack2<F16>(lo, hi);
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
 
 template <int D>
 struct Layout {
@@ -560,8 +572,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int cls = tile_class(a, pr, me, nt, m_tiles, n_tiles);
         if (cls == 0) continue;
         const uint32_t s_col = tmem + lane_base + L::kSCol + (J & 1u) * BN;
-        bool okt = ok && mbar_wait(&s_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err,
-                                   kErrPrefillWait);
+        // tcgen05.ld / st are warp-collective: every decision that guards them
+        // is made the same for the whole warp.
+        bool okt = __all_sync(0xffffffffu, ok && mbar_wait_hot(&s_full[J & 1u], (J >> 1) & 1u,
+                                                               abort_flag, a.err, kErrPrefillWait));
         // This half of the S row: its maximum.  Fully visible tiles work on
         // raw scores and fold the scale into one FMA per element below; other
         // tiles test each key against the row's visibility bits.
@@ -612,8 +626,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (__any_sync(0xffffffffu, o_live)) {
           // O holds the earlier tiles' P V with the old reference: rescale this
           // half once the previous tile's PV has completed.
-          if (mbar_wait(&o_ready[(J - 1) & 1u], ((J - 1) >> 1) & 1u, abort_flag, a.err,
-                        kErrPrefillWait)) {
+          if (__all_sync(0xffffffffu, mbar_wait(&o_ready[(J - 1) & 1u], ((J - 1) >> 1) & 1u,
+                                                abort_flag, a.err, kErrPrefillWait))) {
             tc_fence_after();
             const float f = o_live ? alpha : 1.f;
 #pragma unroll
@@ -654,7 +668,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const float p1 = ((c1 & 7) < kEmuPerEight) ? exp2_poly(x1) : fast_exp2(x1);
             lp[c0 & 7] += p0;
             lp[c1 & 7] += p1;
-            pk[e] = pack2<F16>(p0, p1);
+            pk[e] = pack_p<F16>(p0, p1);
           }
           tmem_st16(s_col + h * (HK / 2) + c * 16, pk);
         }
@@ -668,8 +682,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       if (!live) break;
       // Epilogue: out = O / l for this half row, l being both halves' sum.
-      bool oke = ok && mbar_wait(o_final, static_cast<uint32_t>(it & 1), abort_flag, a.err,
-                                 kErrPrefillWait);
+      bool oke = ok && mbar_wait_hot(o_final, static_cast<uint32_t>(it & 1), abort_flag, a.err,
+                                     kErrPrefillWait);
       const float l_other = trade(l, oke);
       if (!oke) {
         live = false;
