@@ -110,7 +110,7 @@ struct Layout {
   static constexpr int kKOff = kQOff + kQBufs * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 3;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kKStages + 3 * kVStages + 2 + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXOff = kMiscOff + 16;  // float [2][2][128]: per-row values the halves trade
   static constexpr int kBytes = kXOff + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
@@ -300,6 +300,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* o_final = o_ready + 2;           // the item's last PV has completed
   uint64_t* o_free = o_final + 1;            // the epilogue has read O (8 warps)
   uint64_t* mma_done = o_free + 1;
+  uint64_t* v_fix = mma_done + 1;            // [stage]: rows past the length zeroed (partial tiles)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(o_final, 1);
     mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
+    for (int i = 0; i < kVStages; ++i) mbar_init(&v_fix[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -361,15 +363,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIoRegs));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------- producers
-    if (lane == 0) {
+    // The whole warp walks the tiles; lane 0 issues the copies.
+    {
       const bool is_qk = warp == kWarpQK;
       const CUtensorMap* map = is_qk ? &tmk : &tmv;
       uint64_t* full = is_qk ? k_full : v_full;
       uint64_t* empty = is_qk ? k_empty : v_empty;
       uint8_t* ring = smem + (is_qk ? L::kKOff : L::kVOff);
       const int stages = is_qk ? kKStages : kVStages;
-      prefetch_tmap(map);
-      if (is_qk) prefetch_tmap(&tmq);
+      if (lane == 0) {
+        prefetch_tmap(map);
+        if (is_qk) prefetch_tmap(&tmq);
+      }
       uint32_t kt = 0;
       int64_t it = 0, q_issued = 0;
       bool ok = true;
@@ -380,16 +385,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (is_qk) {
           const int qb = static_cast<int>(it % kQBufs);
           if (it >= kQBufs &&
-              !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), abort_flag,
-                         a.err, kErrPrefillWait)) {
+              !__all_sync(0xffffffffu,
+                          mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1),
+                                    abort_flag, a.err, kErrPrefillWait))) {
             ok = false;
             break;
           }
-          uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
-          mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, me.q0,
-                        pr.kv * a.g, pr.b);
+          if (lane == 0) {
+            uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
+            mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, me.q0,
+                          pr.kv * a.g, pr.b);
+          }
           ++q_issued;
         }
         for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
@@ -397,18 +405,41 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int s = static_cast<int>(kt % stages);
           const uint32_t round = kt / stages;
           if (round > 0 &&
-              !mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
+              !__all_sync(0xffffffffu, mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err,
+                                                 kErrPrefillWait))) {
             ok = false;
             break;
           }
           uint8_t* dst = ring + s * L::kTileBytes;
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
+          }
           ++kt;
+          // The V rows of the entry's last tile past its length hold whatever
+          // the cache holds there (NaN included), and P = 0 does not hide a
+          // NaN in P V: once the tile has landed they are zeroed, and the MMA
+          // waits for that too.  Only the last tile a query tile visits can
+          // reach past the length.
+          if (!is_qk && (static_cast<int64_t>(nt) + 1) * BN > pr.len) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], round & 1u, abort_flag, a.err,
+                                                   kErrPrefillWait))) {
+              ok = false;
+              break;
+            }
+            const int valid = pr.len - nt * BN;  // 1 .. BN - 1: the tile holds a key below len
+            for (int c = 0; c < CH; ++c) {
+              uint4* row0 = reinterpret_cast<uint4*>(dst + c * L::kChunkBytes + valid * 128);
+              for (int i = lane; i < (BN - valid) * 8; i += 32) row0[i] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&v_fix[s]);
+          }
         }
       }
-      if (*abort_flag) {  // let every copy in flight land before the CTA exits
+      if (lane == 0 && *abort_flag) {  // let every copy in flight land before the CTA exits
         for (uint32_t j = kt > static_cast<uint32_t>(stages) ? kt - stages : 0; j < kt; ++j)
           mbar_wait_drain(&full[j % stages], (j / stages) & 1u);
         if (is_qk)
@@ -452,12 +483,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_commit(&k_empty[s]);
         return true;
       };
-      // O (+)= P(J) V(J); `first`: the item's first PV overwrites O.
-      auto issue_pv = [&](uint32_t J, bool first) -> bool {
+      // O (+)= P(J) V(J); `first`: the item's first PV overwrites O; `fix`:
+      // the tile reaches past the entry's length, and the V producer zeroes
+      // those rows once it has landed (one phase of v_fix[stage] per such tile).
+      uint32_t fix_parity = 0;  // bit s: parity of the next v_fix[s] phase
+      auto issue_pv = [&](uint32_t J, bool first, bool fix) -> bool {
         const uint32_t s = J % kVStages;
         if (!mbar_wait_hot(&p_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait) ||
             !mbar_wait_hot(&v_full[s], (J / kVStages) & 1u, abort_flag, a.err, kErrPrefillWait))
           return false;
+        if (fix) {
+          if (!mbar_wait_hot(&v_fix[s], (fix_parity >> s) & 1u, abort_flag, a.err,
+                             kErrPrefillWait))
+            return false;
+          fix_parity ^= 1u << s;
+        }
         if (first && it > 0 &&
             !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
                            kErrPrefillWait))
@@ -480,11 +520,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Key tiles the query tile visits: without a mask every tile of
         // [nt_beg, nt_end) holds a key some row may see.
         int n = pr.nt_end - pr.nt_beg;
+        // The last of them reaches past the entry's length: its V rows there
+        // are zeroed by the V producer before its PV.
+        bool last_fix = n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
         if (a.has_mask) {
           const Slot me = slot_of(pr, a, qpt);
           n = 0;
           for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt)
             n += tile_class(a, pr, me, nt, m_tiles, n_tiles) != 0;
+          last_fix = last_fix && tile_class(a, pr, me, pr.nt_end - 1, m_tiles, n_tiles) != 0;
         }
         // Q from its landing buffer into TMEM (the A operand of every QK of
         // this query tile); the copy follows the previous tile's last QK on
@@ -504,7 +548,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // QK runs two tiles ahead of PV: QK(0), QK(1), PV(0), QK(2), PV(1), ...
         for (int i = 0; i < 2 && i < n && ok; ++i) ok = issue_qk(Jq++);
         for (int i = 0; i < n && ok; ++i) {
-          ok = issue_pv(Jp++, i == 0);
+          ok = issue_pv(Jp++, i == 0, last_fix && i == n - 1);
           if (ok && i + 2 < n) ok = issue_qk(Jq++);
         }
         if (!ok) break;

@@ -119,6 +119,37 @@ def test_ragged_prefill(gqa, B, Hq, Hkv, Sq, Sk, D, window, pinned):
     _check(out, ref, "ragged prefill %s" % ((B, Hq, Hkv, Sq, Sk, D, window),))
 
 
+@pytest.mark.parametrize("dtype,D,causal", [("bf16", 128, True), ("bf16", 64, False),
+                                             ("f16", 128, False)])
+def test_ragged_prefill_nan_tail(gqa, dtype, D, causal):
+    """A contiguous cache whose rows past each length are NaN (K and V), on the
+    prefill path: the result must not see them."""
+    B, Hq, Hkv, Sq, Sk = 3, 8, 2, 100, 700
+    seed = 3500 + D
+    if dtype == "bf16":
+        bits = synth.qkv_bf16_bits(seed, B, Hq, Hkv, Sq, Sk, D)
+        qc, kc, vc = (f64(x) for x in bits)
+        tdt = torch.bfloat16
+    else:
+        qc, kc, vc = (x.astype(np.float16).astype(np.float64)
+                      for x in synth.qkv_f32(seed, B, Hq, Hkv, Sq, Sk, D))
+        tdt = torch.float16
+    lens = np.array([700, 333, 129], dtype=np.int32)
+    kn, vn = kc.copy(), vc.copy()
+    for b in range(B):
+        kn[b, :, lens[b]:] = np.nan
+        vn[b, :, lens[b]:] = np.nan
+        kc[b, :, lens[b]:] = 0.0
+        vc[b, :, lens[b]:] = 0.0
+    q, k, v = (torch.from_numpy(x).to(tdt).cuda() for x in (qc, kn, vn))
+    kw = dict(causal=True, causal_offset="bottom_right") if causal else {}
+    out = to_np(gqa.forward(q, k, v, kv_lens=torch.from_numpy(lens).cuda(), **kw))
+    assert _status(gqa) == 0
+    ref = oracle.forward(qc, kc, vc, kv_lens=lens,
+                         **(dict(causal=True, causal_offset=Sk - Sq) if causal else {}))
+    _check(out, ref, "ragged prefill NaN tail %s D=%d causal=%s" % (dtype, D, causal))
+
+
 def test_ragged_prefill_non_causal(gqa):
     B, Hq, Hkv, Sq, Sk, D = 2, 8, 2, 100, 800, 128
     bits, (q, k, v) = bf16_inputs(3400, B, Hq, Hkv, Sq, Sk, D)
