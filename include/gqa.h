@@ -44,9 +44,9 @@
  *    Multi-Head Attention: Understanding GQA Implementation", "Memory
  *    Footprint and KV-Cache Optimization", describes, with a per-sequence T.
  *    A length outside [0, seq_k] is clamped and reported by gqa_device_status
- *    as GQA_ERR_KV_LENGTH.  The decode path never lets cache rows past a
- *    length reach the result; the prefill path multiplies them by zero
- *    weights, so there they must hold finite values (zeros, or old keys).
+ *    as GQA_ERR_KV_LENGTH.  Cache rows past a length never reach the result,
+ *    whatever they hold (NaN included): the decode path masks them, and the
+ *    prefill path zeroes the V rows of the last key tile in shared memory.
  *  - Paged cache (block_table != NULL; decode and fp32 paths): k and v point
  *    to a pool of num_pages pages, each [heads_kv, page_size, head_dim],
  *    described by k_stride / v_stride over (page, h_kv, key in page, d).  Key
