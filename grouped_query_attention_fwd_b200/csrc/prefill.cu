@@ -101,7 +101,9 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
-template <int D>
+// LENS: the launch has per-sequence lengths (two more barriers, for the V
+// rows past a length; without lengths the kernel is built without them).
+template <int D, bool LENS>
 struct Layout {
   static constexpr int CH = D / 64;                  // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 bytes
@@ -110,7 +112,8 @@ struct Layout {
   static constexpr int kKOff = kQOff + kQBufs * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kKStages + 3 * kVStages + 2 + 2 + 2 + 3;
+  static constexpr int kNumBars =
+      2 * kQBufs + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 3 + (LENS ? kVStages : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXOff = kMiscOff + 16;  // float [2][2][128]: per-row values the halves trade
   static constexpr int kBytes = kXOff + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
@@ -271,14 +274,14 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t chunk_
 }
 
 
-template <int D, bool F16>
+template <int D, bool F16, bool LENS>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const PrefillArgs a,
                        const int qpt, const int rows, const int m_tiles, const int n_tiles,
                        const int64_t work) {
-  using L = Layout<D>;
+  using L = Layout<D, LENS>;
   constexpr int CH = L::CH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* o_final = o_ready + 2;           // the item's last PV has completed
   uint64_t* o_free = o_final + 1;            // the epilogue has read O (8 warps)
   uint64_t* mma_done = o_free + 1;
-  uint64_t* v_fix = mma_done + 1;            // [stage]: rows past the length zeroed (partial tiles)
+  uint64_t* v_fix = mma_done + 1;            // [stage] (LENS): rows past the length zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -328,7 +331,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(o_final, 1);
     mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < kVStages; ++i) mbar_init(&v_fix[i], 1);
+    if (LENS)
+      for (int i = 0; i < kVStages; ++i) mbar_init(&v_fix[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -363,18 +367,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIoRegs));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------- producers
-    // The whole warp walks the tiles; lane 0 issues the copies.
-    {
+    if (lane == 0) {
       const bool is_qk = warp == kWarpQK;
       const CUtensorMap* map = is_qk ? &tmk : &tmv;
       uint64_t* full = is_qk ? k_full : v_full;
       uint64_t* empty = is_qk ? k_empty : v_empty;
       uint8_t* ring = smem + (is_qk ? L::kKOff : L::kVOff);
       const int stages = is_qk ? kKStages : kVStages;
-      if (lane == 0) {
-        prefetch_tmap(map);
-        if (is_qk) prefetch_tmap(&tmq);
-      }
+      prefetch_tmap(map);
+      if (is_qk) prefetch_tmap(&tmq);
       uint32_t kt = 0;
       int64_t it = 0, q_issued = 0;
       bool ok = true;
@@ -385,19 +386,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (is_qk) {
           const int qb = static_cast<int>(it % kQBufs);
           if (it >= kQBufs &&
-              !__all_sync(0xffffffffu,
-                          mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1),
-                                    abort_flag, a.err, kErrPrefillWait))) {
+              !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), abort_flag,
+                         a.err, kErrPrefillWait)) {
             ok = false;
             break;
           }
-          if (lane == 0) {
-            uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
-            mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
-            for (int c = 0; c < CH; ++c)
-              tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, me.q0,
-                          pr.kv * a.g, pr.b);
-          }
+          uint8_t* qdst = smem + L::kQOff + qb * L::kTileBytes;
+          mbar_arrive_expect_tx(&q_full[qb], static_cast<uint32_t>(rows * 128 * CH));
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(qdst + c * L::kChunkBytes, &tmq, &q_full[qb], c * 64, me.q0,
+                        pr.kv * a.g, pr.b);
           ++q_issued;
         }
         for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt) {
@@ -405,41 +403,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int s = static_cast<int>(kt % stages);
           const uint32_t round = kt / stages;
           if (round > 0 &&
-              !__all_sync(0xffffffffu, mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err,
-                                                 kErrPrefillWait))) {
+              !mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
             ok = false;
             break;
           }
           uint8_t* dst = ring + s * L::kTileBytes;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
-            for (int c = 0; c < CH; ++c)
-              tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
-          }
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
           ++kt;
           // The V rows of the entry's last tile past its length hold whatever
           // the cache holds there (NaN included), and P = 0 does not hide a
           // NaN in P V: once the tile has landed they are zeroed, and the MMA
           // waits for that too.  Only the last tile a query tile visits can
           // reach past the length.
-          if (!is_qk && (static_cast<int64_t>(nt) + 1) * BN > pr.len) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], round & 1u, abort_flag, a.err,
-                                                   kErrPrefillWait))) {
+          if (LENS && !is_qk && (static_cast<int64_t>(nt) + 1) * BN > pr.len) {
+            if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrPrefillWait)) {
               ok = false;
               break;
             }
             const int valid = pr.len - nt * BN;  // 1 .. BN - 1: the tile holds a key below len
             for (int c = 0; c < CH; ++c) {
               uint4* row0 = reinterpret_cast<uint4*>(dst + c * L::kChunkBytes + valid * 128);
-              for (int i = lane; i < (BN - valid) * 8; i += 32) row0[i] = make_uint4(0, 0, 0, 0);
+              for (int i = 0; i < (BN - valid) * 8; ++i) row0[i] = make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&v_fix[s]);
+            mbar_arrive(&v_fix[s]);
           }
         }
       }
-      if (lane == 0 && *abort_flag) {  // let every copy in flight land before the CTA exits
+      if (*abort_flag) {  // let every copy in flight land before the CTA exits
         for (uint32_t j = kt > static_cast<uint32_t>(stages) ? kt - stages : 0; j < kt; ++j)
           mbar_wait_drain(&full[j % stages], (j / stages) & 1u);
         if (is_qk)
@@ -461,6 +454,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint64_t dv0 = mnmajor_desc(smem_u32(smem + L::kVOff), L::kChunkBytes);
       constexpr uint32_t kStageStep = L::kTileBytes >> 4;
       uint32_t Jq = 0, Jp = 0;  // tiles whose QK / PV have been issued, over the whole kernel
+      uint32_t fix_parity = 0;  // bit s: parity of the next v_fix[s] phase
       int64_t it = 0;
       bool ok = true;
       // This thread issues every MMA of the CTA, one dependent instruction
@@ -483,21 +477,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_commit(&k_empty[s]);
         return true;
       };
-      // O (+)= P(J) V(J); `first`: the item's first PV overwrites O; `fix`:
-      // the tile reaches past the entry's length, and the V producer zeroes
-      // those rows once it has landed (one phase of v_fix[stage] per such tile).
-      uint32_t fix_parity = 0;  // bit s: parity of the next v_fix[s] phase
-      auto issue_pv = [&](uint32_t J, bool first, bool fix) -> bool {
+      // O (+)= P(J) V(J); `first`: the item's first PV overwrites O.
+      auto issue_pv = [&](uint32_t J, bool first) -> bool {
         const uint32_t s = J % kVStages;
         if (!mbar_wait_hot(&p_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait) ||
             !mbar_wait_hot(&v_full[s], (J / kVStages) & 1u, abort_flag, a.err, kErrPrefillWait))
           return false;
-        if (fix) {
-          if (!mbar_wait_hot(&v_fix[s], (fix_parity >> s) & 1u, abort_flag, a.err,
-                             kErrPrefillWait))
-            return false;
-          fix_parity ^= 1u << s;
-        }
         if (first && it > 0 &&
             !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
                            kErrPrefillWait))
@@ -522,7 +507,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         int n = pr.nt_end - pr.nt_beg;
         // The last of them reaches past the entry's length: its V rows there
         // are zeroed by the V producer before its PV.
-        bool last_fix = n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
+        bool last_fix = LENS && n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
         if (a.has_mask) {
           const Slot me = slot_of(pr, a, qpt);
           n = 0;
@@ -548,7 +533,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // QK runs two tiles ahead of PV: QK(0), QK(1), PV(0), QK(2), PV(1), ...
         for (int i = 0; i < 2 && i < n && ok; ++i) ok = issue_qk(Jq++);
         for (int i = 0; i < n && ok; ++i) {
-          ok = issue_pv(Jp++, i == 0, last_fix && i == n - 1);
+          if (last_fix && i == n - 1) {
+            // The tile reaches past the entry's length: the V producer zeroes
+            // those rows once it has landed (one phase of v_fix[stage] each).
+            const uint32_t s = Jp % kVStages;
+            ok = mbar_wait_hot(&v_fix[s], (fix_parity >> s) & 1u, abort_flag, a.err,
+                               kErrPrefillWait);
+            fix_parity ^= 1u << s;
+            if (!ok) break;
+          }
+          ok = issue_pv(Jp++, i == 0);
           if (ok && i + 2 < n) ok = issue_qk(Jq++);
         }
         if (!ok) break;
@@ -834,7 +828,7 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-template <int D, bool F16>
+template <int D, bool F16, bool LENS>
 int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
                      const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
   if (a.has_mask) {
@@ -845,17 +839,17 @@ int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensor
         vec ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
-  auto kern = gqa_prefill_kernel<D, F16>;
+  auto kern = gqa_prefill_kernel<D, F16, LENS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Layout<D>::kBytes) != cudaSuccess)
+                           Layout<D, LENS>::kBytes) != cudaSuccess)
     return GQA_ERR_CUDA;
   // The register split assumes the launch allocation it was sized for: with
   // fewer registers per thread, setmaxnreg.inc could never be granted.
   cudaFuncAttributes fa{};
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQA_ERR_CUDA;
   if (fa.numRegs != kLaunchRegs) return GQA_ERR_CUDA;
-  kern<<<s.grid, kPrefillThreads, Layout<D>::kBytes, stream>>>(tmq, tmk, tmv, a, s.qpt, s.rows,
-                                                                s.m_tiles, s.n_tiles, s.work);
+  kern<<<s.grid, kPrefillThreads, Layout<D, LENS>::kBytes, stream>>>(
+      tmq, tmk, tmv, a, s.qpt, s.rows, s.m_tiles, s.n_tiles, s.work);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -872,7 +866,9 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.work = p.batch * p.heads_kv * s.m_tiles;  // query tiles
   s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
   if (s.grid < 1) s.grid = 1;
-  s.smem_bytes = s.D == 128 ? Layout<128>::kBytes : Layout<64>::kBytes;
+  s.smem_bytes = p.kv_lens != nullptr
+                     ? (s.D == 128 ? Layout<128, true>::kBytes : Layout<64, true>::kBytes)
+                     : (s.D == 128 ? Layout<128, false>::kBytes : Layout<64, false>::kBytes);
   s.summary_offset = kScratchOffset;
   s.workspace_end = s.summary_offset + (p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0);
   return s;
@@ -882,12 +878,21 @@ int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArg
                    const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                    cudaStream_t stream) {
   const bool f16 = p.dtype == GQA_DTYPE_F16;
-  if (s.D == 128)
-    return f16 ? launch_prefill_t<128, true>(s, a, tmq, tmk, tmv, stream)
-               : launch_prefill_t<128, false>(s, a, tmq, tmk, tmv, stream);
-  if (s.D == 64)
-    return f16 ? launch_prefill_t<64, true>(s, a, tmq, tmk, tmv, stream)
-               : launch_prefill_t<64, false>(s, a, tmq, tmk, tmv, stream);
+  const bool lens = a.lens != nullptr;
+  if (s.D == 128) {
+    if (lens)
+      return f16 ? launch_prefill_t<128, true, true>(s, a, tmq, tmk, tmv, stream)
+                 : launch_prefill_t<128, false, true>(s, a, tmq, tmk, tmv, stream);
+    return f16 ? launch_prefill_t<128, true, false>(s, a, tmq, tmk, tmv, stream)
+               : launch_prefill_t<128, false, false>(s, a, tmq, tmk, tmv, stream);
+  }
+  if (s.D == 64) {
+    if (lens)
+      return f16 ? launch_prefill_t<64, true, true>(s, a, tmq, tmk, tmv, stream)
+                 : launch_prefill_t<64, false, true>(s, a, tmq, tmk, tmv, stream);
+    return f16 ? launch_prefill_t<64, true, false>(s, a, tmq, tmk, tmv, stream)
+               : launch_prefill_t<64, false, false>(s, a, tmq, tmk, tmv, stream);
+  }
   return GQA_ERR_UNSUPPORTED;
 }
 
