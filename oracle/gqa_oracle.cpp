@@ -30,7 +30,7 @@
 //  * "Multi-Query Attention" (aiwiki), "Implementation": the same map and a
 //    boolean attn_mask in the library attention call.
 //
-// Readings where the pages are silent or differ (each listed in the design doc):
+// Readings where the pages are silent or differ:
 //  * the scale is an argument and multiplies the dot product (the reference
 //    solution divides by sqrt(head_dim); callers pass 1/sqrt(D) for that);
 //  * a mask value of 1 means "attend" (the reference solution fills where the
