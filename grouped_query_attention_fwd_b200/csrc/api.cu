@@ -163,7 +163,6 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       break;
     }
     case GQA_KERNEL_PREFILL: {
-      if (p.block_table != nullptr) return GQA_ERR_UNSUPPORTED;  // paged: decode and fp32 only
       const PrefillShape s = plan_prefill(p, sm_count);
       plan->grid = s.grid;
       plan->block = kPrefillThreads;
@@ -341,12 +340,19 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   int erc = encode_half_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
                             static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g), f16);
   if (erc != GQA_OK) return erc;
-  erc = encode_half_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 128, 1,
-                        f16);
-  if (erc != GQA_OK) return erc;
-  erc = encode_half_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128, 1,
-                        f16);
-  if (erc != GQA_OK) return erc;
+  if (p.block_table != nullptr) {  // paged: 64-key boxes, one page each
+    erc = encode_decode_kv_map(&tmk, k, p, p.k_stride);
+    if (erc != GQA_OK) return erc;
+    erc = encode_decode_kv_map(&tmv, v, p, p.v_stride);
+    if (erc != GQA_OK) return erc;
+  } else {
+    erc = encode_half_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 128,
+                          1, f16);
+    if (erc != GQA_OK) return erc;
+    erc = encode_half_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128,
+                          1, f16);
+    if (erc != GQA_OK) return erc;
+  }
   PrefillArgs a{};
   a.mask = p.has_mask ? mask : nullptr;
   for (int d = 0; d < 3; ++d) a.ms[d] = p.mask_stride[d];

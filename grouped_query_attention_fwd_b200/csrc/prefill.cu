@@ -101,9 +101,10 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
   return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
-// LENS: the launch has per-sequence lengths (two more barriers, for the V
-// rows past a length; without lengths the kernel is built without them).
-template <int D, bool LENS>
+// KVX: the launch has per-sequence lengths or a paged cache (two more
+// barriers, for the V rows past a length; without either the kernel is built
+// without them).
+template <int D, bool KVX>
 struct Layout {
   static constexpr int CH = D / 64;                  // 64-column (128-byte) chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 bytes
@@ -113,7 +114,7 @@ struct Layout {
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kNumBars =
-      2 * kQBufs + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 3 + (LENS ? kVStages : 0);
+      2 * kQBufs + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 3 + (KVX ? kVStages : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXOff = kMiscOff + 16;  // float [2][2][128]: per-row values the halves trade
   static constexpr int kBytes = kXOff + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
@@ -124,6 +125,15 @@ struct Layout {
 
 __device__ __forceinline__ int64_t imin64(int64_t x, int64_t y) { return x < y ? x : y; }
 __device__ __forceinline__ int64_t imax64(int64_t x, int64_t y) { return x > y ? x : y; }
+
+// Paged K / V cache: a pool of num_pages pages, each [Hkv, page_size, D];
+// key j of entry b is row j % page_size of page bt[b * bt_stride + j /
+// page_size].  bt == nullptr: contiguous caches.
+struct PagedKV {
+  const int32_t* bt;
+  int64_t bt_stride;
+  int page_size, num_pages;
+};
 
 // Work item: one query tile of one (batch, kv head).
 struct Pair {
@@ -274,14 +284,14 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t chunk_
 }
 
 
-template <int D, bool F16, bool LENS>
+template <int D, bool F16, bool KVX>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, const PrefillArgs a,
                        const int qpt, const int rows, const int m_tiles, const int n_tiles,
-                       const int64_t work) {
-  using L = Layout<D, LENS>;
+                       const int64_t work, const PagedKV pg) {
+  using L = Layout<D, KVX>;
   constexpr int CH = L::CH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -303,7 +313,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* o_final = o_ready + 2;           // the item's last PV has completed
   uint64_t* o_free = o_final + 1;            // the epilogue has read O (8 warps)
   uint64_t* mma_done = o_free + 1;
-  uint64_t* v_fix = mma_done + 1;            // [stage] (LENS): rows past the length zeroed
+  uint64_t* v_fix = mma_done + 1;            // [stage] (KVX): rows past the length zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -331,7 +341,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(o_final, 1);
     mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
-    if (LENS)
+    if (KVX)
       for (int i = 0; i < kVStages; ++i) mbar_init(&v_fix[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -409,15 +419,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           uint8_t* dst = ring + s * L::kTileBytes;
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kTileBytes));
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
+          if (KVX && pg.bt != nullptr) {
+            // Two 64-key boxes, each inside one page (page_size is a multiple
+            // of 64).  A box that starts at or past the entry's length reads an
+            // out-of-range page, which the copy fills with zeros; a page index
+            // outside the pool for keys in use is reported and read the same way.
+            for (int hb = 0; hb < 2; ++hb) {
+              const int key = nt * BN + hb * 64;
+              int page = pg.num_pages;
+              if (key < pr.len) {
+                page = __ldg(pg.bt + pr.b * pg.bt_stride + key / pg.page_size);
+                if (page < 0 || page >= pg.num_pages) {
+                  atomicOr(a.err, kErrPage);
+                  page = pg.num_pages;
+                }
+              }
+              for (int c = 0; c < CH; ++c)
+                tma_load_4d(dst + c * L::kChunkBytes + hb * 64 * 128, map, &full[s], c * 64,
+                            key % pg.page_size, pr.kv, page);
+            }
+          } else {
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(dst + c * L::kChunkBytes, map, &full[s], c * 64, nt * BN, pr.kv, pr.b);
+          }
           ++kt;
           // The V rows of the entry's last tile past its length hold whatever
           // the cache holds there (NaN included), and P = 0 does not hide a
           // NaN in P V: once the tile has landed they are zeroed, and the MMA
           // waits for that too.  Only the last tile a query tile visits can
           // reach past the length.
-          if (LENS && !is_qk && (static_cast<int64_t>(nt) + 1) * BN > pr.len) {
+          if (KVX && !is_qk && (static_cast<int64_t>(nt) + 1) * BN > pr.len) {
             if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrPrefillWait)) {
               ok = false;
               break;
@@ -507,7 +538,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         int n = pr.nt_end - pr.nt_beg;
         // The last of them reaches past the entry's length: its V rows there
         // are zeroed by the V producer before its PV.
-        bool last_fix = LENS && n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
+        bool last_fix = KVX && n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
         if (a.has_mask) {
           const Slot me = slot_of(pr, a, qpt);
           n = 0;
@@ -828,9 +859,10 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-template <int D, bool F16, bool LENS>
-int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
-                     const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
+template <int D, bool F16, bool KVX>
+int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const PagedKV& pg,
+                     const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                     cudaStream_t stream) {
   if (a.has_mask) {
     const bool vec = (reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0 && a.ms[0] % 16 == 0 &&
                      a.ms[1] % 16 == 0;
@@ -839,17 +871,17 @@ int launch_prefill_t(const PrefillShape& s, const PrefillArgs& a, const CUtensor
         vec ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
-  auto kern = gqa_prefill_kernel<D, F16, LENS>;
+  auto kern = gqa_prefill_kernel<D, F16, KVX>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Layout<D, LENS>::kBytes) != cudaSuccess)
+                           Layout<D, KVX>::kBytes) != cudaSuccess)
     return GQA_ERR_CUDA;
   // The register split assumes the launch allocation it was sized for: with
   // fewer registers per thread, setmaxnreg.inc could never be granted.
   cudaFuncAttributes fa{};
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQA_ERR_CUDA;
   if (fa.numRegs != kLaunchRegs) return GQA_ERR_CUDA;
-  kern<<<s.grid, kPrefillThreads, Layout<D, LENS>::kBytes, stream>>>(
-      tmq, tmk, tmv, a, s.qpt, s.rows, s.m_tiles, s.n_tiles, s.work);
+  kern<<<s.grid, kPrefillThreads, Layout<D, KVX>::kBytes, stream>>>(
+      tmq, tmk, tmv, a, s.qpt, s.rows, s.m_tiles, s.n_tiles, s.work, pg);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -866,7 +898,7 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.work = p.batch * p.heads_kv * s.m_tiles;  // query tiles
   s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
   if (s.grid < 1) s.grid = 1;
-  s.smem_bytes = p.kv_lens != nullptr
+  s.smem_bytes = (p.kv_lens != nullptr || p.block_table != nullptr)
                      ? (s.D == 128 ? Layout<128, true>::kBytes : Layout<64, true>::kBytes)
                      : (s.D == 128 ? Layout<128, false>::kBytes : Layout<64, false>::kBytes);
   s.summary_offset = kScratchOffset;
@@ -878,20 +910,25 @@ int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArg
                    const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
                    cudaStream_t stream) {
   const bool f16 = p.dtype == GQA_DTYPE_F16;
-  const bool lens = a.lens != nullptr;
+  PagedKV pg{};
+  pg.bt = p.block_table;
+  pg.bt_stride = p.block_table_stride;
+  pg.page_size = static_cast<int>(p.page_size);
+  pg.num_pages = static_cast<int>(p.num_pages);
+  const bool kvx = a.lens != nullptr || pg.bt != nullptr;
   if (s.D == 128) {
-    if (lens)
-      return f16 ? launch_prefill_t<128, true, true>(s, a, tmq, tmk, tmv, stream)
-                 : launch_prefill_t<128, false, true>(s, a, tmq, tmk, tmv, stream);
-    return f16 ? launch_prefill_t<128, true, false>(s, a, tmq, tmk, tmv, stream)
-               : launch_prefill_t<128, false, false>(s, a, tmq, tmk, tmv, stream);
+    if (kvx)
+      return f16 ? launch_prefill_t<128, true, true>(s, a, pg, tmq, tmk, tmv, stream)
+                 : launch_prefill_t<128, false, true>(s, a, pg, tmq, tmk, tmv, stream);
+    return f16 ? launch_prefill_t<128, true, false>(s, a, pg, tmq, tmk, tmv, stream)
+               : launch_prefill_t<128, false, false>(s, a, pg, tmq, tmk, tmv, stream);
   }
   if (s.D == 64) {
-    if (lens)
-      return f16 ? launch_prefill_t<64, true, true>(s, a, tmq, tmk, tmv, stream)
-                 : launch_prefill_t<64, false, true>(s, a, tmq, tmk, tmv, stream);
-    return f16 ? launch_prefill_t<64, true, false>(s, a, tmq, tmk, tmv, stream)
-               : launch_prefill_t<64, false, false>(s, a, tmq, tmk, tmv, stream);
+    if (kvx)
+      return f16 ? launch_prefill_t<64, true, true>(s, a, pg, tmq, tmk, tmv, stream)
+                 : launch_prefill_t<64, false, true>(s, a, pg, tmq, tmk, tmv, stream);
+    return f16 ? launch_prefill_t<64, true, false>(s, a, pg, tmq, tmk, tmv, stream)
+               : launch_prefill_t<64, false, false>(s, a, pg, tmq, tmk, tmv, stream);
   }
   return GQA_ERR_UNSUPPORTED;
 }

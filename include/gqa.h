@@ -47,7 +47,7 @@
  *    as GQA_ERR_KV_LENGTH.  Cache rows past a length never reach the result,
  *    whatever they hold (NaN included): the decode path masks them, and the
  *    prefill path zeroes the V rows of the last key tile in shared memory.
- *  - Paged cache (block_table != NULL; decode and fp32 paths): k and v point
+ *  - Paged cache (block_table != NULL; every path): k and v point
  *    to a pool of num_pages pages, each [heads_kv, page_size, head_dim],
  *    described by k_stride / v_stride over (page, h_kv, key in page, d).  Key
  *    j of batch entry b lives in page block_table[b * block_table_stride +

@@ -293,10 +293,10 @@ def test_paged_validation(gqa):
                        v_stride=pool))[0] == 2        # more keys than the table can address
     assert _rc(gqa, _p(gqa, **dict(base, num_pages=0), page_size=128, k_stride=pool,
                        v_stride=pool))[0] == 2
-    # the prefill path takes contiguous caches only
-    rc, _ = _rc(gqa, _p(gqa, **dict(base, Sq=300, causal=True, causal_offset=724),
-                        page_size=128, k_stride=pool, v_stride=pool))
-    assert rc == gqa.GQA_ERR_UNSUPPORTED
+    # the prefill path reads pages too
+    rc, pl = _rc(gqa, _p(gqa, **dict(base, Sq=300, causal=True, causal_offset=724),
+                         page_size=128, k_stride=pool, v_stride=pool))
+    assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "prefill"
     # fp32 gathers through the table too
     rc, pl = _rc(gqa, _p(gqa, **base, page_size=128, dtype=1, k_stride=pool, v_stride=pool))
     assert rc == 0 and gqa.KERNEL_NAMES[pl.kernel] == "f32"

@@ -96,6 +96,60 @@ def test_paged_short_query_block(gqa):
     assert_bf16_parity(out, ref, "paged short query block")
 
 
+def _check_nan_rows(out, ref, what):
+    nan_ref = np.isnan(ref).all(axis=-1)
+    assert np.array_equal(np.isnan(out).all(axis=-1), nan_ref), what
+    assert_bf16_parity(out[~nan_ref], ref[~nan_ref], what)
+
+
+@pytest.mark.parametrize("page_size,dtype,D", [(64, "bf16", 128), (128, "f16", 128),
+                                               (256, "bf16", 64), (64, "f16", 96)])
+def test_paged_prefill(gqa, page_size, dtype, D):
+    """A block of new queries at the end of each sequence (bottom-right
+    causal) on the prefill path, the cache in shuffled pages of a pool that is
+    NaN outside the valid rows."""
+    B, Hq, Hkv, Sq = 3, 16, 4, 100
+    per_seq = 1024 // page_size
+    lens = np.array([1024, 333, 129], dtype=np.int32)
+    kc, vc, kd, vd, table = _paged(6800 + page_size + D, B, Hkv, D, page_size, per_seq, lens,
+                                   dtype)
+    q, qd = _q(6800 + D, B, Hq, Sq, D, dtype)
+    cap = per_seq * page_size
+    out = to_np(gqa.forward(qd, kd, vd, causal=True, causal_offset="bottom_right",
+                            kv_lens=torch.from_numpy(lens).cuda(), block_table=table))
+    assert gqa.device_status() == 0
+    ref = oracle.forward(q, kc, vc, causal=True, causal_offset=cap - Sq, kv_lens=lens)
+    _check_nan_rows(out, ref, "paged prefill ps=%d %s D=%d" % (page_size, dtype, D))
+
+
+def test_paged_prefill_full_cache_non_causal(gqa):
+    """No lengths: every key of the capacity is in use, non-causal, g = 6."""
+    B, Hq, Hkv, Sq, D, ps, per_seq = 2, 12, 2, 150, 128, 128, 5
+    cap = ps * per_seq
+    lens = np.full(B, cap, dtype=np.int32)
+    kc, vc, kd, vd, table = _paged(6900, B, Hkv, D, ps, per_seq, lens, "bf16")
+    q, qd = _q(6900, B, Hq, Sq, D, "bf16")
+    out = to_np(gqa.forward(qd, kd, vd, block_table=table))
+    assert gqa.device_status() == 0
+    assert_bf16_parity(out, oracle.forward(q, kc, vc), "paged prefill, full cache")
+
+
+def test_paged_prefill_bad_page_is_reported(gqa):
+    B, Hq, Hkv, Sq, D, ps, per_seq = 2, 8, 2, 64, 64, 64, 4
+    lens = np.array([200, 150], dtype=np.int32)
+    kc, vc, kd, vd, table = _paged(7000, B, Hkv, D, ps, per_seq, lens, "bf16")
+    bad = table.clone()
+    bad[1, 1] = -5                      # keys 64..127 of entry 1 are in use
+    q, qd = _q(7000, B, Hq, Sq, D, "bf16")
+    dl = torch.from_numpy(lens).cuda()
+    gqa.forward(qd, kd, vd, causal=True, causal_offset="bottom_right", kv_lens=dl,
+                block_table=bad)
+    assert gqa.device_status() == gqa.GQA_ERR_PAGE
+    gqa.forward(qd, kd, vd, causal=True, causal_offset="bottom_right", kv_lens=dl,
+                block_table=table)
+    assert gqa.device_status() == 0
+
+
 def test_paged_f32(gqa):
     B, Hq, Hkv, D, ps, per_seq = 3, 8, 2, 40, 64, 5
     lens = np.array([320, 1, 100], dtype=np.int32)
