@@ -60,6 +60,11 @@ DECODE_STEP = dict(name="decode_step_append", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096 
 # The ragged cache held in 64-key pages of a shuffled pool (block table per sequence).
 DECODE_PAGED = dict(name="decode_paged_cache", B=16, Hq=32, Hkv=8, Sq=1, Sk=4096, D=128,
                     causal=False, mask=False, seed=6, lens=(256, 4096), append=0, page=64)
+# Chunked prefill on a paged cache: 1024 new queries at the end of each
+# sequence (bottom-right causal) over lengths U[2048, 8192] in 64-key pages.
+PREFILL_CHUNK_PAGED = dict(name="prefill_chunk_paged_cache", B=4, Hq=32, Hkv=8, Sq=1024, Sk=8192,
+                           D=128, causal=True, mask=False, seed=10, lens=(2048, 8192), append=0,
+                           page=64)
 # The Mistral-7B-shaped decode with fp16 operands, and with head dim 96.
 DECODE_F16 = dict(DECODE, name="decode_mistral7b_layer_fp16", dtype="f16", seed=8)
 DECODE_D96 = dict(DECODE, name="decode_head_dim_96", D=96, seed=9)
@@ -372,10 +377,16 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
         mean_keys += n_new * B  # the appended token is read too
     step_bytes = (mean_keys * Hkv * D * 2 * 2 + 2 * qd.numel() * 2 +
                   (4 * B * Hkv * n_new * D * 2 if n_new else 0))
+    # Visible (query, key) pairs per head: bottom-right causal, or every key.
+    Sq = cfg["Sq"]
+    if cfg["causal"]:
+        pairs = sum(Sq * int(n) - Sq * (Sq - 1) // 2 for n in lens0) if not n_new else None
+    else:
+        pairs = Sq * int(lens0.sum())
     res = dict(total_ms=total_ms, per_launch_ms=total_ms / steps,
                single_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
                step_bytes=step_bytes, launches=plan["launches"] + (1 if n_new else 0),
-               mean_len=mean_keys / B)
+               mean_len=mean_keys / B, visible_pairs_per_head=pairs)
     del ks, vs, qd, out, lens
     torch.cuda.empty_cache()
     return res
@@ -471,9 +482,20 @@ def _roofline_ragged(res, hbm, peak_kind, workload):
             "step_ms": round(res["per_launch_ms"], 5)}
 
 
+def _roofline_ragged_prefill(res, cfg, tf_peak, peak_kind):
+    """Tensor roofline of a prefill over per-sequence lengths: 4 * D FLOPs per
+    visible (query, key) pair and query head."""
+    flops = 4.0 * cfg["D"] * cfg["Hq"] * res["visible_pairs_per_head"]
+    achieved = flops / (res["per_launch_ms"] / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": round(achieved / tf_peak, 4), "peak_source": peak_kind, "traffic": None,
+            "algorithmic_flops_per_launch": flops, "mean_len": round(res["mean_len"], 1),
+            "launch_ms": round(res["per_launch_ms"], 5)}
+
+
 WORKLOADS = {c["name"]: c for c in (DECODE, DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED,
                                     DECODE_RAGGED, DECODE_STEP, DECODE_PAGED, DECODE_F16,
-                                    DECODE_D96)}
+                                    DECODE_D96, PREFILL_CHUNK_PAGED)}
 
 
 def run_profile_case(args):
@@ -600,7 +622,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.skip_extra:
         extra = {}
         for c in (DECODE_LONG, PREFILL_CAUSAL, PREFILL_MASKED, DECODE_RAGGED, DECODE_STEP,
-                  DECODE_PAGED, DECODE_F16, DECODE_D96):
+                  DECODE_PAGED, DECODE_F16, DECODE_D96, PREFILL_CHUNK_PAGED):
             timer = _time_ragged if "lens" in c else _time_config
             try:
                 res = timer(gqa, torch, c, steps=max(3, min(args.steps, 50)),
@@ -608,7 +630,11 @@ def run_gpu(args):
             except Exception as e:  # report, keep the primary line
                 extra[c["name"]] = {"unavailable": "%s: %s" % (type(e).__name__, e)}
                 continue
-            if "lens" in c:
+            if "lens" in c and c["Sq"] > 1:
+                rf = _roofline_ragged_prefill(res, c, tf_burst, peak_kind)
+                extra[c["name"]] = {"value": rf["achieved"], "unit": "TFLOP/s", "roofline": rf,
+                                    "frac_of_sustained_peak": round(rf["achieved"] / tf_sus, 4)}
+            elif "lens" in c:
                 rf = _roofline_ragged(res, hbm, peak_kind, c["name"])
                 extra[c["name"]] = {"value": rf["achieved"], "unit": "GB/s", "roofline": rf}
             elif c["Sq"] == 1:
