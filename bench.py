@@ -311,6 +311,22 @@ def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     return res
 
 
+def visible_pairs(Sq, lens, causal):
+    """(query, key) pairs a query head sees over entries with cache lengths
+    `lens`: every key, or, bottom-right causal, query i of the block of Sq
+    sees keys j <= i + len - Sq (and j >= 0)."""
+    total = 0
+    for n in lens:
+        n = int(n)
+        if not causal:
+            total += Sq * n
+            continue
+        # min(max(i + n - Sq + 1, 0), n) summed over i = 0 .. Sq - 1
+        lo = max(0, Sq - n)  # first query that sees a key
+        total += sum(min(i + n - Sq + 1, n) for i in range(lo, Sq))
+    return total
+
+
 def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
     """Device-resident timing of a ragged-cache workload: per step an optional
     gqa_kv_append of one token per sequence, then gqa_forward with kv_lens."""
@@ -377,12 +393,7 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
         mean_keys += n_new * B  # the appended token is read too
     step_bytes = (mean_keys * Hkv * D * 2 * 2 + 2 * qd.numel() * 2 +
                   (4 * B * Hkv * n_new * D * 2 if n_new else 0))
-    # Visible (query, key) pairs per head: bottom-right causal, or every key.
-    Sq = cfg["Sq"]
-    if cfg["causal"]:
-        pairs = sum(Sq * int(n) - Sq * (Sq - 1) // 2 for n in lens0) if not n_new else None
-    else:
-        pairs = Sq * int(lens0.sum())
+    pairs = None if n_new else visible_pairs(cfg["Sq"], lens0, cfg["causal"])
     res = dict(total_ms=total_ms, per_launch_ms=total_ms / steps,
                single_launch_median_ms=statistics.median(per), plan=plan, copies=copies,
                step_bytes=step_bytes, launches=plan["launches"] + (1 if n_new else 0),

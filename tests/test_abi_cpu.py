@@ -306,3 +306,19 @@ def test_paged_append_validation(gqa):
     d = _append(gqa, cap=1024)
     d.block_table, d.block_table_stride, d.page_size, d.num_pages = 256, 4, 128, 16
     assert _append_rc(gqa, d) == gqa.GQA_ERR_SHAPE   # 4 pages of 128 < capacity 1024
+
+
+@pytest.mark.parametrize("Sq,lens,causal", [(5, [7, 3, 5, 0], True), (4, [6, 2], False),
+                                            (1, [9], True), (8, [8, 20], True)])
+def test_bench_visible_pairs_brute_force(Sq, lens, causal):
+    """The bench's FLOP count for prefill over per-sequence lengths counts the
+    (query, key) pairs the oracle's bottom-right causal rule leaves visible."""
+    import bench
+    brute = 0
+    for n in lens:
+        for i in range(Sq):
+            for j in range(n):
+                brute += (not causal) or (j <= i + n - Sq)
+    assert bench.visible_pairs(Sq, lens, causal) == brute
+    if causal and all(n >= Sq for n in lens):  # the closed form used in the docs
+        assert brute == sum(Sq * n - Sq * (Sq - 1) // 2 for n in lens)
