@@ -403,6 +403,42 @@ def test_kv_lens_equal_truncated_cache(oracle_mod):
             np.testing.assert_allclose(out[b:b + 1], ref, rtol=1e-11, atol=1e-12)
 
 
+def test_rows_ex_match_torch_and_full(oracle_mod):
+    """forward_rows with a causal offset, a window and per-sequence lengths
+    (lengths 0 and full included): each requested row equals PyTorch's fp64
+    attention on that entry's first len_b keys under the same visibility
+    rule, and equals the same row of the full-output function bitwise; the
+    rows come back in the order asked for, duplicates included."""
+    rng = np.random.default_rng(47)
+    B, Hq, Hkv, Sq, Sk, D = 3, 6, 2, 4, 15, 8
+    q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+    lens = np.array([15, 0, 9], dtype=np.int32)
+    rows = [(2, 5, 3), (0, 0, 0), (1, 3, 2), (2, 1, 0), (0, 4, 3), (2, 5, 3), (0, 2, 1)]
+    for causal, off, window in ((False, None, 0), (True, Sk - Sq, 0), (True, Sk - Sq, 5),
+                                (True, 3, 2)):
+        full = oracle_mod.forward(q, k, v, causal=causal, causal_offset=off, window=window,
+                                  kv_lens=lens)
+        got = oracle_mod.forward_rows(q, k, v, rows, causal=causal, causal_offset=off,
+                                      window=window, kv_lens=lens)
+        for r, (b, h, i) in enumerate(rows):
+            assert np.array_equal(got[r], full[b, h, i], equal_nan=True), (causal, off, window, r)
+            n = int(lens[b])
+            vis = np.arange(Sk) < n
+            if causal:
+                j = np.arange(Sk)
+                lim = i + off + (n - Sk)
+                vis &= j <= lim
+                if window:
+                    vis &= j > lim - window
+            if not vis.any():
+                assert np.all(np.isnan(got[r]))
+                continue
+            ref = _sdpa(q[b:b + 1, h:h + 1, i:i + 1], k[b:b + 1, h // 3:h // 3 + 1],
+                        v[b:b + 1, h // 3:h // 3 + 1], mask=vis[None, None, :],
+                        scale=1.0 / np.sqrt(D))
+            np.testing.assert_allclose(got[r], ref[0, 0, 0], rtol=1e-11, atol=1e-12)
+
+
 def test_kv_lens_bounds(oracle_mod):
     rng = np.random.default_rng(46)
     q, k = _rand(rng, 2, 2, 1, 4), _rand(rng, 2, 1, 5, 4)
@@ -430,6 +466,15 @@ MUTANTS = {
     "v from q head": ("const double* vbase = p.v + ((b * p.Hkv + kv) * p.Sk) * p.D;",
                       "const double* vbase = p.v + ((b * p.Hkv + (h % p.Hkv)) * p.Sk) * p.D;"),
     "kv bytes factor": ("return 2 * layers * tokens", "return layers * tokens"),
+    # Mistakes confined to the selected-rows entry point with lengths, offset
+    # and window: (function, text, replacement) plants them in that function only.
+    "rows_ex rows written out of order": ("oracle_gqa_forward_rows_ex",
+                                          "row_output(p, b, h, i, w.data(), out + r * D);",
+                                          "row_output(p, b, h, i, w.data(), out + (n - 1 - r) * D);"),
+    "rows_ex ignores the lengths": ("oracle_gqa_forward_rows_ex", "true,\n            kv_lens};",
+                                    "true,\n            nullptr};"),
+    "rows_ex ignores the window": ("oracle_gqa_forward_rows_ex", "causal_offset, window, true",
+                                   "causal_offset, 0, true"),
 }
 
 
@@ -465,6 +510,22 @@ def _pins_hold(oracle_mod, lib):
         ok &= bool(np.allclose(ragged[b:b + 1], ref, rtol=1e-11, atol=1e-12))
         ref, _ = _offset_window_ref(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], n, 0)
         ok &= bool(np.allclose(plain[b:b + 1], ref, rtol=1e-11, atol=1e-12))
+    # Selected rows, plain and with offset / window / lengths, against the
+    # full-output functions pinned above (rows in a scrambled order).
+    q, k, v = _rand(rng, 2, 4, 3, 8), _rand(rng, 2, 2, 11, 8), _rand(rng, 2, 2, 11, 8)
+    rows = [(1, 3, 2), (0, 0, 0), (1, 0, 1), (0, 2, 2)]
+    try:
+        for kw in ({}, dict(causal=True, causal_offset=8, window=4, kv_lens=[11, 6])):
+            full = oracle_mod.forward(q, k, v, lib=lib, **kw)
+            sel = oracle_mod.forward_rows(q, k, v, rows, lib=lib, **kw)
+            ok &= all(np.allclose(sel[r], full[b, h, i], rtol=1e-13, atol=1e-14)
+                      for r, (b, h, i) in enumerate(rows))
+            ref, _ = _offset_window_ref(q[:1], k[:1], v[:1], 8, 4) if kw else (None, None)
+            if kw:
+                ok &= bool(np.allclose(sel[1], ref[0, 0, 0], rtol=1e-11, atol=1e-12))
+                ok &= bool(np.allclose(sel[3], ref[0, 2, 2], rtol=1e-11, atol=1e-12))
+    except oracle_mod.OracleError:
+        return False
     q, k, v = _rand(rng, 1, 4, 5, 8) * 60.0, _rand(rng, 1, 2, 7, 8) * 60.0, _rand(rng, 1, 2, 7, 8)
     big = oracle_mod.forward(q, k, v, scale=1.0, lib=lib)
     ok &= bool(np.allclose(big, _sdpa(q, k, v, scale=1.0), rtol=1e-11, atol=1e-12))
@@ -481,11 +542,20 @@ def test_pins_hold_for_the_real_oracle(oracle_mod):
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(oracle_mod, tmp_path, name):
-    old, new = MUTANTS[name]
+    spec = MUTANTS[name]
     src = open(os.path.join(ROOT, "oracle", "gqa_oracle.cpp")).read()
-    assert src.count(old) >= 1, name
+    if len(spec) == 3:  # only inside the named function (its definition onwards)
+        func, old, new = spec
+        start = src.index("int %s(" % func)
+        at = src.index(old, start)
+        mutated = src[:at] + new + src[at + len(old):]
+    else:
+        old, new = spec
+        assert src.count(old) >= 1, name
+        mutated = src.replace(old, new)
+    assert mutated != src, name
     mutant_src = tmp_path / "mutant.cpp"
-    mutant_src.write_text(src.replace(old, new))
+    mutant_src.write_text(mutated)
     so = str(tmp_path / "libmutant.so")
     oracle_mod.build(force=True, src=str(mutant_src), out=so)
     lib = oracle_mod.load_library(so)
