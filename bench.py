@@ -523,6 +523,110 @@ def run_profile_case(args):
                       "copies": res["copies"], "plan": res["plan"]}), flush=True)
 
 
+def trace_summary(words, grid, launches, kv_bytes_per_unit):
+    """Phase summary of `launches` consecutive decode launches from the
+    per-CTA trace records (see gqa_debug_decode_trace); times in microseconds
+    relative to each launch's first CTA entry."""
+    import numpy as np
+    W = 16
+    t = np.asarray(words, dtype=np.int64).reshape(launches, grid, W)
+    entry, ready, fissue, land, last = (t[:, :, i] for i in (1, 2, 3, 5, 6))
+    merged, done, exit_, units = (t[:, :, i] for i in (7, 8, 9, 10))
+    flushes, midns, kind = t[:, :, 11], t[:, :, 12], t[:, :, 13]
+    t0 = entry.min(axis=1, keepdims=True)
+    us = lambda x: (x - t0) / 1e3  # noqa: E731
+
+    def stat(x):
+        x = np.asarray(x, dtype=np.float64).ravel()
+        return {"min": round(float(x.min()), 2), "median": round(float(np.median(x)), 2),
+                "max": round(float(x.max()), 2)}
+
+    span = (exit_.max(axis=1) - t0[:, 0]) / 1e3
+    period = np.diff(t0[:, 0]) / 1e3
+    gap = (entry.min(axis=1)[1:] - exit_.max(axis=1)[:-1]) / 1e3
+    stream_us = (last - land) / 1e3
+    rate = units * kv_bytes_per_unit / np.maximum(last - land, 1)  # bytes per ns = GB/s
+    slowest = np.argmax(exit_, axis=1)
+    return {
+        "launches": int(launches), "grid": int(grid),
+        "launch_period_us": stat(period),
+        "gap_prev_exit_to_entry_us": stat(gap),
+        "span_entry_to_last_exit_us": stat(span),
+        "entry_us": stat(us(entry)),
+        "ready_us": stat(us(ready)),
+        "first_issue_us": stat(us(fissue)),
+        "first_land_us": stat(us(land)),
+        "last_tile_us": stat(us(last)),
+        "final_merged_us": stat(us(merged)),
+        "final_done_us": stat(us(done)),
+        "exit_us": stat(us(exit_)),
+        "stream_us_per_cta": stat(stream_us),
+        "stream_gbs_per_cta": stat(rate),
+        "stream_gbs_all_ctas": round(float(np.median(units.sum(axis=1) * kv_bytes_per_unit /
+                                                     (last.max(axis=1) - land.min(axis=1)))), 1),
+        "units_per_cta": stat(units),
+        "mid_flush_us_per_cta": stat(midns / 1e3),
+        "flushes_per_cta": stat(flushes),
+        "final_kind_counts": {str(k): int((kind == k).sum()) for k in (0, 1, 2)},
+        "final_merge_us": stat((merged - last) / 1e3),
+        "final_write_us": stat((done - merged) / 1e3),
+        "slowest_cta_units": stat(units[np.arange(launches), slowest]),
+    }
+
+
+def run_trace(args):
+    """Per-CTA phase trace of one decode workload: one CUDA graph of
+    consecutive launches with the trace buffer set, replayed a few times; the
+    summary of the last replay is printed as one JSON line."""
+    import torch
+    import grouped_query_attention_fwd_b200 as gqa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = WORKLOADS[args.trace]
+    if cfg["Sq"] != 1 or "lens" in cfg:
+        raise SystemExit("--trace takes a contiguous single-query decode workload")
+    q, k, v, _ = _host_inputs(cfg, torch)
+    qd = q.to(dev)
+    kv_bytes = 2 * k.numel() * 2
+    copies = max(3, math.ceil(3 * L2_BYTES / kv_bytes))
+    ks = [k.to(dev) for _ in range(copies)]
+    vs = [v.to(dev) for _ in range(copies)]
+    out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
+    plan = gqa.query(qd, ks[0], vs[0])
+    ws = gqa.workspace_for(dev, plan["workspace_bytes"])
+    stream = torch.cuda.current_stream(dev)
+    launches = 32
+    grid = plan["grid"]
+    buf = torch.zeros(launches * grid * 16, dtype=torch.int64, device=dev)
+    for i in range(6):
+        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+    torch.cuda.synchronize()
+    gqa.debug_decode_trace(buf)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(launches):
+            gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+    gqa.debug_decode_trace(None)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = gqa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status after tracing: %s" % gqa.status_string(st))
+    unit_bytes = 2 * 128 * cfg["D"] * 2
+    summ = trace_summary(buf.cpu().numpy(), grid, launches, unit_bytes)
+    ms = e0.elapsed_time(e1) / launches
+    summ.update({"trace_workload": cfg["name"], "launch_ms_graph": round(ms, 5),
+                 "gbs_algorithmic": round(plan["algorithmic_bytes"] / (ms / 1e3) / 1e9, 1)})
+    print(json.dumps(summ), flush=True)
+    del g
+
+
 def run_gpu(args):
     import torch
     import grouped_query_attention_fwd_b200 as gqa
@@ -756,6 +860,8 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--profile", default=None, choices=sorted(WORKLOADS),
                     help="time one workload alone (for ncu captures) and exit")
+    ap.add_argument("--trace", default=None, choices=sorted(WORKLOADS),
+                    help="per-CTA phase trace of one decode workload, then exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -763,6 +869,8 @@ def main():
         run_reference(args)
     elif args.profile:
         run_profile_case(args)
+    elif args.trace:
+        run_trace(args)
     else:
         run_gpu(args)
 

@@ -38,7 +38,7 @@ GQA_DTYPE_BF16, GQA_DTYPE_F32, GQA_DTYPE_F16 = 0, 1, 2
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
 
 EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
-           "gqa_forward_decode_noalloc", "gqa_kv_append")
+           "gqa_forward_decode_noalloc", "gqa_kv_append", "gqa_debug_decode_trace")
 
 
 class Problem(ctypes.Structure):
@@ -101,6 +101,8 @@ _lib.gqa_forward_decode_noalloc.restype = ctypes.c_int
 _lib.gqa_kv_append.argtypes = [ctypes.POINTER(AppendDesc), _vp, _vp, _vp, _vp, _vp, _vp,
                                ctypes.c_size_t, _vp]
 _lib.gqa_kv_append.restype = ctypes.c_int
+_lib.gqa_debug_decode_trace.argtypes = [_vp, ctypes.c_int64]
+_lib.gqa_debug_decode_trace.restype = ctypes.c_int
 
 
 class GQAError(RuntimeError):
@@ -259,14 +261,36 @@ def query(q, k, v, mask=None, causal=False, scale=None, sm_count: int = 0, causa
                          sm_count).as_dict()
 
 
-def workspace_for(device, nbytes: int):
-    """A zeroed, cached device workspace of at least ``nbytes`` for ``device``."""
+def _stream_object(idx: int, stream):
+    """torch stream object for a raw cudaStream_t handle on device ``idx``."""
     torch = _torch()
-    key = torch.device(device).index if torch.device(device).index is not None else \
-        torch.cuda.current_device()
+    cur = torch.cuda.current_stream(idx)
+    if stream is None or int(stream) == cur.cuda_stream:
+        return cur
+    dflt = torch.cuda.default_stream(idx)
+    if int(stream) == dflt.cuda_stream:
+        return dflt
+    return torch.cuda.ExternalStream(int(stream), device=torch.device("cuda", idx))
+
+
+def workspace_for(device, nbytes: int, stream=None):
+    """A zeroed, cached device workspace of at least ``nbytes`` for ``device``
+    and ``stream`` (a cudaStream_t handle; None = the current stream).
+
+    One workspace per (device, stream): calls sharing a workspace must be
+    ordered on one stream, since the split-merge counters it holds are not
+    safe for calls that overlap on the GPU.  A new workspace is allocated and
+    zero-filled on that stream, so the caching allocator orders its reuse
+    after the stream's earlier work."""
+    torch = _torch()
+    dev = torch.device(device)
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    st = _stream_object(idx, stream)
+    key = (idx, int(st.cuda_stream))
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=torch.device("cuda", key))
+        with torch.cuda.device(idx), torch.cuda.stream(st):
+            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=torch.device("cuda", idx))
         _workspaces[key] = ws
     return ws
 
@@ -299,10 +323,10 @@ def forward(q, k, v, mask=None, causal=False, scale=None, out=None, workspace=No
     p = problem_for(q, k, v, mask, causal, scale, out, causal_offset=causal_offset, window=window,
                     kv_lens=kv_lens, block_table=block_table)
     plan = query_problem(p)
-    if workspace is None:
-        workspace = workspace_for(q.device, plan.workspace_bytes)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
+    if workspace is None:
+        workspace = workspace_for(q.device, plan.workspace_bytes, stream)
     forward_ptrs(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                  mask.data_ptr() if mask is not None else None, out.data_ptr(),
                  workspace.data_ptr(), workspace.numel(), stream)
@@ -359,19 +383,32 @@ def kv_append(cache_k, cache_v, k_new, v_new, kv_lens, workspace=None, stream=No
         d.block_table, d.block_table_stride = bt_ptr, bt_stride
         d.page_size, d.num_pages = page_size, num_pages
     lp = _lens_ptr(kv_lens, B)
-    if workspace is None:
-        workspace = workspace_for(cache_k.device, 256)
     if stream is None:
         stream = torch.cuda.current_stream(cache_k.device).cuda_stream
+    if workspace is None:
+        workspace = workspace_for(cache_k.device, 256, stream)
     kv_append_ptrs(d, cache_k.data_ptr(), cache_v.data_ptr(), k_new.data_ptr(),
                    v_new.data_ptr(), lp, workspace.data_ptr(), workspace.numel(), stream)
 
 
 def device_status(workspace=None, stream=None) -> int:
-    """Synchronise and read/clear the workspace error word (GQA_OK or an error)."""
+    """Synchronise and read/clear the workspace error word (GQA_OK or an error);
+    the default workspace is the one of (current device, ``stream``)."""
     torch = _torch()
-    if workspace is None:
-        workspace = workspace_for(torch.cuda.current_device(), 256)
     if stream is None:
         stream = torch.cuda.current_stream().cuda_stream
+    if workspace is None:
+        workspace = workspace_for(torch.cuda.current_device(), 256, stream)
     return _lib.gqa_device_status(workspace.data_ptr(), workspace.numel(), stream)
+
+
+def debug_decode_trace(buf=None) -> None:
+    """Diagnostics: record per-CTA phase timestamps of every following decode
+    launch into ``buf`` (an int64 CUDA tensor; None stops recording).  See
+    gqa_debug_decode_trace in include/gqa.h for the record layout."""
+    if buf is None:
+        rc = _lib.gqa_debug_decode_trace(None, 0)
+    else:
+        rc = _lib.gqa_debug_decode_trace(buf.data_ptr(), buf.numel() * buf.element_size())
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_debug_decode_trace")

@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "gqa.h"
 #include "kernels.h"
@@ -227,6 +228,24 @@ bool aligned(const void* ptr, uintptr_t a) {
 }  // namespace gqa
 
 namespace gqa {
+namespace {
+// Diagnostic trace buffer of the decode kernel (gqa_debug_decode_trace).
+std::mutex g_trace_mu;
+uint64_t* g_trace_buf = nullptr;
+int64_t g_trace_bytes = 0;
+uint64_t g_trace_next = 0;
+}  // namespace
+
+uint64_t* decode_trace_slot(int grid) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  if (g_trace_buf == nullptr || grid <= 0) return nullptr;
+  const int64_t words = static_cast<int64_t>(grid) * kDecodeTraceWords;
+  const int64_t slots = g_trace_bytes / (words * 8);
+  if (slots <= 0) return nullptr;
+  const int64_t slot = static_cast<int64_t>(g_trace_next++ % static_cast<uint64_t>(slots));
+  return g_trace_buf + slot * words;
+}
+
 // K/V tensor map for the decode tile shape, shared with the static-scratch
 // decode entry point.
 int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& p,
@@ -437,6 +456,17 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
   a.page_size = d->page_size;
   a.num_pages = d->num_pages;
   return launch_kv_append(a, static_cast<cudaStream_t>(stream_ptr));
+}
+
+GQA_API int gqa_debug_decode_trace(void* device_buffer, int64_t bytes) {
+  if (device_buffer != nullptr && bytes < 0) return GQA_ERR_ARG;
+  if (device_buffer != nullptr && (reinterpret_cast<uintptr_t>(device_buffer) & 7u) != 0)
+    return GQA_ERR_LAYOUT;
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  g_trace_buf = static_cast<uint64_t*>(device_buffer);
+  g_trace_bytes = device_buffer != nullptr ? bytes : 0;
+  g_trace_next = 0;
+  return GQA_OK;
 }
 
 GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* stream_ptr) {

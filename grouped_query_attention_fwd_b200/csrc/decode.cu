@@ -30,6 +30,17 @@
 //    and the last one merges all partials and writes bf16 `out` (the counters
 //    are zeroed on the stream before the launch).  No CTA ever waits for
 //    another one.
+//  * The CTA that finishes a split group last usually knows it in advance:
+//    the group's other contributors flushed it early in their ranges.  Once
+//    the consumers are on the range's last tile, the producer warp (idle by
+//    then) reads the final group's ticket count; if every other partial is
+//    already published the consumers merge them directly with their own
+//    states and write `out`, without publishing a partial or taking a ticket,
+//    which shortens the launch's tail.
+//  * Launched with programmatic stream serialisation: the next launch's CTAs
+//    may start, initialise their barriers and wait (griddepcontrol.wait) while
+//    this grid's last CTAs finish; nothing global is read or written before
+//    that wait.
 //  * Per-sequence cache lengths (kv_lens): each CTA reads the B lengths,
 //    counts the tiles every batch entry needs and prefix-sums them in shared
 //    memory, so the units -- and the cut into CTA ranges -- cover only keys
@@ -156,11 +167,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int* len_s = reinterpret_cast<int*>(tail + 16);
   int* pre_s = len_s + a.B;
 
+  volatile int* fast_flag = abort_flag + 2;  // the final split group is merged here directly
+  // Ticket count of the final split group read by the producer near the end
+  // of the range (kNoPeek until then; the producer's fence precedes the write).
+  volatile uint32_t* peek_count = reinterpret_cast<volatile uint32_t*>(abort_flag + 3);
+  constexpr uint32_t kNoPeek = 0xFFFFFFFFu;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool ragged = a.lens != nullptr;
   const int gpb = a.Hkv * passes;
+  // Trace record of this CTA (diagnostics only; the address is recomputed
+  // from the parameter at each use rather than held in a register).
+  auto trace = [&]() { return a.trace + blockIdx.x * kDecodeTraceWords; };
+  const uint64_t t_entry = (a.trace != nullptr && threadIdx.x == 0) ? globaltimer_ns() : 0;
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&full_v[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    *abort_flag = 0;
+    *fast_flag = 0;
+    *peek_count = kNoPeek;
+    fence_mbar_init();
+  }
+  // Everything above touches shared memory only; from here on global memory
+  // written by earlier work on the stream (lengths, caches, counters) is read.
+  griddep_wait();
+  griddep_launch_dependents();
   if (ragged) {
     for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
       int len = a.lens[b];
@@ -171,16 +206,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       len_s[b] = len;
     }
   }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&full_v[s], 1);
-      mbar_init(&empty[s], NCW);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
   __syncthreads();
+  if (a.trace != nullptr && threadIdx.x == 0) {
+    uint64_t* tr = trace();
+    for (int w = 0; w < kDecodeTraceWords; ++w) tr[w] = 0;
+    tr[kTrEntry] = t_entry;
+    tr[kTrReady] = globaltimer_ns();
+  }
   if (ragged) {
     if (warp == 0) {
       // pre[b + 1] = sum over entries <= b of (groups per entry) x (tiles of the entry).
@@ -287,16 +319,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             for (int c = 0; c < CHUNKS; ++c)
               tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES + h * kDecodePageBox * 128, &tmv,
                           &full_v[s], c * 64, prow[h], kv, page[h]);
+          if (a.trace != nullptr && it == 0) trace()[kTrFirstIssue] = globaltimer_ns();
           continue;
         }
         mbar_arrive_expect_tx(&full[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c)
           tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, key0, kv, b);
+        if (a.trace != nullptr && it == 0) trace()[kTrFirstIssue] = globaltimer_ns();
         mbar_arrive_expect_tx(&full_v[s], L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c)
           tma_load_4d(st + L::kTileBytes + c * CHUNK_BYTES, &tmv, &full_v[s], c * 64, key0, kv, b);
+      }
+      if (a.trace != nullptr) trace()[kTrLastIssue] = globaltimer_ns();
+      // Final group split over several CTAs: once the consumers have released
+      // the range's second-to-last tile, read the group's ticket count for
+      // the consumers' final flush (a fence makes the partials published
+      // before those tickets visible to this CTA).
+      if (!*abort_flag && u_begin < u_end) {
+        seek(cu, u_end - 1, sc, a);
+        const int gi = (u_end - 1 - cu.beg) / cu.kr.tiles;
+        const int g_beg = cu.beg + gi * cu.kr.tiles;
+        if (cta_of_unit(g_beg, sc.total, sc.P) !=
+            cta_of_unit(g_beg + cu.kr.tiles - 1, sc.total, sc.P)) {
+          const int j = it - 2;  // second-to-last unit of the range
+          const bool ready =
+              j < 0 || mbar_wait(&empty[j % stages], static_cast<uint32_t>((j / stages) & 1),
+                                 abort_flag, a.err, kErrDecodeWait);
+          if (ready) {
+            const uint32_t n = ld_relaxed_gpu(&counters[cu.b * gpb + gi]);
+            fence_acq_rel_gpu();
+            *peek_count = n;
+          }
+        }
       }
       // Unwind: make sure no copy is still landing in this CTA's shared memory.
       if (*abort_flag) {
@@ -407,8 +463,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // hold the same fragment positions of different keys: w + 4 hands its
     // state over, then the four merged states combine per output element.
     // The scratch rows keep (m, l) in the padding after the D values.
-    auto flush = [&]() {
+    auto flush = [&](bool final_flush) {
       constexpr int R = L::kScrRow;
+      // CTAs sharing this group (every CTA computes the same ranges).
+      const int c_lo = cta_of_unit(cur_beg, sc.total, sc.P);
+      const int c_hi = cta_of_unit(cur_beg + cur_tiles - 1, sc.total, sc.P);
+      const int n_contrib = c_hi - c_lo + 1;
+      // Fast final merge: every other contributor has published (the early
+      // ticket read saw n - 1) and one 4-wide column group per thread covers
+      // the group's output.
+      constexpr bool kOneQuadPerThread = HP * D / 4 <= NCW * 32;
+      if (kOneQuadPerThread && final_flush && threadIdx.x == 0) {
+        int fast = 0;
+        if (n_contrib > 1 && n_contrib <= kFastMerge &&
+            *peek_count == static_cast<uint32_t>(n_contrib - 1)) {
+          // The producer read the tickets and fenced at gpu scope before
+          // publishing the count in shared memory; acquiring that store at
+          // CTA scope orders the partial loads below after the other CTAs'
+          // releases.
+          fence_acq_rel_cta();
+          fast = 1;
+        }
+        *fast_flag = fast;
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -445,6 +522,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       };
       if (warp >= kMergeWarps) put_state();
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      // Partial slot of CTA cc for this group: only a range's first and last
+      // groups can be split, so two slots per CTA suffice.
+      auto slot_of = [&](int cc) -> int {
+        const int first = group_of(range_start(cc, sc.total, sc.P), sc, a);
+        return (cc * 2 + (first == cur ? 0 : 1)) * HP;
+      };
+      // Fast final merge: this thread's quad of every other partial is
+      // requested now, so that the loads overlap the eight-warp merge.
+      const bool fast = kOneQuadPerThread && final_flush && *fast_flag != 0;
+      float2 rml[kFastMerge];
+      float4 rov[kFastMerge];
+      if (fast && threadIdx.x < HP * D / 4) {
+        const int h = threadIdx.x / (D / 4), d = (threadIdx.x % (D / 4)) * 4;
+#pragma unroll
+        for (int k = 0; k < kFastMerge; ++k) {
+          const int cc = c_lo + k;
+          if (k < n_contrib && cc != static_cast<int>(blockIdx.x)) {
+            const int base = slot_of(cc);
+            rml[k] = __ldcg(&a.part_ml[base + h]);
+            rov[k] = __ldcg(reinterpret_cast<const float4*>(&a.part_o[(base + h) * D + d]));
+          }
+        }
+      }
       if (warp < kMergeWarps) {
         float wa[NT][2], wb[NT][2];
 #pragma unroll
@@ -473,17 +573,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         put_state();
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      if (a.trace != nullptr && final_flush && threadIdx.x == 0) trace()[kTrFinalMerged] = globaltimer_ns();
       auto m_of = [&](int w, int h) { return scr_o[(w * HP + h) * R + D]; };
       auto l_of = [&](int w, int h) { return scr_o[(w * HP + h) * R + D + 1]; };
-      // Which CTAs share this group?  Every CTA computes the same ranges.
-      const int c_lo = cta_of_unit(cur_beg, sc.total, sc.P);
-      const int c_hi = cta_of_unit(cur_beg + cur_tiles - 1, sc.total, sc.P);
-      // Partial slot of CTA cc for this group: only a range's first and last
-      // groups can be split, so two slots per CTA suffice.
-      auto slot_of = [&](int cc) -> int {
-        const int first = group_of(range_start(cc, sc.total, sc.P), sc, a);
-        return (cc * 2 + (first == cur ? 0 : 1)) * HP;
-      };
       // Output row of row hr of this pass (a head, or a (head, query) pair).
       auto out_row = [&](int hr) -> uint16_t* {
         const int r = pass * HP + hr;
@@ -516,6 +608,65 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           *reinterpret_cast<uint32_t*>(out_row(h) + d) = pack2<F16>(acc0 * inv, acc1 * inv);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+        if (a.trace != nullptr && final_flush && threadIdx.x == 0) {
+          trace()[kTrFinalDone] = globaltimer_ns();
+          trace()[kTrFinalKind] = 0;
+        }
+        return;
+      }
+      if (fast) {
+        // Every other partial of the group is published and was requested
+        // above: merge them with the eight warps' states and write out.
+        if (threadIdx.x < HP * D / 4) {
+          const int h = threadIdx.x / (D / 4), d = (threadIdx.x % (D / 4)) * 4;
+          if (pass * HP + h < a.rows && d < a.Dv) {
+            auto other = [&](int k) { return k < n_contrib && c_lo + k != static_cast<int>(blockIdx.x); };
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, m_of(w, h));
+#pragma unroll
+            for (int k = 0; k < kFastMerge; ++k)
+              if (other(k)) M = fmaxf(M, rml[k].x);
+            float Lsum = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (M != -INFINITY) {
+#pragma unroll
+              for (int w = 0; w < kMergeWarps; ++w) {
+                const float wt = fast_exp2(m_of(w, h) - M);
+                Lsum += wt * l_of(w, h);
+                const float4 ov = *reinterpret_cast<const float4*>(&scr_o[(w * HP + h) * R + d]);
+                acc.x += wt * ov.x;
+                acc.y += wt * ov.y;
+                acc.z += wt * ov.z;
+                acc.w += wt * ov.w;
+              }
+#pragma unroll
+              for (int k = 0; k < kFastMerge; ++k) {
+                if (other(k)) {
+                  const float wt = fast_exp2(rml[k].x - M);
+                  Lsum += wt * rml[k].y;
+                  acc.x += wt * rov[k].x;
+                  acc.y += wt * rov[k].y;
+                  acc.z += wt * rov[k].z;
+                  acc.w += wt * rov[k].w;
+                }
+              }
+            }
+            const float inv = 1.f / Lsum;  // Lsum == 0: NaN
+            uint2 pk;
+            pk.x = pack2<F16>(acc.x * inv, acc.y * inv);
+            pk.y = pack2<F16>(acc.z * inv, acc.w * inv);
+            *reinterpret_cast<uint2*>(out_row(h) + d) = pk;
+          }
+        }
+        // Every contributor has arrived: the counter goes back to zero for
+        // the next launch (which reads it only after this grid completes).
+        if (threadIdx.x == 0) counters[cur] = 0u;
+        asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+        if (a.trace != nullptr && threadIdx.x == 0) {
+          trace()[kTrFinalDone] = globaltimer_ns();
+          trace()[kTrFinalKind] = 2;
+        }
         return;
       }
       // Split group: publish this CTA's partial (float4 stores), then take a
@@ -651,6 +802,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (threadIdx.x == 0) atomicExch(&counters[cur], 0u);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+      if (a.trace != nullptr && final_flush && threadIdx.x == 0) {
+        trace()[kTrFinalDone] = globaltimer_ns();
+        trace()[kTrFinalKind] = 1;
+      }
     };
 
     int it = 0;
@@ -662,7 +817,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int grp = cu.b * gpb + gi;
       const int tile = r - gi * cu.kr.tiles + cu.kr.t0;
       if (grp != cur) {
-        if (cur >= 0) flush();
+        if (cur >= 0) {
+          const uint64_t t0 = (a.trace != nullptr && threadIdx.x == 0) ? globaltimer_ns() : 0;
+          flush(false);
+          if (a.trace != nullptr && threadIdx.x == 0) {
+            trace()[kTrMidFlushNs] += globaltimer_ns() - t0;
+            trace()[kTrFlushes] += 1;
+          }
+        }
         cur = grp;
         cur_beg = cu.beg + gi * cu.kr.tiles;
         cur_tiles = cu.kr.tiles;
@@ -686,6 +848,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
         continue;
       }
+      if (a.trace != nullptr && it == 0 && threadIdx.x == 0) trace()[kTrFirstLand] = globaltimer_ns();
       const uint32_t kbase = smem_u32(ring + s * L::kStageBytes);
       const uint32_t vbase = kbase + L::kTileBytes;
 
@@ -816,9 +979,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (cur >= 0) flush();  // after an abort too (its output is undefined, the error word set)
+    if (a.trace != nullptr && threadIdx.x == 0) trace()[kTrLastTile] = globaltimer_ns();
+    if (cur >= 0) {
+      flush(true);  // after an abort too (its output is undefined, the error word set)
+      if (a.trace != nullptr && threadIdx.x == 0) trace()[kTrFlushes] += 1;
+    }
   }
   __syncthreads();
+  if (a.trace != nullptr && threadIdx.x == 0) {
+    uint64_t* tr = trace();
+    tr[kTrExit] = globaltimer_ns();
+    tr[kTrSm] = static_cast<uint64_t>(sm_id()) | (static_cast<uint64_t>(blockIdx.x) << 32);
+    tr[kTrUnits] = static_cast<uint64_t>(u_end - u_begin);
+  }
 }
 
 template <int D, int NT, bool MQ, bool F16>
@@ -828,10 +1001,22 @@ int launch_decode_t(const DecodeShape& s, const DecodeArgs& a, const CUtensorMap
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_bytes) !=
       cudaSuccess)
     return GQA_ERR_CUDA;
-  kern<<<s.grid, kDecodeThreads, s.smem_bytes, stream>>>(tmk, tmv, a, s.tiles_per_group,
-                                                          s.passes, static_cast<int>(s.units),
-                                                          s.stages, a.counters);
-  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(s.grid));
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(s.smem_bytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, a, s.tiles_per_group, s.passes,
+                         static_cast<int>(s.units), s.stages, a.counters) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  return GQA_OK;
 }
 
 }  // namespace
@@ -916,6 +1101,7 @@ DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const vo
   a.causal_offset = p.causal_offset;
   a.window = p.window;
   a.scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634073599);
+  a.trace = decode_trace_slot(s.grid);
   return a;
 }
 

@@ -100,7 +100,31 @@ struct DecodeArgs {
   int causal;
   int64_t causal_offset, window;
   float scale_log2;  // scale * log2(e)
+  uint64_t* trace;   // per-CTA phase timestamps (kDecodeTraceWords each), or nullptr
 };
+
+// Diagnostic trace of the decode kernel: one record of kDecodeTraceWords
+// 64-bit words per CTA and launch (gqa_debug_decode_trace).
+constexpr int kDecodeTraceWords = 16;
+enum DecodeTraceWord : int {
+  kTrSm = 0,           // SM id (low 32 bits), CTA index (high 32 bits)
+  kTrEntry = 1,        // %globaltimer at kernel entry
+  kTrReady = 2,        // set-up done, earlier grids complete (after the dependent-launch wait)
+  kTrFirstIssue = 3,   // producer: first K tile copy issued
+  kTrLastIssue = 4,    // producer: last V tile copy issued
+  kTrFirstLand = 5,    // consumer warp 0: first K tile landed
+  kTrLastTile = 6,     // consumer warp 0: last tile consumed
+  kTrFinalMerged = 7,  // final group merged across the eight warps
+  kTrFinalDone = 8,    // final group written (out, or a partial and its ticket)
+  kTrExit = 9,         // after the closing barrier
+  kTrUnits = 10,       // tiles in this CTA's range
+  kTrFlushes = 11,     // groups flushed
+  kTrMidFlushNs = 12,  // consumer warp 0: time spent in flushes before the final one
+  kTrFinalKind = 13,   // final group: 0 whole, 1 split (published), 2 split (merged here directly)
+};
+// Device buffer and slot count set by gqa_debug_decode_trace (api.cu), or
+// nullptr; each decode launch takes the next slot.
+uint64_t* decode_trace_slot(int grid);
 
 // Arguments of one decode launch; the workspace `ws` holds the error word at
 // offset 0 and the plan's counters and partials.

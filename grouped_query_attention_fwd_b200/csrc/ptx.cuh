@@ -24,6 +24,46 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+__device__ __forceinline__ uint32_t sm_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %smid;" : "=r"(r));
+  return r;
+}
+
+// Programmatic dependent launch.  griddep_wait: block until the grids this
+// launch depends on have completed and their memory is visible (a no-op for a
+// launch without the programmatic-serialization attribute); nothing written by
+// earlier work on the stream may be read, and nothing may be written, before
+// it.  griddep_launch_dependents: let the next launch on the stream be
+// scheduled before this grid has finished (it still waits in its own
+// griddep_wait for this grid's completion).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Relaxed 32-bit load at gpu scope (no ordering of later accesses).
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* addr) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Acquire-release fence at gpu scope: after a relaxed load that observed a
+// value written by a release operation, accesses after the fence see what the
+// releasing thread wrote before it.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// The same at CTA scope: for a value another thread of this CTA released.
+__device__ __forceinline__ void fence_acq_rel_cta() {
+  asm volatile("fence.acq_rel.cta;" ::: "memory");
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

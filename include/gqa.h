@@ -272,6 +272,23 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
                           const void* k_new, const void* v_new, int32_t* kv_lens,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gqa_debug_decode_trace -- diagnostics: record per-CTA phase timestamps of
+ * the decode kernel.  Not part of the operation (the pages have no
+ * counterpart); used to account for the time of a launch that is not spent
+ * streaming K/V.
+ *   device_buffer: device memory of `bytes` bytes, 8-byte aligned, owned by
+ *                  the caller, or NULL to stop recording.
+ * While set, every decode launch (gqa_forward, gqa_forward_decode_noalloc)
+ * writes, per CTA, 16 unsigned 64-bit words (%globaltimer nanoseconds and
+ * counts; layout: kDecodeTraceWords / DecodeTraceWord in the library's
+ * csrc/kernels.h) into the next slot of grid * 128 bytes; launch k uses slot
+ * k mod (bytes / slot size).  The setting is process-wide and is captured
+ * into CUDA graphs with the launch.  Returns GQA_OK, GQA_ERR_ARG for a
+ * negative size or GQA_ERR_LAYOUT for a misaligned buffer.
+ */
+GQA_API int gqa_debug_decode_trace(void* device_buffer, int64_t bytes);
+
 /* Static English description of a status code (never NULL). */
 GQA_API const char* gqa_status_string(int status);
 

@@ -298,3 +298,30 @@ def test_decode_many_groups_zeroes_its_counters(gqa):
     for b in (0, 777, 2099):
         ref = oracle_bf16(bits[0][b:b + 1], bits[1][b:b + 1], bits[2][b:b + 1])
         assert_bf16_parity(out[b:b + 1], ref, "many groups b=%d" % b)
+
+
+def test_default_workspaces_on_two_streams(gqa):
+    """Decodes issued on two streams with the default arguments each get the
+    workspace of their own stream: split groups merge correctly on both even
+    when the launches overlap on the GPU."""
+    dev = torch.device("cuda")
+    cases = []
+    for seed in (41, 42):
+        (qb, kb, vb), (q, k, v) = bf16_inputs(seed, 2, 8, 2, 1, 8192, 128)
+        cases.append(((qb, kb, vb), (q, k, v)))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    outs = [[], []]
+    for _ in range(6):
+        for i, s in enumerate(streams):
+            with torch.cuda.stream(s):
+                outs[i].append(gqa.forward(*cases[i][1]))
+    torch.cuda.synchronize()
+    ws = [gqa.workspace_for(dev, 256, s.cuda_stream) for s in streams]
+    assert ws[0].data_ptr() != ws[1].data_ptr()
+    for i, s in enumerate(streams):
+        assert gqa.device_status(stream=s.cuda_stream) == 0
+        ref = oracle_bf16(*cases[i][0])
+        for o in outs[i]:
+            assert_bf16_parity(to_np(o), ref, "stream %d" % i)
