@@ -228,20 +228,24 @@ def weak_scaling_gbs(bytes_per_step: int, steps: int, world: int, elapsed_ms: fl
 
 # ------------------------------------------------------------------ GPU arm
 
-def _graph_timed(torch, calls, steps, warmup, stream, per_launch_samples=200):
-    """Time exactly `steps` launches, launch i being calls[i % len(calls)].
+def _graph_timed(torch, calls, steps, warmup, stream, repeats=1, per_launch_samples=100,
+                 before_each=None):
+    """Time exactly `steps` launches, launch i being calls[i % len(calls)],
+    `repeats` times over.
 
-    Whole run: the launches are captured into CUDA graphs of many launches
-    each (one host call per ~32 launches, so the host never starves the GPU)
-    and the run is bracketed by two events.  Per launch: a separate pass
-    replays one-launch graphs with an event pair around each.  Returns
-    (total_ms for the `steps` launches, per-launch ms list, host seconds per
-    launch spent enqueuing the whole run)."""
+    The launches are captured into CUDA graphs (one graph of up to ~64
+    launches, a whole number of rounds over the calls, replayed, plus one for
+    the remainder), so the host never paces the GPU.  Each repetition of the
+    `steps` launches is bracketed by a device synchronise (after
+    `before_each()`, e.g. a barrier over ranks) and two events on `stream`.
+    A separate pass replays one-launch graphs with an event pair around each.
+    Returns (ms of each repetition, per-launch ms list, host seconds per
+    launch spent enqueuing a repetition)."""
     for i in range(warmup):
         calls[i % len(calls)]()
     torch.cuda.synchronize()
     n = len(calls)
-    reps = max(1, 32 // n)
+    chunk = n * max(1, min(64, steps) // n) if steps >= n else steps
 
     def capture(count, start):
         g = torch.cuda.CUDAGraph()
@@ -250,26 +254,32 @@ def _graph_timed(torch, calls, steps, warmup, stream, per_launch_samples=200):
                 calls[(start + j) % n]()
         return g
 
-    chain = capture(n * reps, 0)            # a whole number of rounds over the copies
-    tail = capture(steps % (n * reps), 0) if steps % (n * reps) else None
+    chain = capture(chunk, 0)
+    tail = capture(steps % chunk, 0) if steps % chunk else None
     singles = [capture(1, i) for i in range(n)]
     chain.replay()
+    if tail is not None:
+        tail.replay()
     for g in singles:
         g.replay()
     torch.cuda.synchronize()
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    h0 = time.perf_counter()
-    e0.record(stream)
-    for _ in range(steps // (n * reps)):
-        chain.replay()
-    if tail is not None:
-        tail.replay()
-    e1.record(stream)
-    h1 = time.perf_counter()
-    torch.cuda.synchronize()
-    total_ms = e0.elapsed_time(e1)
+    times, host = [], []
+    for _ in range(repeats):
+        if before_each is not None:
+            before_each()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
+        e0.record(stream)
+        for _ in range(steps // chunk):
+            chain.replay()
+        if tail is not None:
+            tail.replay()
+        e1.record(stream)
+        host.append(time.perf_counter() - h0)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
 
     k = min(steps, per_launch_samples)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -281,7 +291,13 @@ def _graph_timed(torch, calls, steps, warmup, stream, per_launch_samples=200):
     torch.cuda.synchronize()
     per = [a.elapsed_time(b) for a, b in ev]
     del chain, tail, singles
-    return total_ms, per, (h1 - h0) / steps
+    return times, per, statistics.median(host) / steps
+
+
+def timing_repeats(steps: int) -> int:
+    """Repetitions of the `steps`-launch timed region: about 2000 launches in
+    all, at least 3 and at most 50 repetitions."""
+    return max(3, min(50, -(-2000 // max(1, steps))))
 
 
 def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYTES):
@@ -299,7 +315,8 @@ def _time_config(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
     stream = torch.cuda.current_stream(dev)
     calls = [(lambda i=i: gqa.forward(qd, ks[i], vs[i], mask=md, causal=cfg["causal"], out=out,
                                       workspace=ws)) for i in range(copies)]
-    total_ms, per, _ = _graph_timed(torch, calls, steps, warmup, stream)
+    times, per, _ = _graph_timed(torch, calls, steps, warmup, stream, repeats=5)
+    total_ms = statistics.median(times)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
@@ -376,12 +393,13 @@ def _time_ragged(gqa, torch, cfg, steps, warmup, dev, rotate_to_bytes=3 * L2_BYT
 
     calls = [(lambda i=i: call(i)) for i in range(copies)]
     if n_new:  # every call of a copy appends n_new tokens: they must fit the capacity
-        rounds = max(1, 32 // copies) * copies  # warm replay of the many-launch graph
-        executed = warmup + rounds + copies + steps + min(steps, 200)
+        chunk = copies * max(1, min(64, steps) // copies)  # warm replay of the graphs
+        executed = warmup + chunk + steps % chunk + copies + 5 * steps + min(steps, 100)
         calls_per_copy = math.ceil(executed / copies)
         if hi + calls_per_copy * n_new > Sk:
             raise ValueError("%d steps overflow the %d-key cache; use fewer" % (steps, Sk))
-    total_ms, per, _ = _graph_timed(torch, calls, steps, warmup, stream)
+    times, per, _ = _graph_timed(torch, calls, steps, warmup, stream, repeats=5)
+    total_ms = statistics.median(times)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
@@ -436,30 +454,109 @@ def _e2e(gqa, torch, cfg, steps, dev):
     return ms, h2d, out_h.numel() * 2
 
 
-def _cpu_baseline(cfg, budget_s=12.0):
-    """The fp64 oracle as it stands, single-threaded, on whole (batch, kv head)
-    groups of the workload until about ``budget_s`` of CPU time."""
-    import oracle
-    B, Hq, Hkv, Sq, Sk, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sq", "Sk", "D"))
-    g = Hq // Hkv
-    qb = synth.normal_bf16_bits(cfg["seed"], synth.STREAM_Q, B * Hq * Sq * D).reshape(B, Hq, Sq, D)
-    groups, nbytes, t_used = 0, 0, 0.0
-    order = [(b, kv) for b in range(B) for kv in range(Hkv)]
-    while t_used < budget_s and groups < len(order) * 64:
-        b, kv = order[groups % len(order)]
-        ks = synth.bf16_bits_to_f64(
-            synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_K, B, Hkv, Sk, D, b, kv))[None, None]
-        vs = synth.bf16_bits_to_f64(
-            synth.kv_slice_bf16_bits(cfg["seed"], synth.STREAM_V, B, Hkv, Sk, D, b, kv))[None, None]
-        qs = synth.bf16_bits_to_f64(qb[b:b + 1, kv * g:(kv + 1) * g])
+def _time_oracle(fn, budget_s, max_calls=100000):
+    """Call fn() until about budget_s of wall time; returns (calls, seconds)."""
+    calls, used = 0, 0.0
+    while used < budget_s and calls < max_calls:
         t0 = time.perf_counter()
-        oracle.forward(qs, ks, vs, causal=cfg["causal"])
-        t_used += time.perf_counter() - t0
-        groups += 1
-        nbytes += 2 * (qs.size * 2) + 2 * (Sk * D * 2)
-    return dict(value=nbytes / t_used / 1e9, unit="GB/s", cores=1, kind="oracle",
-                sample="%d (batch, kv-head) groups of %d query heads x %d keys (of %d groups), "
-                       "fp64 single-threaded, %.1f s" % (groups, g, Sk, B * Hkv, t_used))
+        fn(calls)
+        used += time.perf_counter() - t0
+        calls += 1
+    return calls, used
+
+
+def _cpu_baseline(budget_s=16.0):
+    """The fp64 oracle as it stands (single-threaded C++, unchanged), timed on
+    bounded samples of all five workloads, about budget_s of CPU time in all.
+    The headline value is the Mistral-7B-shaped decode's; `per_config` holds
+    every workload's rate in its own unit with the sample it was taken on."""
+    import oracle
+    per = {}
+
+    # Page-1 toy, fp32: the whole problem, repeatedly.
+    q, k, v = synth.qkv_f32(1, 1, 4, 2, 5, 5, 4)
+    n, t = _time_oracle(lambda i: oracle.forward(q, k, v, scale=0.5), 0.05 * budget_s, 20000)
+    per["page1_toy_f32"] = {"value": round(t / n * 1e6, 2), "unit": "us per forward",
+                            "sample": "the whole (1,4,5,4) problem, %d calls" % n}
+
+    def decode_groups(cfg, share, distinct):
+        B, Hq, Hkv, Sk, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sk", "D"))
+        g = Hq // Hkv
+        qb = synth.normal_bf16_bits(cfg["seed"], synth.STREAM_Q, B * Hq * D).reshape(B, Hq, 1, D)
+        # Cycle over the first `distinct` groups (generating their inputs is
+        # not timed, and takes longer than the oracle on the long cache).
+        order = [(b, kv) for b in range(B) for kv in range(Hkv)][:distinct]
+        cache = {}
+
+        def one(i):
+            b, kv = order[i % len(order)]
+            if (b, kv) not in cache:
+                ks = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(
+                    cfg["seed"], synth.STREAM_K, B, Hkv, Sk, D, b, kv))[None, None]
+                vs = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(
+                    cfg["seed"], synth.STREAM_V, B, Hkv, Sk, D, b, kv))[None, None]
+                cache.clear()
+                cache[(b, kv)] = (synth.bf16_bits_to_f64(qb[b:b + 1, kv * g:(kv + 1) * g]), ks, vs)
+            oracle.forward(*cache[(b, kv)], causal=cfg["causal"])
+
+        # Input generation is not timed: only the oracle calls.
+        calls, used = 0, 0.0
+        slices = {}
+        while used < share * budget_s and calls < 1000 * len(order):
+            b, kv = order[calls % len(order)]
+            if (b, kv) not in slices:
+                cache.clear()
+                one(calls)  # builds the slice (untimed) and runs once (untimed)
+                slices[(b, kv)] = cache[(b, kv)]
+            cache[(b, kv)] = slices[(b, kv)]
+            t0 = time.perf_counter()
+            oracle.forward(*cache[(b, kv)], causal=cfg["causal"])
+            used += time.perf_counter() - t0
+            calls += 1
+        nbytes = calls * (2 * g * D * 2 + 2 * Sk * D * 2)
+        return {"value": round(nbytes / used / 1e9, 4), "unit": "GB/s",
+                "sample": "%d calls over %d (batch, kv-head) groups of %d query heads x %d keys "
+                          "(of %d groups), %.1f s" % (calls, len(order), g, Sk, B * Hkv, used)}
+
+    def prefill_rows(cfg, share, causal_flops):
+        B, Hq, Hkv, S, D = (cfg[x] for x in ("B", "Hq", "Hkv", "Sq", "D"))
+        g = Hq // Hkv
+        b, kv = B - 1, Hkv - 1
+        qs = np.stack([synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(
+            cfg["seed"], synth.STREAM_Q, B, Hq, S, D, b, kv * g + h)) for h in range(g)])[None]
+        ks = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(
+            cfg["seed"], synth.STREAM_K, B, Hkv, S, D, b, kv))[None, None]
+        vs = synth.bf16_bits_to_f64(synth.kv_slice_bf16_bits(
+            cfg["seed"], synth.STREAM_V, B, Hkv, S, D, b, kv))[None, None]
+        mask = None
+        if cfg["mask"]:
+            lens = synth.uniform_int(cfg["seed"], synth.STREAM_MASK, B, 256, S)
+            mask = synth.mask_from_lengths(lens, S, S)[b:b + 1]
+        rows = [(0, h, i) for i in range(0, S, 61) for h in range(g)]
+        flops, n, used = 0.0, 0, 0.0
+        while used < share * budget_s and n < 50 * len(rows):
+            at = n % len(rows)
+            chunk = rows[at:at + 64]
+            t0 = time.perf_counter()
+            oracle.forward_rows(qs, ks, vs, chunk, mask=mask, causal=cfg["causal"])
+            used += time.perf_counter() - t0
+            n += len(chunk)
+            flops += sum(4.0 * D * ((i + 1) if causal_flops else S) for (_, _, i) in chunk)
+        return {"value": round(flops / used / 1e9, 3), "unit": "GFLOP/s",
+                "sample": "%d rows (cycling over query positions 0, 61, 122, ... of every head "
+                          "of batch entry %d, kv head %d), %.1f s; FLOPs counted %s" % (
+                              n, b, kv, used, "4*D per visible (causal) key" if causal_flops
+                              else "4*D*Sk per row (the dense formula)")}
+
+    per["decode_mistral7b_layer"] = decode_groups(DECODE, 0.35, 16)
+    per["decode_llama2_70b_layer"] = decode_groups(DECODE_LONG, 0.2, 2)
+    per["prefill_causal"] = prefill_rows(PREFILL_CAUSAL, 0.2, True)
+    per["prefill_padded_mask"] = prefill_rows(PREFILL_MASKED, 0.2, False)
+    head = per["decode_mistral7b_layer"]
+    return dict(value=head["value"], unit="GB/s", cores=1, threads_used=1,
+                host_cores=os.cpu_count(), kind="oracle",
+                sample="decode workload: " + head["sample"] + "; every workload in per_config",
+                per_config=per)
 
 
 def _roofline_decode(res, hbm, peak_kind, workload, kernel_file="decode.cu"):
@@ -619,7 +716,10 @@ def run_trace(args):
     if st != 0:
         raise RuntimeError("device status after tracing: %s" % gqa.status_string(st))
     unit_bytes = 2 * 128 * cfg["D"] * 2
-    summ = trace_summary(buf.cpu().numpy(), grid, launches, unit_bytes)
+    raw = buf.cpu().numpy()
+    if getattr(args, "trace_out", None):
+        np.save(args.trace_out, raw.reshape(launches, grid, 16))
+    summ = trace_summary(raw, grid, launches, unit_bytes)
     ms = e0.elapsed_time(e1) / launches
     summ.update({"trace_workload": cfg["name"], "launch_ms_graph": round(ms, 5),
                  "gbs_algorithmic": round(plan["algorithmic_bytes"] / (ms / 1e3) / 1e9, 1)})
@@ -672,19 +772,27 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    elapsed_ms, per, host_s = _graph_timed(torch, calls, args.steps, args.warmup, stream)
+    # The timed region (exactly --steps launches, a barrier and a device
+    # synchronise before it) is repeated; every repetition is timed on the
+    # device and reduced to its maximum over ranks, and the median
+    # repetition gives the reported value.
+    repeats = timing_repeats(args.steps)
+    times, per, host_s = _graph_timed(torch, calls, args.steps, args.warmup, stream,
+                                      repeats=repeats,
+                                      before_each=(dist.barrier if dist is not None else None))
     t_wall1 = time.time()
     if dist is not None:
         dist.barrier()
     sampler.stop()
-    # Average launch duration over the timed region (graphs of many launches);
-    # the one-launch-graph pass adds the graph launch to every launch.
-    per_launch = elapsed_ms / args.steps
     single_launch = statistics.median(per)
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after timing: %s" % gqa.status_string(st))
-    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
+    times = [max_over_ranks(t, dist, dev) for t in times]
+    elapsed_ms = statistics.median(times)
+    # Average launch duration over the median timed region (graphs of many
+    # launches); the one-launch-graph pass adds the graph launch to every launch.
+    per_launch = elapsed_ms / args.steps
     del ks, vs
     torch.cuda.empty_cache()
 
@@ -699,6 +807,9 @@ def run_gpu(args):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "timing": {"repeats": repeats, "statistic": "median repetition (max over ranks)",
+                   "ms_per_step_min": round(min(times) / args.steps, 5),
+                   "ms_per_step_max": round(max(times) / args.steps, 5)},
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -711,10 +822,11 @@ def run_gpu(args):
             "parallelism": "replicas" if world == 1 else "dp%d (independent problems per rank)" % world,
             "l2": "K/V rotated over %d device copies (%.0f MB) so no launch finds its K/V in L2"
                   % (copies, copies * kv_bytes / 1e6),
-            "launch": "one gqa_forward per step; the steps are replayed from CUDA graphs of "
-                      "%d launches (host enqueue %.2f us per step); per-launch times from a "
-                      "separate pass of one-launch graphs" % (max(1, 32 // copies) * copies,
-                                                              host_s * 1e6),
+            "launch": "one gqa_forward per step; each repetition of the %d steps is replayed "
+                      "from CUDA graphs of up to %d launches (host enqueue %.2f us per step); "
+                      "per-launch times from a separate pass of one-launch graphs"
+                      % (args.steps, copies * max(1, min(64, args.steps) // copies)
+                         if args.steps >= copies else args.steps, host_s * 1e6),
         },
         "gpu_launches": args.steps * plan["launches"],
         "clocks": {k_: v_ for k_, v_ in clocks.items()},
@@ -729,7 +841,8 @@ def run_gpu(args):
             "kernel": "gqa_decode_kernel (split merge fused; the counter memset is in the same graph)",
             "algorithmic_bytes_per_launch": plan["algorithmic_bytes"],
             "launch_ms": round(per_launch, 5),
-            "launch_ms_basis": "timed region / steps (CUDA events around the graphs of launches)",
+            "launch_ms_basis": "median timed region / steps (CUDA events around the graphs of "
+                               "launches)",
             "single_launch_graph_median_ms": round(single_launch, 5),
         },
     }
@@ -771,7 +884,7 @@ def run_gpu(args):
                        "ms_per_step": round(ms, 4),
                        "note": "pinned host q/k/v copied to the device, gqa_forward, out copied back, every step"}
     if rank == 0 and world == 1 and not args.skip_cpu:
-        line["cpu_baseline"] = _cpu_baseline(DECODE)
+        line["cpu_baseline"] = _cpu_baseline()
 
     if dist is not None:
         dist.barrier()
@@ -841,8 +954,8 @@ def run_reference(args):
         "data": "synthetic: same seeded inputs as the GPU arm",
         "config": {"workload": "decode, Mistral-7B-shaped layer: B=16 Hq=32 Hkv=8 Sq=1 Sk=4096 "
                                "D=128, bounded sample per step (see cpu_baseline.sample)"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "threads_used": 1,
+                         "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -862,6 +975,8 @@ def main():
                     help="time one workload alone (for ncu captures) and exit")
     ap.add_argument("--trace", default=None, choices=sorted(WORKLOADS),
                     help="per-CTA phase trace of one decode workload, then exit")
+    ap.add_argument("--trace-out", default=None,
+                    help="with --trace: also save the raw records (.npy, [launch, CTA, word])")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -38,7 +38,8 @@ GQA_DTYPE_BF16, GQA_DTYPE_F32, GQA_DTYPE_F16 = 0, 1, 2
 KERNEL_NAMES = {0: "none", 1: "decode", 2: "prefill", 3: "f32", 4: "zero", 5: "nan"}
 
 EXPORTS = ("gqa_query", "gqa_forward", "gqa_device_status", "gqa_status_string", "gqa_version",
-           "gqa_forward_decode_noalloc", "gqa_kv_append", "gqa_debug_decode_trace")
+           "gqa_forward_decode_noalloc", "gqa_kv_append", "gqa_debug_decode_trace",
+           "gqa_debug_decode_withhold")
 
 
 class Problem(ctypes.Structure):
@@ -103,6 +104,8 @@ _lib.gqa_kv_append.argtypes = [ctypes.POINTER(AppendDesc), _vp, _vp, _vp, _vp, _
 _lib.gqa_kv_append.restype = ctypes.c_int
 _lib.gqa_debug_decode_trace.argtypes = [_vp, ctypes.c_int64]
 _lib.gqa_debug_decode_trace.restype = ctypes.c_int
+_lib.gqa_debug_decode_withhold.argtypes = [ctypes.c_int64, ctypes.c_int64]
+_lib.gqa_debug_decode_withhold.restype = ctypes.c_int
 
 
 class GQAError(RuntimeError):
@@ -412,3 +415,13 @@ def debug_decode_trace(buf=None) -> None:
         rc = _lib.gqa_debug_decode_trace(buf.data_ptr(), buf.numel() * buf.element_size())
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_debug_decode_trace")
+
+
+def debug_decode_withhold(unit: int, wait_limit_ns: int) -> None:
+    """Test of the bounded waits: the next decode launch withholds the copies
+    of `unit` and gives up its waits after `wait_limit_ns`; device_status()
+    then reports GQA_ERR_TIMEOUT.  See gqa_debug_decode_withhold in
+    include/gqa.h."""
+    rc = _lib.gqa_debug_decode_withhold(int(unit), int(wait_limit_ns))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_debug_decode_withhold")

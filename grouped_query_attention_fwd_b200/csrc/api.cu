@@ -236,6 +236,17 @@ int64_t g_trace_bytes = 0;
 uint64_t g_trace_next = 0;
 }  // namespace
 
+int g_withhold_unit = -1;  // one-shot test settings (gqa_debug_decode_withhold)
+uint64_t g_wait_ns = kWaitLimitNs;
+
+void decode_test_settings(int* withhold_unit, uint64_t* wait_ns) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  *withhold_unit = g_withhold_unit;
+  *wait_ns = g_wait_ns;
+  g_withhold_unit = -1;
+  g_wait_ns = kWaitLimitNs;
+}
+
 uint64_t* decode_trace_slot(int grid) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   if (g_trace_buf == nullptr || grid <= 0) return nullptr;
@@ -359,7 +370,14 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   int erc = encode_half_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
                             static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g), f16);
   if (erc != GQA_OK) return erc;
-  if (p.block_table != nullptr) {  // paged: 64-key boxes, one page each
+  if (s.pair) {  // each CTA of a pair loads 64 keys of a K tile and 64 columns of a V tile
+    erc = encode_half_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 64, 1,
+                          f16);
+    if (erc != GQA_OK) return erc;
+    erc = encode_half_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128,
+                          1, f16);
+    if (erc != GQA_OK) return erc;
+  } else if (p.block_table != nullptr) {  // paged: 64-key boxes, one page each
     erc = encode_decode_kv_map(&tmk, k, p, p.k_stride);
     if (erc != GQA_OK) return erc;
     erc = encode_decode_kv_map(&tmv, v, p, p.v_stride);
@@ -392,6 +410,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.lens = p.kv_lens;
   a.Dv = static_cast<int>(p.head_dim);
   a.scale_log2 = scale_log2;
+  if (s.pair) return launch_prefill_pair(p, s, a, tmq, tmk, tmv, stream);
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
 }
 
@@ -466,6 +485,16 @@ GQA_API int gqa_debug_decode_trace(void* device_buffer, int64_t bytes) {
   g_trace_buf = static_cast<uint64_t*>(device_buffer);
   g_trace_bytes = device_buffer != nullptr ? bytes : 0;
   g_trace_next = 0;
+  return GQA_OK;
+}
+
+GQA_API int gqa_debug_decode_withhold(int64_t unit, int64_t wait_limit_ns) {
+  if (unit < -1 || unit >= (int64_t(1) << 31)) return GQA_ERR_ARG;
+  if (wait_limit_ns < 1000 || wait_limit_ns > static_cast<int64_t>(kWaitLimitNs))
+    return GQA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  g_withhold_unit = static_cast<int>(unit);
+  g_wait_ns = static_cast<uint64_t>(wait_limit_ns);
   return GQA_OK;
 }
 

@@ -181,6 +181,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   auto trace = [&]() { return a.trace + blockIdx.x * kDecodeTraceWords; };
   const uint64_t t_entry = (a.trace != nullptr && threadIdx.x == 0) ? globaltimer_ns() : 0;
 
+  if (warp == NCW && lane == 0) {
+    // The tensor maps are kernel parameters: fetch them before the wait.
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
@@ -252,8 +257,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tmk);
-      prefetch_tmap(&tmv);
       int it = 0;
       Cursor cu;
       // Paged cache: each 128-key tile is two 64-key boxes, each in one page.
@@ -284,8 +287,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int s = it % stages;
         const uint32_t round = static_cast<uint32_t>(it / stages);
         if (round > 0 &&
-            !mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, a.err, kErrDecodeWait))
+            !mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, a.err, kErrDecodeWait, a.wait_ns))
           break;
+        if (u == a.withhold_unit) {
+          // Test of the bounded waits (gqa_debug_decode_withhold): this
+          // unit's copies are never issued, so the consumers' wait for it
+          // runs out and aborts the CTA; nothing more is issued, so every
+          // copy in flight belongs to an earlier unit and lands.
+          const uint64_t t0 = globaltimer_ns();
+          while (!*abort_flag && globaltimer_ns() - t0 < 4 * a.wait_ns) {
+          }
+          break;
+        }
         seek(cu, u, sc, a);
         const int r = u - cu.beg;
         const int gi = r / cu.kr.tiles;  // group within the entry: kv * passes + pass
@@ -346,7 +359,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const int j = it - 2;  // second-to-last unit of the range
           const bool ready =
               j < 0 || mbar_wait(&empty[j % stages], static_cast<uint32_t>((j / stages) & 1),
-                                 abort_flag, a.err, kErrDecodeWait);
+                                 abort_flag, a.err, kErrDecodeWait, a.wait_ns);
           if (ready) {
             const uint32_t n = ld_relaxed_gpu(&counters[cu.b * gpb + gi]);
             fence_acq_rel_gpu();
@@ -358,8 +371,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (*abort_flag) {
         const int issued = it;
         for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j) {
-          mbar_wait_drain(&full[j % stages], static_cast<uint32_t>((j / stages) & 1));
-          mbar_wait_drain(&full_v[j % stages], static_cast<uint32_t>((j / stages) & 1));
+          mbar_wait_drain(&full[j % stages], static_cast<uint32_t>((j / stages) & 1),
+                          a.wait_ns / 4);
+          mbar_wait_drain(&full_v[j % stages], static_cast<uint32_t>((j / stages) & 1),
+                          a.wait_ns / 4);
         }
       }
     }
@@ -843,7 +858,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // A wait that gives up sets the abort flag; from then on every wait
       // fails at once and the warps skip the arithmetic but keep walking the
       // units, so that all eight reach the same flush() barriers.
-      if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
+      if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrDecodeWait, a.wait_ns)) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         continue;
@@ -940,7 +955,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
 
       // O^T[D x 8] += V^T[D x 16 keys] P^T[16 keys x 8], once the V tile is in.
-      if (!mbar_wait(&full_v[s], round & 1u, abort_flag, a.err, kErrDecodeWait)) {
+      if (!mbar_wait(&full_v[s], round & 1u, abort_flag, a.err, kErrDecodeWait, a.wait_ns)) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         continue;
@@ -1102,6 +1117,7 @@ DecodeArgs make_decode_args(const gqa_problem& p, const DecodeShape& s, const vo
   a.window = p.window;
   a.scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634073599);
   a.trace = decode_trace_slot(s.grid);
+  decode_test_settings(&a.withhold_unit, &a.wait_ns);
   return a;
 }
 

@@ -101,7 +101,14 @@ struct DecodeArgs {
   int64_t causal_offset, window;
   float scale_log2;  // scale * log2(e)
   uint64_t* trace;   // per-CTA phase timestamps (kDecodeTraceWords each), or nullptr
+  uint64_t wait_ns;  // limit of every wait of the launch (1 s unless a test shortens it)
+  int withhold_unit; // test only (gqa_debug_decode_withhold): the producer never issues
+                     // this unit's copies and stops there; -1 = none
 };
+
+// One-shot settings of the next decode launch made by gqa_debug_decode_withhold
+// (api.cu): the unit to withhold (-1: none) and the wait limit.
+void decode_test_settings(int* withhold_unit, uint64_t* wait_ns);
 
 // Diagnostic trace of the decode kernel: one record of kDecodeTraceWords
 // 64-bit words per CTA and launch (gqa_debug_decode_trace).
@@ -141,7 +148,14 @@ int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& 
 // ------------------------------------------------------------ prefill
 constexpr int kPrefillThreads = 12 * 32;  // two softmax warpgroups, load, MMA and V-load warps
 
+// Key tiles a work item of the pair prefill kernel may span (Sk <= 32768).
+constexpr int kMaxPairTiles = 256;
+// The pair prefill kernel is parity-green but not yet faster than the one-SM
+// kernel on the causal workload: plans do not choose it until it is.
+constexpr bool kPairPrefill = false;
+
 struct PrefillShape {
+  bool pair;         // pairs of SMs (prefill_pair.cu), else one SM per query tile
   int D;             // 64 or 128
   int qpt;           // query positions per 128-row tile (rows = qpt * g)
   int rows;          // qpt * g <= 128
@@ -169,6 +183,16 @@ struct PrefillArgs {
   int64_t causal_offset, window;
   float scale_log2;
 };
+
+// Mask pre-pass shared by both prefill kernels: per (batch, query tile, key
+// tile) 0 all hidden, 1 mixed, 2 all visible.
+int launch_mask_summary(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+
+// Pair prefill: tmk_half is K with 64-key boxes, tmv V with 128-key boxes.
+int pair_smem_bytes();
+int launch_prefill_pair(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
+                        const CUtensorMap& tmq, const CUtensorMap& tmk_half,
+                        const CUtensorMap& tmv, cudaStream_t stream);
 
 int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
                    const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,

@@ -201,26 +201,36 @@ GQA_API int gqa_device_status(void* workspace, size_t workspace_bytes, void* str
 #define GQA_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
 /*
- * gqa_forward_decode_noalloc -- the decode path (bf16, seq_q == 1) without a
+ * gqa_forward_decode_noalloc -- gqa_forward for the decode path without a
  * caller workspace.  The pages have no counterpart: this is a deployment
- * variant of gqa_forward for callers that cannot allocate device memory --
- * code that is only handed the q/k/v/out buffers by a host framework and has
- * no allocator of its own, or a steady-state loop that must not call
- * cudaMalloc because it can synchronise the device.
+ * variant for callers that cannot allocate device memory -- code that is only
+ * handed the q/k/v/out buffers by a host framework and has no allocator of its
+ * own, or a steady-state loop that must not call cudaMalloc because it can
+ * synchronise the device.
  *   p, q, k, v, mask, out, stream: as for gqa_forward (device pointers).
+ * Accepts what gqa_forward sends to the decode kernel (GQA_KERNEL_DECODE):
+ * bf16 or fp16, seq_q == 1 or (heads_q / heads_kv) * seq_q <= 16, with any of
+ * mask, causal_offset, window, kv_lens and a paged cache.  seq_k == 0 fills
+ * `out` with zeros and a problem in which no query sees a key fills it with
+ * NaN, as gqa_forward does.  Longer query blocks (GQA_KERNEL_PREFILL) and
+ * fp32 return GQA_ERR_UNSUPPORTED.
  * Scratch: a file-scope static device array of GQA_STATIC_SCRATCH_BYTES inside
- * the library.  The first call on each device looks up that array's device
- * address (cudaGetSymbolAddress, with the device current); make that first
- * call before any stream capture.  The call allocates nothing (no cudaMalloc,
- * no cudaFree, no allocating library routine).  Every call on a device
- * shares the one array: each call zeroes the part that must start at zero
- * (with cudaMemsetAsync on `stream`) and leaves the rest as the last call
- * left it, so calls that overlap on the GPU race -- order them on one stream.
- * Returns GQA_OK once enqueued; GQA_ERR_UNSUPPORTED for anything but the
- * decode path; GQA_ERR_SCRATCH_LIMIT when the problem's scratch (the
- * workspace_bytes gqa_query reports) exceeds GQA_STATIC_SCRATCH_BYTES; the
- * argument errors of gqa_forward otherwise.  A kernel wait that runs out is
- * recorded only in the static array and is not reported to the caller.
+ * the library.  The call looks up that array's device address on the current
+ * device (cudaGetSymbolAddress) and caches it; during a stream capture only
+ * the cached address is used, so make the first call on each device before
+ * any capture.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).  Every call on a device shares the one array:
+ * each call zeroes the part that must start at zero (with cudaMemsetAsync on
+ * `stream`) and leaves the rest as the last call left it, so calls that
+ * overlap on the GPU race -- order them on one stream.
+ * Returns GQA_OK once enqueued; GQA_ERR_UNSUPPORTED as above;
+ * GQA_ERR_SCRATCH_LIMIT when the problem's scratch (the workspace_bytes
+ * gqa_query reports) exceeds GQA_STATIC_SCRATCH_BYTES; the argument errors of
+ * gqa_forward otherwise.  Errors found by the kernel are NOT reported: a wait
+ * that runs out, a kv_lens entry outside [0, seq_k] (clamped) and a block-table
+ * entry outside [0, num_pages) (read as zeros) are recorded only in the static
+ * array, which the next call clears.  Use gqa_forward with gqa_device_status
+ * where those must be detected.
  */
 GQA_API int gqa_forward_decode_noalloc(const gqa_problem* p, const void* q, const void* k,
                                        const void* v, const uint8_t* mask, void* out,
@@ -288,6 +298,20 @@ GQA_API int gqa_kv_append(const gqa_kv_append_desc* d, void* cache_k, void* cach
  * negative size or GQA_ERR_LAYOUT for a misaligned buffer.
  */
 GQA_API int gqa_debug_decode_trace(void* device_buffer, int64_t bytes);
+
+/*
+ * gqa_debug_decode_withhold -- test of the kernels' bounded waits (failure
+ * detection without a GPU fault; the pages have no counterpart).  The NEXT
+ * decode launch of the process (gqa_forward or gqa_forward_decode_noalloc)
+ * uses `wait_limit_ns` (1000 .. 1e9) as the limit of every internal wait and,
+ * if `unit` >= 0, its producer never issues the copies of that 128-key unit
+ * (index in launch order) and issues nothing after it: the consumers' wait
+ * for the unit runs out, the CTA unwinds (every copy already issued lands
+ * first), the output is undefined and gqa_device_status then returns
+ * GQA_ERR_TIMEOUT and re-zeroes the workspace.  The setting is consumed by
+ * that one launch.  Returns GQA_OK or GQA_ERR_ARG.
+ */
+GQA_API int gqa_debug_decode_withhold(int64_t unit, int64_t wait_limit_ns);
 
 /* Static English description of a status code (never NULL). */
 GQA_API const char* gqa_status_string(int status);

@@ -58,3 +58,27 @@ def f16_inputs(seed, B, Hq, Hkv, Sq, Sk, D, device="cuda"):
     q, k, v = synth.qkv_f32(seed, B, Hq, Hkv, Sq, Sk, D)
     h = [x.astype(np.float16) for x in (q, k, v)]
     return tuple(x.astype(np.float64) for x in h), tuple(torch.from_numpy(x).to(device) for x in h)
+
+
+def oracle_rows_threaded(q, k, v, rows, mask=None, causal=False, threads=None):
+    """oracle.forward_rows over chunks of ``rows`` on several host threads
+    (the oracle's ctypes calls release the GIL); the per-row arithmetic is the
+    oracle's own, unchanged.  Returns [len(rows), D] float64 in row order."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    rows = list(rows)
+    n = max(1, min(threads or os.cpu_count() or 1, 64, len(rows)))
+    chunks = [rows[i::n] for i in range(n)]
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        parts = list(ex.map(lambda c: oracle.forward_rows(q, k, v, c, mask=mask, causal=causal),
+                            chunks))
+    out = np.empty((len(rows), q.shape[-1]))
+    for i, part in enumerate(parts):
+        out[i::n] = part
+    return out
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """x rounded to the nearest bf16 (ties to even), as float64."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).bfloat16()
+    return t.float().numpy().astype(np.float64)

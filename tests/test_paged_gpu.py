@@ -134,6 +134,29 @@ def test_paged_prefill_full_cache_non_causal(gqa):
     assert_bf16_parity(out, oracle.forward(q, kc, vc), "paged prefill, full cache")
 
 
+@pytest.mark.parametrize("Sq,causal", [(150, False), (150, True), (1, False), (3, True)])
+def test_paged_capacity_not_a_page_multiple(gqa, Sq, causal):
+    """A block table without lengths and seq_k = 600 (not a multiple of the
+    128-key page or tile): keys 600..639 of the last page hold NaN in the pool
+    and must not reach the result, causal (bottom-right) or not."""
+    B, Hq, Hkv, D, ps, per_seq, Sk = 2, 12, 2, 128, 128, 5, 600
+    lens = np.full(B, Sk, dtype=np.int32)
+    kc, vc, kd, vd, table = _paged(7100 + Sq, B, Hkv, D, ps, per_seq, lens, "bf16")
+    q, qd = _q(7100 + Sq, B, Hq, Sq, D, "bf16")
+    out = torch.empty_like(qd)
+    p = gqa.problem_for(qd, kd, vd, causal=causal, out=out,
+                        causal_offset=(Sk - Sq) if causal else None, block_table=table)
+    p.seq_k = Sk
+    plan = gqa.query_problem(p)
+    ws = gqa.workspace_for(qd.device, plan.workspace_bytes)
+    gqa.forward_ptrs(p, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), None, out.data_ptr(),
+                     ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert gqa.device_status() == 0
+    ref = oracle.forward(q, kc[:, :, :Sk], vc[:, :, :Sk], causal=causal,
+                         causal_offset=(Sk - Sq) if causal else None)
+    assert_bf16_parity(to_np(out), ref, "paged, seq_k %d, Sq %d, causal %s" % (Sk, Sq, causal))
+
+
 def test_paged_prefill_bad_page_is_reported(gqa):
     B, Hq, Hkv, Sq, D, ps, per_seq = 2, 8, 2, 64, 64, 64, 4
     lens = np.array([200, 150], dtype=np.int32)

@@ -6,7 +6,8 @@ import torch
 import oracle
 import synth
 
-from gpu_util import assert_bf16_parity, bf16_inputs, bits_to_dev, f64, oracle_bf16, to_np
+from gpu_util import (assert_bf16_parity, bf16_inputs, bf16_round, bits_to_dev, f64, oracle_bf16,
+                      oracle_rows_threaded, rel_rms, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -121,7 +122,10 @@ def test_prefill_fully_hidden_rows_are_nan(gqa):
 
 # ------------------------------------------------------------ full size
 
-def _sampled(gqa, seed, B, Hq, Hkv, S, D, causal, mask_lens, samples):
+def _full_size(gqa, seed, B, Hq, Hkv, S, D, causal, mask_lens, whole):
+    """One full-size workload: every output row of the (b, kv) group `whole`,
+    and from every other (b, kv) group one row of every query tile of the
+    kernel (qpt = 128 // g query positions per tile), against the oracle."""
     bits, (q, k, v) = bf16_inputs(seed, B, Hq, Hkv, S, S, D)
     mask = None
     if mask_lens:
@@ -132,33 +136,54 @@ def _sampled(gqa, seed, B, Hq, Hkv, S, D, causal, mask_lens, samples):
     _status_ok(gqa)
     qb, kb, vb = bits
     g = Hq // Hkv
-    got, ref = [], []
-    for (b, kv, rows) in samples:
-        qs = f64(qb[b:b + 1, kv * g:(kv + 1) * g])
-        ks = f64(kb[b:b + 1, kv:kv + 1])
-        vs = f64(vb[b:b + 1, kv:kv + 1])
-        ms = mask[b:b + 1] if mask is not None else None
-        r = oracle.forward_rows(qs, ks, vs, [(0, hh, i) for (hh, i) in rows], mask=ms,
-                                causal=causal)
-        ref.append(r)
-        got.append(np.stack([out[b, kv * g + hh, i] for (hh, i) in rows]))
+    qpt = 128 // g
+    m_tiles = -(-S // qpt)
+    got, ref, tiles_seen = [], [], set()
+    for b in range(B):
+        for kv in range(Hkv):
+            if (b, kv) == whole:
+                rows = [(hh, i) for hh in range(g) for i in range(S)]
+            else:
+                rows = []
+                for mt in range(m_tiles):
+                    hh = (mt + 3 * b + kv) % g
+                    i = min(S - 1, mt * qpt + (7 * mt + b + 5 * kv) % qpt)
+                    rows.append((hh, i))
+                    tiles_seen.add((b, kv, i // qpt))
+            qs = f64(qb[b:b + 1, kv * g:(kv + 1) * g])
+            ks, vs = f64(kb[b:b + 1, kv:kv + 1]), f64(vb[b:b + 1, kv:kv + 1])
+            ms = mask[b:b + 1] if mask is not None else None
+            ref.append(oracle_rows_threaded(qs, ks, vs, [(0, hh, i) for (hh, i) in rows],
+                                            mask=ms, causal=causal))
+            got.append(np.stack([out[b, kv * g + hh, i] for (hh, i) in rows]))
+    assert len(tiles_seen) == (B * Hkv - 1) * m_tiles
     return np.concatenate(got), np.concatenate(ref)
 
 
-def test_prefill_causal_full_size_sampled(gqa):
-    """B=4, Hq=32, Hkv=8, S=4096, D=128, causal: sampled rows of every kind of tile."""
-    rows = [(hh, i) for hh in range(4) for i in (0, 1, 31, 32, 127, 128, 2047, 2048, 4000, 4095)]
-    got, ref = _sampled(gqa, 4, 4, 32, 8, 4096, 128, True, False,
-                        [(0, 0, rows), (3, 7, rows), (2, 5, rows[::3])])
-    assert_bf16_parity(got, ref, "causal prefill full size")
+def _report(name, got, ref):
+    """The parity bar, plus the diagnostic split of the error: against the
+    unrounded oracle (what the bar checks) and against the oracle rounded to
+    bf16 (the error left once the output rounding is taken out)."""
+    max_abs, rr = assert_bf16_parity(got, ref, name)
+    rr_rounded = rel_rms(got, bf16_round(ref))
+    print("%s: rows %d, max_abs %.3e, rel_rms %.3e (vs oracle rounded to bf16: %.3e)"
+          % (name, got.shape[0], max_abs, rr, rr_rounded))
 
 
-def test_prefill_masked_full_size_sampled(gqa):
-    """B=8, Hq=12, Hkv=2, S=2048, D=64, padding mask len_b ~ U[256, 2048]."""
-    rows = [(hh, i) for hh in range(6) for i in (0, 20, 21, 1000, 2047)]
-    got, ref = _sampled(gqa, 5, 8, 12, 2, 2048, 64, False, True,
-                        [(0, 0, rows), (7, 1, rows), (4, 0, rows)])
-    assert_bf16_parity(got, ref, "masked prefill full size")
+def test_prefill_causal_full_size(gqa):
+    """B=4, Hq=32, Hkv=8, S=4096, D=128, causal: one whole (b, kv) group (4 heads
+    x 4096 rows) element by element, and a row of every query tile of every
+    other group."""
+    got, ref = _full_size(gqa, 4, 4, 32, 8, 4096, 128, True, False, whole=(1, 3))
+    _report("causal prefill full size", got, ref)
+
+
+def test_prefill_masked_full_size(gqa):
+    """B=8, Hq=12, Hkv=2, S=2048, D=64, padding mask len_b ~ U[256, 2048]: one
+    whole (b, kv) group (6 heads x 2048 rows) and a row of every query tile of
+    every other group."""
+    got, ref = _full_size(gqa, 5, 8, 12, 2, 2048, 64, False, True, whole=(5, 1))
+    _report("masked prefill full size", got, ref)
 
 
 # ----------------------------------------------- causal offset and sliding window
