@@ -81,12 +81,6 @@ static_assert(128 * kIoRegs + 256 * kSoftmaxRegs <= kPrefillThreads * kLaunchReg
               "register split must fit in the launch allocation");
 static_assert(kPrefillThreads == 12 * 32, "two softmax warpgroups and one producer / MMA warpgroup");
 constexpr uint32_t kTmemCols = 512;
-// Exponentials of every eight computed on the FMA pipe (exp2_poly) rather
-// than the MUFU unit; the rest use ex2.approx.
-#ifndef GQA_PREFILL_EXP_EMU
-#define GQA_PREFILL_EXP_EMU 0
-#endif
-constexpr int kEmuPerEight = GQA_PREFILL_EXP_EMU;
 
 // KVX: the launch has per-sequence lengths or a paged cache (two more
 // barriers, for the V rows past a length; without either the kernel is built
@@ -581,10 +575,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = c * 32 + 2 * e, c1 = c0 + 1;
-            const float x0 = fmaf(__uint_as_float(r[c0]), sc, -ref);
-            const float x1 = fmaf(__uint_as_float(r[c1]), sc, -ref);
-            const float p0 = ((c0 & 7) < kEmuPerEight) ? exp2_poly(x0) : fast_exp2(x0);
-            const float p1 = ((c1 & 7) < kEmuPerEight) ? exp2_poly(x1) : fast_exp2(x1);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[c0]), sc, -ref));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(r[c1]), sc, -ref));
             lp[c0 & 7] += p0;
             lp[c1 & 7] += p1;
             pk[e] = pack_p<F16>(p0, p1);
