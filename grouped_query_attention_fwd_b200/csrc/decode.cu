@@ -71,17 +71,22 @@ __host__ __device__ inline int cta_of_unit(int u, int T, int P) {
   return static_cast<int>(((static_cast<int64_t>(u) + 1) * P + T - 1) / T) - 1;
 }
 
+// Shared memory of one CTA: the K / V ring, one Q area per stage (one 8-row
+// column tile: a group's Q rows arrive with its first K tile), the flush
+// scratch, the barriers and flags, then (ragged launches) the B lengths and
+// B + 1 prefix sums.
 template <int D, int NT>
 struct DecodeSmem {
   static constexpr int kTileBytes = KT * D * 2;        // K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
   static constexpr int HP = 8 * NT;
+  static constexpr int kQRow = D * 2 + 16;             // bytes per Q row (padded: no bank conflicts)
+  static constexpr int kQAreaBytes = NT == 1 ? HP * kQRow : 0;
   static constexpr int kScrRow = D + 4;  // one row's O, then (m, l), padded (floats)
   static constexpr int kScrOBytes = kMergeWarps * HP * kScrRow * 4;
-  // Ragged launches keep the B lengths and B + 1 prefix sums after the flags.
   static int bytes(int stages, int ragged_batch) {
-    return 1024 /*alignment slack*/ + stages * kStageBytes + kScrOBytes + 3 * stages * 8 + 16 +
-           (ragged_batch > 0 ? ((8 * ragged_batch + 4 + 15) / 16) * 16 : 0);
+    return 1024 /*alignment slack*/ + stages * (kStageBytes + kQAreaBytes) + kScrOBytes +
+           3 * stages * 8 + 16 + (ragged_batch > 0 ? ((8 * ragged_batch + 4 + 15) / 16) * 16 : 0);
   }
 };
 
@@ -157,7 +162,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
-  float* scr_o = reinterpret_cast<float*>(ring + stages * L::kStageBytes);
+  uint8_t* qarea = ring + stages * L::kStageBytes;  // stage s: qarea + s * kQAreaBytes
+  float* scr_o = reinterpret_cast<float*>(qarea + stages * L::kQAreaBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scr_o) + L::kScrOBytes);
   uint64_t* full_v = full + stages;  // full: the stage's K tile landed; full_v: its V tile
   uint64_t* empty = full_v + stages;
@@ -197,6 +203,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     *peek_count = kNoPeek;
     fence_mbar_init();
   }
+  // Q areas: columns past head_dim and rows past the group stay zero.
+  for (int x = threadIdx.x; x < stages * L::kQAreaBytes / 16; x += blockDim.x)
+    reinterpret_cast<uint4*>(qarea)[x] = make_uint4(0u, 0u, 0u, 0u);
+  if (L::kQAreaBytes > 0) fence_proxy_async_smem();  // before the bulk copies into it
   // Everything above touches shared memory only; from here on global memory
   // written by earlier work on the stream (lengths, caches, counters) is read.
   griddep_wait();
@@ -306,6 +316,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int kv = gi / passes;
         const int b = cu.b;
         uint8_t* st = ring + s * L::kStageBytes;
+        // The first tile of a group in this range brings the group's Q rows
+        // (one 8-row column tile) into the stage's Q area, on the same
+        // barrier: the consumers then start the group without a global load.
+        const bool q_rows = L::kQAreaBytes > 0 && (u == u_begin || r - gi * cu.kr.tiles == 0);
+        const int pass = gi % passes;
+        const int nq = q_rows ? min(HP, a.rows - pass * HP) : 0;
+        const uint32_t q_bytes = static_cast<uint32_t>(nq * a.Dv * 2);
+        auto issue_q = [&]() {
+          uint8_t* qd = qarea + s * L::kQAreaBytes;
+          for (int hr = 0; hr < nq; ++hr) {
+            const int hl = pass * HP + hr;
+            const int hh = MQ ? hl / a.Sq : hl;
+            const int qi = MQ ? hl % a.Sq : 0;
+            const uint16_t* src = a.q + b * a.qs[0] + static_cast<int64_t>(kv * a.g + hh) * a.qs[1] +
+                                  static_cast<int64_t>(qi) * a.qs[2];
+            bulk_load(qd + hr * L::kQRow, src, static_cast<uint32_t>(a.Dv * 2), &full[s]);
+          }
+        };
         if (paged) {
           int page[2], prow[2];
 #pragma unroll
@@ -318,7 +346,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
           }
           if (u + 1 < u_end) fetch_pages(u + 1);
-          mbar_arrive_expect_tx(&full[s], L::kTileBytes);
+          mbar_arrive_expect_tx(&full[s], L::kTileBytes + q_bytes);
+          issue_q();
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -335,10 +364,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           if (a.trace != nullptr && it == 0) trace()[kTrFirstIssue] = globaltimer_ns();
           continue;
         }
-        mbar_arrive_expect_tx(&full[s], L::kTileBytes);
+        mbar_arrive_expect_tx(&full[s], L::kTileBytes + q_bytes);
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c)
           tma_load_4d(st + c * CHUNK_BYTES, &tmk, &full[s], c * 64, key0, kv, b);
+        issue_q();
         if (a.trace != nullptr && it == 0) trace()[kTrFirstIssue] = globaltimer_ns();
         mbar_arrive_expect_tx(&full_v[s], L::kTileBytes);
 #pragma unroll
@@ -380,12 +410,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // Q as MMA B fragments: in registers for one column tile; for two, in
+    // Q as MMA B fragments: for one column tile, in registers, read from the
+    // Q area of the stage that brought the group's first tile; for two, in
     // shared memory (head rows padded to D * 2 + 16 bytes, conflict-free for
     // ldmatrix), aliasing the flush scratch, to stay within the registers
     // that 288 threads may hold.
     constexpr bool kQSmem = NT == 2;
-    constexpr int kQRow = D * 2 + 16;
+    constexpr int kQRow = L::kQRow;
     static_assert(!kQSmem || HP * kQRow <= L::kScrOBytes, "Q rows must fit the scratch");
     uint32_t bq[kQSmem ? 1 : NT][kQSmem ? 1 : KSTEPS][2];
     uint8_t* q_smem = reinterpret_cast<uint8_t*>(scr_o);
@@ -398,6 +429,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     int b = 0, kv = 0, pass = 0;
     const uint8_t* mrow = nullptr;
     const int first_grp = u_begin < u_end ? group_of(u_begin, sc, a) : -1;
+    bool q_pending = false;  // the group's Q fragments come with its first stage
 
     auto reset_state = [&]() {
 #pragma unroll
@@ -437,19 +469,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        if (!kQSmem) {
-          const int hl = pass * HP + nt * 8 + (lane >> 2);  // row within the group
-          const bool ok = hl < a.rows;
-          const uint16_t* qrow = q_row(ok ? hl : 0);
-#pragma unroll
-          for (int ks = 0; ks < KSTEPS; ++ks) {
-            const int d0 = ks * 16 + (lane & 3) * 2;
-            bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][0] =
-                (ok && d0 < a.Dv) ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
-            bq[kQSmem ? 0 : nt][kQSmem ? 0 : ks][1] =
-                (ok && d0 + 8 < a.Dv) ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
-          }
-        }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           if (MQ) {
@@ -469,6 +488,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             vhi[nt][e] = cur_hi;
             vmask[nt][e] = mrow;
           }
+        }
+      }
+    };
+
+    // One column tile: the group's B fragments from the Q area of stage st
+    // (rows past the group and columns past head_dim are zero there).
+    auto load_q_stage = [&](int st) {
+      if (!kQSmem) {
+        const uint8_t* qrow = qarea + st * L::kQAreaBytes + (lane >> 2) * kQRow;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int d0 = ks * 16 + (lane & 3) * 2;
+          bq[0][kQSmem ? 0 : ks][0] = *reinterpret_cast<const uint32_t*>(qrow + d0 * 2);
+          bq[0][kQSmem ? 0 : ks][1] = *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2);
         }
       }
     };
@@ -852,6 +885,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         mrow = a.mask ? a.mask + b * a.ms[0] : nullptr;
         load_q();
         reset_state();
+        q_pending = true;
       }
       const int s = it % stages;
       const uint32_t round = static_cast<uint32_t>(it / stages);
@@ -864,6 +898,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         continue;
       }
       if (a.trace != nullptr && it == 0 && threadIdx.x == 0) trace()[kTrFirstLand] = globaltimer_ns();
+      if (q_pending) {
+        load_q_stage(s);
+        q_pending = false;
+      }
       const uint32_t kbase = smem_u32(ring + s * L::kStageBytes);
       const uint32_t vbase = kbase + L::kTileBytes;
 
