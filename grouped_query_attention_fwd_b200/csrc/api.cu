@@ -411,6 +411,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.Dv = static_cast<int>(p.head_dim);
   a.scale_log2 = scale_log2;
   if (s.pair) return launch_prefill_pair(p, s, a, tmq, tmk, tmv, stream);
+  if (s.pp) return launch_prefill_pp(p, s, a, tmq, tmk, tmv, stream);
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
 }
 

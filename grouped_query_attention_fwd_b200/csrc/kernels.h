@@ -154,8 +154,13 @@ constexpr int kMaxPairTiles = 256;
 // kernel on the causal workload: plans do not choose it until it is.
 constexpr bool kPairPrefill = false;
 
+// Key tiles a work item of the two-tile prefill kernel may span (Sk <= 131072).
+constexpr int kMaxPPTiles = 1024;
+constexpr bool kPPPrefill = true;
+
 struct PrefillShape {
-  bool pair;         // pairs of SMs (prefill_pair.cu), else one SM per query tile
+  bool pair;         // pairs of SMs (prefill_pair.cu)
+  bool pp;           // two query tiles per SM (prefill_pp.cu); else one query tile per SM
   int D;             // 64 or 128
   int qpt;           // query positions per 128-row tile (rows = qpt * g)
   int rows;          // qpt * g <= 128
@@ -193,6 +198,12 @@ int pair_smem_bytes();
 int launch_prefill_pair(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
                         const CUtensorMap& tmq, const CUtensorMap& tmk_half,
                         const CUtensorMap& tmv, cudaStream_t stream);
+
+// Two query tiles per SM: K and V with 128-key boxes, as for the one-tile kernel.
+int pp_smem_bytes(int D);
+int launch_prefill_pp(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
+                      const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                      cudaStream_t stream);
 
 int launch_prefill(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
                    const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,

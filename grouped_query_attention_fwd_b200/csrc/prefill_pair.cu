@@ -50,8 +50,7 @@ constexpr int kPairThreads = 12 * 32;
 constexpr int kWarpQK = 8;   // TMA producer of Q tiles and K halves
 constexpr int kWarpMMA = 9;  // TMEM allocation; the leader's MMA issuer
 constexpr int kWarpV = 10;   // TMA producer of V halves (warp 11 idles)
-constexpr int kKStages = 4;
-constexpr int kVStages = 4;
+constexpr int kStages = 4;  // K and V stages (a K half and a V half per key tile)
 constexpr int kLaunchRegs = 168;
 constexpr int kIoRegs = 120;
 constexpr int kSoftmaxRegs = 192;
@@ -71,13 +70,14 @@ struct PairLayout {
   static constexpr int kVHalf = BN * 128;               // 128 keys x this CTA's 64 columns
   static constexpr int kQOff = 0;                       // Q_A, then Q_B
   static constexpr int kKOff = kQOff + 2 * kQTile;
-  static constexpr int kVOff = kKOff + kKStages * kKHalf;
-  static constexpr int kBarOff = kVOff + kVStages * kVHalf;
-  // q_full[2], q_empty[2], k_full, k_empty, v_full, v_empty, s_full[2],
-  // p_full[2], o_ready[2], o_final[2], o_free[2], mma_done
-  static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 10 + 1;
+  static constexpr int kVOff = kKOff + kStages * kKHalf;
+  static constexpr int kBarOff = kVOff + kStages * kVHalf;
+  // q_full[2], q_empty[2], k_full[S], v_full[S], kv_empty[S], s_full[2],
+  // p_full[2], o_final[2], o_free[2], mma_done
+  static constexpr int kNumBars = 4 + 3 * kStages + 8 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  static constexpr int kSchedOff = kMiscOff + 16;  // the MMA thread's key-tile list of an item
+  static constexpr int kBytes = kSchedOff + kMaxPairTiles + 1024;  // + alignment slack
   // TMEM columns of S_X and O_X (X = 0: tile A, 1: tile B).
   __device__ static constexpr uint32_t s_col(int X) { return static_cast<uint32_t>(X) * 128u; }
   __device__ static constexpr uint32_t o_col(int X) { return 256u + static_cast<uint32_t>(X) * 128u; }
@@ -163,16 +163,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* q_full = bars;                  // [X] leader: both CTAs' Q_X landed
   uint64_t* q_empty = q_full + 2;           // [X] every CTA: the item's QK_X done
   uint64_t* k_full = q_empty + 2;           // [stage] leader: both K halves landed
-  uint64_t* k_empty = k_full + kKStages;    // [stage] every CTA: the QKs reading it done
-  uint64_t* v_full = k_empty + kKStages;    // [stage] leader: both V halves landed
-  uint64_t* v_empty = v_full + kVStages;    // [stage] every CTA: the PVs reading it done
-  uint64_t* s_full = v_empty + kVStages;    // [X] every CTA: QK_X done
-  uint64_t* p_full = s_full + 2;            // [X] leader: P_X written (8 warps, both CTAs)
-  uint64_t* o_ready = p_full + 2;           // [X] every CTA: PV_X done
-  uint64_t* o_final = o_ready + 2;          // [X] every CTA: the item's last PV_X done
+  uint64_t* v_full = k_full + kStages;      // [stage] leader: both V halves landed
+  uint64_t* kv_empty = v_full + kStages;    // [stage] every CTA: the products reading it done
+  // S_X done.  The commit follows QK_X, which follows the previous PV_X from
+  // the same thread, so it also means that PV_X has completed: the softmax
+  // may rescale O_X once it has seen S_X.
+  uint64_t* s_full = kv_empty + kStages;    // [X] every CTA
+  uint64_t* p_full = s_full + 2;            // [X] leader: P_X written (one arrival per CTA)
+  uint64_t* o_final = p_full + 2;           // [X] every CTA: the item's last PV_X done
   uint64_t* o_free = o_final + 2;           // [X] leader: O_X read by both epilogues
   uint64_t* mma_done = o_free + 2;          // leader: every MMA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  uint8_t* sched = smem + L::kSchedOff;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5;
@@ -189,18 +191,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);   // four warps of each CTA
-      mbar_init(&o_ready[i], 1);
+      mbar_init(&p_full[i], 2);   // one arrival per CTA
       mbar_init(&o_final[i], 1);
-      mbar_init(&o_free[i], 8);
+      mbar_init(&o_free[i], 2);
     }
-    for (int i = 0; i < kKStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-    }
-    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -234,8 +232,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const bool is_qk = warp == kWarpQK;
       const CUtensorMap* map = is_qk ? &tmk : &tmv;
       uint64_t* full = is_qk ? k_full : v_full;
-      uint64_t* empty = is_qk ? k_empty : v_empty;
-      const int stages = is_qk ? kKStages : kVStages;
+      uint64_t* empty = kv_empty;
+      const int stages = kStages;
       const uint32_t bytes = is_qk ? L::kKHalf : L::kVHalf;
       uint8_t* ring = smem + (is_qk ? L::kKOff : L::kVOff);
       prefetch_tmap(map);
@@ -298,13 +296,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t dq0 = kmajor_desc(smem_u32(smem + L::kQOff));
       const uint64_t dk0 = kmajor_desc(smem_u32(smem + L::kKOff));
       const uint64_t dv0 = mnmajor_desc(smem_u32(smem + L::kVOff), L::kVHalf);
-      uint32_t kt = 0, vt = 0;       // K / V tiles consumed over the kernel
+      uint32_t kt = 0;               // key tiles (K / V stages) consumed over the kernel
       uint32_t np[2] = {0, 0};       // P_X tiles consumed over the kernel
       int64_t it = 0;
       bool ok = true;
-      auto qk = [&](int X, uint32_t ks_idx) {
+      auto qk = [&](int X, uint32_t idx) {
         const uint64_t dq = dq0 + ((X * L::kQTile) >> 4);
-        const uint64_t dk = dk0 + (((ks_idx % kKStages) * L::kKHalf) >> 4);
+        const uint64_t dk = dk0 + (((idx % kStages) * L::kKHalf) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           tc_mma_ss_pair(tmem + L::s_col(X), dq + (((k >> 2) * L::kQChunk + (k & 3) * 32) >> 4),
@@ -312,41 +310,29 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                          k > 0 ? 1u : 0u);
         tc_commit_pair_mc(&s_full[X], kBothCtas);
       };
-      auto pv = [&](int X, uint32_t vs_idx, bool first) {
-        const uint64_t dv = dv0 + (((vs_idx % kVStages) * L::kVHalf) >> 4);
+      auto pv = [&](int X, uint32_t idx, bool first) {
+        const uint64_t dv = dv0 + (((idx % kStages) * L::kVHalf) >> 4);
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
           tc_mma_ts_pair(tmem + L::o_col(X), tmem + L::s_col(X) + k * 8,
                          dv + ((k * 16 * 128) >> 4), idesc_pv, (!first || k > 0) ? 1u : 0u);
-        tc_commit_pair_mc(&o_ready[X], kBothCtas);
       };
       for (int64_t x = snake(0, pair, npairs); x < items && ok; ++it, x = snake(it, pair, npairs)) {
         const ItemGeom g = item_geom(x, a, m_tiles, qpt, n_tiles);
-        // Key tiles the pair computes for A and for B, as bit sets relative
-        // to t_lo (tile classes read mask summaries from global memory: they
-        // are taken once per item, off the per-tile path).
-        uint32_t bits[2][kMaxPairTiles / 32];
-        int nX[2] = {0, 0};
-        for (int w = 0; w < kMaxPairTiles / 32; ++w) bits[0][w] = bits[1][w] = 0u;
-        for (int t = g.t_lo; t < g.t_hi; ++t)
-          for (int X = 0; X < 2; ++X)
-            if (pair_does(g, X, t, a, m_tiles, n_tiles)) {
-              bits[X][(t - g.t_lo) >> 5] |= 1u << ((t - g.t_lo) & 31);
-              ++nX[X];
-            }
-        auto does = [&](int X, int t) {
-          return ((bits[X][(t - g.t_lo) >> 5] >> ((t - g.t_lo) & 31)) & 1u) != 0u;
-        };
-        // The next tile at or after t that some tile computes (t_hi if none).
-        auto next_tile = [&](int t) {
-          for (; t < g.t_hi; ++t) {
-            const int w = (t - g.t_lo) >> 5, sh = (t - g.t_lo) & 31;
-            const uint32_t m = (bits[0][w] | bits[1][w]) >> sh;
-            if (m != 0u) return t + __ffs(m) - 1;
-            t += 31 - sh;  // to the end of this word
+        // The item's key tiles that some tile works on, in order, as one byte
+        // each in shared memory (bit X: tile X computes it); tile classes read
+        // mask summaries from global memory, so they are taken here once per
+        // item, off the per-tile path.
+        int n = 0, nX[2] = {0, 0};
+        for (int t = g.t_lo; t < g.t_hi; ++t) {
+          const uint32_t f = (pair_does(g, 0, t, a, m_tiles, n_tiles) ? 1u : 0u) |
+                             (pair_does(g, 1, t, a, m_tiles, n_tiles) ? 2u : 0u);
+          if (f != 0u) {
+            sched[n++] = static_cast<uint8_t>(f);
+            nX[0] += f & 1u;
+            nX[1] += f >> 1;
           }
-          return g.t_hi;
-        };
+        }
         for (int X = 0; X < 2 && ok; ++X)
           ok = mbar_wait_hot(&q_full[X], static_cast<uint32_t>(it & 1), abort_flag, a.err,
                              kErrPrefillWait);
@@ -354,61 +340,57 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         int qkX[2] = {0, 0};  // QK_X / PV_X issued for this item
         int pvX[2] = {0, 0};
-        int t = next_tile(g.t_lo);
-        if (t < g.t_hi) {  // the first key tile: its QKs
-          ok = mbar_wait_hot(&k_full[kt % kKStages], (kt / kKStages) & 1u, abort_flag, a.err,
+        if (n > 0) {  // the first key tile: its QKs
+          ok = mbar_wait_hot(&k_full[kt % kStages], (kt / kStages) & 1u, abort_flag, a.err,
                              kErrPrefillWait);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t f = sched[0];
           for (int X = 0; X < 2; ++X)
-            if (does(X, t)) {
+            if ((f >> X) & 1u) {
               qk(X, kt);
               if (++qkX[X] == nX[X]) tc_commit_pair_mc(&q_empty[X], kBothCtas);
             }
-          tc_commit_pair_mc(&k_empty[kt % kKStages], kBothCtas);
-          ++kt;
         }
-        while (t < g.t_hi && ok) {
-          // Per key tile: PV_A(t), QK_A(tn), PV_B(t), QK_B(tn).
-          const int tn = next_tile(t + 1);
-          ok = mbar_wait_hot(&v_full[vt % kVStages], (vt / kVStages) & 1u, abort_flag, a.err,
+        for (int i = 0; i < n && ok; ++i) {
+          // Per key tile: PV_A(i), QK_A(i+1), PV_B(i), QK_B(i+1).
+          const uint32_t f = sched[i];
+          const uint32_t fn = i + 1 < n ? sched[i + 1] : 0u;
+          const uint32_t cur = kt + static_cast<uint32_t>(i), nxt = cur + 1;
+          ok = mbar_wait_hot(&v_full[cur % kStages], (cur / kStages) & 1u, abort_flag, a.err,
                              kErrPrefillWait);
           if (!ok) break;
-          bool k_ready = false;  // K(tn) waited for, right before its first QK
+          bool k_ready = false;  // K(i+1) waited for, right before its first QK
           for (int X = 0; X < 2 && ok; ++X) {
-            if (does(X, t)) {
+            if ((f >> X) & 1u) {
               ok = mbar_wait_cluster(&p_full[X], np[X] & 1u, abort_flag, a.err, kErrPrefillWait);
               if (ok && pvX[X] == 0 && it > 0)  // O_X still holds the last item's result
                 ok = mbar_wait_cluster(&o_free[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
                                        a.err, kErrPrefillWait);
               if (!ok) break;
               tc_fence_after();
-              pv(X, vt, pvX[X] == 0);
+              pv(X, cur, pvX[X] == 0);
               ++np[X];
               if (++pvX[X] == nX[X]) tc_commit_pair_mc(&o_final[X], kBothCtas);
             }
-            if (tn < g.t_hi && does(X, tn)) {
+            if ((fn >> X) & 1u) {
               if (!k_ready) {
-                ok = mbar_wait_hot(&k_full[kt % kKStages], (kt / kKStages) & 1u, abort_flag,
+                ok = mbar_wait_hot(&k_full[nxt % kStages], (nxt / kStages) & 1u, abort_flag,
                                    a.err, kErrPrefillWait);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
               }
-              qk(X, kt);
+              qk(X, nxt);
               if (++qkX[X] == nX[X]) tc_commit_pair_mc(&q_empty[X], kBothCtas);
             }
           }
           if (!ok) break;
-          tc_commit_pair_mc(&v_empty[vt % kVStages], kBothCtas);
-          ++vt;
-          if (tn < g.t_hi) {
-            tc_commit_pair_mc(&k_empty[kt % kKStages], kBothCtas);
-            ++kt;
-          }
-          t = tn;
+          // Stage i is free once its PVs (and the QKs issued before them) are done.
+          tc_commit_pair_mc(&kv_empty[cur % kStages], kBothCtas);
         }
         if (!ok) break;
+        kt += static_cast<uint32_t>(n);
         // A tile of the item that sees no key at all: release Q_X and let the
         // epilogue run (it writes NaN rows) once the last item's O_X is read.
         for (int X = 0; X < 2 && ok; ++X)
@@ -453,11 +435,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int t = g.t_lo; t < g.t_hi && ok; ++t) {
         if (!pair_does(g, X, t, a, m_tiles, n_tiles)) continue;
         const int cls = cls_of(g, X, static_cast<int>(rank), t, a, m_tiles, n_tiles);
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_hot(&s_full[X], J & 1u, abort_flag, a.err, kErrPrefillWait));
-        if (!ok) break;
-        tc_fence_after();
-        if (cls == 0) {
+        // okt: warp-uniform, so that every TMEM access it guards is made by
+        // the whole warp; the warpgroup meets once per tile below and leaves
+        // the loop together.
+        bool okt = __all_sync(0xffffffffu, mbar_wait_hot(&s_full[X], J & 1u, abort_flag, a.err,
+                                                         kErrPrefillWait));
+        if (!okt) {
+        } else if (cls == 0) {
+          tc_fence_after();
           // No row of this CTA's tile sees the tile: P = 0 for the pair's PV.
           uint32_t z[16];
 #pragma unroll
@@ -465,6 +450,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_st16(s_col + c * 16, z);
         } else {
+          tc_fence_after();
           uint32_t r[BN];
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -496,22 +482,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.f;
           const bool o_live = grow && nloc > 0 && m_ref != -INFINITY;
           if (__any_sync(0xffffffffu, o_live)) {
-            // O_X holds the earlier tiles' P V with the old reference:
-            // rescale it once the previous PV_X has completed.
-            ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[X], (J - 1) & 1u, abort_flag, a.err,
-                                                   kErrPrefillWait));
-            if (!ok) break;
-            tc_fence_after();
-            const float f = o_live ? alpha : 1.f;
+            // O_X holds the earlier tiles' P V with the old reference; the
+            // previous PV_X has completed (S_X follows it): rescale it.
+            {
+              const float f = o_live ? alpha : 1.f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(o_col + c * 32, o);
-              tmem_ld_wait();
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(o_col + c * 32, o);
+                tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-              tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-              tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+                tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+              }
             }
           }
           if (grow) {
@@ -541,30 +525,40 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(p_full_at);
+        // The four warps of the warpgroup have written P_X (or given up):
+        // one arrival per CTA on the leader's barrier.
+        if (!bar_and(1 + X, 128, okt)) {
+          ok = false;
+          break;
+        }
+        if ((threadIdx.x & 127) == 0) mbar_arrive_cluster(p_full_at);
         ++J;
         ++nloc;
       }
       if (!ok) break;
       // Epilogue: out = O / l for this row.
-      ok = __all_sync(0xffffffffu, mbar_wait_hot(&o_final[X], static_cast<uint32_t>(it & 1),
-                                                 abort_flag, a.err, kErrPrefillWait));
-      if (!ok) break;
-      tc_fence_after();
+      bool oke = __all_sync(0xffffffffu, mbar_wait_hot(&o_final[X], static_cast<uint32_t>(it & 1),
+                                                       abort_flag, a.err, kErrPrefillWait));
+      if (oke) tc_fence_after();
       uint16_t* orow = a.out + pr.b * a.os[0] +
                        static_cast<int64_t>(pr.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
                        static_cast<int64_t>(q) * a.os[2];
       const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
       if (nloc > 0) {
+        // (After a failed wait the values read are discarded: the output of
+        // an aborted launch is undefined.)
         uint32_t r[D];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c)
           tmem_ld32(o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
         tmem_ld_wait();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(o_free_at);  // the next item's first PV_X may start
+        if (!bar_and(1 + X, 128, oke)) {
+          ok = false;
+          break;
+        }
+        // O_X is in registers: the next item's first PV_X may overwrite it.
+        if ((threadIdx.x & 127) == 0) mbar_arrive_cluster(o_free_at);
         if (row_valid) {
 #pragma unroll
           for (int v8 = 0; v8 < D / 8; ++v8) {
@@ -589,8 +583,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
         }
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(o_free_at);
+        if (!bar_and(1 + X, 128, oke)) {
+          ok = false;
+          break;
+        }
+        if ((threadIdx.x & 127) == 0) mbar_arrive_cluster(o_free_at);
       }
     }
   }

@@ -1,0 +1,602 @@
+// Prefill with two query tiles in flight per SM.
+//
+// The g query heads of a kv head are packed into 128-row tiles as in the
+// other prefill kernel (row r: head h0 + r / qpt, query q0 + r % qpt), and
+// one K / V tile serves every head of the group ("Multi-Query Attention",
+// "Implementation": the shared K/V head is read once; the expanded K/V of
+// "28. Grouped-Query Attention (GQA)", "Reference solution", never exists).
+//
+// A work item is two consecutive query tiles A = 2i and B = 2i + 1 of one
+// (batch, kv head).  TMEM holds S_A, S_B (128 columns each) and O_A, O_B (D
+// each); Q_A and Q_B stay in shared memory:
+//
+//   S_X = Q_X K^T    tcgen05.mma, A = Q_X and B = K from shared memory
+//   O_X += P_X V     tcgen05.mma, A = P_X from TMEM (over the first half of
+//                    S_X), B = V from shared memory
+//
+// One softmax warpgroup per query tile, one thread per row holding all 128
+// keys of its S row: the maximum and the row sum need no exchange between
+// threads, and while warpgroup A turns S_A into P_A the tensor core computes
+// tile B's products, and the other way round.  The MMA thread issues, per
+// key tile u:  PV_A(u), QK_A(u+1), PV_B(u), QK_B(u+1).  tcgen05 operations of
+// one thread execute in issue order, so QK_X(u+1), which overwrites P_X(u),
+// follows PV_X(u), and the commit that signals S_X(u+1) also means that
+// PV_X(u) has completed: the softmax may rescale O_X as soon as it sees S_X.
+// Each K / V tile is staged once for both query tiles.
+//
+// Warp roles (384 threads, one CTA per SM, persistent over items):
+//   warps 0-3  softmax, O rescale and epilogue of tile A (thread t: row t)
+//   warps 4-7  the same for tile B
+//   warp 8     TMA producer of Q tiles and K tiles
+//   warp 9     TMEM allocator and single-thread MMA issuer
+//   warp 10    TMA producer of V tiles (warp 11 idles)
+// Every wait is bounded; a thread that gives up sets the abort flag and the
+// error word, every role leaves its loop, copies in flight are waited for and
+// TMEM is freed after a block-wide barrier.
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "prefill_common.cuh"
+#include "ptx.cuh"
+
+namespace gqa {
+namespace {
+
+using namespace prefill;
+
+constexpr int kPPThreads = 12 * 32;
+constexpr int kWarpQK = 8;
+constexpr int kWarpMMA = 9;
+constexpr int kWarpV = 10;
+// Register split (setmaxnreg): the softmax threads keep a whole S row (128
+// values) in registers.
+constexpr int kLaunchRegs = 168;
+constexpr int kIoRegs = 120;
+constexpr int kSoftmaxRegs = 192;
+static_assert(128 * kIoRegs + 256 * kSoftmaxRegs <= kPPThreads * kLaunchRegs,
+              "register split must fit in the launch allocation");
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct PPLayout {
+  static_assert(D == 64 || D == 128, "head_dim is padded to 64 or 128");
+  static constexpr int CH = D / 64;                  // 64-column (128-byte) chunks
+  static constexpr int kChunk = 128 * 128;           // 128 rows (or keys) x 128 bytes
+  static constexpr int kTile = CH * kChunk;          // one Q, K or V tile
+  static constexpr int kStages = D == 128 ? 2 : 4;   // depth of the K ring and of the V ring
+  static constexpr int kQOff = 0;                    // Q_A, then Q_B
+  static constexpr int kKOff = kQOff + 2 * kTile;
+  static constexpr int kVOff = kKOff + kStages * kTile;
+  static constexpr int kBarOff = kVOff + kStages * kTile;
+  // q_full[2], q_empty[2], k_full[S], k_empty[S], v_full[S], v_empty[S],
+  // s_full[2], p_full[2], o_final[2], o_free[2], mma_done
+  static constexpr int kNumBars = 4 + 4 * kStages + 8 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSchedOff = kMiscOff + 16;  // the MMA thread's key-tile list of an item
+  static constexpr int kBytes = kSchedOff + kMaxPPTiles + 1024;  // + alignment slack
+  // TMEM columns of S_X and O_X (X = 0: tile A, 1: tile B).
+  __device__ static constexpr uint32_t s_col(int X) { return static_cast<uint32_t>(X) * 128u; }
+  __device__ static constexpr uint32_t o_col(int X) {
+    return 256u + static_cast<uint32_t>(X) * static_cast<uint32_t>(D);
+  }
+};
+
+// Query tile X of item x (late, long causal items first), with its key
+// range; a tile index past the last query tile gives a dead tile (no keys).
+struct PPTile {
+  Pair pr;
+  Slot sl;
+};
+
+__device__ __forceinline__ PPTile pp_tile(int64_t x, int X, const PrefillArgs& a, int m_tiles,
+                                          int qpt, int n_tiles) {
+  PPTile t;
+  const int64_t bh = static_cast<int64_t>(a.B) * a.Hkv;
+  const int n2 = (m_tiles + 1) / 2;
+  const int bk = static_cast<int>(x % bh);
+  const int mt = 2 * (n2 - 1 - static_cast<int>(x / bh)) + X;
+  t.pr.b = bk / a.Hkv;
+  t.pr.kv = bk % a.Hkv;
+  t.pr.mt0 = mt;
+  t.pr.len = a.Sk;
+  t.sl = slot_of(t.pr, a, qpt);
+  t.sl.live = mt < m_tiles;
+  if (!t.sl.live || t.sl.key_hi <= t.sl.key_lo) {
+    t.pr.nt_beg = t.pr.nt_end = 0;
+  } else {
+    t.pr.nt_beg = static_cast<int>(t.sl.key_lo / BN);
+    t.pr.nt_end = min(n_tiles, static_cast<int>((t.sl.key_hi + BN - 1) / BN));
+  }
+  return t;
+}
+
+// Class of key tile u for a query tile: 0 skipped, 1 mixed, 2 fully visible.
+__device__ __forceinline__ int pp_class(const PPTile& q, int u, const PrefillArgs& a, int m_tiles,
+                                        int n_tiles) {
+  if (u < q.pr.nt_beg || u >= q.pr.nt_end) return 0;
+  return tile_class(a, q.pr, q.sl, u, m_tiles, n_tiles);
+}
+
+template <int D, bool F16>
+__global__ void __launch_bounds__(kPPThreads, 1)
+    gqa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmq,
+                          const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv, const PrefillArgs a,
+                          const int qpt, const int rows, const int m_tiles, const int n_tiles,
+                          const int64_t items) {
+  using L = PPLayout<D>;
+  constexpr int CH = L::CH;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars;              // [X] Q_X landed
+  uint64_t* q_empty = q_full + 2;       // [X] the item's last QK_X done
+  uint64_t* k_full = q_empty + 2;       // [stage] K tile landed
+  uint64_t* k_empty = k_full + S;       // [stage] the QKs reading it done
+  uint64_t* v_full = k_empty + S;       // [stage] V tile landed
+  uint64_t* v_empty = v_full + S;       // [stage] the PVs reading it done
+  uint64_t* s_full = v_empty + S;       // [X] S_X done (and every earlier PV_X)
+  uint64_t* p_full = s_full + 2;        // [X] P_X written (one arrival per warpgroup)
+  uint64_t* o_final = p_full + 2;       // [X] the item's last PV_X done
+  uint64_t* o_free = o_final + 2;       // [X] O_X read by the epilogue
+  uint64_t* mma_done = o_free + 2;      // every MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  uint8_t* sched = smem + L::kSchedOff;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 1);
+      mbar_init(&o_final[i], 1);
+      mbar_init(&o_free[i], 1);
+    }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // Q rows past qpt * g of a tile are never written by TMA: zero them once.
+  if (rows < BM && threadIdx.x < 8) {
+    for (int X = 0; X < 2; ++X)
+      for (int c = 0; c < CH; ++c) {
+        uint8_t* base = smem + L::kQOff + X * L::kTile + c * L::kChunk;
+        for (int r = rows; r < BM; ++r)
+          reinterpret_cast<uint4*>(base + r * 128)[threadIdx.x] = make_uint4(0, 0, 0, 0);
+      }
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIoRegs));
+    if ((warp == kWarpQK || warp == kWarpV) && lane == 0) {
+      // ------------------------------------------------------------ producers
+      const bool is_qk = warp == kWarpQK;
+      const CUtensorMap* map = is_qk ? &tmk : &tmv;
+      uint64_t* full = is_qk ? k_full : v_full;
+      uint64_t* empty = is_qk ? k_empty : v_empty;
+      uint8_t* ring = smem + (is_qk ? L::kKOff : L::kVOff);
+      prefetch_tmap(map);
+      if (is_qk) prefetch_tmap(&tmq);
+      uint32_t kt = 0;         // key tiles loaded over the kernel
+      uint32_t nq[2] = {0, 0};  // Q tiles loaded into each buffer
+      int64_t it = 0;
+      bool ok = true;
+      for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
+           ++it, x = snake(it, blockIdx.x, gridDim.x)) {
+        const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
+        const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
+        if (is_qk) {
+#pragma unroll
+          for (int X = 0; X < 2; ++X) {
+            if (it > 0 && !mbar_wait(&q_empty[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
+                                     a.err, kErrPrefillWait)) {
+              ok = false;
+              break;
+            }
+            const Pair& pr = X == 0 ? qa.pr : qb.pr;
+            mbar_arrive_expect_tx(&q_full[X], static_cast<uint32_t>(rows * 128 * CH));
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(smem + L::kQOff + X * L::kTile + c * L::kChunk, &tmq, &q_full[X], c * 64,
+                          pr.mt0 * qpt, pr.kv * a.g, pr.b);
+            ++nq[X];
+          }
+        }
+        const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
+                             qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
+        const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
+        for (int t = t_lo; t < t_hi && ok; ++t) {
+          if (pp_class(qa, t, a, m_tiles, n_tiles) == 0 && pp_class(qb, t, a, m_tiles, n_tiles) == 0)
+            continue;
+          const int s = static_cast<int>(kt % S);
+          const uint32_t round = kt / S;
+          if (round > 0 &&
+              !mbar_wait(&empty[s], (round - 1) & 1u, abort_flag, a.err, kErrPrefillWait)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kTile);
+          uint8_t* dst = ring + s * L::kTile;
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(dst + c * L::kChunk, map, &full[s], c * 64, t * BN, qa.pr.kv, qa.pr.b);
+          ++kt;
+        }
+      }
+      // On an abort, the copies still in flight land before the CTA leaves.
+      if (*abort_flag) {
+        for (uint32_t j = kt > static_cast<uint32_t>(S) ? kt - S : 0; j < kt; ++j)
+          mbar_wait_drain(&full[j % S], (j / S) & 1u);
+        for (int X = 0; X < 2; ++X)
+          if (nq[X] > 0) mbar_wait_drain(&q_full[X], (nq[X] - 1) & 1u);
+      }
+    } else if (warp == kWarpMMA && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_qk = F16 ? idesc_f16_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idesc_pv = F16 ? idesc_f16_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
+      const uint64_t dq0 = kmajor_desc(smem_u32(smem + L::kQOff));
+      const uint64_t dk0 = kmajor_desc(smem_u32(smem + L::kKOff));
+      const uint64_t dv0 = mnmajor_desc(smem_u32(smem + L::kVOff), L::kChunk);
+      uint32_t kt = 0;          // key tiles (K / V stages) consumed over the kernel
+      uint32_t np[2] = {0, 0};  // P_X tiles consumed over the kernel
+      int64_t it = 0;
+      bool ok = true;
+      auto qk = [&](int X, uint32_t idx) {
+        const uint64_t dq = dq0 + ((X * L::kTile) >> 4);
+        const uint64_t dk = dk0 + (((idx % S) * L::kTile) >> 4);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          tc_mma_ss(tmem + L::s_col(X), dq + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4),
+                    dk + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4), idesc_qk, k > 0 ? 1u : 0u);
+        tc_commit(&s_full[X]);
+      };
+      auto pv = [&](int X, uint32_t idx, bool first) {
+        const uint64_t dv = dv0 + (((idx % S) * L::kTile) >> 4);
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          tc_mma_ts(tmem + L::o_col(X), tmem + L::s_col(X) + k * 8, dv + ((k * 16 * 128) >> 4),
+                    idesc_pv, (!first || k > 0) ? 1u : 0u);
+      };
+      for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
+           ++it, x = snake(it, blockIdx.x, gridDim.x)) {
+        const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
+        const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
+        // The item's key tiles that some tile works on, in order, one byte
+        // each in shared memory (bit X: tile X computes it); tile classes may
+        // read mask summaries from global memory, so they are taken once per
+        // item, off the per-tile path.
+        const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
+                             qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
+        const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
+        int n = 0, nX[2] = {0, 0};
+        for (int t = t_lo; t < t_hi; ++t) {
+          const uint32_t f = (pp_class(qa, t, a, m_tiles, n_tiles) != 0 ? 1u : 0u) |
+                             (pp_class(qb, t, a, m_tiles, n_tiles) != 0 ? 2u : 0u);
+          if (f != 0u) {
+            sched[n++] = static_cast<uint8_t>(f);
+            nX[0] += f & 1u;
+            nX[1] += f >> 1;
+          }
+        }
+#pragma unroll
+        for (int X = 0; X < 2; ++X)
+          if (ok)
+            ok = mbar_wait_hot(&q_full[X], static_cast<uint32_t>(it & 1), abort_flag, a.err,
+                               kErrPrefillWait);
+        if (!ok) break;
+        tc_fence_after();
+        int qkX[2] = {0, 0};  // QK_X / PV_X issued for this item
+        int pvX[2] = {0, 0};
+        if (n > 0) {  // the first key tile: its QKs
+          ok = mbar_wait_hot(&k_full[kt % S], (kt / S) & 1u, abort_flag, a.err, kErrPrefillWait);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t f = sched[0];
+#pragma unroll
+          for (int X = 0; X < 2; ++X)
+            if ((f >> X) & 1u) {
+              qk(X, kt);
+              if (++qkX[X] == nX[X]) tc_commit(&q_empty[X]);
+            }
+          tc_commit(&k_empty[kt % S]);
+        }
+        for (int i = 0; i < n && ok; ++i) {
+          // Per key tile: PV_A(i), QK_A(i+1), PV_B(i), QK_B(i+1).
+          const uint32_t f = sched[i];
+          const uint32_t fn = i + 1 < n ? sched[i + 1] : 0u;
+          const uint32_t cur = kt + static_cast<uint32_t>(i), nxt = cur + 1;
+          ok = mbar_wait_hot(&v_full[cur % S], (cur / S) & 1u, abort_flag, a.err, kErrPrefillWait);
+          if (!ok) break;
+          bool k_ready = false;  // K(i+1) waited for, right before its first QK
+#pragma unroll
+          for (int X = 0; X < 2; ++X) {
+            if (!ok) break;
+            if ((f >> X) & 1u) {
+              ok = mbar_wait_hot(&p_full[X], np[X] & 1u, abort_flag, a.err, kErrPrefillWait);
+              if (ok && pvX[X] == 0 && it > 0)  // O_X still holds the last item's result
+                ok = mbar_wait_hot(&o_free[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
+                                   a.err, kErrPrefillWait);
+              if (!ok) break;
+              tc_fence_after();
+              pv(X, cur, pvX[X] == 0);
+              ++np[X];
+              if (++pvX[X] == nX[X]) tc_commit(&o_final[X]);
+            }
+            if ((fn >> X) & 1u) {
+              if (!k_ready) {
+                ok = mbar_wait_hot(&k_full[nxt % S], (nxt / S) & 1u, abort_flag, a.err,
+                                   kErrPrefillWait);
+                if (!ok) break;
+                tc_fence_after();
+                k_ready = true;
+              }
+              qk(X, nxt);
+              if (++qkX[X] == nX[X]) tc_commit(&q_empty[X]);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&v_empty[cur % S]);          // V(i): its PVs are issued
+          if (fn != 0u) tc_commit(&k_empty[nxt % S]);  // K(i+1): its QKs are issued
+        }
+        if (!ok) break;
+        kt += static_cast<uint32_t>(n);
+        // A tile of the item that sees no key at all: release Q_X and let the
+        // epilogue run (it writes NaN rows) once the last item's O_X is read.
+#pragma unroll
+        for (int X = 0; X < 2; ++X)
+          if (ok && nX[X] == 0) {
+            tc_commit(&q_empty[X]);
+            if (it > 0)
+              ok = mbar_wait_hot(&o_free[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
+                                 a.err, kErrPrefillWait);
+            tc_commit(&o_final[X]);
+          }
+      }
+      tc_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    const int X = warp >> 2;  // query tile of this warpgroup
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + L::s_col(X);
+    const uint32_t o_col = tmem + lane_base + L::o_col(X);
+    const int hh = row / qpt, qi = row % qpt;
+    const bool mask_vec = a.has_mask && ((reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0) &&
+                          (a.ms[0] % 16 == 0) && (a.ms[1] % 16 == 0);
+    uint32_t J = 0;  // S_X tiles over the kernel
+    int64_t it = 0;
+    bool ok = true;
+    for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
+         ++it, x = snake(it, blockIdx.x, gridDim.x)) {
+      const PPTile me = pp_tile(x, X, a, m_tiles, qpt, n_tiles);
+      const Pair& pr = me.pr;
+      const int q = me.sl.q0 + qi;
+      const bool row_valid = me.sl.live && row < rows && q < a.Sq;
+      const uint8_t* mrow =
+          (a.has_mask && row_valid) ? a.mask + pr.b * a.ms[0] + static_cast<int64_t>(q) * a.ms[1]
+                                    : nullptr;
+      float m_ref = -INFINITY, l = 0.f;
+      int nloc = 0;
+      for (int t = pr.nt_beg; t < pr.nt_end && ok; ++t) {
+        const int cls = tile_class(a, pr, me.sl, t, m_tiles, n_tiles);
+        if (cls == 0) continue;
+        // okt: warp-uniform, so that every TMEM access it guards is made by
+        // the whole warp; the warpgroup meets once per tile below and leaves
+        // the loop together.
+        const bool okt = __all_sync(0xffffffffu, mbar_wait_hot(&s_full[X], J & 1u, abort_flag,
+                                                               a.err, kErrPrefillWait));
+        if (okt) {
+          tc_fence_after();
+          uint32_t r[BN];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+          tmem_ld_wait();
+          // Fully visible tiles work on raw scores and fold the scale into
+          // one FMA per element below; other tiles test each key against the
+          // row's visibility bits.
+          const bool fast = cls == 2 && a.scale_log2 >= 0.f;
+          if (!fast) {
+            uint32_t vb[4];
+            visible_bits<4>(vb, row_valid ? mrow : nullptr, t * BN, a, pr, q, mask_vec);
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              r[c] = __float_as_uint(((vb[c >> 5] >> (c & 31)) & 1u)
+                                         ? __uint_as_float(r[c]) * a.scale_log2
+                                         : -INFINITY);
+          }
+          // Eight independent running maxima, two elements per three-input max.
+          float part[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part[e] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < BN; c += 16)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              part[e] = fmax3(part[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
+          float mx = fmax3(fmax3(part[0], part[1], part[2]), fmax3(part[3], part[4], part[5]),
+                           fmaxf(part[6], part[7]));
+          if (fast) mx *= a.scale_log2;
+          const float m_new = fmaxf(m_ref, mx);
+          const bool grow = m_new > m_ref + kRescaleLog2;  // also true for -inf -> finite
+          const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.f;
+          const bool o_live = grow && nloc > 0 && m_ref != -INFINITY;
+          if (grow) {
+            l *= alpha;
+            m_ref = m_new;
+          }
+          const float ref = exp_ref(m_ref);
+          const float sc = fast ? a.scale_log2 : 1.f;
+          // P = 2^(t - ref) as 16-bit pairs over the first 64 columns of S_X.
+          float lp[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lp[e] = 0.f;
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = c * 32 + 2 * e, c1 = c0 + 1;
+              const float p0 = fast_exp2(fmaf(__uint_as_float(r[c0]), sc, -ref));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(r[c1]), sc, -ref));
+              lp[c0 & 7] += p0;
+              lp[c1 & 7] += p1;
+              pk[e] = pack_p<F16>(p0, p1);
+            }
+            tmem_st16(s_col + c * 16, pk);
+          }
+          l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+          if (__any_sync(0xffffffffu, o_live)) {
+            // O_X holds the earlier tiles' P V with the old reference; the
+            // previous PV_X has completed (S_X follows it) and the next waits
+            // for this tile's P: rescale it now, the S row being dead.
+            const float f = o_live ? alpha : 1.f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(o_col + c * 32, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st16(o_col + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+              tmem_st16(o_col + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+            }
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        // The four warps of the warpgroup have written P_X (or given up).
+        if (!bar_and(1 + X, 128, okt)) {
+          ok = false;
+          break;
+        }
+        if ((threadIdx.x & 127) == 0) mbar_arrive(&p_full[X]);
+        ++J;
+        ++nloc;
+      }
+      if (!ok) break;
+      // Epilogue: out = O / l for this row.
+      const bool oke = __all_sync(
+          0xffffffffu, mbar_wait_hot(&o_final[X], static_cast<uint32_t>(it & 1), abort_flag,
+                                     a.err, kErrPrefillWait));
+      if (oke) tc_fence_after();
+      uint16_t* orow = a.out + pr.b * a.os[0] +
+                       static_cast<int64_t>(pr.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
+                       static_cast<int64_t>(q) * a.os[2];
+      const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
+      if (nloc > 0) {
+        // (After a failed wait the values read are discarded: the output of
+        // an aborted launch is undefined.)
+        uint32_t r[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        if (!bar_and(1 + X, 128, oke)) {
+          ok = false;
+          break;
+        }
+        // O_X is in registers: the next item's first PV_X may overwrite it.
+        if ((threadIdx.x & 127) == 0) mbar_arrive(&o_free[X]);
+        if (row_valid) {
+#pragma unroll
+          for (int v8 = 0; v8 < D / 8; ++v8) {
+            if (v8 * 8 >= a.Dv) break;
+            uint4 w;
+            w.x = pack2<F16>(__uint_as_float(r[v8 * 8 + 0]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 1]) * inv_l);
+            w.y = pack2<F16>(__uint_as_float(r[v8 * 8 + 2]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 3]) * inv_l);
+            w.z = pack2<F16>(__uint_as_float(r[v8 * 8 + 4]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 5]) * inv_l);
+            w.w = pack2<F16>(__uint_as_float(r[v8 * 8 + 6]) * inv_l,
+                             __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+            reinterpret_cast<uint4*>(orow)[v8] = w;
+          }
+        }
+      } else {
+        if (row_valid) {
+          const float nanv = __int_as_float(0x7fc00000);
+          const uint32_t nn = pack2<F16>(nanv, nanv);
+          for (int d = 0; d < a.Dv; d += 8)
+            *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
+        }
+        tc_fence_before();
+        if (!bar_and(1 + X, 128, oke)) {
+          ok = false;
+          break;
+        }
+        if ((threadIdx.x & 127) == 0) mbar_arrive(&o_free[X]);
+      }
+    }
+  }
+
+  // Every role is done with TMEM (the MMA thread has seen its last MMA
+  // complete) before it is freed.
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int D, bool F16>
+int launch_pp_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
+                const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
+  auto kern = gqa_prefill_pp_kernel<D, F16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           PPLayout<D>::kBytes) != cudaSuccess)
+    return GQA_ERR_CUDA;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQA_ERR_CUDA;
+  if (fa.numRegs != kLaunchRegs) return GQA_ERR_CUDA;  // the register split assumes it
+  kern<<<s.grid, kPPThreads, PPLayout<D>::kBytes, stream>>>(tmq, tmk, tmv, a, s.qpt, s.rows,
+                                                            s.m_tiles, s.n_tiles, s.work);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+
+int pp_smem_bytes(int D) { return D == 128 ? PPLayout<128>::kBytes : PPLayout<64>::kBytes; }
+
+int launch_prefill_pp(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
+                      const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                      cudaStream_t stream) {
+  if (a.has_mask) {
+    const int rc = launch_mask_summary(s, a, stream);
+    if (rc != GQA_OK) return rc;
+  }
+  const bool f16 = p.dtype == GQA_DTYPE_F16;
+  if (s.D == 128)
+    return f16 ? launch_pp_t<128, true>(s, a, tmq, tmk, tmv, stream)
+               : launch_pp_t<128, false>(s, a, tmq, tmk, tmv, stream);
+  if (s.D == 64)
+    return f16 ? launch_pp_t<64, true>(s, a, tmq, tmk, tmv, stream)
+               : launch_pp_t<64, false>(s, a, tmq, tmk, tmv, stream);
+  return GQA_ERR_UNSUPPORTED;
+}
+
+}  // namespace gqa
