@@ -370,14 +370,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   int erc = encode_half_map(&tmq, q, p.batch, p.heads_q, p.seq_q, p.head_dim, p.q_stride,
                             static_cast<uint32_t>(s.qpt), static_cast<uint32_t>(g), f16);
   if (erc != GQA_OK) return erc;
-  if (s.pair) {  // each CTA of a pair loads 64 keys of a K tile and 64 columns of a V tile
-    erc = encode_half_map(&tmk, k, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.k_stride, 64, 1,
-                          f16);
-    if (erc != GQA_OK) return erc;
-    erc = encode_half_map(&tmv, v, p.batch, p.heads_kv, p.seq_k, p.head_dim, p.v_stride, 128,
-                          1, f16);
-    if (erc != GQA_OK) return erc;
-  } else if (p.block_table != nullptr) {  // paged: 64-key boxes, one page each
+  if (p.block_table != nullptr) {  // paged: 64-key boxes, one page each
     erc = encode_decode_kv_map(&tmk, k, p, p.k_stride);
     if (erc != GQA_OK) return erc;
     erc = encode_decode_kv_map(&tmv, v, p, p.v_stride);
@@ -410,7 +403,6 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   a.lens = p.kv_lens;
   a.Dv = static_cast<int>(p.head_dim);
   a.scale_log2 = scale_log2;
-  if (s.pair) return launch_prefill_pair(p, s, a, tmq, tmk, tmv, stream);
   if (s.pp) return launch_prefill_pp(p, s, a, tmq, tmk, tmv, stream);
   return launch_prefill(p, s, a, tmq, tmk, tmv, stream);
 }

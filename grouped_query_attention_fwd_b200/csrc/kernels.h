@@ -148,19 +148,11 @@ int encode_decode_kv_map(CUtensorMap* map, const void* base, const gqa_problem& 
 // ------------------------------------------------------------ prefill
 constexpr int kPrefillThreads = 12 * 32;  // two softmax warpgroups, load, MMA and V-load warps
 
-// Key tiles a work item of the pair prefill kernel may span (Sk <= 32768).
-constexpr int kMaxPairTiles = 256;
-// The pair prefill kernel is parity-green but not yet faster than the one-SM
-// kernel on the causal workload: plans do not choose it until it is.
-constexpr bool kPairPrefill = false;
-
 // Key tiles a work item of the two-tile prefill kernel may span (Sk <= 131072).
 constexpr int kMaxPPTiles = 1024;
-constexpr bool kPPPrefill = true;
 
 struct PrefillShape {
-  bool pair;         // pairs of SMs (prefill_pair.cu)
-  bool pp;           // two query tiles per SM (prefill_pp.cu); else one query tile per SM
+  bool pp;           // two query tiles per SM (prefill_pp.cu); else one (prefill.cu)
   int D;             // 64 or 128
   int qpt;           // query positions per 128-row tile (rows = qpt * g)
   int rows;          // qpt * g <= 128
@@ -192,12 +184,6 @@ struct PrefillArgs {
 // Mask pre-pass shared by both prefill kernels: per (batch, query tile, key
 // tile) 0 all hidden, 1 mixed, 2 all visible.
 int launch_mask_summary(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
-
-// Pair prefill: tmk_half is K with 64-key boxes, tmv V with 128-key boxes.
-int pair_smem_bytes();
-int launch_prefill_pair(const gqa_problem& p, const PrefillShape& s, const PrefillArgs& a,
-                        const CUtensorMap& tmq, const CUtensorMap& tmk_half,
-                        const CUtensorMap& tmv, cudaStream_t stream);
 
 // Two query tiles per SM: K and V with 128-key boxes, as for the one-tile kernel.
 int pp_smem_bytes(int D);

@@ -742,22 +742,14 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.rows = static_cast<int>(s.qpt * g);
   s.m_tiles = static_cast<int>((p.seq_q + s.qpt - 1) / s.qpt);
   s.n_tiles = static_cast<int>((p.seq_k + BN - 1) / BN);
-  // Pairs of SMs for head_dim 128 over contiguous caches without lengths
-  // (work item: four query tiles); one SM per query tile otherwise.
-  s.pair = kPairPrefill && s.D == 128 && p.kv_lens == nullptr && p.block_table == nullptr &&
-           s.n_tiles <= kMaxPairTiles && sm_count >= 2;
-  s.pp = !s.pair && kPPPrefill && p.kv_lens == nullptr && p.block_table == nullptr &&
-         s.n_tiles <= kMaxPPTiles;
+  // Two query tiles per SM over contiguous caches without lengths; one
+  // query tile per SM (the kernel that reads lengths and block tables) otherwise.
+  s.pp = p.kv_lens == nullptr && p.block_table == nullptr && s.n_tiles <= kMaxPPTiles;
   if (s.pp) {
     s.work = p.batch * p.heads_kv * ((s.m_tiles + 1) / 2);  // pairs of query tiles
     s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
     if (s.grid < 1) s.grid = 1;
     s.smem_bytes = pp_smem_bytes(s.D);
-  } else if (s.pair) {
-    s.work = p.batch * p.heads_kv * ((s.m_tiles + 3) / 4);
-    const int64_t pairs = sm_count / 2;
-    s.grid = static_cast<int>(2 * (s.work < pairs ? s.work : pairs));
-    s.smem_bytes = pair_smem_bytes();
   } else {
     s.work = p.batch * p.heads_kv * s.m_tiles;  // query tiles
     s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);

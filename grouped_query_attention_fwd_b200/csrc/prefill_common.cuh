@@ -1,5 +1,5 @@
-// Pieces shared by the two prefill kernels (one SM per query tile, and a
-// pair of SMs per two query tiles): the geometry of a query tile's visible
+// Pieces shared by the two prefill kernels (one query tile per SM, and two
+// query tiles per SM): the geometry of a query tile's visible
 // keys, the classification of key tiles, per-key visibility bits, the
 // shared-memory matrix descriptors and the packing of P.
 #pragma once
