@@ -150,6 +150,9 @@ constexpr int kPrefillThreads = 12 * 32;  // two softmax warpgroups, load, MMA a
 
 // Key tiles a work item of the two-tile prefill kernel may span (Sk <= 131072).
 constexpr int kMaxPPTiles = 1024;
+// Largest items x key tiles for which the two-tile kernel's item order is
+// sorted on the device (one CTA classifies every item's key tiles).
+constexpr int64_t kMaxOrderWork = int64_t(1) << 21;
 
 struct PrefillShape {
   bool pp;           // two query tiles per SM (prefill_pp.cu); else one (prefill.cu)
@@ -162,6 +165,9 @@ struct PrefillShape {
   int grid;
   int smem_bytes;
   int64_t summary_offset, workspace_end;
+  // Two-tile kernel with a mask: the order in which the items are taken
+  // (heaviest first, from the mask summary), int32 per item, or -1 (none).
+  int64_t order_offset;
 };
 
 PrefillShape plan_prefill(const gqa_problem& p, int sm_count);
@@ -172,6 +178,7 @@ struct PrefillArgs {
   uint16_t* out;
   int64_t os[4];
   uint8_t* summary;  // [B][m_tiles][n_tiles]: 0 all hidden, 1 mixed, 2 all visible
+  int32_t* order;    // item taken at position x of the schedule, or nullptr (x itself)
   uint32_t* err;
   const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
   int Dv;               // head_dim (<= the kernel's D; a multiple of 8)

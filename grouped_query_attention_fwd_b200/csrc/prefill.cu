@@ -760,6 +760,14 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   }
   s.summary_offset = kScratchOffset;
   s.workspace_end = s.summary_offset + (p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0);
+  s.order_offset = -1;
+  // With a mask the items' costs vary (a padding mask: with the entry's
+  // length): the two-tile kernel takes them heaviest first, in an order
+  // sorted on the device from the mask summary, when sorting is cheap.
+  if (s.pp && p.has_mask && s.work * s.n_tiles <= kMaxOrderWork) {
+    s.order_offset = ((s.workspace_end + 255) / 256) * 256;
+    s.workspace_end = s.order_offset + s.work * 4;
+  }
   return s;
 }
 

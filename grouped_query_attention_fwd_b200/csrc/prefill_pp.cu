@@ -205,8 +205,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       bool ok = true;
       for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
            ++it, x = snake(it, blockIdx.x, gridDim.x)) {
-        const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
-        const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
+        const int64_t xi = a.order != nullptr ? a.order[x] : x;
+        const PPTile qa = pp_tile(xi, 0, a, m_tiles, qpt, n_tiles);
+        const PPTile qb = pp_tile(xi, 1, a, m_tiles, qpt, n_tiles);
         if (is_qk) {
 #pragma unroll
           for (int X = 0; X < 2; ++X) {
@@ -279,8 +280,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       };
       for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
            ++it, x = snake(it, blockIdx.x, gridDim.x)) {
-        const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
-        const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
+        const int64_t xi = a.order != nullptr ? a.order[x] : x;
+        const PPTile qa = pp_tile(xi, 0, a, m_tiles, qpt, n_tiles);
+        const PPTile qb = pp_tile(xi, 1, a, m_tiles, qpt, n_tiles);
         // The item's key tiles that some tile works on, in order, one byte
         // each in shared memory (bit X: tile X computes it); tile classes may
         // read mask summaries from global memory, so they are taken once per
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     bool ok = true;
     for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
          ++it, x = snake(it, blockIdx.x, gridDim.x)) {
-      const PPTile me = pp_tile(x, X, a, m_tiles, qpt, n_tiles);
+      const PPTile me = pp_tile(a.order != nullptr ? a.order[x] : x, X, a, m_tiles, qpt, n_tiles);
       const Pair& pr = me.pr;
       const int q = me.sl.q0 + qi;
       const bool row_valid = me.sl.live && row < rows && q < a.Sq;
@@ -563,6 +565,59 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
 }
 
+// The items of a masked launch in decreasing order of cost (the key tiles
+// that either query tile computes, from the mask summary): a counting sort in
+// one CTA, written to a.order.  Position x of the kernels' schedule then takes
+// item a.order[x], so the heaviest items are spread first over the CTAs and
+// the lightest fill in last.
+__global__ void __launch_bounds__(1024)
+    gqa_pp_order_kernel(const PrefillArgs a, const int qpt, const int m_tiles, const int n_tiles,
+                        const int64_t items) {
+  __shared__ int slot[1024];  // per cost bucket (bucket 0: the heaviest): count, then next position
+  __shared__ int warp_base[32];
+  const int tid = threadIdx.x;
+  auto bucket_of = [&](int64_t x) -> int {
+    const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
+    const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
+    const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
+                         qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
+    const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
+    int n = 0;
+    for (int t = t_lo; t < t_hi; ++t)
+      n += (pp_class(qa, t, a, m_tiles, n_tiles) != 0 || pp_class(qb, t, a, m_tiles, n_tiles) != 0)
+               ? 1
+               : 0;
+    return 1023 - min(n, 1023);
+  };
+  slot[tid] = 0;
+  __syncthreads();
+  for (int64_t x = tid; x < items; x += blockDim.x) atomicAdd(&slot[bucket_of(x)], 1);
+  __syncthreads();
+  // Exclusive prefix sum of the bucket counts: the first position of each bucket.
+  const int v = slot[tid];
+  int incl = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((tid & 31) >= o) incl += y;
+  }
+  if ((tid & 31) == 31) warp_base[tid >> 5] = incl;
+  __syncthreads();
+  if (tid < 32) {
+    const int w = warp_base[tid];
+    int wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (tid >= o) wi += y;
+    }
+    warp_base[tid] = wi - w;
+  }
+  __syncthreads();
+  slot[tid] = warp_base[tid >> 5] + incl - v;
+  __syncthreads();
+  for (int64_t x = tid; x < items; x += blockDim.x)
+    a.order[atomicAdd(&slot[bucket_of(x)], 1)] = static_cast<int32_t>(x);
+}
+
 template <int D, bool F16>
 int launch_pp_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
                 const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
@@ -588,6 +643,10 @@ int launch_prefill_pp(const gqa_problem& p, const PrefillShape& s, const Prefill
   if (a.has_mask) {
     const int rc = launch_mask_summary(s, a, stream);
     if (rc != GQA_OK) return rc;
+  }
+  if (a.order != nullptr) {
+    gqa_pp_order_kernel<<<1, 1024, 0, stream>>>(a, s.qpt, s.m_tiles, s.n_tiles, s.work);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
   const bool f16 = p.dtype == GQA_DTYPE_F16;
   if (s.D == 128)
