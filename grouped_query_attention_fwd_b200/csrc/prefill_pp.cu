@@ -573,25 +573,41 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 __global__ void __launch_bounds__(1024)
     gqa_pp_order_kernel(const PrefillArgs a, const int qpt, const int m_tiles, const int n_tiles,
                         const int64_t items) {
+  constexpr int kKeep = 8192;  // items whose bucket is kept in shared memory
   __shared__ int slot[1024];  // per cost bucket (bucket 0: the heaviest): count, then next position
   __shared__ int warp_base[32];
+  __shared__ uint16_t kept[kKeep];
   const int tid = threadIdx.x;
   auto bucket_of = [&](int64_t x) -> int {
     const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
     const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
-    const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
-                         qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
-    const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
     int n = 0;
-    for (int t = t_lo; t < t_hi; ++t)
-      n += (pp_class(qa, t, a, m_tiles, n_tiles) != 0 || pp_class(qb, t, a, m_tiles, n_tiles) != 0)
-               ? 1
-               : 0;
+    if (!a.causal) {
+      // Mask only: a key tile is computed iff its summary byte is nonzero
+      // for either live query tile.
+      const uint8_t* ra = a.summary + (static_cast<int64_t>(qa.pr.b) * m_tiles + qa.pr.mt0) * n_tiles;
+      const uint8_t* rb = a.summary + (static_cast<int64_t>(qb.pr.b) * m_tiles + qb.pr.mt0) * n_tiles;
+      const bool la = qa.pr.nt_end > qa.pr.nt_beg, lb = qb.pr.nt_end > qb.pr.nt_beg;
+      for (int t = 0; t < n_tiles; ++t)
+        n += ((la && ra[t] != 0) || (lb && rb[t] != 0)) ? 1 : 0;
+    } else {
+      const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
+                           qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
+      const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
+      for (int t = t_lo; t < t_hi; ++t)
+        n += (pp_class(qa, t, a, m_tiles, n_tiles) != 0 || pp_class(qb, t, a, m_tiles, n_tiles) != 0)
+                 ? 1
+                 : 0;
+    }
     return 1023 - min(n, 1023);
   };
   slot[tid] = 0;
   __syncthreads();
-  for (int64_t x = tid; x < items; x += blockDim.x) atomicAdd(&slot[bucket_of(x)], 1);
+  for (int64_t x = tid; x < items; x += blockDim.x) {
+    const int k = bucket_of(x);
+    if (x < kKeep) kept[x] = static_cast<uint16_t>(k);
+    atomicAdd(&slot[k], 1);
+  }
   __syncthreads();
   // Exclusive prefix sum of the bucket counts: the first position of each bucket.
   const int v = slot[tid];
@@ -615,7 +631,7 @@ __global__ void __launch_bounds__(1024)
   slot[tid] = warp_base[tid >> 5] + incl - v;
   __syncthreads();
   for (int64_t x = tid; x < items; x += blockDim.x)
-    a.order[atomicAdd(&slot[bucket_of(x)], 1)] = static_cast<int32_t>(x);
+    a.order[atomicAdd(&slot[x < kKeep ? kept[x] : bucket_of(x)], 1)] = static_cast<int32_t>(x);
 }
 
 template <int D, bool F16>
