@@ -84,12 +84,15 @@ def _peaks():
 
 
 TRAFFIC_SOURCES = ("kernels.h", "ptx.cuh", "epilogue.cuh")
+# Headers a prefill kernel also includes.
+PREFILL_SOURCES = ("prefill_common.cuh",)
 
 
 def kernel_source_sha256(kernel_file: str) -> str:
     """Hash of a kernel's source and the headers it includes."""
     h = hashlib.sha256()
-    for name in (kernel_file,) + TRAFFIC_SOURCES:
+    extra = PREFILL_SOURCES if kernel_file.startswith("prefill") else ()
+    for name in (kernel_file,) + TRAFFIC_SOURCES + extra:
         with open(os.path.join(ROOT, "grouped_query_attention_fwd_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -570,13 +573,14 @@ def _roofline_decode(res, hbm, peak_kind, workload, kernel_file="decode.cu"):
             "launch_ms": round(res["per_launch_ms"], 5)}
 
 
-def _roofline_prefill(res, tflops, peak_kind, workload):
+def _roofline_prefill(res, tflops, peak_kind, workload, kernel_file="prefill_pp.cu"):
+    """Contiguous caches without lengths run on the two-tile kernel."""
     per_s = res["per_launch_ms"] / 1e3
     fl = res["plan"]["algorithmic_flops"]
     achieved = fl / per_s / 1e12
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tflops, "unit": "TFLOP/s",
             "frac": round(achieved / tflops, 4), "peak_source": peak_kind,
-            "traffic": _traffic_for("prefill.cu", workload),
+            "traffic": _traffic_for(kernel_file, workload),
             "algorithmic_flops_per_launch": fl, "launch_ms": round(res["per_launch_ms"], 5)}
 
 
