@@ -168,7 +168,8 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       plan->grid = s.grid;
       plan->block = kPrefillThreads;
       plan->smem_bytes = s.smem_bytes;
-      plan->launches = p.has_mask ? 2 : 1;
+      // (+ the mask summary pre-pass, and the sort of the items by cost)
+      plan->launches = p.has_mask ? (s.order_offset >= 0 ? 3 : 2) : 1;
       plan->work_units = static_cast<int32_t>(s.work);
       plan->workspace_bytes = s.workspace_end;
       break;
