@@ -601,7 +601,7 @@ def _roofline_ragged_prefill(res, cfg, tf_peak, peak_kind):
     achieved = flops / (res["per_launch_ms"] / 1e3) / 1e12
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tf_peak, "unit": "TFLOP/s",
             "frac": round(achieved / tf_peak, 4), "peak_source": peak_kind,
-            "traffic": _traffic_for("prefill.cu", cfg["name"]),
+            "traffic": _traffic_for("prefill_pp.cu", cfg["name"]),
             "algorithmic_flops_per_launch": flops, "mean_len": round(res["mean_len"], 1),
             "launch_ms": round(res["per_launch_ms"], 5)}
 

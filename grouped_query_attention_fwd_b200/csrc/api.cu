@@ -169,7 +169,7 @@ int fill_plan(const gqa_problem& p, int sm_count, gqa_plan* plan) {
       plan->block = kPrefillThreads;
       plan->smem_bytes = s.smem_bytes;
       // (+ the mask summary pre-pass, and the sort of the items by cost)
-      plan->launches = p.has_mask ? (s.order_offset >= 0 ? 3 : 2) : 1;
+      plan->launches = 1 + (p.has_mask ? 1 : 0) + (s.order_offset >= 0 ? 1 : 0);
       plan->work_units = static_cast<int32_t>(s.work);
       plan->workspace_bytes = s.workspace_end;
       break;

@@ -62,7 +62,10 @@ constexpr int CHUNK_BYTES = KT * 128;   // one 64-wide bf16 column chunk of a ti
 constexpr int kFastMerge = 4;           // split groups merged with all loads in flight
 
 __host__ __device__ inline int range_start(int c, int T, int P) {
-  return static_cast<int>((static_cast<int64_t>(c) * T) / P);
+  // floor(c T / P) = c q + floor(c r / P) with T = q P + r: 32-bit operations
+  // only (c <= P, so c r < P^2), on every CTA's path to its first copy.
+  const int q = T / P, r = T - q * P;
+  return c * q + (c * r) / P;
 }
 
 // The CTA whose range [range_start(c), range_start(c + 1)) holds unit u:

@@ -1,4 +1,7 @@
-// Prefill kernel (longer query blocks) on the 5th-generation tensor cores.
+// Prefill kernel (longer query blocks) on the 5th-generation tensor cores,
+// one query tile per SM.  Plans use it for key lengths beyond the two-tile
+// kernel's per-item step list (more than 1024 key tiles); the two-tile
+// kernel (prefill_pp.cu) takes every other prefill.
 //
 // The g query heads that share a kv head are packed into the 128 rows (M) of
 // one tcgen05 tile: row r holds head h0 + r / qpt at query position
@@ -742,9 +745,9 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.rows = static_cast<int>(s.qpt * g);
   s.m_tiles = static_cast<int>((p.seq_q + s.qpt - 1) / s.qpt);
   s.n_tiles = static_cast<int>((p.seq_k + BN - 1) / BN);
-  // Two query tiles per SM over contiguous caches without lengths; one
-  // query tile per SM (the kernel that reads lengths and block tables) otherwise.
-  s.pp = p.kv_lens == nullptr && p.block_table == nullptr && s.n_tiles <= kMaxPPTiles;
+  // Two query tiles per SM; one query tile per SM when an item's key tiles
+  // would overflow the two-tile kernel's per-item step list.
+  s.pp = s.n_tiles <= kMaxPPTiles;
   if (s.pp) {
     s.work = p.batch * p.heads_kv * ((s.m_tiles + 1) / 2);  // pairs of query tiles
     s.grid = static_cast<int>(s.work < sm_count ? s.work : sm_count);
@@ -761,10 +764,13 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   s.summary_offset = kScratchOffset;
   s.workspace_end = s.summary_offset + (p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0);
   s.order_offset = -1;
-  // With a mask the items' costs vary (a padding mask: with the entry's
-  // length): the two-tile kernel takes them heaviest first, in an order
-  // sorted on the device from the mask summary, when sorting is cheap.
-  if (s.pp && p.has_mask && s.work * s.n_tiles <= kMaxOrderWork) {
+  // With a mask or per-sequence lengths the items' costs vary (with each
+  // entry's length): the two-tile kernel takes them heaviest first, in an
+  // order sorted on the device, when sorting is cheap (a mask: every item's
+  // tiles are classified; lengths alone: a range per item).
+  const bool sort_cost = p.has_mask ? s.work * s.n_tiles <= kMaxOrderWork
+                                    : (p.kv_lens != nullptr && s.work <= kMaxOrderWork);
+  if (s.pp && sort_cost) {
     s.order_offset = ((s.workspace_end + 255) / 256) * 256;
     s.workspace_end = s.order_offset + s.work * 4;
   }

@@ -30,6 +30,13 @@
 //   warp 8     TMA producer of Q tiles and K tiles
 //   warp 9     TMEM allocator and single-thread MMA issuer
 //   warp 10    TMA producer of V tiles (warp 11 idles)
+// Per-sequence lengths and paged caches (the KVX instances): an item's key
+// range ends at its entry's length; the one key tile that reaches past it has
+// its V rows there zeroed in shared memory by the V producer before its PVs
+// (0 times a NaN left in the cache would still reach O); a paged cache's
+// 128-key tile is two 64-key boxes, each inside one page.  With a mask or
+// lengths the items' costs differ, and a one-CTA sort orders them heaviest
+// first before the launch.
 // Every wait is bounded; a thread that gives up sets the abort flag and the
 // error word, every role leaves its loop, copies in flight are waited for and
 // TMEM is freed after a block-wide barrier.
@@ -70,8 +77,8 @@ struct PPLayout {
   static constexpr int kVOff = kKOff + kStages * kTile;
   static constexpr int kBarOff = kVOff + kStages * kTile;
   // q_full[2], q_empty[2], k_full[S], k_empty[S], v_full[S], v_empty[S],
-  // s_full[2], p_full[2], o_final[2], o_free[2], mma_done
-  static constexpr int kNumBars = 4 + 4 * kStages + 8 + 1;
+  // s_full[2], p_full[2], o_final[2], o_free[2], mma_done, v_fix[S]
+  static constexpr int kNumBars = 4 + 4 * kStages + 8 + 1 + kStages;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSchedOff = kMiscOff + 16;  // the MMA thread's key-tile list of an item
   static constexpr int kBytes = kSchedOff + kMaxPPTiles + 1024;  // + alignment slack
@@ -100,6 +107,10 @@ __device__ __forceinline__ PPTile pp_tile(int64_t x, int X, const PrefillArgs& a
   t.pr.kv = bk % a.Hkv;
   t.pr.mt0 = mt;
   t.pr.len = a.Sk;
+  if (a.lens != nullptr) {  // out-of-range lengths are clamped (and reported at kernel start)
+    const int len = a.lens[t.pr.b];
+    t.pr.len = len < 0 ? 0 : (len > a.Sk ? a.Sk : len);
+  }
   t.sl = slot_of(t.pr, a, qpt);
   t.sl.live = mt < m_tiles;
   if (!t.sl.live || t.sl.key_hi <= t.sl.key_lo) {
@@ -118,13 +129,16 @@ __device__ __forceinline__ int pp_class(const PPTile& q, int u, const PrefillArg
   return tile_class(a, q.pr, q.sl, u, m_tiles, n_tiles);
 }
 
-template <int D, bool F16>
+// KVX: the launch has per-sequence lengths or a paged cache (the V rows past
+// a length are zeroed before their PV; K / V tiles of a paged cache are two
+// 64-key boxes, each inside one page).
+template <int D, bool F16, bool KVX>
 __global__ void __launch_bounds__(kPPThreads, 1)
     gqa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmq,
                           const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv, const PrefillArgs a,
                           const int qpt, const int rows, const int m_tiles, const int n_tiles,
-                          const int64_t items) {
+                          const int64_t items, const PagedKV pg) {
   using L = PPLayout<D>;
   constexpr int CH = L::CH;
   constexpr int S = L::kStages;
@@ -143,6 +157,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   uint64_t* o_final = p_full + 2;       // [X] the item's last PV_X done
   uint64_t* o_free = o_final + 2;       // [X] O_X read by the epilogue
   uint64_t* mma_done = o_free + 2;      // every MMA done
+  uint64_t* v_fix = mma_done + 1;       // [stage] (KVX): the V rows past the length zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   uint8_t* sched = smem + L::kSchedOff;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -166,8 +181,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       mbar_init(&v_empty[i], 1);
     }
     mbar_init(mma_done, 1);
+    if (KVX)
+      for (int i = 0; i < S; ++i) mbar_init(&v_fix[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (KVX && a.lens != nullptr && blockIdx.x == 0) {
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+      const int len = a.lens[b];
+      if (len < 0 || len > a.Sk) atomicOr(a.err, kErrKvLength);
+    }
   }
   // Q rows past qpt * g of a tile are never written by TMA: zero them once.
   if (rows < BM && threadIdx.x < 8) {
@@ -239,9 +262,48 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           mbar_arrive_expect_tx(&full[s], L::kTile);
           uint8_t* dst = ring + s * L::kTile;
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(dst + c * L::kChunk, map, &full[s], c * 64, t * BN, qa.pr.kv, qa.pr.b);
+          if (KVX && pg.bt != nullptr) {
+            // Two 64-key boxes, each inside one page (page_size is a multiple
+            // of 64).  A box that starts at or past the entry's length reads an
+            // out-of-range page, which the copy fills with zeros; a page index
+            // outside the pool for keys in use is reported and read the same way.
+            for (int hb = 0; hb < 2; ++hb) {
+              const int key = t * BN + hb * 64;
+              int page = pg.num_pages;
+              if (key < qa.pr.len) {
+                page = __ldg(pg.bt + qa.pr.b * pg.bt_stride + key / pg.page_size);
+                if (page < 0 || page >= pg.num_pages) {
+                  atomicOr(a.err, kErrPage);
+                  page = pg.num_pages;
+                }
+              }
+              for (int c = 0; c < CH; ++c)
+                tma_load_4d(dst + c * L::kChunk + hb * 64 * 128, map, &full[s], c * 64,
+                            key % pg.page_size, qa.pr.kv, page);
+            }
+          } else {
+            for (int c = 0; c < CH; ++c)
+              tma_load_4d(dst + c * L::kChunk, map, &full[s], c * 64, t * BN, qa.pr.kv, qa.pr.b);
+          }
           ++kt;
+          // The V rows of the entry's last tile past its length hold whatever
+          // the cache holds there (NaN included), and P = 0 does not hide a
+          // NaN in P V: once the tile has landed they are zeroed, and the MMA
+          // waits for that too.  Only the last tile an item visits can reach
+          // past the length.
+          if (KVX && !is_qk && (static_cast<int64_t>(t) + 1) * BN > qa.pr.len) {
+            if (!mbar_wait(&full[s], round & 1u, abort_flag, a.err, kErrPrefillWait)) {
+              ok = false;
+              break;
+            }
+            const int valid = qa.pr.len - t * BN;  // 1 .. BN - 1: the tile holds a key below len
+            for (int c = 0; c < CH; ++c) {
+              uint4* row0 = reinterpret_cast<uint4*>(dst + c * L::kChunk + valid * 128);
+              for (int i = 0; i < (BN - valid) * 8; ++i) row0[i] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&v_fix[s]);
+          }
         }
       }
       // On an abort, the copies still in flight land before the CTA leaves.
@@ -260,6 +322,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       const uint64_t dv0 = mnmajor_desc(smem_u32(smem + L::kVOff), L::kChunk);
       uint32_t kt = 0;          // key tiles (K / V stages) consumed over the kernel
       uint32_t np[2] = {0, 0};  // P_X tiles consumed over the kernel
+      uint32_t fix_parity = 0;  // bit s (KVX): parity of the next v_fix[s] phase
       int64_t it = 0;
       bool ok = true;
       auto qk = [&](int X, uint32_t idx) {
@@ -291,6 +354,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                              qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
         const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
         int n = 0, nX[2] = {0, 0};
+        int t_last = -1;  // the last key tile computed
         for (int t = t_lo; t < t_hi; ++t) {
           const uint32_t f = (pp_class(qa, t, a, m_tiles, n_tiles) != 0 ? 1u : 0u) |
                              (pp_class(qb, t, a, m_tiles, n_tiles) != 0 ? 2u : 0u);
@@ -298,8 +362,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             sched[n++] = static_cast<uint8_t>(f);
             nX[0] += f & 1u;
             nX[1] += f >> 1;
+            t_last = t;
           }
         }
+        // That tile reaches past the entry's length: its V rows there are
+        // zeroed by the V producer before its PVs.
+        const bool last_fix = KVX && n > 0 && (static_cast<int64_t>(t_last) + 1) * BN > qa.pr.len;
 #pragma unroll
         for (int X = 0; X < 2; ++X)
           if (ok)
@@ -328,6 +396,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           const uint32_t fn = i + 1 < n ? sched[i + 1] : 0u;
           const uint32_t cur = kt + static_cast<uint32_t>(i), nxt = cur + 1;
           ok = mbar_wait_hot(&v_full[cur % S], (cur / S) & 1u, abort_flag, a.err, kErrPrefillWait);
+          if (ok && last_fix && i == n - 1) {
+            const uint32_t sf = cur % S;
+            ok = mbar_wait_hot(&v_fix[sf], (fix_parity >> sf) & 1u, abort_flag, a.err,
+                               kErrPrefillWait);
+            fix_parity ^= 1u << sf;
+          }
           if (!ok) break;
           bool k_ready = false;  // K(i+1) waited for, right before its first QK
 #pragma unroll
@@ -565,9 +639,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
 }
 
-// The items of a masked launch in decreasing order of cost (the key tiles
-// that either query tile computes, from the mask summary): a counting sort in
-// one CTA, written to a.order.  Position x of the kernels' schedule then takes
+// The items of a launch with a mask or per-sequence lengths in decreasing
+// order of cost (the key tiles that either query tile computes): a counting
+// sort in one CTA, written to a.order.  Position x of the kernels' schedule then takes
 // item a.order[x], so the heaviest items are spread first over the CTAs and
 // the lightest fill in last.
 __global__ void __launch_bounds__(1024)
@@ -582,7 +656,14 @@ __global__ void __launch_bounds__(1024)
     const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
     const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
     int n = 0;
-    if (!a.causal) {
+    if (!a.has_mask) {
+      // Every key tile of a query tile's range is computed: the union of the
+      // two ranges (consecutive query tiles: they overlap or touch).
+      const int lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
+                         qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
+      const int hi = max(qa.pr.nt_end, qb.pr.nt_end);
+      n = hi > lo ? hi - lo : 0;
+    } else if (!a.causal && a.lens == nullptr) {
       // Mask only: a key tile is computed iff its summary byte is nonzero
       // for either live query tile.
       const uint8_t* ra = a.summary + (static_cast<int64_t>(qa.pr.b) * m_tiles + qa.pr.mt0) * n_tiles;
@@ -634,10 +715,11 @@ __global__ void __launch_bounds__(1024)
     a.order[atomicAdd(&slot[x < kKeep ? kept[x] : bucket_of(x)], 1)] = static_cast<int32_t>(x);
 }
 
-template <int D, bool F16>
-int launch_pp_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& tmq,
-                const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream) {
-  auto kern = gqa_prefill_pp_kernel<D, F16>;
+template <int D, bool F16, bool KVX>
+int launch_pp_t(const PrefillShape& s, const PrefillArgs& a, const PagedKV& pg,
+                const CUtensorMap& tmq, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                cudaStream_t stream) {
+  auto kern = gqa_prefill_pp_kernel<D, F16, KVX>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            PPLayout<D>::kBytes) != cudaSuccess)
     return GQA_ERR_CUDA;
@@ -645,7 +727,7 @@ int launch_pp_t(const PrefillShape& s, const PrefillArgs& a, const CUtensorMap& 
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return GQA_ERR_CUDA;
   if (fa.numRegs != kLaunchRegs) return GQA_ERR_CUDA;  // the register split assumes it
   kern<<<s.grid, kPPThreads, PPLayout<D>::kBytes, stream>>>(tmq, tmk, tmv, a, s.qpt, s.rows,
-                                                            s.m_tiles, s.n_tiles, s.work);
+                                                            s.m_tiles, s.n_tiles, s.work, pg);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -665,12 +747,26 @@ int launch_prefill_pp(const gqa_problem& p, const PrefillShape& s, const Prefill
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   }
   const bool f16 = p.dtype == GQA_DTYPE_F16;
-  if (s.D == 128)
-    return f16 ? launch_pp_t<128, true>(s, a, tmq, tmk, tmv, stream)
-               : launch_pp_t<128, false>(s, a, tmq, tmk, tmv, stream);
-  if (s.D == 64)
-    return f16 ? launch_pp_t<64, true>(s, a, tmq, tmk, tmv, stream)
-               : launch_pp_t<64, false>(s, a, tmq, tmk, tmv, stream);
+  PagedKV pg{};
+  pg.bt = p.block_table;
+  pg.bt_stride = p.block_table_stride;
+  pg.page_size = static_cast<int>(p.page_size);
+  pg.num_pages = static_cast<int>(p.num_pages);
+  const bool kvx = a.lens != nullptr || pg.bt != nullptr;
+  if (s.D == 128) {
+    if (kvx)
+      return f16 ? launch_pp_t<128, true, true>(s, a, pg, tmq, tmk, tmv, stream)
+                 : launch_pp_t<128, false, true>(s, a, pg, tmq, tmk, tmv, stream);
+    return f16 ? launch_pp_t<128, true, false>(s, a, pg, tmq, tmk, tmv, stream)
+               : launch_pp_t<128, false, false>(s, a, pg, tmq, tmk, tmv, stream);
+  }
+  if (s.D == 64) {
+    if (kvx)
+      return f16 ? launch_pp_t<64, true, true>(s, a, pg, tmq, tmk, tmv, stream)
+                 : launch_pp_t<64, false, true>(s, a, pg, tmq, tmk, tmv, stream);
+    return f16 ? launch_pp_t<64, true, false>(s, a, pg, tmq, tmk, tmv, stream)
+               : launch_pp_t<64, false, false>(s, a, pg, tmq, tmk, tmv, stream);
+  }
   return GQA_ERR_UNSUPPORTED;
 }
 
