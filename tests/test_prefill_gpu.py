@@ -211,3 +211,36 @@ def test_prefill_offset_window(gqa, B, Hq, Hkv, Sq, Sk, D, off, window, mask_kin
     nan_ref = np.isnan(ref).all(axis=-1)
     assert np.array_equal(np.isnan(out).all(axis=-1), nan_ref)
     assert_bf16_parity(out[~nan_ref], ref[~nan_ref], "prefill offset/window")
+
+
+def test_prefill_long_keys_one_tile(gqa):
+    """Keys past 1024 tiles (131072) per item: plans take the one-query-tile
+    kernel (its work units are single query tiles).  Contiguous cache with a
+    bottom-right causal block, then a ragged batch in 64-key pages of a pool
+    that is NaN outside the valid rows."""
+    import test_paged_gpu as pg
+    # contiguous, bottom-right causal (g = 4: 32 queries per tile)
+    B, Hq, Hkv, Sq, Sk, D = 1, 4, 1, 40, 132000, 64
+    bits, (q, k, v) = bf16_inputs(7100, B, Hq, Hkv, Sq, Sk, D)
+    plan = gqa.query(q, k, v, causal=True, causal_offset="bottom_right")
+    m_tiles = -(-Sq // 32)
+    assert plan["kernel_name"] == "prefill" and plan["work_units"] == B * Hkv * m_tiles
+    out = to_np(gqa.forward(q, k, v, causal=True, causal_offset="bottom_right"))
+    _status_ok(gqa)
+    ref = oracle.forward(f64(bits[0]), f64(bits[1]), f64(bits[2]), causal=True,
+                         causal_offset=Sk - Sq)
+    assert_bf16_parity(out, ref, "prefill, 132000 keys, one query tile per SM")
+    # ragged and paged: capacity 2100 pages of 64 keys, lengths 134000 and 5000
+    B, Hq, Hkv, Sq, D, ps, per_seq = 2, 4, 1, 64, 64, 64, 2100
+    lens = np.array([134000, 5000], dtype=np.int32)
+    kc, vc, kd, vd, table = pg._paged(7200, B, Hkv, D, ps, per_seq, lens, "bf16")
+    qh, qd = pg._q(7200, B, Hq, Sq, D, "bf16")
+    cap = ps * per_seq
+    plan = gqa.query(qd, kd, vd, causal=True, causal_offset="bottom_right",
+                     kv_lens=torch.from_numpy(lens).cuda(), block_table=table)
+    assert plan["work_units"] == B * Hkv * 2  # two query tiles of 32 positions
+    out = to_np(gqa.forward(qd, kd, vd, causal=True, causal_offset="bottom_right",
+                            kv_lens=torch.from_numpy(lens).cuda(), block_table=table))
+    _status_ok(gqa)
+    ref = oracle.forward(qh, kc, vc, causal=True, causal_offset=cap - Sq, kv_lens=lens)
+    pg._check_nan_rows(out, ref, "paged prefill, 134000 keys, one query tile per SM")
