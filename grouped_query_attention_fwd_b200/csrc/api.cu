@@ -391,6 +391,7 @@ GQA_API int gqa_forward(const gqa_problem* pp, const void* q, const void* k, con
   for (int d = 0; d < 4; ++d) a.os[d] = p.o_stride[d];
   a.summary = ws + s.summary_offset;
   a.order = s.order_offset >= 0 ? reinterpret_cast<int32_t*>(ws + s.order_offset) : nullptr;
+  a.bounds = s.bounds_offset >= 0 ? reinterpret_cast<int32_t*>(ws + s.bounds_offset) : nullptr;
   a.err = err;
   a.B = static_cast<int>(p.batch);
   a.Hq = static_cast<int>(p.heads_q);

@@ -168,6 +168,7 @@ struct PrefillShape {
   // Two-tile kernel with a mask: the order in which the items are taken
   // (heaviest first, from the mask summary), int32 per item, or -1 (none).
   int64_t order_offset;
+  int64_t bounds_offset;  // with a mask: the summary's per-query-tile key-tile bounds
 };
 
 PrefillShape plan_prefill(const gqa_problem& p, int sm_count);
@@ -179,6 +180,7 @@ struct PrefillArgs {
   int64_t os[4];
   uint8_t* summary;  // [B][m_tiles][n_tiles]: 0 all hidden, 1 mixed, 2 all visible
   int32_t* order;    // item taken at position x of the schedule, or nullptr (x itself)
+  int32_t* bounds;   // with a mask: [B][m_tiles][2] first and past-last key tile not hidden
   uint32_t* err;
   const int32_t* lens;  // per-sequence cache lengths, or nullptr (all seq_k)
   int Dv;               // head_dim (<= the kernel's D; a multiple of 8)

@@ -660,11 +660,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 // mask[b, q0 : q0 + qpt, nt*BN : nt*BN + BN].  Each thread owns a 16-byte
 // column piece and reads it down the tile's rows (one 16-byte load per row
 // when the rows are 16-byte aligned); the BN / 16 threads of a key tile then
-// combine their flags with warp shuffles.
+// combine their flags with warp shuffles.  bounds[b][mt] = the first key tile
+// not all hidden and one past the last (0, 0 when every tile is hidden), so
+// that the prefill kernels never walk the hidden tiles at either end.
 __global__ void __launch_bounds__(128)
     gqa_mask_summary_kernel(const uint8_t* __restrict__ mask, int64_t ms0, int64_t ms1,
-                            uint8_t* __restrict__ summary, int Sq, int Sk, int qpt, int m_tiles,
-                            int n_tiles, int BN, int vec) {
+                            uint8_t* __restrict__ summary, int32_t* __restrict__ bounds, int Sq,
+                            int Sk, int qpt, int m_tiles, int n_tiles, int BN, int vec) {
+  __shared__ int lo_s, hi_s;
+  if (threadIdx.x == 0) {
+    lo_s = n_tiles;
+    hi_s = 0;
+  }
+  __syncthreads();
   const int mt = blockIdx.x, b = blockIdx.y;
   const int q0 = mt * qpt;
   const int qn = min(qpt, Sq - q0);
@@ -698,9 +706,20 @@ __global__ void __launch_bounds__(128)
       any1 |= __shfl_xor_sync(0xffffffffu, any1, o) != 0;
       any0 |= __shfl_xor_sync(0xffffffffu, any0, o) != 0;
     }
-    if (c < pieces && threadIdx.x % per_tile == 0)
+    if (c < pieces && threadIdx.x % per_tile == 0) {
       summary[(static_cast<int64_t>(b) * m_tiles + mt) * n_tiles + c / per_tile] =
           static_cast<uint8_t>(any1 ? (any0 ? 1 : 2) : 0);
+      if (any1) {
+        atomicMin(&lo_s, c / per_tile);
+        atomicMax(&hi_s, c / per_tile + 1);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && bounds != nullptr) {
+    int32_t* bd = bounds + (static_cast<int64_t>(b) * m_tiles + mt) * 2;
+    bd[0] = hi_s > lo_s ? lo_s : 0;
+    bd[1] = hi_s > lo_s ? hi_s : 0;
   }
 }
 
@@ -732,7 +751,7 @@ int launch_mask_summary(const PrefillShape& s, const PrefillArgs& a, cudaStream_
   const bool vec = (reinterpret_cast<uintptr_t>(a.mask) & 15u) == 0 && a.ms[0] % 16 == 0 &&
                    a.ms[1] % 16 == 0;
   gqa_mask_summary_kernel<<<dim3(s.m_tiles, a.B), 128, 0, stream>>>(
-      a.mask, a.ms[0], a.ms[1], a.summary, a.Sq, a.Sk, s.qpt, s.m_tiles, s.n_tiles, BN,
+      a.mask, a.ms[0], a.ms[1], a.summary, a.bounds, a.Sq, a.Sk, s.qpt, s.m_tiles, s.n_tiles, BN,
       vec ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
@@ -763,6 +782,11 @@ PrefillShape plan_prefill(const gqa_problem& p, int sm_count) {
   }
   s.summary_offset = kScratchOffset;
   s.workspace_end = s.summary_offset + (p.has_mask ? p.batch * s.m_tiles * s.n_tiles : 0);
+  s.bounds_offset = -1;
+  if (p.has_mask) {
+    s.bounds_offset = ((s.workspace_end + 255) / 256) * 256;
+    s.workspace_end = s.bounds_offset + p.batch * s.m_tiles * 8;
+  }
   s.order_offset = -1;
   // With a mask or per-sequence lengths the items' costs vary (with each
   // entry's length): the two-tile kernel takes them heaviest first, in an

@@ -118,6 +118,13 @@ __device__ __forceinline__ PPTile pp_tile(int64_t x, int X, const PrefillArgs& a
   } else {
     t.pr.nt_beg = static_cast<int>(t.sl.key_lo / BN);
     t.pr.nt_end = min(n_tiles, static_cast<int>((t.sl.key_hi + BN - 1) / BN));
+    if (a.bounds != nullptr) {  // with a mask: drop the all-hidden tiles at either end
+      const int2 bd = *reinterpret_cast<const int2*>(a.bounds + (static_cast<int64_t>(t.pr.b) *
+                                                                 m_tiles + mt) * 2);
+      t.pr.nt_beg = max(t.pr.nt_beg, bd.x);
+      t.pr.nt_end = min(t.pr.nt_end, bd.y);
+      if (t.pr.nt_end <= t.pr.nt_beg) t.pr.nt_beg = t.pr.nt_end = 0;
+    }
   }
   return t;
 }

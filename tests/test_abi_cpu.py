@@ -262,11 +262,13 @@ def test_workspace_layout_keeps_counters_apart(gqa):
     assert rc == 0 and dec.workspace_bytes > region and dec.launches == 1
     rc, pre = _rc(gqa, _p(gqa, B=2, Hq=8, Hkv=2, Sq=300, Sk=300, mask=True))
     # after it: the tile classes [B][m_tiles][n_tiles], then (256-aligned) the
-    # item order of the two-tile kernel, one int32 per pair of query tiles
+    # key-tile bounds of every query tile (two int32), then the item order of
+    # the two-tile kernel, one int32 per pair of query tiles
     # (g = 4: 32 query positions per tile, 10 query tiles, 3 key tiles)
     classes_end = (region + 2 * 10 * 3 + 255) // 256 * 256
+    bounds_end = (classes_end + 2 * 10 * 8 + 255) // 256 * 256
     assert rc == 0 and pre.launches == 3
-    assert pre.workspace_bytes == (classes_end + 2 * 2 * 5 * 4 + 255) // 256 * 256
+    assert pre.workspace_bytes == (bounds_end + 2 * 2 * 5 * 4 + 255) // 256 * 256
     rc, huge = _rc(gqa, _p(gqa, B=2100, Hq=32, Hkv=8, Sq=1, Sk=100))
     assert rc == 0 and huge.launches == 2 and huge.workspace_bytes > region + 2100 * 8 * 4
 
