@@ -663,9 +663,12 @@ __global__ void __launch_bounds__(1024)
     const PPTile qa = pp_tile(x, 0, a, m_tiles, qpt, n_tiles);
     const PPTile qb = pp_tile(x, 1, a, m_tiles, qpt, n_tiles);
     int n = 0;
-    if (!a.has_mask) {
-      // Every key tile of a query tile's range is computed: the union of the
-      // two ranges (consecutive query tiles: they overlap or touch).
+    if (!a.has_mask || a.bounds != nullptr) {
+      // The union of the two query tiles' key-tile ranges (consecutive query
+      // tiles: they overlap or touch).  Without a mask every tile of a range
+      // is computed; with one the ranges are already trimmed to the first and
+      // last tiles that are not all hidden (tiles hidden in between count too:
+      // the order needs a cost, not the exact work).
       const int lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
                          qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
       const int hi = max(qa.pr.nt_end, qb.pr.nt_end);
