@@ -679,35 +679,64 @@ def trace_summary(words, grid, launches, kv_bytes_per_unit):
 def run_trace(args):
     """Per-CTA phase trace of one decode workload: one CUDA graph of
     consecutive launches with the trace buffer set, replayed a few times; the
-    summary of the last replay is printed as one JSON line."""
+    summary of the last replay is printed as one JSON line.  Ragged and paged
+    caches are traced without the append step (the lengths stay fixed)."""
     import torch
+    import numpy as np
     import grouped_query_attention_fwd_b200 as gqa
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     cfg = WORKLOADS[args.trace]
-    if cfg["Sq"] != 1 or "lens" in cfg:
-        raise SystemExit("--trace takes a contiguous single-query decode workload")
+    if cfg["Sq"] != 1 or cfg.get("append"):
+        raise SystemExit("--trace takes a single-query decode workload without an append")
     q, k, v, _ = _host_inputs(cfg, torch)
     qd = q.to(dev)
-    kv_bytes = 2 * k.numel() * 2
+    B, Hkv, Sk, D = cfg["B"], cfg["Hkv"], cfg["Sk"], cfg["D"]
+    lens = table = None
+    if "lens" in cfg:
+        lo, hi = cfg["lens"]
+        lens0 = synth.uniform_int(cfg["seed"], synth.STREAM_MASK, B, lo, hi).astype(np.int32)
+        lens = torch.from_numpy(lens0).to(dev)
+        kv_bytes = int(lens0.sum()) * Hkv * D * 2 * 2
+    else:
+        kv_bytes = 2 * k.numel() * 2
     copies = max(3, math.ceil(3 * L2_BYTES / kv_bytes))
     ks = [k.to(dev) for _ in range(copies)]
     vs = [v.to(dev) for _ in range(copies)]
+    tables = [None] * copies
+    ps = cfg.get("page")
+    if ps:  # every (sequence, page) of the cache at a random slot of a pool
+        per_seq = Sk // ps
+        gen = torch.Generator().manual_seed(cfg["seed"])
+        for i in range(copies):
+            perm = torch.randperm(B * per_seq, generator=gen)
+            inv = torch.empty_like(perm)
+            inv[perm] = torch.arange(B * per_seq)
+
+            def pool(x):
+                return x.view(B, Hkv, per_seq, ps, D).permute(0, 2, 1, 3, 4).reshape(
+                    B * per_seq, Hkv, ps, D)[perm.to(dev)].contiguous()
+            ks[i], vs[i] = pool(ks[i]), pool(vs[i])
+            tables[i] = inv.view(B, per_seq).to(torch.int32).to(dev)
     out = torch.empty(qd.shape, dtype=qd.dtype, device=dev)
-    plan = gqa.query(qd, ks[0], vs[0])
+    plan = gqa.query(qd, ks[0], vs[0], kv_lens=lens, block_table=tables[0])
     ws = gqa.workspace_for(dev, plan["workspace_bytes"])
     stream = torch.cuda.current_stream(dev)
     launches = 32
     grid = plan["grid"]
+
+    def call(i):
+        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws, kv_lens=lens,
+                    block_table=tables[i % copies])
     buf = torch.zeros(launches * grid * 16, dtype=torch.int64, device=dev)
     for i in range(6):
-        gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+        call(i)
     torch.cuda.synchronize()
     gqa.debug_decode_trace(buf)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(launches):
-            gqa.forward(qd, ks[i % copies], vs[i % copies], out=out, workspace=ws)
+            call(i)
     gqa.debug_decode_trace(None)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(3):
@@ -720,14 +749,15 @@ def run_trace(args):
     st = gqa.device_status(ws)
     if st != 0:
         raise RuntimeError("device status after tracing: %s" % gqa.status_string(st))
-    unit_bytes = 2 * 128 * cfg["D"] * 2
+    unit_bytes = 2 * 128 * D * 2
     raw = buf.cpu().numpy()
     if getattr(args, "trace_out", None):
         np.save(args.trace_out, raw.reshape(launches, grid, 16))
     summ = trace_summary(raw, grid, launches, unit_bytes)
     ms = e0.elapsed_time(e1) / launches
     summ.update({"trace_workload": cfg["name"], "launch_ms_graph": round(ms, 5),
-                 "gbs_algorithmic": round(plan["algorithmic_bytes"] / (ms / 1e3) / 1e9, 1)})
+                 "gbs_algorithmic": round(plan["algorithmic_bytes"] / (ms / 1e3) / 1e9, 1)
+                 if lens is None else round((kv_bytes + 2 * qd.numel() * 2) / (ms / 1e3) / 1e9, 1)})
     print(json.dumps(summ), flush=True)
     del g
 
