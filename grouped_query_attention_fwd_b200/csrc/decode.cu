@@ -194,6 +194,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // The tensor maps are kernel parameters: fetch them before the wait.
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
+    // Without lengths or a block table the range and its first tiles follow
+    // from the arguments alone: start their K and V towards L2 before the
+    // grid dependency resolves.
+    if (!ragged && a.bt == nullptr) {
+      const int P = static_cast<int>(gridDim.x) < units ? static_cast<int>(gridDim.x) : units;
+      if (static_cast<int>(blockIdx.x) < P) {
+        const int ub = range_start(blockIdx.x, units, P);
+        const int ue = range_start(blockIdx.x + 1, units, P);
+        const KeyRange kr =
+            decode_key_range(a.Sk, a.Sk, a.Sq, a.causal, a.causal_offset, a.window);
+        const int per_b = gpb * tiles_per_group;
+        for (int u = ub; u < ub + 2 && u < ue; ++u) {
+          const int b = u / per_b, r = u - b * per_b, gi = r / tiles_per_group;
+          const int kv = gi / passes, key0 = (r - gi * tiles_per_group + kr.t0) * KT;
+#pragma unroll
+          for (int c = 0; c < CHUNKS; ++c) {
+            tma_prefetch_4d(&tmk, c * 64, key0, kv, b);
+            tma_prefetch_4d(&tmv, c * 64, key0, kv, b);
+          }
+        }
+      }
+    }
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {

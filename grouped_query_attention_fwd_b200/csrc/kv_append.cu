@@ -17,6 +17,10 @@ namespace {
 
 template <typename V>
 __global__ void __launch_bounds__(256) gqa_kv_append_kernel(const AppendArgs a) {
+  // A decode launched after this one as a programmatic dependent may start its
+  // prologue now; it waits for this launch to complete before reading the
+  // lengths and rows written here.
+  griddep_launch_dependents();
   const int per_row = a.row_bytes / static_cast<int>(sizeof(V));
   const int64_t per_tensor = static_cast<int64_t>(a.B) * a.H * a.n_new * per_row;
   const int64_t total = 2 * per_tensor;

@@ -208,6 +208,17 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Prefetch of a 4-D tile into L2 (no copy into shared memory, no completion):
+// L2 is where later writes land, so a prefetch cannot serve stale data.
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 // 4-D tiled tensor load global -> shared, completion counted on `bar`.
 // The innermost coordinate c0 must keep c0 * sizeof(elem) a multiple of 16 B.
 __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map,
