@@ -160,9 +160,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   uint64_t* v_full = k_empty + S;       // [stage] V tile landed
   uint64_t* v_empty = v_full + S;       // [stage] the PVs reading it done
   uint64_t* s_full = v_empty + S;       // [X] S_X done (and every earlier PV_X)
-  uint64_t* p_full = s_full + 2;        // [X] P_X written (one arrival per warpgroup)
+  uint64_t* p_full = s_full + 2;        // [X] P_X written (one arrival per softmax warp)
   uint64_t* o_final = p_full + 2;       // [X] the item's last PV_X done
-  uint64_t* o_free = o_final + 2;       // [X] O_X read by the epilogue
+  uint64_t* o_free = o_final + 2;       // [X] O_X read by the epilogue (one arrival per warp)
   uint64_t* mma_done = o_free + 2;      // every MMA done
   uint64_t* v_fix = mma_done + 1;       // [stage] (KVX): the V rows past the length zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -177,9 +177,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 1);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&o_final[i], 1);
-      mbar_init(&o_free[i], 1);
+      mbar_init(&o_free[i], 4);  // one arrival per softmax warp
     }
     for (int i = 0; i < S; ++i) {
       mbar_init(&k_full[i], 1);
@@ -487,8 +487,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         const int cls = tile_class(a, pr, me.sl, t, m_tiles, n_tiles);
         if (cls == 0) continue;
         // okt: warp-uniform, so that every TMEM access it guards is made by
-        // the whole warp; the warpgroup meets once per tile below and leaves
-        // the loop together.
+        // the whole warp.  The softmax warps meet no barrier of their own: each
+        // signals the MMA thread per warp, and a warp that gives up leaves
+        // while the others stop at their next wait, which sees the abort flag.
         const bool okt = __all_sync(0xffffffffu, mbar_wait_hot(&s_full[X], J & 1u, abort_flag,
                                                                a.err, kErrPrefillWait));
         if (okt) {
@@ -533,25 +534,29 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           const float ref = exp_ref(m_ref);
           const float sc = fast ? a.scale_log2 : 1.f;
-          // P = 2^(t - ref) as 16-bit pairs over the first 64 columns of S_X.
-          float lp[8];
+          // P = 2^(t - ref) as 16-bit pairs over the first 64 columns of S_X;
+          // the scaling and the row sum take two columns per instruction.
+          const uint64_t sc2 = f2_pack(sc, sc), nref2 = f2_pack(-ref, -ref);
+          uint64_t lp[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) lp[e] = 0.f;
+          for (int e = 0; e < 4; ++e) lp[e] = 0;
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const int c0 = c * 32 + 2 * e, c1 = c0 + 1;
-              const float p0 = fast_exp2(fmaf(__uint_as_float(r[c0]), sc, -ref));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(r[c1]), sc, -ref));
-              lp[c0 & 7] += p0;
-              lp[c1 & 7] += p1;
+              const int c0 = c * 32 + 2 * e;
+              const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[c0]), __uint_as_float(r[c0 + 1])),
+                                        sc2, nref2);
+              const float p0 = fast_exp2(f2_lo(x));
+              const float p1 = fast_exp2(f2_hi(x));
+              lp[e & 3] = f2_add(lp[e & 3], f2_pack(p0, p1));
               pk[e] = pack_p<F16>(p0, p1);
             }
             tmem_st16(s_col + c * 16, pk);
           }
-          l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+          l += ((f2_lo(lp[0]) + f2_hi(lp[0])) + (f2_lo(lp[1]) + f2_hi(lp[1]))) +
+               ((f2_lo(lp[2]) + f2_hi(lp[2])) + (f2_lo(lp[3]) + f2_hi(lp[3])));
           if (__any_sync(0xffffffffu, o_live)) {
             // O_X holds the earlier tiles' P V with the old reference; the
             // previous PV_X has completed (S_X follows it) and the next waits
@@ -571,12 +576,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        // The four warps of the warpgroup have written P_X (or given up).
-        if (!bar_and(1 + X, 128, okt)) {
+        // Each warp reports its 32 rows of P_X on its own: a named barrier of
+        // the warpgroup here would sit on every tile's critical path.  A warp
+        // that gave up leaves; the others see the abort flag in their next wait.
+        if (!okt) {
           ok = false;
           break;
         }
-        if ((threadIdx.x & 127) == 0) mbar_arrive(&p_full[X]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[X]);
         ++J;
         ++nloc;
       }
@@ -599,12 +607,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           tmem_ld32(o_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
         tmem_ld_wait();
         tc_fence_before();
-        if (!bar_and(1 + X, 128, oke)) {
+        if (!oke) {
           ok = false;
           break;
         }
-        // O_X is in registers: the next item's first PV_X may overwrite it.
-        if ((threadIdx.x & 127) == 0) mbar_arrive(&o_free[X]);
+        // This warp's rows of O_X are in registers: once all four warps have
+        // said so, the next item's first PV_X may overwrite O_X.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[X]);
         if (row_valid) {
 #pragma unroll
           for (int v8 = 0; v8 < D / 8; ++v8) {
@@ -629,11 +639,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             *reinterpret_cast<uint4*>(orow + d) = make_uint4(nn, nn, nn, nn);
         }
         tc_fence_before();
-        if (!bar_and(1 + X, 128, oke)) {
+        if (!oke) {
           ok = false;
           break;
         }
-        if ((threadIdx.x & 127) == 0) mbar_arrive(&o_free[X]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[X]);
       }
     }
   }
