@@ -17,7 +17,7 @@
 // One softmax warpgroup per query tile, one thread per row holding all 128
 // keys of its S row: the maximum and the row sum need no exchange between
 // threads, and while warpgroup A turns S_A into P_A the tensor core computes
-// tile B's products, and the other way round.  The MMA thread issues, per
+// tile B's products, and the other way round.  The MMA warp issues, per
 // key tile u:  PV_A(u), QK_A(u+1), PV_B(u), QK_B(u+1).  tcgen05 operations of
 // one thread execute in issue order, so QK_X(u+1), which overwrites P_X(u),
 // follows PV_X(u), and the commit that signals S_X(u+1) also means that
@@ -28,7 +28,7 @@
 //   warps 0-3  softmax, O rescale and epilogue of tile A (thread t: row t)
 //   warps 4-7  the same for tile B
 //   warp 8     TMA producer of Q tiles and K tiles
-//   warp 9     TMEM allocator and single-thread MMA issuer
+//   warp 9     TMEM allocator and MMA warp (one elected lane issues)
 //   warp 10    TMA producer of V tiles (warp 11 idles)
 // Per-sequence lengths and paged caches (the KVX instances): an item's key
 // range ends at its entry's length; the one key tile that reaches past it has
@@ -80,7 +80,7 @@ struct PPLayout {
   // s_full[2], p_full[2], o_final[2], o_free[2], mma_done, v_fix[S]
   static constexpr int kNumBars = 4 + 4 * kStages + 8 + 1 + kStages;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSchedOff = kMiscOff + 16;  // the MMA thread's key-tile list of an item
+  static constexpr int kSchedOff = kMiscOff + 16;  // the MMA warp's key-tile list of an item
   static constexpr int kBytes = kSchedOff + kMaxPPTiles + 1024;  // + alignment slack
   // TMEM columns of S_X and O_X (X = 0: tile A, 1: tile B).
   __device__ static constexpr uint32_t s_col(int X) { return static_cast<uint32_t>(X) * 128u; }
@@ -320,8 +320,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int X = 0; X < 2; ++X)
           if (nq[X] > 0) mbar_wait_drain(&q_full[X], (nq[X] - 1) & 1u);
       }
-    } else if (warp == kWarpMMA && lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpMMA) {
+      // ------------------------------------------------------------ MMA warp
+      // The whole warp walks the schedule and takes every wait (made
+      // warp-uniform by a vote); one elected lane issues the MMAs and their
+      // commits.  A lone issuing thread in a diverged warp leaves the tensor
+      // core idle ~200 cycles at each wait or data-dependent branch between
+      // MMA groups; a converged warp does not.  elect.sync picks the lowest
+      // lane of a full warp, so one thread issues every tcgen05 operation
+      // and they execute in issue order.
       constexpr uint32_t idesc_qk = F16 ? idesc_f16_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = F16 ? idesc_f16_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
       const uint64_t dq0 = kmajor_desc(smem_u32(smem + L::kQOff));
@@ -332,21 +339,34 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       uint32_t fix_parity = 0;  // bit s (KVX): parity of the next v_fix[s] phase
       int64_t it = 0;
       bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait_hot(bar, parity, abort_flag, a.err, kErrPrefillWait));
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+      };
       auto qk = [&](int X, uint32_t idx) {
         const uint64_t dq = dq0 + ((X * L::kTile) >> 4);
         const uint64_t dk = dk0 + (((idx % S) * L::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          tc_mma_ss(tmem + L::s_col(X), dq + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4),
-                    dk + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4), idesc_qk, k > 0 ? 1u : 0u);
-        tc_commit(&s_full[X]);
+          for (int k = 0; k < D / 16; ++k)
+            tc_mma_ss(tmem + L::s_col(X), dq + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4),
+                      dk + (((k >> 2) * L::kChunk + (k & 3) * 32) >> 4), idesc_qk, k > 0 ? 1u : 0u);
+          tc_commit(&s_full[X]);
+        }
+        __syncwarp();
       };
       auto pv = [&](int X, uint32_t idx, bool first) {
         const uint64_t dv = dv0 + (((idx % S) * L::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          tc_mma_ts(tmem + L::o_col(X), tmem + L::s_col(X) + k * 8, dv + ((k * 16 * 128) >> 4),
-                    idesc_pv, (!first || k > 0) ? 1u : 0u);
+          for (int k = 0; k < BN / 16; ++k)
+            tc_mma_ts(tmem + L::o_col(X), tmem + L::s_col(X) + k * 8, dv + ((k * 16 * 128) >> 4),
+                      idesc_pv, (!first || k > 0) ? 1u : 0u);
+        }
+        __syncwarp();
       };
       for (int64_t x = snake(0, blockIdx.x, gridDim.x); x < items && ok;
            ++it, x = snake(it, blockIdx.x, gridDim.x)) {
@@ -356,36 +376,38 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         // The item's key tiles that some tile works on, in order, one byte
         // each in shared memory (bit X: tile X computes it); tile classes may
         // read mask summaries from global memory, so they are taken once per
-        // item, off the per-tile path.
+        // item, 32 key tiles at a time across the warp, off the per-tile path.
         const int t_lo = min(qa.pr.nt_end > qa.pr.nt_beg ? qa.pr.nt_beg : 1 << 30,
                              qb.pr.nt_end > qb.pr.nt_beg ? qb.pr.nt_beg : 1 << 30);
         const int t_hi = max(qa.pr.nt_end, qb.pr.nt_end);
         int n = 0, nX[2] = {0, 0};
         int t_last = -1;  // the last key tile computed
-        for (int t = t_lo; t < t_hi; ++t) {
-          const uint32_t f = (pp_class(qa, t, a, m_tiles, n_tiles) != 0 ? 1u : 0u) |
-                             (pp_class(qb, t, a, m_tiles, n_tiles) != 0 ? 2u : 0u);
-          if (f != 0u) {
-            sched[n++] = static_cast<uint8_t>(f);
-            nX[0] += f & 1u;
-            nX[1] += f >> 1;
-            t_last = t;
-          }
+        for (int t0 = t_lo; t0 < t_hi; t0 += 32) {
+          const int t = t0 + lane;
+          uint32_t f = 0;
+          if (t < t_hi)
+            f = (pp_class(qa, t, a, m_tiles, n_tiles) != 0 ? 1u : 0u) |
+                (pp_class(qb, t, a, m_tiles, n_tiles) != 0 ? 2u : 0u);
+          const uint32_t any = __ballot_sync(0xffffffffu, f != 0u);
+          if (f != 0u) sched[n + __popc(any & ((1u << lane) - 1u))] = static_cast<uint8_t>(f);
+          n += __popc(any);
+          nX[0] += __popc(__ballot_sync(0xffffffffu, (f & 1u) != 0u));
+          nX[1] += __popc(__ballot_sync(0xffffffffu, (f & 2u) != 0u));
+          if (any != 0u) t_last = t0 + 31 - __clz(any);
         }
+        __syncwarp();  // sched written by every lane, read by every lane below
         // That tile reaches past the entry's length: its V rows there are
         // zeroed by the V producer before its PVs.
         const bool last_fix = KVX && n > 0 && (static_cast<int64_t>(t_last) + 1) * BN > qa.pr.len;
 #pragma unroll
         for (int X = 0; X < 2; ++X)
-          if (ok)
-            ok = mbar_wait_hot(&q_full[X], static_cast<uint32_t>(it & 1), abort_flag, a.err,
-                               kErrPrefillWait);
+          if (ok) ok = wait(&q_full[X], static_cast<uint32_t>(it & 1));
         if (!ok) break;
         tc_fence_after();
         int qkX[2] = {0, 0};  // QK_X / PV_X issued for this item
         int pvX[2] = {0, 0};
         if (n > 0) {  // the first key tile: its QKs
-          ok = mbar_wait_hot(&k_full[kt % S], (kt / S) & 1u, abort_flag, a.err, kErrPrefillWait);
+          ok = wait(&k_full[kt % S], (kt / S) & 1u);
           if (!ok) break;
           tc_fence_after();
           const uint32_t f = sched[0];
@@ -393,20 +415,19 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           for (int X = 0; X < 2; ++X)
             if ((f >> X) & 1u) {
               qk(X, kt);
-              if (++qkX[X] == nX[X]) tc_commit(&q_empty[X]);
+              if (++qkX[X] == nX[X]) commit(&q_empty[X]);
             }
-          tc_commit(&k_empty[kt % S]);
+          commit(&k_empty[kt % S]);
         }
         for (int i = 0; i < n && ok; ++i) {
           // Per key tile: PV_A(i), QK_A(i+1), PV_B(i), QK_B(i+1).
           const uint32_t f = sched[i];
           const uint32_t fn = i + 1 < n ? sched[i + 1] : 0u;
           const uint32_t cur = kt + static_cast<uint32_t>(i), nxt = cur + 1;
-          ok = mbar_wait_hot(&v_full[cur % S], (cur / S) & 1u, abort_flag, a.err, kErrPrefillWait);
+          ok = wait(&v_full[cur % S], (cur / S) & 1u);
           if (ok && last_fix && i == n - 1) {
             const uint32_t sf = cur % S;
-            ok = mbar_wait_hot(&v_fix[sf], (fix_parity >> sf) & 1u, abort_flag, a.err,
-                               kErrPrefillWait);
+            ok = wait(&v_fix[sf], (fix_parity >> sf) & 1u);
             fix_parity ^= 1u << sf;
           }
           if (!ok) break;
@@ -415,31 +436,29 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           for (int X = 0; X < 2; ++X) {
             if (!ok) break;
             if ((f >> X) & 1u) {
-              ok = mbar_wait_hot(&p_full[X], np[X] & 1u, abort_flag, a.err, kErrPrefillWait);
+              ok = wait(&p_full[X], np[X] & 1u);
               if (ok && pvX[X] == 0 && it > 0)  // O_X still holds the last item's result
-                ok = mbar_wait_hot(&o_free[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
-                                   a.err, kErrPrefillWait);
+                ok = wait(&o_free[X], static_cast<uint32_t>((it - 1) & 1));
               if (!ok) break;
               tc_fence_after();
               pv(X, cur, pvX[X] == 0);
               ++np[X];
-              if (++pvX[X] == nX[X]) tc_commit(&o_final[X]);
+              if (++pvX[X] == nX[X]) commit(&o_final[X]);
             }
             if ((fn >> X) & 1u) {
               if (!k_ready) {
-                ok = mbar_wait_hot(&k_full[nxt % S], (nxt / S) & 1u, abort_flag, a.err,
-                                   kErrPrefillWait);
+                ok = wait(&k_full[nxt % S], (nxt / S) & 1u);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
               }
               qk(X, nxt);
-              if (++qkX[X] == nX[X]) tc_commit(&q_empty[X]);
+              if (++qkX[X] == nX[X]) commit(&q_empty[X]);
             }
           }
           if (!ok) break;
-          tc_commit(&v_empty[cur % S]);          // V(i): its PVs are issued
-          if (fn != 0u) tc_commit(&k_empty[nxt % S]);  // K(i+1): its QKs are issued
+          commit(&v_empty[cur % S]);          // V(i): its PVs are issued
+          if (fn != 0u) commit(&k_empty[nxt % S]);  // K(i+1): its QKs are issued
         }
         if (!ok) break;
         kt += static_cast<uint32_t>(n);
@@ -448,14 +467,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
         for (int X = 0; X < 2; ++X)
           if (ok && nX[X] == 0) {
-            tc_commit(&q_empty[X]);
-            if (it > 0)
-              ok = mbar_wait_hot(&o_free[X], static_cast<uint32_t>((it - 1) & 1), abort_flag,
-                                 a.err, kErrPrefillWait);
-            tc_commit(&o_final[X]);
+            commit(&q_empty[X]);
+            if (it > 0) ok = wait(&o_free[X], static_cast<uint32_t>((it - 1) & 1));
+            commit(&o_final[X]);
           }
+        __syncwarp();  // the next item's schedule overwrites sched
       }
-      tc_commit(mma_done);
+      commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
   } else {
@@ -488,7 +506,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         if (cls == 0) continue;
         // okt: warp-uniform, so that every TMEM access it guards is made by
         // the whole warp.  The softmax warps meet no barrier of their own: each
-        // signals the MMA thread per warp, and a warp that gives up leaves
+        // signals the MMA warp per warp, and a warp that gives up leaves
         // while the others stop at their next wait, which sees the abort flag.
         const bool okt = __all_sync(0xffffffffu, mbar_wait_hot(&s_full[X], J & 1u, abort_flag,
                                                                a.err, kErrPrefillWait));
@@ -649,7 +667,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
   }
 
-  // Every role is done with TMEM (the MMA thread has seen its last MMA
+  // Every role is done with TMEM (the MMA warp has seen its last MMA
   // complete) before it is freed.
   tc_fence_before();
   __syncthreads();
