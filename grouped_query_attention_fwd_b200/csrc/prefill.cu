@@ -319,8 +319,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
     }
   } else if (warp == kWarpMMA) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------- MMA warp
+    // The whole warp walks the work and takes every wait (made warp-uniform
+    // by a vote); one elect.sync lane -- lane 0 of the full warp, so always
+    // the same thread -- issues the copies, MMAs and commits.  A lone issuing
+    // lane in a diverged warp leaves the tensor core idle for a while at each
+    // wait or data-dependent branch between MMA groups; a converged warp does
+    // not.
+    {
       constexpr uint32_t idesc_qk = F16 ? idesc_f16_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = F16 ? idesc_f16_f32(BM, D, 0, 1) : idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t q_base = smem_u32(smem + L::kQOff);
@@ -335,45 +341,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t fix_parity = 0;  // bit s: parity of the next v_fix[s] phase
       int64_t it = 0;
       bool ok = true;
-      // This thread issues every MMA of the CTA, one dependent instruction
-      // every few cycles: its path per tile is kept to the waits, the
-      // MMAs and the commits.
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait_hot(bar, parity, abort_flag, a.err, kErrPrefillWait));
+      };
 
       // S(J & 1) = Q K(J)^T; the K stage is released when the MMA completes.
       auto issue_qk = [&](uint32_t J) -> bool {
         const uint32_t s = J % kKStages;
-        if (!mbar_wait_hot(&k_full[s], (J / kKStages) & 1u, abort_flag, a.err, kErrPrefillWait))
-          return false;
+        if (!wait(&k_full[s], (J / kKStages) & 1u)) return false;
         tc_fence_after();
         const uint64_t dk = dk0 + s * kStageStep;
         const uint32_t d_s = tmem + L::kSCol + (J & 1u) * BN;
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          tc_mma_ts(d_s, t_q + ks * 8, dk + (((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4),
-                    idesc_qk, ks > 0 ? 1u : 0u);
-        tc_commit(&s_full[J & 1u]);
-        tc_commit(&k_empty[s]);
+          for (int ks = 0; ks < D / 16; ++ks)
+            tc_mma_ts(d_s, t_q + ks * 8, dk + (((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4),
+                      idesc_qk, ks > 0 ? 1u : 0u);
+          tc_commit(&s_full[J & 1u]);
+          tc_commit(&k_empty[s]);
+        }
+        __syncwarp();
         return true;
       };
       // O (+)= P(J) V(J); `first`: the item's first PV overwrites O.
       auto issue_pv = [&](uint32_t J, bool first) -> bool {
         const uint32_t s = J % kVStages;
-        if (!mbar_wait_hot(&p_full[J & 1u], (J >> 1) & 1u, abort_flag, a.err, kErrPrefillWait) ||
-            !mbar_wait_hot(&v_full[s], (J / kVStages) & 1u, abort_flag, a.err, kErrPrefillWait))
+        if (!wait(&p_full[J & 1u], (J >> 1) & 1u) || !wait(&v_full[s], (J / kVStages) & 1u))
           return false;
-        if (first && it > 0 &&
-            !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
-                           kErrPrefillWait))
-          return false;
+        if (first && it > 0 && !wait(o_free, static_cast<uint32_t>((it - 1) & 1))) return false;
         tc_fence_after();
         const uint64_t dv = dv0 + s * kStageStep;
         const uint32_t p_t = tmem + L::kSCol + (J & 1u) * BN;
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks)
-          tc_mma_ts(t_o, p_t + ks * 8, dv + ((ks * 16 * 128) >> 4), idesc_pv,
-                    (!first || ks > 0) ? 1u : 0u);
-        tc_commit(&o_ready[J & 1u]);
-        tc_commit(&v_empty[s]);
+          for (int ks = 0; ks < BN / 16; ++ks)
+            tc_mma_ts(t_o, p_t + ks * 8, dv + ((ks * 16 * 128) >> 4), idesc_pv,
+                      (!first || ks > 0) ? 1u : 0u);
+          tc_commit(&o_ready[J & 1u]);
+          tc_commit(&v_empty[s]);
+        }
+        __syncwarp();
         return true;
       };
 
@@ -386,28 +393,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // The last of them reaches past the entry's length: its V rows there
         // are zeroed by the V producer before its PV.
         bool last_fix = KVX && n > 0 && static_cast<int64_t>(pr.nt_end) * BN > pr.len;
-        if (a.has_mask) {
+        if (a.has_mask) {  // classes taken 32 key tiles at a time across the warp
           const Slot me = slot_of(pr, a, qpt);
           n = 0;
-          for (int nt = pr.nt_beg; nt < pr.nt_end; ++nt)
-            n += tile_class(a, pr, me, nt, m_tiles, n_tiles) != 0;
+          for (int nt0 = pr.nt_beg; nt0 < pr.nt_end; nt0 += 32) {
+            const int nt = nt0 + lane;
+            n += __popc(__ballot_sync(
+                0xffffffffu, nt < pr.nt_end && tile_class(a, pr, me, nt, m_tiles, n_tiles) != 0));
+          }
           last_fix = last_fix && tile_class(a, pr, me, pr.nt_end - 1, m_tiles, n_tiles) != 0;
         }
         // Q from its landing buffer into TMEM (the A operand of every QK of
         // this query tile); the copy follows the previous tile's last QK on
         // the tensor core, and the buffer is released when the copy is done.
         const int qb = static_cast<int>(it % kQBufs);
-        if (!mbar_wait_hot(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1), abort_flag,
-                           a.err, kErrPrefillWait)) {
+        if (!wait(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t qs = q_base + qb * L::kTileBytes;
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          tc_cp_128x256b(t_q + ks * 8, kmajor_desc(qs + (ks >> 2) * L::kChunkBytes + (ks & 3) * 32));
-        tc_commit(&q_empty[qb]);
+          for (int ks = 0; ks < D / 16; ++ks)
+            tc_cp_128x256b(t_q + ks * 8,
+                           kmajor_desc(qs + (ks >> 2) * L::kChunkBytes + (ks & 3) * 32));
+          tc_commit(&q_empty[qb]);
+        }
+        __syncwarp();
         // QK runs two tiles ahead of PV: QK(0), QK(1), PV(0), QK(2), PV(1), ...
         for (int i = 0; i < 2 && i < n && ok; ++i) ok = issue_qk(Jq++);
         for (int i = 0; i < n && ok; ++i) {
@@ -415,8 +428,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // The tile reaches past the entry's length: the V producer zeroes
             // those rows once it has landed (one phase of v_fix[stage] each).
             const uint32_t s = Jp % kVStages;
-            ok = mbar_wait_hot(&v_fix[s], (fix_parity >> s) & 1u, abort_flag, a.err,
-                               kErrPrefillWait);
+            ok = wait(&v_fix[s], (fix_parity >> s) & 1u);
             fix_parity ^= 1u << s;
             if (!ok) break;
           }
@@ -425,15 +437,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (!ok) break;
         if (n == 0 && it > 0 &&  // no PV: O is left as it is, but the epilogue must be done
-            !mbar_wait_hot(o_free, static_cast<uint32_t>((it - 1) & 1), abort_flag, a.err,
-                           kErrPrefillWait)) {
+            !wait(o_free, static_cast<uint32_t>((it - 1) & 1))) {
           ok = false;
           break;
         }
-        tc_commit(o_final);
+        if (elect_one()) tc_commit(o_final);
+        __syncwarp();
       }
       // Every MMA issued so far has completed before TMEM is released.
-      tc_commit(mma_done);
+      if (elect_one()) tc_commit(mma_done);
+      __syncwarp();
       mbar_wait_drain(mma_done, 0);
     }
   }
