@@ -64,6 +64,66 @@ constexpr int kSoftmaxRegs = 192;
 static_assert(128 * kIoRegs + 256 * kSoftmaxRegs <= kPPThreads * kLaunchRegs,
               "register split must fit in the launch allocation");
 constexpr uint32_t kTmemCols = 512;
+// At head dim 64, one pair of columns in four takes its exponentials on the
+// FMA pipe (exp2_poly_x2), the others on the MUFU unit: 16 exponentials per
+// clock per SM, which the two tiles' 2 x 128 x 128 per key tile otherwise keep
+// busy for 2048 cycles, about 80% of the key tile's time at that head dim.  At
+// head dim 128 the tensor core's share is twice as large and the exponentials
+// all stay on the MUFU unit (a share on the FMA pipe was slower there), and so
+// they do in the instances with lengths or a paged cache, whose softmax has no
+// registers to spare for it.
+template <int D, bool KVX>
+__host__ __device__ constexpr bool poly_pair(int e) {
+  return D == 64 && !KVX && e % 4 == 3;
+}
+
+// 2^x for two packed fp32 lanes on the FMA pipe.  Cody and Waite style
+// reduction: n = round(x) (the low mantissa bits of x + 1.5 * 2^23), f = x - n
+// in [-1/2, 1/2]; 2^f by the degree-3 polynomial of least maximum relative
+// error on [-1/2, 1/2] (own Remez exchange fit: c3 = 5.517166853e-02,
+// c2 = 2.426111251e-01, c1 = 6.932609677e-01, c0 = 9.999280572e-01, maximum
+// relative error 7.5e-5, below the 16-bit rounding of P); 2^n by adding n to
+// the exponent field ((t's bits << 23) is n << 23: the bits of 1.5 * 2^23
+// shift out).  x is first raised to -126 (NaN kept) so that the exponent
+// cannot wrap: -inf and anything below -126 give 2^-126 instead of 0, which
+// the softmax tolerates (a row with no visible key is told by its running
+// maximum, not by its sum).  One asm block, so that the packed constants live
+// only inside it.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  uint64_t y;
+  asm("{\n\t"
+      ".reg .f32 a0, a1;\n\t"
+      ".reg .b64 xc, t, nf, f, q, k, k2;\n\t"
+      ".reg .b32 q0, q1, t0, t1;\n\t"
+      "mov.b64 {a0, a1}, %1;\n\t"
+      "max.NaN.f32 a0, a0, 0fC2FC0000;\n\t"
+      "max.NaN.f32 a1, a1, 0fC2FC0000;\n\t"
+      "mov.b64 xc, {a0, a1};\n\t"
+      "mov.b64 k, 0x4B4000004B400000;\n\t"
+      "add.rn.f32x2 t, xc, k;\n\t"
+      "mov.b64 k, 0xCB400000CB400000;\n\t"
+      "add.rn.f32x2 nf, t, k;\n\t"
+      "mov.b64 k, 0xBF800000BF800000;\n\t"
+      "fma.rn.f32x2 f, nf, k, xc;\n\t"
+      "mov.b64 k, 0x3D61FBB03D61FBB0;\n\t"
+      "mov.b64 k2, 0x3E786F0D3E786F0D;\n\t"
+      "fma.rn.f32x2 q, f, k, k2;\n\t"
+      "mov.b64 k, 0x3F31798D3F31798D;\n\t"
+      "fma.rn.f32x2 q, q, f, k;\n\t"
+      "mov.b64 k, 0x3F7FFB493F7FFB49;\n\t"
+      "fma.rn.f32x2 q, q, f, k;\n\t"
+      "mov.b64 {q0, q1}, q;\n\t"
+      "mov.b64 {t0, t1}, t;\n\t"
+      "shl.b32 t0, t0, 23;\n\t"
+      "shl.b32 t1, t1, 23;\n\t"
+      "add.u32 q0, q0, t0;\n\t"
+      "add.u32 q1, q1, t1;\n\t"
+      "mov.b64 %0, {q0, q1};\n\t"
+      "}"
+      : "=l"(y)
+      : "l"(x));
+  return y;
+}
 
 template <int D>
 struct PPLayout {
@@ -566,8 +626,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               const int c0 = c * 32 + 2 * e;
               const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[c0]), __uint_as_float(r[c0 + 1])),
                                         sc2, nref2);
-              const float p0 = fast_exp2(f2_lo(x));
-              const float p1 = fast_exp2(f2_hi(x));
+              float p0, p1;
+              if (poly_pair<D, KVX>(e)) {
+                const uint64_t pp = exp2_poly_x2(x);
+                p0 = f2_lo(pp);
+                p1 = f2_hi(pp);
+              } else {
+                p0 = fast_exp2(f2_lo(x));
+                p1 = fast_exp2(f2_hi(x));
+              }
               lp[e & 3] = f2_add(lp[e & 3], f2_pack(p0, p1));
               pk[e] = pack_p<F16>(p0, p1);
             }
@@ -615,7 +682,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       uint16_t* orow = a.out + pr.b * a.os[0] +
                        static_cast<int64_t>(pr.kv * a.g + (hh < a.g ? hh : 0)) * a.os[1] +
                        static_cast<int64_t>(q) * a.os[2];
-      const float inv_l = 1.f / l;  // l == 0: no visible key, NaN output
+      // No visible key (the running maximum never left -inf): NaN output.
+      const float inv_l = m_ref == -INFINITY ? __int_as_float(0x7fc00000) : 1.f / l;
       if (nloc > 0) {
         // (After a failed wait the values read are discarded: the output of
         // an aborted launch is undefined.)
