@@ -39,8 +39,10 @@
 //    which shortens the launch's tail.
 //  * Launched with programmatic stream serialisation: the next launch's CTAs
 //    may start, initialise their barriers and wait (griddepcontrol.wait) while
-//    this grid's last CTAs finish; nothing global is read or written before
-//    that wait.
+//    this grid's last CTAs finish; before that wait nothing global is written,
+//    and global memory is read only to place L2 prefetch hints for the first
+//    tiles of a contiguous cache (lengths read then are clamped, and read
+//    again after the wait).
 //  * Per-sequence cache lengths (kv_lens): each CTA reads the B lengths,
 //    counts the tiles every batch entry needs and prefix-sums them in shared
 //    memory, so the units -- and the cut into CTA ranges -- cover only keys
@@ -190,28 +192,76 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   auto trace = [&]() { return a.trace + blockIdx.x * kDecodeTraceWords; };
   const uint64_t t_entry = (a.trace != nullptr && threadIdx.x == 0) ? globaltimer_ns() : 0;
 
-  if (warp == NCW && lane == 0) {
+  if (warp == NCW) {
     // The tensor maps are kernel parameters: fetch them before the wait.
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-    // Without lengths or a block table the range and its first tiles follow
-    // from the arguments alone: start their K and V towards L2 before the
-    // grid dependency resolves.
-    if (!ragged && a.bt == nullptr) {
-      const int P = static_cast<int>(gridDim.x) < units ? static_cast<int>(gridDim.x) : units;
-      if (static_cast<int>(blockIdx.x) < P) {
-        const int ub = range_start(blockIdx.x, units, P);
-        const int ue = range_start(blockIdx.x + 1, units, P);
-        const KeyRange kr =
-            decode_key_range(a.Sk, a.Sk, a.Sq, a.causal, a.causal_offset, a.window);
-        const int per_b = gpb * tiles_per_group;
-        for (int u = ub; u < ub + 2 && u < ue; ++u) {
-          const int b = u / per_b, r = u - b * per_b, gi = r / tiles_per_group;
-          const int kv = gi / passes, key0 = (r - gi * tiles_per_group + kr.t0) * KT;
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+    }
+    // Contiguous caches: start the range's first two tiles towards L2 before
+    // the grid dependency resolves.  Lengths may still be being written by
+    // earlier work on the stream: they are read here only to place these
+    // prefetch hints, clamped into range (a stale one warms the wrong lines,
+    // nothing more), and read again after the wait.  (With a block table the
+    // page entries would cost a second dependent round trip before the wait,
+    // which measured slower than no hints.)
+    auto hint_len = [&](int b) -> int {
+      if (!ragged) return a.Sk;
+      const int l = __ldcg(a.lens + b);
+      return l < 0 ? 0 : (l > a.Sk ? a.Sk : l);
+    };
+    auto hint_tiles = [&](int b) -> int {  // key tiles of each group of entry b
+      return decode_key_range(hint_len(b), a.Sk, a.Sq, a.causal, a.causal_offset, a.window).tiles;
+    };
+    int total = a.bt == nullptr ? units : 0;
+    if (ragged && a.bt == nullptr) {
+      total = 0;
+      for (int b0 = 0; b0 < a.B; b0 += 32)
+        total += __reduce_add_sync(0xffffffffu, b0 + lane < a.B ? gpb * hint_tiles(b0 + lane) : 0);
+    }
+    const int P = static_cast<int>(gridDim.x) < total ? static_cast<int>(gridDim.x) : total;
+    if (static_cast<int>(blockIdx.x) < P) {
+      const int ub = range_start(blockIdx.x, total, P);
+      const int ue = range_start(blockIdx.x + 1, total, P);
+      for (int u = ub; u < ub + 2 && u < ue; ++u) {
+        int b = -1, beg = 0;  // entry of unit u and its first unit
+        if (!ragged) {
+          b = u / (gpb * tiles_per_group);
+          beg = b * gpb * tiles_per_group;
+        } else {
+          int carry = 0;
+          for (int b0 = 0; b0 < a.B && b < 0; b0 += 32) {
+            const int bb = b0 + lane;
+            const int v = bb < a.B ? gpb * hint_tiles(bb) : 0;
+            int incl = v;
 #pragma unroll
-          for (int c = 0; c < CHUNKS; ++c) {
-            tma_prefetch_4d(&tmk, c * 64, key0, kv, b);
-            tma_prefetch_4d(&tmv, c * 64, key0, kv, b);
+            for (int o = 1; o < 32; o <<= 1) {
+              const int n = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += n;
+            }
+            const uint32_t hit = __ballot_sync(0xffffffffu, bb < a.B && carry + incl > u);
+            if (hit != 0u) {
+              const int l = __ffs(hit) - 1;
+              b = b0 + l;
+              beg = carry + __shfl_sync(0xffffffffu, incl - v, l);
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+          }
+          if (b < 0) break;
+        }
+        const int len = hint_len(b);
+        const KeyRange kr = decode_key_range(len, a.Sk, a.Sq, a.causal, a.causal_offset, a.window);
+        const int tpg = ragged ? kr.tiles : tiles_per_group;
+        if (tpg <= 0) break;
+        const int r = u - beg, gi = r / tpg;
+        const int kv = gi / passes, key0 = (r - gi * tpg + kr.t0) * KT;
+        if (lane == 0) {
+          if (a.bt == nullptr) {
+#pragma unroll
+            for (int c = 0; c < CHUNKS; ++c) {
+              tma_prefetch_4d(&tmk, c * 64, key0, kv, b);
+              tma_prefetch_4d(&tmv, c * 64, key0, kv, b);
+            }
           }
         }
       }
@@ -232,8 +282,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   for (int x = threadIdx.x; x < stages * L::kQAreaBytes / 16; x += blockDim.x)
     reinterpret_cast<uint4*>(qarea)[x] = make_uint4(0u, 0u, 0u, 0u);
   if (L::kQAreaBytes > 0) fence_proxy_async_smem();  // before the bulk copies into it
-  // Everything above touches shared memory only; from here on global memory
-  // written by earlier work on the stream (lengths, caches, counters) is read.
+  // Above, only shared memory is written and global memory is read for L2
+  // hints alone; from here on global memory written by earlier work on the
+  // stream (lengths, caches, counters) is read.
   griddep_wait();
   griddep_launch_dependents();
   if (ragged) {
