@@ -22,12 +22,7 @@
 // one thread execute in issue order, so QK_X(u+1), which overwrites P_X(u),
 // follows PV_X(u), and the commit that signals S_X(u+1) also means that
 // PV_X(u) has completed: the softmax may rescale O_X as soon as it sees S_X.
-// Each K / V tile is staged once for both query tiles.  The period of a key
-// tile is one tile's chain (its PV and QK, its softmax, the hand-offs), so the
-// softmax keeps its per-tile path short: packed fp32 arithmetic for the
-// scaling and the row sum, a signal per warp instead of a warpgroup barrier,
-// and at head dim 64, where the exponentials keep the MUFU unit busy most of
-// the key tile, a quarter of them on the FMA pipe.
+// Each K / V tile is staged once for both query tiles.
 //
 // Warp roles (384 threads, one CTA per SM, persistent over items):
 //   warps 0-3  softmax, O rescale and epilogue of tile A (thread t: row t)
