@@ -213,8 +213,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     auto hint_tiles = [&](int b) -> int {  // key tiles of each group of entry b
       return decode_key_range(hint_len(b), a.Sk, a.Sq, a.causal, a.causal_offset, a.window).tiles;
     };
-    int total = a.bt == nullptr ? units : 0;
-    if (ragged && a.bt == nullptr) {
+    // With lengths, a batch of more than 32 entries gets no hints: its scan
+    // would take a round trip per 32 entries before the wait.
+    int total = a.bt == nullptr && (!ragged || a.B <= 32) ? units : 0;
+    if (ragged && total > 0) {
       total = 0;
       for (int b0 = 0; b0 < a.B; b0 += 32)
         total += __reduce_add_sync(0xffffffffu, b0 + lane < a.B ? gpb * hint_tiles(b0 + lane) : 0);
